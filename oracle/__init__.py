@@ -1,0 +1,116 @@
+"""WKV-7 oracle: plain fp64 CPU recurrence (test infrastructure only).
+
+Only the test suite, the smoke check and the benchmark's CPU-baseline leg may
+import this package.  It loads ``libwkv7_oracle.so`` built from
+``wkv7_oracle.c`` (see :func:`build`), which shares no code with the CUDA
+library.  Inputs are taken as float64 numpy arrays holding the values *after*
+rounding to their storage dtype (bf16 or fp32); the oracle upcasts nothing else
+and rounds nothing.
+
+What is computed, and the passages it follows, is documented in the header of
+``wkv7_oracle.c``.  Every function here is argument marshalling only.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "wkv7_oracle.c")
+_LIB_PATH = os.path.join(_HERE, "libwkv7_oracle.so")
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile the oracle shared object with gcc (no fast-math: the evaluation
+    order is the one written in the C source)."""
+    if force or not os.path.exists(_LIB_PATH) or os.path.getmtime(_LIB_PATH) < os.path.getmtime(_SRC):
+        cmd = ["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-pthread", "-o", _LIB_PATH, _SRC, "-lm"]
+        subprocess.run(cmd, check=True)
+    return _LIB_PATH
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        build()
+        lib = ctypes.CDLL(_LIB_PATH)
+        dp = ctypes.POINTER(ctypes.c_double)
+        ip = ctypes.POINTER(ctypes.c_int32)
+        lib.wkv7_oracle_forward.argtypes = [dp] * 9 + [ctypes.c_int] * 4 + [ip, ctypes.c_int]
+        lib.wkv7_oracle_forward.restype = ctypes.c_int
+        lib.wkv7_oracle_decode_step.argtypes = [dp] * 9 + [ctypes.c_int] * 4
+        lib.wkv7_oracle_decode_step.restype = ctypes.c_int
+        _lib = lib
+    return _lib
+
+
+def _f64(x):
+    if x is None:
+        return None
+    if hasattr(x, "detach"):  # torch tensor (CPU)
+        x = x.detach().to("cpu").double().numpy()
+    return np.ascontiguousarray(np.asarray(x, dtype=np.float64))
+
+
+def _ptr(x):
+    if x is None:
+        return None
+    return x.ctypes.data_as(ctypes.POINTER(ctypes.c_double))
+
+
+def default_threads() -> int:
+    return max(1, os.cpu_count() or 1)
+
+
+def forward(r, w_log, k, v, a, b, s0=None, seq_offsets=None, n_threads=None, want_y=True):
+    """Run the recurrence over whole sequences.
+
+    Dense: r, w_log, k, v, a, b are [B, T, H, D]; packed (``seq_offsets`` given,
+    B+1 int32 entries): they are [T, H, D].  ``s0`` is [B, H, D, D] or None.
+    Returns ``(y, sT)`` as float64 arrays (``y`` is None when ``want_y`` is false).
+    """
+    lib = _load()
+    r, w_log, k, v, a, b = (_f64(t) for t in (r, w_log, k, v, a, b))
+    if seq_offsets is not None:
+        offs = np.ascontiguousarray(np.asarray(seq_offsets, dtype=np.int32))
+        T, H, D = r.shape
+        B = offs.shape[0] - 1
+        offs_p = offs.ctypes.data_as(ctypes.POINTER(ctypes.c_int32))
+    else:
+        B, T, H, D = r.shape
+        offs_p = None
+    for t in (w_log, k, v, a, b):
+        if t.shape != r.shape:
+            raise ValueError("input shapes differ")
+    s0 = _f64(s0)
+    if s0 is not None and s0.shape != (B, H, D, D):
+        raise ValueError("s0 must be [B, H, D, D]")
+    y = np.empty_like(r) if want_y else None
+    sT = np.empty((B, H, D, D), dtype=np.float64)
+    nt = default_threads() if n_threads is None else n_threads
+    rc = lib.wkv7_oracle_forward(_ptr(r), _ptr(w_log), _ptr(k), _ptr(v), _ptr(a), _ptr(b),
+                                 _ptr(s0), _ptr(y), _ptr(sT), B, T, H, D, offs_p, nt)
+    if rc != 0:
+        raise RuntimeError(f"wkv7_oracle_forward failed with status {rc}")
+    return y, sT
+
+
+def decode_step(r, w_log, k, v, a, b, s_in, n_threads=None):
+    """One token per sequence: inputs [B, H, D], state [B, H, D, D].
+    Returns ``(y, s_out)`` as float64 arrays."""
+    lib = _load()
+    r, w_log, k, v, a, b = (_f64(t) for t in (r, w_log, k, v, a, b))
+    B, H, D = r.shape
+    s = _f64(s_in)
+    s_out = np.array(s, dtype=np.float64, copy=True) if s is not None else np.zeros((B, H, D, D))
+    y = np.empty_like(r)
+    nt = default_threads() if n_threads is None else n_threads
+    rc = lib.wkv7_oracle_decode_step(_ptr(r), _ptr(w_log), _ptr(k), _ptr(v), _ptr(a), _ptr(b),
+                                     _ptr(s_out), _ptr(y), _ptr(s_out), B, H, D, nt)
+    if rc != 0:
+        raise RuntimeError(f"wkv7_oracle_decode_step failed with status {rc}")
+    return y, s_out

@@ -1,0 +1,191 @@
+/*
+ * WKV-7 oracle: the plain sequential recurrence in double precision, on the CPU.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing on the product path may call, link or load
+ * this file; only the test suite, the smoke check and the benchmark's CPU
+ * baseline leg use it.  It shares no code, header or constant with the CUDA
+ * library: it parses its own arguments and computes everything from scratch.
+ *
+ * What it computes (per sequence n, head h; S is a D x D matrix, row index i is
+ * the value channel, column index j is the key channel):
+ *
+ *   w_j   = exp(-exp(l_j))                                      (decay)
+ *   sa_i  = sum_j S_ij a_j                                      (uses S_{t-1})
+ *   S_ij <- S_ij w_j + sa_i b_j + v_i k_j                       (state update)
+ *   y_i   = sum_j S_ij r_j                                      (uses S_t)
+ *
+ * Sources:
+ *  - State update S_t = S_{t-1}(diag(w_t) - k^T (a (.) k)) + v^T k: the note
+ *    "RWKV-7 Goose: Expressive Dynamic State Evolution" (myWiki, peng-rwkv7),
+ *    section "Generalized Delta rule", the full state-update formula.  Written
+ *    with a = -kk and b = kk*a_lr the rank-one term is (S a) b^T, which is the
+ *    argument order of the WKV call in the forward listing of
+ *    "RWKV hxa07D architecture explainer" (zenn.dev/openmose), where the
+ *    kernel receives (r, log_neglog_w, k, v, -kk, kk*a).
+ *  - Decay w = exp(-exp(log_neglog_w)): the same listing, where w is formed
+ *    from log_neglog_w by two exponentials and the kernel is handed the inner
+ *    argument.
+ *  - Read-out after the update (y_t = S_t r_t): "RWKV-7 Goose architecture
+ *    analysis" (youngju.dev), section "Dynamic State Evolution", whose
+ *    per-token loop updates the state and then reads the output from it.
+ *  - Padding / variable length: the same WKV call takes an attention mask "for
+ *    variable length and padding"; here sequences are given by offsets into a
+ *    packed token axis and each sequence starts from its own initial state.
+ *
+ * Layouts (all double, contiguous, the fastest index last):
+ *  dense  (seq_offsets == NULL): r, w_log, k, v, a, b, y are [B][T][H][D]
+ *  packed (seq_offsets != NULL): they are [T][H][D] with T the packed length and
+ *          sequence n occupying tokens [seq_offsets[n], seq_offsets[n+1]).
+ *  s0, sT: [B][H][D][D] with S[i][j], i = value, j = key.  s0 == NULL means a
+ *          zero initial state; sT == NULL means the final state is not stored.
+ */
+#include <math.h>
+#include <pthread.h>
+#include <stddef.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+typedef struct {
+    const double *r, *w_log, *k, *v, *a, *b, *s0;
+    double *y, *sT;
+    int B, T, H, D;
+    const int32_t *seq_offsets;
+    long next_unit; /* shared work counter, guarded by lock */
+    pthread_mutex_t lock;
+    int status;
+} oracle_job;
+
+/* One (sequence, head) unit: tokens [t_begin, t_end) of the token axis. */
+static void run_unit(const oracle_job *job, int n, int h, long t_begin, long t_end,
+                     long token_stride, double *S, double *sa, double *w) {
+    const int D = job->D;
+    const long head_off = (long)h * D;
+    if (job->s0) {
+        memcpy(S, job->s0 + ((long)n * job->H + h) * D * D, sizeof(double) * D * D);
+    } else {
+        memset(S, 0, sizeof(double) * D * D);
+    }
+    for (long t = t_begin; t < t_end; ++t) {
+        const long off = t * token_stride + head_off;
+        const double *r = job->r + off, *wl = job->w_log + off, *k = job->k + off;
+        const double *v = job->v + off, *a = job->a + off, *b = job->b + off;
+        for (int j = 0; j < D; ++j) w[j] = exp(-exp(wl[j]));
+        for (int i = 0; i < D; ++i) {
+            double acc = 0.0;
+            for (int j = 0; j < D; ++j) acc += S[i * D + j] * a[j];
+            sa[i] = acc;
+        }
+        for (int i = 0; i < D; ++i)
+            for (int j = 0; j < D; ++j)
+                S[i * D + j] = S[i * D + j] * w[j] + sa[i] * b[j] + v[i] * k[j];
+        if (job->y) {
+            double *y = job->y + off;
+            for (int i = 0; i < D; ++i) {
+                double acc = 0.0;
+                for (int j = 0; j < D; ++j) acc += S[i * D + j] * r[j];
+                y[i] = acc;
+            }
+        }
+    }
+    if (job->sT) memcpy(job->sT + ((long)n * job->H + h) * D * D, S, sizeof(double) * D * D);
+}
+
+static void *worker(void *arg) {
+    oracle_job *job = (oracle_job *)arg;
+    const int D = job->D;
+    double *S = (double *)malloc(sizeof(double) * D * D);
+    double *sa = (double *)malloc(sizeof(double) * D);
+    double *w = (double *)malloc(sizeof(double) * D);
+    if (!S || !sa || !w) {
+        pthread_mutex_lock(&job->lock);
+        job->status = -2;
+        pthread_mutex_unlock(&job->lock);
+        free(S); free(sa); free(w);
+        return NULL;
+    }
+    const long n_units = (long)job->B * job->H;
+    for (;;) {
+        pthread_mutex_lock(&job->lock);
+        long u = job->next_unit++;
+        pthread_mutex_unlock(&job->lock);
+        if (u >= n_units) break;
+        const int n = (int)(u / job->H), h = (int)(u % job->H);
+        long t_begin, t_end, token_stride;
+        if (job->seq_offsets) {
+            t_begin = job->seq_offsets[n];
+            t_end = job->seq_offsets[n + 1];
+            token_stride = (long)job->H * D;
+        } else {
+            /* dense [B][T][H][D] viewed as a packed axis of B*T tokens */
+            t_begin = (long)n * job->T;
+            t_end = t_begin + job->T;
+            token_stride = (long)job->H * D;
+        }
+        run_unit(job, n, h, t_begin, t_end, token_stride, S, sa, w);
+    }
+    free(S); free(sa); free(w);
+    return NULL;
+}
+
+/*
+ * Returns 0 on success, -1 on an invalid argument, -2 on allocation failure.
+ * n_threads <= 0 means one thread.  y may be NULL (no outputs stored).
+ */
+int wkv7_oracle_forward(const double *r, const double *w_log, const double *k,
+                        const double *v, const double *a, const double *b,
+                        const double *s0, double *y, double *sT,
+                        int B, int T, int H, int D, const int32_t *seq_offsets,
+                        int n_threads) {
+    if (!r || !w_log || !k || !v || !a || !b) return -1;
+    if (B <= 0 || T < 0 || H <= 0 || D <= 0) return -1;
+    if (seq_offsets) {
+        if (seq_offsets[0] != 0 || seq_offsets[B] != T) return -1;
+        for (int n = 0; n < B; ++n)
+            if (seq_offsets[n + 1] < seq_offsets[n]) return -1;
+    }
+    oracle_job job;
+    job.r = r; job.w_log = w_log; job.k = k; job.v = v; job.a = a; job.b = b;
+    job.s0 = s0; job.y = y; job.sT = sT;
+    job.B = B; job.T = T; job.H = H; job.D = D;
+    job.seq_offsets = seq_offsets;
+    job.next_unit = 0;
+    job.status = 0;
+    pthread_mutex_init(&job.lock, NULL);
+    if (n_threads <= 1) {
+        worker(&job);
+    } else {
+        pthread_t *tid = (pthread_t *)malloc(sizeof(pthread_t) * n_threads);
+        if (!tid) { pthread_mutex_destroy(&job.lock); return -2; }
+        int started = 0;
+        for (int i = 0; i < n_threads; ++i) {
+            if (pthread_create(&tid[i], NULL, worker, &job) != 0) break;
+            ++started;
+        }
+        if (started == 0) worker(&job);
+        for (int i = 0; i < started; ++i) pthread_join(tid[i], NULL);
+        free(tid);
+    }
+    pthread_mutex_destroy(&job.lock);
+    return job.status;
+}
+
+/*
+ * One recurrent decoding step (a single token per sequence), the RNN mode of
+ * "RWKV-7 Goose architecture analysis", section on RNN-mode inference: the
+ * state [B][H][D][D] is read from s_in and written to s_out (they may alias);
+ * inputs and y are [B][H][D].
+ */
+int wkv7_oracle_decode_step(const double *r, const double *w_log, const double *k,
+                            const double *v, const double *a, const double *b,
+                            const double *s_in, double *y, double *s_out,
+                            int B, int H, int D, int n_threads) {
+    if (!s_out) return -1;
+    if (s_in && s_in != s_out)
+        memmove(s_out, s_in, sizeof(double) * (size_t)B * H * D * D);
+    else if (!s_in)
+        memset(s_out, 0, sizeof(double) * (size_t)B * H * D * D);
+    /* a dense call with T = 1 whose initial and final state are the same buffer */
+    return wkv7_oracle_forward(r, w_log, k, v, a, b, s_out, y, s_out, B, 1, H, D, NULL,
+                               n_threads);
+}
