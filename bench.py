@@ -1,0 +1,338 @@
+"""WKV-7 benchmark: chunked prefill tokens/s (headline) and decode steps/s on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+One JSON line on rank 0.  `value` is prefill tokens/s of the whole job for the
+B4 T1024 H32 D64 prefill (bf16 inputs, fp32 decay logits, zero initial state),
+timed with CUDA events per launch on the launching stream, L2 flushed (a
+256 MB write) between timed launches.  `e2e` is the same metric through the
+public API from pinned host buffers (host->device copies of the inputs and
+device->host copies of y and sT inside the timed region).  `decode` reports
+the B256 H40 decode step with the fp32 state carried through 128 steps.
+Multi-GPU: every rank runs the same per-GPU workload on its own device
+(independent (sequence, head) units, no collective on the data path); the job
+time is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "WKV7 prefill tokens/s and decode steps/s on 1 B200; % of roofline"
+PREFILL_WORKLOAD = "prefill_1p5b"
+DECODE_WORKLOAD = "decode_2p9b"
+D = 64
+L2_FLUSH_BYTES = 256 << 20
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d.get("hbm_gbs", 6650.0), d.get("bf16_tflops", 1590.0), "measured"
+    return 6650.0, 1590.0, "fallback"
+
+
+def prefill_bytes(n_tokens_heads, io_b, w_b, n_states, with_s0):
+    """Algorithmic HBM bytes: r, k, v, a, b read and y written once (io_b each),
+    w_log read once (w_b), sT written once (and s0 read once when given)."""
+    per = D * (6 * io_b + w_b)
+    return n_tokens_heads * per + n_states * D * D * 4 * (2 if with_s0 else 1)
+
+
+def prefill_flops(n_tokens_heads, L=64):
+    return n_tokens_heads * (15 * L * D + 8 * D * D)
+
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons during a timed region."""
+
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except (FileNotFoundError, OSError):
+            self.proc = None
+        time.sleep(0.3)
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.2)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax.append(float(parts[2]))
+            except ValueError:
+                continue
+            for nm, val in zip(names, parts[5:9]):
+                if val.lower().startswith("active"):
+                    reasons.add(nm)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def time_launches(fn, steps, stream, flush=None):
+    """Per-launch CUDA-event times (ms) on `stream`; `flush` runs between launches, untimed."""
+    import torch
+
+    times = []
+    for _ in range(steps):
+        if flush is not None:
+            flush()
+        s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s.record(stream)
+        fn()
+        e.record(stream)
+        times.append((s, e))
+    torch.cuda.synchronize()
+    return [s.elapsed_time(e) for s, e in times]
+
+
+def oracle_baseline(budget_s=20.0):
+    """The oracle, as it stands, on a bounded sample of the prefill workload:
+    whole sequences of a subset of heads, grown until ~budget_s of CPU work."""
+    import numpy as np
+
+    import oracle
+    import wkv7_inputs as W
+
+    oracle.build()
+    inp = W.make_workload(PREFILL_WORKLOAD)
+    t = inp.tensors()
+    threads = oracle.default_threads()
+    heads = 1
+    total_tokens, total_s = 0, 0.0
+    while True:
+        hs = list(range(heads))
+        sub = {k: v[:, :, hs].contiguous().double().numpy() for k, v in t.items()}
+        t0 = time.perf_counter()
+        oracle.forward(sub["r"], sub["w_log"], sub["k"], sub["v"], sub["a"], sub["b"], None, n_threads=threads)
+        dt = time.perf_counter() - t0
+        total_tokens += inp.B * inp.T * heads
+        total_s += dt
+        if total_s >= budget_s or heads >= inp.H:
+            break
+        heads = min(inp.H, heads * 2)
+    # tokens/s in units of full-width tokens (all H heads), like the GPU number
+    tok_s = total_tokens / inp.H / total_s
+    return {"value": tok_s, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+            "sample": f"prefill_1p5b (B4 T1024), whole sequences of 1..{heads} of 32 heads, "
+                      f"{total_tokens} token-heads in {total_s:.1f} s; tokens counted as token-heads/32"}
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    cb = oracle_baseline(budget_s=max(5.0, min(60.0, 3.0 * args.steps)))
+    line = {"impl": "reference", "metric": METRIC, "value": cb["value"], "unit": "tokens/s",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": 1000.0 * 4 * 1024 / cb["value"], "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": PREFILL_WORKLOAD, "B": 4, "T": 1024, "H": 32, "D": D},
+            "cpu_baseline": cb,
+            "e2e": {"value": cb["value"], "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+
+    import linear_recurrent_lm_wkv7_b200 as wk
+    import wkv7_inputs as W
+
+    hbm_peak, bf16_peak, peak_src = measured_peaks()
+    stream = torch.cuda.current_stream()
+    flush_buf = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+    flush = lambda: flush_buf.zero_()
+
+    # ---------------- prefill (headline)
+    inp = W.make_workload(PREFILL_WORKLOAD, seed=1 + 1000 * rank)
+    B, T, H = inp.B, inp.T, inp.H
+    host = {k: v.pin_memory() for k, v in inp.tensors().items()}
+    dev = {k: v.cuda() for k, v in host.items()}
+    y = torch.empty_like(dev["r"])
+    sT = torch.empty((B, H, D, D), dtype=torch.float32, device="cuda")
+
+    def step():
+        wk.wkv7_forward(dev["r"], dev["w_log"], dev["k"], dev["v"], dev["a"], dev["b"], None, y, sT, B, T, H, D,
+                        None, stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if wk.wkv7_get_device_status() != 0:
+        raise RuntimeError("device status set during warm-up")
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    clk = ClockSampler(local)
+    clk.start()
+    times = time_launches(step, args.steps, stream, flush)
+    clocks = clk.stop()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    ms = sum(times) / len(times)
+    if world > 1:
+        t = torch.tensor([ms], device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    tokens = B * T
+    value = world * tokens / (ms * 1e-3)
+    bytes_alg = prefill_bytes(B * T * H, 2, 4, B * H, with_s0=False)
+    achieved = bytes_alg / (ms * 1e-3) / 1e9
+    flops = prefill_flops(B * T * H)
+
+    # ---------------- end to end through the public API from pinned host memory
+    y_h = torch.empty(y.shape, dtype=y.dtype).pin_memory()
+    sT_h = torch.empty(sT.shape, dtype=sT.dtype).pin_memory()
+    h2d = sum(v.numel() * v.element_size() for v in host.values())
+    d2h = y_h.numel() * y_h.element_size() + sT_h.numel() * sT_h.element_size()
+
+    def e2e_step():
+        for k_, v_ in host.items():
+            dev[k_].copy_(v_, non_blocking=True)
+        step()
+        y_h.copy_(y, non_blocking=True)
+        sT_h.copy_(sT, non_blocking=True)
+
+    for _ in range(2):
+        e2e_step()
+    torch.cuda.synchronize()
+    e2e_times = time_launches(e2e_step, max(3, args.steps // 4), stream, flush)
+    e2e_ms = sum(e2e_times) / len(e2e_times)
+    if world > 1:
+        t = torch.tensor([e2e_ms], device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    e2e_value = world * tokens / (e2e_ms * 1e-3)
+    del dev, host
+
+    # ---------------- decode step (B256 H40, state carried through 128 steps)
+    cfg = W.WORKLOADS[DECODE_WORKLOAD]
+    dB, dH, nsteps = cfg["B"], cfg["H"], cfg["steps"]
+    state = W.make_state(dB, dH, std=cfg["s0_std"], seed=cfg["seed"]).cuda()
+    dsteps = [{k: v.cuda() for k, v in W.make_decode_step(dB, dH, io=cfg["io"], wdt=cfg["wdt"], seed=cfg["seed"],
+                                                          step=s).tensors().items()} for s in range(nsteps)]
+    dy = torch.empty((dB, dH, D), dtype=torch.bfloat16, device="cuda")
+    it = {"i": 0}
+
+    def dstep():
+        d = dsteps[it["i"] % nsteps]
+        it["i"] += 1
+        wk.wkv7_decode_step(d["r"], d["w_log"], d["k"], d["v"], d["a"], d["b"], state, dy, state, dB, dH, D, stream)
+
+    for _ in range(max(3, args.warmup)):
+        dstep()
+    torch.cuda.synchronize()
+    it["i"] = 0
+    dtimes = time_launches(dstep, nsteps, stream, None)  # state (168 MB x2) exceeds L2 by itself
+    if wk.wkv7_get_device_status() != 0:
+        raise RuntimeError("device status set during the run")
+    dms = sum(dtimes) / len(dtimes)
+    if world > 1:
+        t = torch.tensor([dms], device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        dms = float(t.item())
+    dbytes = 2 * dB * dH * D * D * 4 + dB * dH * D * (6 * 2 + 2)
+    dach = dbytes / (dms * 1e-3) / 1e9
+
+    if rank == 0:
+        cb = oracle_baseline(budget_s=20.0) if (world == 1 and not args.no_cpu_baseline) else None
+        line = {
+            "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": PREFILL_WORKLOAD, "B": B, "T": T, "H": H, "D": D, "io": "bf16",
+                       "w_log": "f32", "s0": "zero", "chunk": 64, "l2": "flushed (256 MB write) between launches",
+                       "parallelism": f"replicas{world}" if world > 1 else "single"},
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
+                         "frac": achieved / hbm_peak, "traffic": None, "peak_source": peak_src,
+                         "algorithmic_bytes_per_launch": bytes_alg,
+                         "tensor_flop_per_launch": flops,
+                         "tensor_time_floor_us": flops / (bf16_peak * 1e12) * 1e6,
+                         "hbm_time_floor_us": bytes_alg / (hbm_peak * 1e9) * 1e6},
+            "cpu_baseline": cb,
+            "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                    "ms_per_step": e2e_ms},
+            "gpu_launches": args.steps,
+            "clocks": clocks,
+            "decode": {"workload": DECODE_WORKLOAD, "B": dB, "H": dH, "steps_per_s": 1000.0 / dms,
+                       "tokens_per_s": world * dB / (dms * 1e-3), "ms_per_step": dms,
+                       "roofline": {"bound": "hbm", "achieved": dach, "peak": hbm_peak, "unit": "GB/s",
+                                    "frac": dach / hbm_peak, "algorithmic_bytes_per_launch": dbytes}},
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,129 @@
+/*
+ * wkv7.h — C ABI of the B200 (sm_100a) WKV-7 library, libwkv7.so.
+ *
+ * The operator is the RWKV-7 "Goose" time-mixing recurrence.  Per sequence n
+ * and head h it keeps a D x D fp32 state S (S[i][j]: i = value channel, j = key
+ * channel) and, for every token t,
+ *
+ *     w_t = exp(-exp(w_log_t))                              (per key channel)
+ *     S_t = S_{t-1} diag(w_t) + (S_{t-1} a_t) b_t^T + v_t k_t^T
+ *     y_t = S_t r_t
+ *
+ * Sources: the state update is the generalized delta rule of the note
+ * "RWKV-7 Goose: Expressive Dynamic State Evolution" (section "Generalized
+ * Delta rule", full state-update formula), S_t = S_{t-1}(diag(w_t) -
+ * kk^T (a (.) kk)) + v^T k, written here with a = -kk and b = kk (.) a_lr as in
+ * the WKV call of the forward listing of "RWKV hxa07D architecture explainer"
+ * (zenn.dev/openmose), which hands the kernel (r, log_neglog_w, k, v, -kk,
+ * kk*a) as B,T,C tensors; w_log is that listing's log_neglog_w.  The output is
+ * read from the updated state ("RWKV-7 Goose architecture analysis",
+ * youngju.dev, section "Dynamic State Evolution").  Constant-size state and
+ * token-by-token decoding: the same page's RNN-mode section.
+ *
+ * Conventions shared by every entry point
+ *  - All tensor arguments are caller-owned DEVICE memory, contiguous, with the
+ *    fastest index last.  The library allocates no device memory and keeps no
+ *    handle between calls; it only launches kernels on `stream` (a
+ *    cudaStream_t; NULL is the legacy default stream) and never synchronizes
+ *    the host, except in wkv7_get_device_status.
+ *  - Element types are passed as codes (enum wkv7_dtype): `io_dtype` for r, k,
+ *    v, a, b and y; `w_dtype` for w_log.  States are always fp32.
+ *  - D must be 64 (the head size of the RWKV-7 layers the pages describe);
+ *    other head sizes return WKV7_ERR_UNSUPPORTED.
+ *  - Every pointer must be 16-byte aligned (WKV7_ERR_MISALIGNED otherwise).
+ *  - Documented, unchecked precondition: w_log <= -0.5 or w_log = -inf, i.e.
+ *    w in [exp(-exp(-0.5)), 1] ~= [0.545, 1], the range produced by the
+ *    hxa07D decay parametrisation -softplus(-x) - 0.5.  w_log = -inf gives
+ *    w = 1 exactly (used for padding).
+ *  - Errors in the arguments are detected on the host before anything is
+ *    launched and returned as a negative status; nothing is written then.
+ *    Errors that only the device can see (a bounded wait that expired, packed
+ *    offsets out of range) are recorded in a per-device status word and
+ *    reported by wkv7_get_device_status.  No kernel traps or asserts.
+ */
+#ifndef WKV7_H
+#define WKV7_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    WKV7_F32 = 0,  /* IEEE binary32 */
+    WKV7_BF16 = 1  /* bfloat16 */
+} wkv7_dtype;
+
+typedef enum {
+    WKV7_OK = 0,
+    WKV7_ERR_INVALID_ARG = -1,    /* null pointer, bad size, bad dtype code, aliasing */
+    WKV7_ERR_UNSUPPORTED = -2,    /* D != 64, or no sm_100 device */
+    WKV7_ERR_MISALIGNED = -3,     /* a pointer not 16-byte aligned */
+    WKV7_ERR_CUDA = -4,           /* a CUDA runtime call or a launch failed */
+    WKV7_ERR_DEVICE_TIMEOUT = -5, /* a bounded device-side wait expired */
+    WKV7_ERR_DEVICE_BOUNDS = -6   /* packed offsets not monotone or beyond T */
+} wkv7_status;
+
+/*
+ * wkv7_forward — chunked prefill over whole sequences.
+ *
+ * Dense batch (seq_offsets == NULL):
+ *   r, w_log, k, v, a, b, y : [B][T][H][D]  (the B,T,C layout with C = H*D)
+ * Packed variable-length batch (seq_offsets != NULL):
+ *   r, w_log, k, v, a, b, y : [T][H][D] with T the packed token count;
+ *   seq_offsets: DEVICE int32[B+1], non-decreasing, seq_offsets[0] = 0,
+ *   seq_offsets[B] = T; sequence n owns tokens [seq_offsets[n], seq_offsets[n+1]).
+ *   Pad tokens are ordinary tokens carrying w_log = -inf and k = v = a = b = 0,
+ *   which leave the state unchanged (the "attention_mask ... for variable length
+ *   and padding" of the hxa07D WKV call).
+ * s0 : [B][H][D][D] fp32 initial states, or NULL for zero states.
+ * sT : [B][H][D][D] fp32 final states, or NULL to skip writing them.  sT == s0
+ *      (state carried in place) is allowed; any other overlap is not.
+ * y  : output, same shape and dtype code as r; must not overlap any input.
+ * T == 0 is valid: y is empty and sT receives s0 (or zeros).
+ * Returns WKV7_OK once the work is enqueued on `stream`.
+ */
+int wkv7_forward(const void* r, const void* w_log, const void* k, const void* v,
+                 const void* a, const void* b, const float* s0, void* y, float* sT,
+                 int B, int T, int H, int D, const int32_t* seq_offsets,
+                 int io_dtype, int w_dtype, void* stream);
+
+/*
+ * wkv7_decode_step — one token per sequence (RNN mode).
+ *   r, w_log, k, v, a, b, y : [B][H][D]
+ *   s_in, s_out            : [B][H][D][D] fp32; s_in == s_out (in place) is
+ *                            allowed, any other overlap is not.  s_in == NULL
+ *                            means a zero state.
+ * Returns WKV7_OK once the step is enqueued on `stream`.
+ */
+int wkv7_decode_step(const void* r, const void* w_log, const void* k, const void* v,
+                     const void* a, const void* b, const float* s_in, void* y, float* s_out,
+                     int B, int H, int D, int io_dtype, int w_dtype, void* stream);
+
+/* Human-readable text for a status code (static storage, never NULL). */
+const char* wkv7_status_string(int status);
+
+/*
+ * Synchronizes `stream`, then reads and clears the status word of the current
+ * device.  Returns WKV7_OK, WKV7_ERR_DEVICE_TIMEOUT, WKV7_ERR_DEVICE_BOUNDS, or
+ * WKV7_ERR_CUDA if the synchronization itself failed.
+ */
+int wkv7_get_device_status(void* stream);
+
+/*
+ * Test hook for the bounded-wait path: launches one block that waits on a
+ * barrier nothing ever completes, with a limit of `spins` polls, then records
+ * WKV7_ERR_DEVICE_TIMEOUT in the status word and returns.  Nothing else runs
+ * and nothing is left in flight.  spins must be in [1, 1<<20].
+ */
+int wkv7_debug_expire_wait(int spins, void* stream);
+
+/* Library version as major*10000 + minor*100 + patch. */
+int wkv7_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* WKV7_H */

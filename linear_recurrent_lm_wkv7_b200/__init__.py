@@ -1,0 +1,56 @@
+"""B200 (sm_100a) WKV-7 operator: chunked tensor-core prefill and streaming
+decode step behind a C ABI (``include/wkv7.h``, ``libwkv7.so``).
+
+The Python layer only marshals arguments to the CUDA library; importing the
+package loads ``libwkv7.so`` and fails loudly if it has not been built.
+Convenience wrappers ``forward`` and ``decode_step`` allocate outputs with
+torch and call the C entry points.
+"""
+from __future__ import annotations
+
+from ._binding import (  # noqa: F401
+    EXPORTS,
+    LIB_PATH,
+    STATUS,
+    WKV7_BF16,
+    WKV7_F32,
+    Wkv7Error,
+    _lib,
+    wkv7_debug_expire_wait,
+    wkv7_decode_step,
+    wkv7_forward,
+    wkv7_get_device_status,
+    wkv7_status_string,
+    wkv7_version,
+)
+
+_lib()  # load now: a missing or broken library is an import error, never a silent fallback
+
+
+def forward(r, w_log, k, v, a, b, s0=None, seq_offsets=None, want_state=True, stream=None):
+    """Chunked prefill.  Dense inputs are [B, T, H, D]; packed inputs are
+    [T, H, D] with int32 ``seq_offsets`` [B+1] on the device.  Returns
+    ``(y, sT)`` (``sT`` is None when ``want_state`` is false)."""
+    import torch
+
+    if seq_offsets is not None:
+        T, H, D = r.shape
+        B = seq_offsets.numel() - 1
+    else:
+        B, T, H, D = r.shape
+    y = torch.empty_like(r)
+    sT = torch.empty((B, H, D, D), dtype=torch.float32, device=r.device) if want_state else None
+    wkv7_forward(r, w_log, k, v, a, b, s0, y, sT, B, T, H, D, seq_offsets, stream)
+    return y, sT
+
+
+def decode_step(r, w_log, k, v, a, b, state, y=None, stream=None):
+    """One decoding step, updating ``state`` ([B, H, D, D] fp32) in place.
+    Returns y ([B, H, D])."""
+    import torch
+
+    B, H, D = r.shape
+    if y is None:
+        y = torch.empty_like(r)
+    wkv7_decode_step(r, w_log, k, v, a, b, state, y, state, B, H, D, stream)
+    return y

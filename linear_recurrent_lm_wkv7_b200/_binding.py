@@ -1,0 +1,142 @@
+"""ctypes binding of libwkv7.so (include/wkv7.h).
+
+Argument marshalling only: tensors are passed as raw device pointers, dtype
+codes are derived from the tensors, and the current torch CUDA stream is used
+unless one is given.  Every call runs in the CUDA library; there is no fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(PKG, "libwkv7.so")
+
+WKV7_F32 = 0
+WKV7_BF16 = 1
+
+STATUS = {
+    0: "WKV7_OK",
+    -1: "WKV7_ERR_INVALID_ARG",
+    -2: "WKV7_ERR_UNSUPPORTED",
+    -3: "WKV7_ERR_MISALIGNED",
+    -4: "WKV7_ERR_CUDA",
+    -5: "WKV7_ERR_DEVICE_TIMEOUT",
+    -6: "WKV7_ERR_DEVICE_BOUNDS",
+}
+# every symbol include/wkv7.h declares
+EXPORTS = (
+    "wkv7_forward",
+    "wkv7_decode_step",
+    "wkv7_status_string",
+    "wkv7_get_device_status",
+    "wkv7_debug_expire_wait",
+    "wkv7_version",
+)
+
+
+class Wkv7Error(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {STATUS.get(status, status)} ({_lib().wkv7_status_string(status).decode()})")
+
+
+_LIB = None
+
+
+def _lib():
+    global _LIB
+    if _LIB is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(
+                f"{LIB_PATH} is missing: build it with `python -m linear_recurrent_lm_wkv7_b200.build`")
+        lib = ctypes.CDLL(LIB_PATH)
+        vp, i = ctypes.c_void_p, ctypes.c_int
+        lib.wkv7_forward.argtypes = [vp] * 9 + [i] * 4 + [vp, i, i, vp]
+        lib.wkv7_forward.restype = i
+        lib.wkv7_decode_step.argtypes = [vp] * 9 + [i] * 3 + [i, i, vp]
+        lib.wkv7_decode_step.restype = i
+        lib.wkv7_status_string.argtypes = [i]
+        lib.wkv7_status_string.restype = ctypes.c_char_p
+        lib.wkv7_get_device_status.argtypes = [vp]
+        lib.wkv7_get_device_status.restype = i
+        lib.wkv7_debug_expire_wait.argtypes = [i, vp]
+        lib.wkv7_debug_expire_wait.restype = i
+        lib.wkv7_version.argtypes = []
+        lib.wkv7_version.restype = i
+        _LIB = lib
+    return _LIB
+
+
+def _dtype_code(t):
+    import torch
+
+    if t.dtype == torch.float32:
+        return WKV7_F32
+    if t.dtype == torch.bfloat16:
+        return WKV7_BF16
+    raise TypeError(f"unsupported dtype {t.dtype}")
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("tensors must live on a CUDA device")
+    if not t.is_contiguous():
+        raise ValueError("tensors must be contiguous")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    import torch
+
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
+
+
+def wkv7_forward(r, w_log, k, v, a, b, s0, y, sT, B, T, H, D, seq_offsets=None, stream=None):
+    """Enqueue the chunked prefill (see include/wkv7.h).  Raises Wkv7Error on a
+    non-OK status."""
+    st = _lib().wkv7_forward(_ptr(r), _ptr(w_log), _ptr(k), _ptr(v), _ptr(a), _ptr(b), _ptr(s0), _ptr(y),
+                             _ptr(sT), int(B), int(T), int(H), int(D), _ptr(seq_offsets), _dtype_code(r),
+                             _dtype_code(w_log), _stream(stream))
+    if st != 0:
+        raise Wkv7Error(st, "wkv7_forward")
+
+
+def wkv7_decode_step(r, w_log, k, v, a, b, s_in, y, s_out, B, H, D, stream=None):
+    """Enqueue one decoding step (see include/wkv7.h)."""
+    st = _lib().wkv7_decode_step(_ptr(r), _ptr(w_log), _ptr(k), _ptr(v), _ptr(a), _ptr(b), _ptr(s_in), _ptr(y),
+                                 _ptr(s_out), int(B), int(H), int(D), _dtype_code(r), _dtype_code(w_log),
+                                 _stream(stream))
+    if st != 0:
+        raise Wkv7Error(st, "wkv7_decode_step")
+
+
+def wkv7_get_device_status(stream=None) -> int:
+    return int(_lib().wkv7_get_device_status(_stream(stream)))
+
+
+def wkv7_debug_expire_wait(spins: int, stream=None) -> None:
+    st = _lib().wkv7_debug_expire_wait(int(spins), _stream(stream))
+    if st != 0:
+        raise Wkv7Error(st, "wkv7_debug_expire_wait")
+
+
+def wkv7_status_string(status: int) -> str:
+    return _lib().wkv7_status_string(int(status)).decode()
+
+
+def wkv7_version() -> int:
+    return int(_lib().wkv7_version())
+
+
+def raw_call_forward(*args):
+    """Direct C call with raw integer pointers (used by host-validation tests)."""
+    return int(_lib().wkv7_forward(*args))
+
+
+def raw_call_decode(*args):
+    return int(_lib().wkv7_decode_step(*args))

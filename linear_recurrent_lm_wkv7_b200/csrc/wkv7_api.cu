@@ -1,0 +1,187 @@
+// wkv7_api.cu — the C ABI declared in include/wkv7.h: argument validation on
+// the host, dispatch to the kernels, and the per-device status word.
+#include <cstdint>
+#include <cstring>
+
+#include "wkv7_internal.cuh"
+
+namespace {
+
+// One status word per device that loads the library: kernels record the first
+// device-side error here (atomicCAS from 0); wkv7_get_device_status reads and
+// clears it.
+__device__ int g_status = 0;
+
+constexpr int kMaxDevices = 64;
+int* g_status_ptr[kMaxDevices] = {};
+
+int status_ptr(int** out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return WKV7_ERR_CUDA;
+    if (!g_status_ptr[dev]) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_status) != cudaSuccess) return WKV7_ERR_CUDA;
+        g_status_ptr[dev] = static_cast<int*>(p);
+    }
+    *out = g_status_ptr[dev];
+    return WKV7_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool dtype_ok(int d) { return d == WKV7_F32 || d == WKV7_BF16; }
+size_t dtype_bytes(int d) { return d == WKV7_F32 ? 4 : 2; }
+
+bool overlaps(const void* p, size_t pn, const void* q, size_t qn) {
+    if (!p || !q || pn == 0 || qn == 0) return false;
+    const uintptr_t a = reinterpret_cast<uintptr_t>(p), b = reinterpret_cast<uintptr_t>(q);
+    return a < b + qn && b < a + pn;
+}
+
+int check_device() {
+    int dev = 0;
+    cudaDeviceProp prop;
+    if (cudaGetDevice(&dev) != cudaSuccess) return WKV7_ERR_CUDA;
+    if (cudaGetDeviceProperties(&prop, dev) != cudaSuccess) return WKV7_ERR_CUDA;
+    if (prop.major != 10) return WKV7_ERR_UNSUPPORTED;
+    return WKV7_OK;
+}
+
+int cached_device_check() {
+    static int cache[kMaxDevices] = {};  // 0 unknown, 1 ok, else status
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return WKV7_ERR_CUDA;
+    if (cache[dev] == 0) {
+        const int s = check_device();
+        cache[dev] = (s == WKV7_OK) ? 1 : s;
+    }
+    return cache[dev] == 1 ? WKV7_OK : cache[dev];
+}
+
+// Zero-token call: sT <- s0 (or zeros).
+__global__ void copy_or_zero_states(const float* __restrict__ s0, float* __restrict__ sT, long n) {
+    const long i = static_cast<long>(blockIdx.x) * blockDim.x + threadIdx.x;
+    const long stride = static_cast<long>(gridDim.x) * blockDim.x;
+    for (long e = i; e < n; e += stride) sT[e] = s0 ? s0[e] : 0.f;
+}
+
+}  // namespace
+
+extern "C" {
+
+int wkv7_version(void) { return 1 * 10000 + 0 * 100 + 0; }
+
+const char* wkv7_status_string(int status) {
+    switch (status) {
+        case WKV7_OK: return "ok";
+        case WKV7_ERR_INVALID_ARG: return "invalid argument";
+        case WKV7_ERR_UNSUPPORTED: return "unsupported (head size must be 64 on an sm_100 device)";
+        case WKV7_ERR_MISALIGNED: return "pointer not 16-byte aligned";
+        case WKV7_ERR_CUDA: return "CUDA runtime error";
+        case WKV7_ERR_DEVICE_TIMEOUT: return "device-side bounded wait expired";
+        case WKV7_ERR_DEVICE_BOUNDS: return "packed sequence offsets out of range";
+        default: return "unknown status";
+    }
+}
+
+int wkv7_forward(const void* r, const void* w_log, const void* k, const void* v, const void* a, const void* b,
+                 const float* s0, void* y, float* sT, int B, int T, int H, int D, const int32_t* seq_offsets,
+                 int io_dtype, int w_dtype, void* stream) {
+    // ---- host-side validation; nothing is launched on failure
+    if (B <= 0 || T < 0 || H <= 0 || D <= 0) return WKV7_ERR_INVALID_ARG;
+    if (!dtype_ok(io_dtype) || !dtype_ok(w_dtype)) return WKV7_ERR_INVALID_ARG;
+    if (D != wkv7::kHead) return WKV7_ERR_UNSUPPORTED;
+    if (T > 0 && (!r || !w_log || !k || !v || !a || !b || !y)) return WKV7_ERR_INVALID_ARG;
+    const void* ptrs[] = {r, w_log, k, v, a, b, s0, y, sT, seq_offsets};
+    for (const void* p : ptrs)
+        if (p && !aligned16(p)) return WKV7_ERR_MISALIGNED;
+    const long tokens = seq_offsets ? static_cast<long>(T) : static_cast<long>(B) * T;
+    const size_t n_act = static_cast<size_t>(tokens) * H * D;
+    const size_t n_state = static_cast<size_t>(B) * H * D * D;
+    const size_t io_b = dtype_bytes(io_dtype), w_b = dtype_bytes(w_dtype);
+    const void* ins[] = {r, k, v, a, b};
+    for (const void* p : ins)
+        if (overlaps(y, n_act * io_b, p, n_act * io_b)) return WKV7_ERR_INVALID_ARG;
+    if (overlaps(y, n_act * io_b, w_log, n_act * w_b) || overlaps(y, n_act * io_b, s0, n_state * 4) ||
+        overlaps(y, n_act * io_b, sT, n_state * 4))
+        return WKV7_ERR_INVALID_ARG;
+    // sT == s0 is allowed: each (sequence, head) block reads its own initial state
+    // before it writes its own final state.  Any other overlap is rejected.
+    if (sT && sT != s0 && overlaps(sT, n_state * 4, s0, n_state * 4)) return WKV7_ERR_INVALID_ARG;
+    if (n_act > 0) {
+        for (const void* p : ins)
+            if (overlaps(sT, n_state * 4, p, n_act * io_b)) return WKV7_ERR_INVALID_ARG;
+        if (overlaps(sT, n_state * 4, w_log, n_act * w_b)) return WKV7_ERR_INVALID_ARG;
+    }
+
+    int dev_ok = cached_device_check();
+    if (dev_ok != WKV7_OK) return dev_ok;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (T == 0) {
+        if (!sT) return WKV7_OK;
+        const long n = static_cast<long>(n_state);
+        const int blocks = static_cast<int>((n + 255) / 256 < 1184 ? (n + 255) / 256 : 1184);
+        copy_or_zero_states<<<blocks, 256, 0, st>>>(s0, sT, n);
+        return cudaGetLastError() == cudaSuccess ? WKV7_OK : WKV7_ERR_CUDA;
+    }
+    int* status = nullptr;
+    if (status_ptr(&status) != WKV7_OK) return WKV7_ERR_CUDA;
+    wkv7::PrefillArgs p{r, w_log, k, v, a, b, s0, y, sT, B, T, H, seq_offsets, status};
+    return wkv7::launch_prefill(p, io_dtype, w_dtype, st) == cudaSuccess ? WKV7_OK : WKV7_ERR_CUDA;
+}
+
+int wkv7_decode_step(const void* r, const void* w_log, const void* k, const void* v, const void* a, const void* b,
+                     const float* s_in, void* y, float* s_out, int B, int H, int D, int io_dtype, int w_dtype,
+                     void* stream) {
+    if (B <= 0 || H <= 0 || D <= 0) return WKV7_ERR_INVALID_ARG;
+    if (!dtype_ok(io_dtype) || !dtype_ok(w_dtype)) return WKV7_ERR_INVALID_ARG;
+    if (D != wkv7::kHead) return WKV7_ERR_UNSUPPORTED;
+    if (!r || !w_log || !k || !v || !a || !b || !y || !s_out) return WKV7_ERR_INVALID_ARG;
+    const void* ptrs[] = {r, w_log, k, v, a, b, s_in, y, s_out};
+    for (const void* p : ptrs)
+        if (p && !aligned16(p)) return WKV7_ERR_MISALIGNED;
+    const size_t n_act = static_cast<size_t>(B) * H * D;
+    const size_t n_state = static_cast<size_t>(B) * H * D * D;
+    const size_t io_b = dtype_bytes(io_dtype), w_b = dtype_bytes(w_dtype);
+    const void* ins[] = {r, k, v, a, b};
+    for (const void* p : ins) {
+        if (overlaps(y, n_act * io_b, p, n_act * io_b)) return WKV7_ERR_INVALID_ARG;
+        if (overlaps(s_out, n_state * 4, p, n_act * io_b)) return WKV7_ERR_INVALID_ARG;
+    }
+    if (overlaps(y, n_act * io_b, w_log, n_act * w_b) || overlaps(y, n_act * io_b, s_in, n_state * 4) ||
+        overlaps(y, n_act * io_b, s_out, n_state * 4) || overlaps(s_out, n_state * 4, w_log, n_act * w_b))
+        return WKV7_ERR_INVALID_ARG;
+    if (s_in && s_in != s_out && overlaps(s_in, n_state * 4, s_out, n_state * 4)) return WKV7_ERR_INVALID_ARG;
+
+    int dev_ok = cached_device_check();
+    if (dev_ok != WKV7_OK) return dev_ok;
+    wkv7::DecodeArgs p{r, w_log, k, v, a, b, s_in, y, s_out, B, H};
+    return wkv7::launch_decode(p, io_dtype, w_dtype, static_cast<cudaStream_t>(stream)) == cudaSuccess
+               ? WKV7_OK
+               : WKV7_ERR_CUDA;
+}
+
+int wkv7_get_device_status(void* stream) {
+    if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return WKV7_ERR_CUDA;
+    int* dptr = nullptr;
+    if (status_ptr(&dptr) != WKV7_OK) return WKV7_ERR_CUDA;
+    int host = 0;
+    if (cudaMemcpy(&host, dptr, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return WKV7_ERR_CUDA;
+    if (host != 0) {
+        const int zero = 0;
+        if (cudaMemcpy(dptr, &zero, sizeof(int), cudaMemcpyHostToDevice) != cudaSuccess) return WKV7_ERR_CUDA;
+    }
+    return host;
+}
+
+int wkv7_debug_expire_wait(int spins, void* stream) {
+    if (spins < 1 || spins > (1 << 20)) return WKV7_ERR_INVALID_ARG;
+    int dev_ok = cached_device_check();
+    if (dev_ok != WKV7_OK) return dev_ok;
+    int* status = nullptr;
+    if (status_ptr(&status) != WKV7_OK) return WKV7_ERR_CUDA;
+    return wkv7::launch_expire_wait(spins, status, static_cast<cudaStream_t>(stream)) == cudaSuccess
+               ? WKV7_OK
+               : WKV7_ERR_CUDA;
+}
+
+}  // extern "C"

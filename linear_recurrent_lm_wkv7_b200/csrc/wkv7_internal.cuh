@@ -1,0 +1,61 @@
+// wkv7_internal.cuh — launch interface between the C-ABI layer (wkv7_api.cu)
+// and the kernels (wkv7_decode.cu, wkv7_prefill.cu).  Not part of the ABI.
+#pragma once
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+#include "wkv7.h"
+
+namespace wkv7 {
+
+constexpr int kHead = 64;  // D: head size supported by every kernel
+
+struct PrefillArgs {
+    const void* r;
+    const void* w_log;
+    const void* k;
+    const void* v;
+    const void* a;
+    const void* b;
+    const float* s0;
+    void* y;
+    float* sT;
+    int B, T, H;
+    const int32_t* seq_offsets;
+    int* status;  // device status word of the current device
+};
+
+struct DecodeArgs {
+    const void* r;
+    const void* w_log;
+    const void* k;
+    const void* v;
+    const void* a;
+    const void* b;
+    const float* s_in;
+    void* y;
+    float* s_out;
+    int B, H;
+};
+
+cudaError_t launch_prefill(const PrefillArgs& p, int io_dtype, int w_dtype, cudaStream_t stream);
+cudaError_t launch_decode(const DecodeArgs& p, int io_dtype, int w_dtype, cudaStream_t stream);
+cudaError_t launch_expire_wait(int spins, int* status, cudaStream_t stream);
+
+// Records the first device-side error of a call sequence (first writer wins).
+__device__ __forceinline__ void report_status(int* status, int code) {
+    if (status) atomicCAS(status, 0, code);
+}
+
+__device__ __forceinline__ float to_f32(__nv_bfloat16 x) { return __bfloat162float(x); }
+__device__ __forceinline__ float to_f32(float x) { return x; }
+template <typename T>
+__device__ __forceinline__ T from_f32(float x);
+template <>
+__device__ __forceinline__ float from_f32<float>(float x) { return x; }
+template <>
+__device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float x) { return __float2bfloat16_rn(x); }
+
+}  // namespace wkv7

@@ -1,0 +1,625 @@
+// wkv7_prefill.cu — chunked WKV-7 prefill on the sm_100a tensor cores.
+//
+// The recurrence (generalized delta rule of "RWKV-7 Goose: Expressive Dynamic
+// State Evolution", section "Generalized Delta rule"; argument roles from the
+// WKV call of the hxa07D forward listing) is
+//     S_t = S_{t-1} diag(w_t) + (S_{t-1} a_t) b_t^T + v_t k_t^T,   y_t = S_t r_t.
+// The pages state that the WKV computation parallelises chunk-wise ("RWKV-7
+// Goose architecture analysis", training section); the chunk algebra below is
+// derived here from the recurrence.
+//
+// One chunk of L = 64 tokens, start state S0, Gamma_t = prod_{s<=t} w_s (per key
+// channel, Gamma_0 = 1).  Scaled operands (rows = tokens):
+//   Rt = r (.) Gamma_t       At = a (.) Gamma_{t-1}
+//   Kt = k / Gamma_t         Bt = b / Gamma_t
+//   Kh = k (.) Gamma_L / Gamma_t,  Bh = b (.) Gamma_L / Gamma_t
+// With u_t = S_{t-1} a_t (rows of U), unrolling the recurrence gives
+//   U = At S0^T + Mak V + Nab U,   Nab = strict_tril(At Bt^T), Mak = strict_tril(At Kt^T)
+//   Y = Rt S0^T + Mrk V + Mrb U,   Mrk = tril(Rt Kt^T),        Mrb = tril(Rt Bt^T)
+//   S_L = S0 diag(Gamma_L) + V^T Kh + U^T Bh.
+// Solving the unit lower-triangular system, [W | Z] = (I - Nab)^{-1} [At | Mak],
+// gives U = W S0^T + Z V, hence the chunk is an affine map of the state:
+//   Y     = (Rt + Mrb W) S0^T + (Mrk + Mrb Z) V
+//   S_L^T = Gamma_L (.) S0^T  + (Bh^T W) S0^T + (Kh^T + Bh^T Z) V
+// Everything except the two products with S0^T is independent of the state.
+//
+// Tensor-core schedule per chunk (M = 128 rows by stacking two 64-row blocks):
+//   G   = [Rt; At] [Bt; Kt]^T               -> Mrb | Mrk over Nab | Mak   (TMEM)
+//   P   = [Mrb; Bh^T] [W | Z]               -> Mrb W | Mrb Z over Bh^T W | Bh^T Z
+//   OUT = [Er; Eq] V + [R'; Bh^T W] S0^T    -> Y over S_L^T - Gamma_L (.) S0^T
+// with R' = Rt + Mrb W, Er = Mrk + Mrb Z, Eq = Kh^T + Bh^T Z.  The triangular
+// solve runs on the CUDA cores in fp32 (one column per thread).  The state is
+// kept in fp32 registers of the threads that own TMEM lanes 64..127 (one key
+// channel each); its decay Gamma_L is applied there in fp32, and a rounded copy
+// of S^T is the B operand of the last product.
+//
+// Operand precision: bf16 tiles and kind::f16 MMAs for bf16 inputs, tf32 tiles
+// and kind::tf32 MMAs for fp32 inputs; accumulation, the solve, the decay and
+// the state are fp32.  All A operands and [W | Z] are K-major.  V and S^T are
+// MN-major B operands (rows = tokens / keys, as they arrive) for bf16; for tf32
+// they are stored transposed, K-major, because kind::tf32 with an MN-major
+// SWIZZLE_128B operand does not produce the product (measured on B200).
+#include "sm100_ptx.cuh"
+#include "wkv7_internal.cuh"
+
+namespace wkv7 {
+namespace {
+
+constexpr int L = 64;          // chunk length (tokens)
+constexpr int NT = 128;        // threads per block: one per TMEM lane
+constexpr int NSTRIDE = 68;    // fp32 row stride of the solver matrices (bank-conflict padding)
+constexpr uint32_t COL_G = 0;    // TMEM columns of G   (128)
+constexpr uint32_t COL_P = 128;  // TMEM columns of P   (128)
+constexpr uint32_t COL_O = 0;    // TMEM columns of OUT (64): reuses G columns 0..63, dead by then
+constexpr uint32_t TMEM_COLS = 256;
+constexpr uint64_t WAIT_LIMIT_NS = 1000000000ull;  // 1 s: far above any legitimate wait
+
+template <bool TF32>
+struct OpType {
+    static constexpr uint32_t EB = TF32 ? 4 : 2;       // bytes per operand element
+    static constexpr uint32_t FMT = TF32 ? 2 : 1;      // instruction-descriptor format
+    static constexpr uint32_t KSTEP = TF32 ? 8 : 16;   // K per tcgen05.mma
+    static constexpr uint32_t KSTEPS = 64 / KSTEP;     // MMAs per K = 64
+    static constexpr uint32_t TILE64 = 64 * 64 * EB;   // 64 rows x 64 elements
+    static constexpr uint32_t TILE128 = 128 * 64 * EB; // 128 rows x 64 elements
+};
+
+__device__ __forceinline__ float round_tf32(float x) {
+    uint32_t u;
+    asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(u) : "f"(x));
+    return __uint_as_float(u);
+}
+
+// element (row, col) of a swizzled operand tile with R rows
+template <bool TF32>
+__device__ __forceinline__ void st_op(uint8_t* tile, uint32_t R, uint32_t row, uint32_t col, float x) {
+    if constexpr (TF32) {
+        *reinterpret_cast<float*>(tile + swz(row, col * 4, R)) = round_tf32(x);
+    } else {
+        *reinterpret_cast<__nv_bfloat16*>(tile + swz(row, col * 2, R)) = __float2bfloat16_rn(x);
+    }
+}
+template <bool TF32>
+__device__ __forceinline__ float ld_op(const uint8_t* tile, uint32_t R, uint32_t row, uint32_t col) {
+    if constexpr (TF32) {
+        return *reinterpret_cast<const float*>(tile + swz(row, col * 4, R));
+    } else {
+        return __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(tile + swz(row, col * 2, R)));
+    }
+}
+// 32 consecutive elements [c0, c0+32) of one row, written with 16-byte stores
+template <bool TF32>
+__device__ __forceinline__ void st_op_row32(uint8_t* tile, uint32_t R, uint32_t row, uint32_t c0, const float* x) {
+    if constexpr (TF32) {
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+            float4 v = make_float4(round_tf32(x[4 * q]), round_tf32(x[4 * q + 1]), round_tf32(x[4 * q + 2]),
+                                   round_tf32(x[4 * q + 3]));
+            *reinterpret_cast<float4*>(tile + swz(row, (c0 + 4 * q) * 4, R)) = v;
+        }
+    } else {
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            uint4 v;
+            uint32_t* w = reinterpret_cast<uint32_t*>(&v);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                __nv_bfloat162 p = __floats2bfloat162_rn(x[8 * q + 2 * e], x[8 * q + 2 * e + 1]);
+                w[e] = *reinterpret_cast<uint32_t*>(&p);
+            }
+            *reinterpret_cast<uint4*>(tile + swz(row, (c0 + 8 * q) * 2, R)) = v;
+        }
+    }
+}
+template <bool TF32>
+__device__ __forceinline__ void ld_op_row32(const uint8_t* tile, uint32_t R, uint32_t row, uint32_t c0, float* x) {
+    if constexpr (TF32) {
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+            const float4 v = *reinterpret_cast<const float4*>(tile + swz(row, (c0 + 4 * q) * 4, R));
+            x[4 * q] = v.x; x[4 * q + 1] = v.y; x[4 * q + 2] = v.z; x[4 * q + 3] = v.w;
+        }
+    } else {
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const uint4 v = *reinterpret_cast<const uint4*>(tile + swz(row, (c0 + 8 * q) * 2, R));
+            const uint32_t* w = reinterpret_cast<const uint32_t*>(&v);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[e]));
+                x[8 * q + 2 * e] = f.x;
+                x[8 * q + 2 * e + 1] = f.y;
+            }
+        }
+    }
+}
+
+// Descriptor of K-step s of a K-major operand tile with R rows (K = 64 elements).
+template <bool TF32>
+__device__ __forceinline__ uint64_t kmajor_desc(const uint8_t* tile, uint32_t R, uint32_t s) {
+    const uint32_t kbyte = s * 32u;  // 16 bf16 or 8 tf32 per step
+    const uint32_t addr = smem_u32(tile) + (kbyte >> 7) * (R << 7) + (kbyte & 127u);
+    return sdesc_sw128(addr, 16, 1024);
+}
+// Descriptor of K-step s of an MN-major operand tile whose rows are K (R rows).
+template <bool TF32>
+__device__ __forceinline__ uint64_t mnmajor_desc(const uint8_t* tile, uint32_t R, uint32_t s) {
+    const uint32_t addr = smem_u32(tile) + s * OpType<TF32>::KSTEP * 128u;
+    return sdesc_sw128(addr, R * 128u, 1024);
+}
+
+struct Smem {
+    uint8_t* RA;   // [Rt ; At]            128 x 64, K-major over key channels
+    uint8_t* BK;   // [Bt ; Kt]            128 x 64, K-major over key channels   (then [W | Z])
+    uint8_t* WZ;   // [W | Z]^T            128 columns x 64 tokens, K-major       (aliases BK)
+    uint8_t* BH;   // [Mrb ; Bh^T]         128 x 64, K-major over tokens          (then [Er ; Eq])
+    uint8_t* AQ;   // [Er ; Eq]            128 x 64, K-major over tokens          (aliases BH)
+    uint8_t* KH;   // Kh^T                 64 keys x 64 tokens
+    float* NAB;    // Nab fp32             64 x NSTRIDE                           (then AS)
+    float* MAK;    // Mak fp32             64 x NSTRIDE
+    uint8_t* AS;   // [R' ; Bh^T W]        128 x 64, K-major over key channels    (aliases NAB, MAK)
+    uint8_t* V;    // V: bf16 64 tokens x 64 values (MN-major); tf32 64 values x 64 tokens (K-major)
+    uint8_t* S;    // S^T: bf16 64 keys x 64 values (MN-major); tf32 64 values x 64 keys (K-major)
+    float* gammaL; // Gamma_L per key channel
+    float* red;    // per-half products of w (2 x 64)
+    uint64_t* bar; // MMA completion barrier
+    uint32_t* tmem_slot;
+};
+
+template <bool TF32>
+__host__ __device__ constexpr uint32_t smem_bytes_needed() {
+    using O = OpType<TF32>;
+    constexpr uint32_t solver = 2u * 64u * NSTRIDE * 4u;
+    constexpr uint32_t r4 = ((solver > O::TILE128 ? solver : O::TILE128) + 1023u) & ~1023u;
+    return 1024u /* alignment slack */ + 3u * O::TILE128 + O::TILE64 + r4 + 2u * O::TILE64 + 64u * 4u +
+           128u * 4u + 64u;
+}
+
+template <bool TF32>
+__device__ __forceinline__ Smem carve(uint8_t* raw) {
+    using O = OpType<TF32>;
+    constexpr uint32_t solver = 2u * 64u * NSTRIDE * 4u;
+    constexpr uint32_t r4 = ((solver > O::TILE128 ? solver : O::TILE128) + 1023u) & ~1023u;
+    uint8_t* p = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(raw) + 1023u) & ~uintptr_t(1023));
+    Smem s;
+    s.RA = p; p += O::TILE128;
+    s.BK = p; s.WZ = p; p += O::TILE128;
+    s.BH = p; s.AQ = p; p += O::TILE128;
+    s.KH = p; p += O::TILE64;
+    s.NAB = reinterpret_cast<float*>(p); s.MAK = s.NAB + 64 * NSTRIDE; s.AS = p; p += r4;
+    s.V = p; p += O::TILE64;
+    s.S = p; p += O::TILE64;
+    s.gammaL = reinterpret_cast<float*>(p); p += 64 * 4;
+    s.red = reinterpret_cast<float*>(p); p += 128 * 4;
+    s.bar = reinterpret_cast<uint64_t*>(p); p += 8;
+    s.tmem_slot = reinterpret_cast<uint32_t*>(p);
+    return s;
+}
+
+// Row jj of S^T (key channel jj, all 64 value channels) into the S operand tile.
+template <bool TF32>
+__device__ __forceinline__ void store_state_operand(uint8_t* tile, int jj, const float* S) {
+    if constexpr (TF32) {
+#pragma unroll
+        for (int i = 0; i < 64; ++i) st_op<true>(tile, 64, i, jj, S[i]);  // K-major: row = value channel
+    } else {
+        st_op_row32<false>(tile, 64, jj, 0, S);  // MN-major: row = key channel
+        st_op_row32<false>(tile, 64, jj, 32, S + 32);
+    }
+}
+
+// Loads 16 bytes of one value row into the V tile (rows beyond nv are zeroed).
+template <typename IO, bool TF32>
+__device__ __forceinline__ void load_v_tile(const IO* __restrict__ v, long row0, long tstride, long hoff, int nv,
+                                            uint8_t* tile, int tid) {
+    if constexpr (TF32) {
+        // fp32 values: 16 chunks of 4 per row, 64 rows
+#pragma unroll
+        for (int it = 0; it < 8; ++it) {
+            const int q = tid + it * NT;
+            const int row = q >> 4, ch = q & 15;
+            float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (row < nv) {
+                const float* src = reinterpret_cast<const float*>(v) + (row0 + row) * tstride + hoff + 4 * ch;
+                x = __ldg(reinterpret_cast<const float4*>(src));
+            }
+            // K-major: row = value channel, column = token
+            st_op<true>(tile, 64, 4 * ch + 0, row, x.x);
+            st_op<true>(tile, 64, 4 * ch + 1, row, x.y);
+            st_op<true>(tile, 64, 4 * ch + 2, row, x.z);
+            st_op<true>(tile, 64, 4 * ch + 3, row, x.w);
+        }
+    } else {
+        // bf16 values: 8 chunks of 8 per row, 64 rows
+#pragma unroll
+        for (int it = 0; it < 4; ++it) {
+            const int q = tid + it * NT;
+            const int row = q >> 3, ch = q & 7;
+            uint4 x = make_uint4(0, 0, 0, 0);
+            if (row < nv) {
+                const __nv_bfloat16* src =
+                    reinterpret_cast<const __nv_bfloat16*>(v) + (row0 + row) * tstride + hoff + 8 * ch;
+                x = __ldg(reinterpret_cast<const uint4*>(src));
+            }
+            *reinterpret_cast<uint4*>(tile + swz(row, ch * 16, 64)) = x;
+        }
+    }
+}
+
+template <typename IO, typename WT, bool TF32>
+__global__ void __launch_bounds__(NT, 1)
+    wkv7_prefill_kernel(const IO* __restrict__ r, const WT* __restrict__ wl, const IO* __restrict__ k,
+                        const IO* __restrict__ v, const IO* __restrict__ a, const IO* __restrict__ b,
+                        const float* s0, IO* __restrict__ y, float* sT, int T, int H,
+                        const int32_t* __restrict__ seq_offsets, int* status) {
+    using O = OpType<TF32>;
+    extern __shared__ uint8_t smem_raw[];
+    const Smem sm = carve<TF32>(smem_raw);
+    const int tid = threadIdx.x;
+    const int warp = tid >> 5;
+
+    // ---- which (sequence, head) unit, and its tokens
+    const int unit = blockIdx.x;
+    const int n = unit / H, h = unit % H;
+    long tb = 0, len = 0;
+    bool bad = false;
+    if (seq_offsets) {
+        const long o0 = seq_offsets[n], o1 = seq_offsets[n + 1];
+        if (o0 < 0 || o1 < o0 || o1 > T) {
+            bad = true;
+        } else {
+            tb = o0;
+            len = o1 - o0;
+        }
+    } else {
+        tb = static_cast<long>(n) * T;
+        len = T;
+    }
+    if (bad) {
+        if (tid == 0) report_status(status, WKV7_ERR_DEVICE_BOUNDS);
+        return;  // nothing allocated yet
+    }
+    const long tstride = static_cast<long>(H) * kHead;  // elements between consecutive tokens
+    const long hoff = static_cast<long>(h) * kHead;
+    const long sbase = (static_cast<long>(n) * H + h) * kHead * kHead;
+
+    // ---- set-up: barrier, TMEM
+    if (tid == 0) {
+        mbar_init(sm.bar, 1);
+        fence_mbar_init();
+    }
+    if (warp == 0) {
+        tmem_alloc(sm.tmem_slot, TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *sm.tmem_slot;
+    const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
+
+    // ---- state: threads 64..127 own key channel j = tid - 64 (a row of S^T)
+    float S[64];
+    const int jj = tid - 64;
+    if (tid >= 64) {
+#pragma unroll
+        for (int i = 0; i < 64; ++i) S[i] = s0 ? s0[sbase + i * kHead + jj] : 0.f;
+        store_state_operand<TF32>(sm.S, jj, S);
+    }
+
+    bool ok = true;
+    uint32_t phase = 0;
+    const int nchunks = static_cast<int>((len + L - 1) / L);
+    for (int c = 0; c < nchunks && ok; ++c) {
+        const long row0 = tb + static_cast<long>(c) * L;  // first token of the chunk
+        const int nv = static_cast<int>(len - static_cast<long>(c) * L < L ? len - static_cast<long>(c) * L : L);
+
+        // ---- p1: decay products and scaled operand tiles.  Thread (j, half).
+        {
+            const int j = tid & 63, hf = tid >> 6;
+            float cp[32];
+            float prod = 1.f;
+#pragma unroll
+            for (int q = 0; q < 32; ++q) {
+                const int t = hf * 32 + q;
+                float w = 1.f;
+                if (t < nv) w = expf(-expf(to_f32(wl[(row0 + t) * tstride + hoff + j])));
+                prod *= w;
+                cp[q] = prod;
+            }
+            sm.red[hf * 64 + j] = prod;
+            __syncthreads();
+            const float pre = hf ? sm.red[j] : 1.f;
+            const float GL = sm.red[j] * sm.red[64 + j];
+            if (hf == 0) sm.gammaL[j] = GL;
+            float gprev = pre;
+#pragma unroll
+            for (int q = 0; q < 32; ++q) {
+                const int t = hf * 32 + q;
+                const float G = pre * cp[q];
+                const float inv = 1.f / G;
+                float rr = 0.f, kk = 0.f, aa = 0.f, bb = 0.f;
+                if (t < nv) {
+                    const long off = (row0 + t) * tstride + hoff + j;
+                    rr = to_f32(r[off]);
+                    kk = to_f32(k[off]);
+                    aa = to_f32(a[off]);
+                    bb = to_f32(b[off]);
+                }
+                const float invL = inv * GL;
+                st_op<TF32>(sm.RA, 128, t, j, rr * G);
+                st_op<TF32>(sm.RA, 128, 64 + t, j, aa * gprev);
+                st_op<TF32>(sm.BK, 128, t, j, bb * inv);
+                st_op<TF32>(sm.BK, 128, 64 + t, j, kk * inv);
+                st_op<TF32>(sm.BH, 128, 64 + j, t, bb * invL);
+                st_op<TF32>(sm.KH, 64, j, t, kk * invL);
+                gprev = G;
+            }
+            load_v_tile<IO, TF32>(v, row0, tstride, hoff, nv, sm.V, tid);
+        }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        __syncthreads();
+
+        // ---- G = [Rt; At] [Bt; Kt]^T
+        if (tid == 0) {
+            tc_fence_after();
+            constexpr uint32_t idesc = idesc_f32acc(O::FMT, 128, 128, 0, 0);
+#pragma unroll
+            for (uint32_t s = 0; s < O::KSTEPS; ++s)
+                mma_ss<TF32>(tmem + COL_G, kmajor_desc<TF32>(sm.RA, 128, s), kmajor_desc<TF32>(sm.BK, 128, s), idesc,
+                             s > 0);
+            mma_commit(sm.bar);
+        }
+        ok = __syncthreads_and(mbar_wait(sm.bar, phase, WAIT_LIMIT_NS));
+        if (!ok) break;
+        phase ^= 1u;
+        tc_fence_after();
+
+        // ---- masks: Mrb (incl. diagonal) -> BH rows 0..63; Nab, Mak (strict) -> fp32 solver inputs
+        {
+            float g[32];
+            if (tid < 64) {
+                const int t = tid;
+#pragma unroll
+                for (int q = 0; q < 2; ++q) {
+                    tmem_load32(tmem + lane_base + COL_G + 32 * q, g);
+#pragma unroll
+                    for (int i = 0; i < 32; ++i)
+                        if (32 * q + i > t) g[i] = 0.f;
+                    st_op_row32<TF32>(sm.BH, 128, t, 32 * q, g);
+                }
+            } else {
+                const int t = tid - 64;
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    tmem_load32(tmem + lane_base + COL_G + 32 * q, g);
+                    float* dst = (q < 2 ? sm.NAB : sm.MAK) + t * NSTRIDE + 32 * (q & 1);
+#pragma unroll
+                    for (int i = 0; i < 32; i += 4) {
+                        float4 x;
+                        x.x = (32 * (q & 1) + i + 0 < t) ? g[i + 0] : 0.f;
+                        x.y = (32 * (q & 1) + i + 1 < t) ? g[i + 1] : 0.f;
+                        x.z = (32 * (q & 1) + i + 2 < t) ? g[i + 2] : 0.f;
+                        x.w = (32 * (q & 1) + i + 3 < t) ? g[i + 3] : 0.f;
+                        *reinterpret_cast<float4*>(dst + i) = x;
+                    }
+                }
+            }
+        }
+        tc_fence_before();
+        __syncthreads();
+
+        // ---- [W | Z] = (I - Nab)^{-1} [At | Mak]: forward substitution, column `tid`
+        {
+            const int col = tid;
+            float x[64];
+#pragma unroll
+            for (int t = 0; t < 64; ++t) x[t] = 0.f;
+#pragma unroll
+            for (int t = 0; t < 64; ++t) {
+                float acc = col < 64 ? ld_op<TF32>(sm.RA, 128, 64 + t, col) : sm.MAK[t * NSTRIDE + (col - 64)];
+                const float* nrow = sm.NAB + t * NSTRIDE;
+#pragma unroll
+                for (int i = 0; i < t; i += 4) {
+                    const float4 nv4 = *reinterpret_cast<const float4*>(nrow + i);
+                    acc = fmaf(nv4.x, x[i], acc);
+                    acc = fmaf(nv4.y, x[i + 1], acc);
+                    acc = fmaf(nv4.z, x[i + 2], acc);
+                    acc = fmaf(nv4.w, x[i + 3], acc);
+                }
+                x[t] = acc;
+            }
+            st_op_row32<TF32>(sm.WZ, 128, col, 0, x);
+            st_op_row32<TF32>(sm.WZ, 128, col, 32, x + 32);
+        }
+        fence_proxy_async_smem();
+        __syncthreads();
+
+        // ---- P = [Mrb; Bh^T] [W | Z]
+        if (tid == 0) {
+            tc_fence_after();
+            constexpr uint32_t idesc = idesc_f32acc(O::FMT, 128, 128, 0, 0);
+#pragma unroll
+            for (uint32_t s = 0; s < O::KSTEPS; ++s)
+                mma_ss<TF32>(tmem + COL_P, kmajor_desc<TF32>(sm.BH, 128, s), kmajor_desc<TF32>(sm.WZ, 128, s),
+                             idesc, s > 0);
+            mma_commit(sm.bar);
+        }
+        ok = __syncthreads_and(mbar_wait(sm.bar, phase, WAIT_LIMIT_NS));
+        if (!ok) break;
+        phase ^= 1u;
+        tc_fence_after();
+
+        // ---- R' = Rt + Mrb W, Er = Mrk + Mrb Z (lanes 0..63); Bh^T W, Eq = Kh^T + Bh^T Z (lanes 64..127)
+        {
+            float p[32], e[32];
+            if (tid < 64) {
+                const int t = tid;
+#pragma unroll
+                for (int q = 0; q < 2; ++q) {
+                    tmem_load32(tmem + lane_base + COL_P + 32 * q, p);
+                    ld_op_row32<TF32>(sm.RA, 128, t, 32 * q, e);
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) p[i] += e[i];
+                    st_op_row32<TF32>(sm.AS, 128, t, 32 * q, p);
+                }
+#pragma unroll
+                for (int q = 0; q < 2; ++q) {
+                    tmem_load32(tmem + lane_base + COL_P + 64 + 32 * q, p);
+                    tmem_load32(tmem + lane_base + COL_G + 64 + 32 * q, e);
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) p[i] += (32 * q + i <= t) ? e[i] : 0.f;
+                    st_op_row32<TF32>(sm.AQ, 128, t, 32 * q, p);
+                }
+            } else {
+                const int j = tid - 64;
+#pragma unroll
+                for (int q = 0; q < 2; ++q) {
+                    tmem_load32(tmem + lane_base + COL_P + 32 * q, p);
+                    st_op_row32<TF32>(sm.AS, 128, 64 + j, 32 * q, p);
+                }
+#pragma unroll
+                for (int q = 0; q < 2; ++q) {
+                    tmem_load32(tmem + lane_base + COL_P + 64 + 32 * q, p);
+                    ld_op_row32<TF32>(sm.KH, 64, j, 32 * q, e);
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) p[i] += e[i];
+                    st_op_row32<TF32>(sm.AQ, 128, 64 + j, 32 * q, p);
+                }
+            }
+        }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        __syncthreads();
+
+        // ---- OUT = [Er; Eq] V + [R'; Bh^T W] S0^T
+        if (tid == 0) {
+            tc_fence_after();
+            constexpr uint32_t idesc = idesc_f32acc(O::FMT, 128, 64, 0, TF32 ? 0 : 1);
+#pragma unroll
+            for (uint32_t s = 0; s < O::KSTEPS; ++s) {
+                const uint64_t bd = TF32 ? kmajor_desc<TF32>(sm.V, 64, s) : mnmajor_desc<TF32>(sm.V, 64, s);
+                mma_ss<TF32>(tmem + COL_O, kmajor_desc<TF32>(sm.AQ, 128, s), bd, idesc, s > 0);
+            }
+#pragma unroll
+            for (uint32_t s = 0; s < O::KSTEPS; ++s) {
+                const uint64_t bd = TF32 ? kmajor_desc<TF32>(sm.S, 64, s) : mnmajor_desc<TF32>(sm.S, 64, s);
+                mma_ss<TF32>(tmem + COL_O, kmajor_desc<TF32>(sm.AS, 128, s), bd, idesc, 1);
+            }
+            mma_commit(sm.bar);
+        }
+        ok = __syncthreads_and(mbar_wait(sm.bar, phase, WAIT_LIMIT_NS));
+        if (!ok) break;
+        phase ^= 1u;
+        tc_fence_after();
+
+        // ---- y rows (lanes 0..63) and the state update (lanes 64..127)
+        {
+            float o[32];
+            if (tid < 64) {
+                const int t = tid;
+#pragma unroll
+                for (int q = 0; q < 2; ++q) {
+                    tmem_load32(tmem + lane_base + COL_O + 32 * q, o);
+                    if (t < nv) {
+                        IO* dst = y + (row0 + t) * tstride + hoff + 32 * q;
+                        if constexpr (TF32) {
+#pragma unroll
+                            for (int i = 0; i < 32; i += 4)
+                                *reinterpret_cast<float4*>(dst + i) = make_float4(o[i], o[i + 1], o[i + 2], o[i + 3]);
+                        } else {
+#pragma unroll
+                            for (int i = 0; i < 32; i += 8) {
+                                uint4 pk;
+                                uint32_t* w = reinterpret_cast<uint32_t*>(&pk);
+#pragma unroll
+                                for (int e2 = 0; e2 < 4; ++e2) {
+                                    __nv_bfloat162 bb2 = __floats2bfloat162_rn(o[i + 2 * e2], o[i + 2 * e2 + 1]);
+                                    w[e2] = *reinterpret_cast<uint32_t*>(&bb2);
+                                }
+                                *reinterpret_cast<uint4*>(dst + i) = pk;
+                            }
+                        }
+                    }
+                }
+            } else {
+                const float GL = sm.gammaL[jj];
+#pragma unroll
+                for (int q = 0; q < 2; ++q) {
+                    tmem_load32(tmem + lane_base + COL_O + 32 * q, o);
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) S[32 * q + i] = fmaf(GL, S[32 * q + i], o[i]);
+                }
+                store_state_operand<TF32>(sm.S, jj, S);
+            }
+        }
+        tc_fence_before();
+        __syncthreads();
+    }
+
+    if (!ok) {
+        if (tid == 0) report_status(status, WKV7_ERR_DEVICE_TIMEOUT);
+        // let any MMA still in flight finish (bounded) before TMEM is released
+        mbar_wait(sm.bar, phase, WAIT_LIMIT_NS);
+    } else if (sT && tid >= 64) {
+#pragma unroll
+        for (int i = 0; i < 64; ++i) sT[sbase + i * kHead + jj] = S[i];
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem, TMEM_COLS);
+    }
+}
+
+template <typename IO, typename WT, bool TF32>
+cudaError_t launch_typed(const PrefillArgs& p, cudaStream_t stream) {
+    constexpr uint32_t smem = smem_bytes_needed<TF32>();
+    auto kern = wkv7_prefill_kernel<IO, WT, TF32>;
+    static unsigned long long configured = 0;  // one bit per device ordinal
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    const unsigned long long bit = 1ull << (dev & 63);
+    if (!(configured & bit)) {
+        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        if (e != cudaSuccess) return e;
+        configured |= bit;
+    }
+    const long units = static_cast<long>(p.B) * p.H;
+    kern<<<static_cast<unsigned>(units), NT, smem, stream>>>(
+        static_cast<const IO*>(p.r), static_cast<const WT*>(p.w_log), static_cast<const IO*>(p.k),
+        static_cast<const IO*>(p.v), static_cast<const IO*>(p.a), static_cast<const IO*>(p.b), p.s0,
+        static_cast<IO*>(p.y), p.sT, p.T, p.H, p.seq_offsets, p.status);
+    return cudaGetLastError();
+}
+
+__global__ void expire_wait_kernel(int spins, int* status) {
+    __shared__ uint64_t bar;
+    if (threadIdx.x == 0) {
+        mbar_init(&bar, 1);
+        fence_mbar_init();
+        // nothing ever arrives on `bar`: the bounded wait must give up
+        if (!mbar_wait_spins(&bar, 0, static_cast<uint32_t>(spins))) report_status(status, WKV7_ERR_DEVICE_TIMEOUT);
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_prefill(const PrefillArgs& p, int io_dtype, int w_dtype, cudaStream_t stream) {
+    if (io_dtype == WKV7_BF16) {
+        return w_dtype == WKV7_BF16 ? launch_typed<__nv_bfloat16, __nv_bfloat16, false>(p, stream)
+                                    : launch_typed<__nv_bfloat16, float, false>(p, stream);
+    }
+    return w_dtype == WKV7_BF16 ? launch_typed<float, __nv_bfloat16, true>(p, stream)
+                                : launch_typed<float, float, true>(p, stream);
+}
+
+cudaError_t launch_expire_wait(int spins, int* status, cudaStream_t stream) {
+    expire_wait_kernel<<<1, 32, 0, stream>>>(spins, status);
+    return cudaGetLastError();
+}
+
+}  // namespace wkv7

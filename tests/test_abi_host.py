@@ -1,0 +1,94 @@
+"""C-ABI checks that need no GPU: the library loads, exports every symbol the
+header declares, and rejects bad arguments on the host before launching
+anything (these calls return before any CUDA call is made)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def wk():
+    from linear_recurrent_lm_wkv7_b200 import build
+
+    build.build()
+    import linear_recurrent_lm_wkv7_b200 as wk
+
+    return wk
+
+
+def test_header_symbols_exported(wk):
+    hdr = open(os.path.join(ROOT, "include", "wkv7.h")).read()
+    declared = set(re.findall(r"^(?:int|const char\*)\s+(wkv7_\w+)\s*\(", hdr, flags=re.M))
+    assert declared == set(wk.EXPORTS)
+    lib = ctypes.CDLL(wk.LIB_PATH)
+    for name in declared:
+        assert hasattr(lib, name), name
+
+
+def test_status_strings(wk):
+    for code in wk.STATUS:
+        assert wk.wkv7_status_string(code)
+    assert wk.wkv7_version() >= 10000
+
+
+# argument tuple for wkv7_forward: 9 pointers, B, T, H, D, offsets, io, w, stream
+def _fwd(ptr=0x1000, B=1, T=8, H=1, D=64, offs=None, io=1, wd=0, **over):
+    p = dict(r=ptr, w=ptr + 0x100000, k=ptr + 0x200000, v=ptr + 0x300000, a=ptr + 0x400000, b=ptr + 0x500000,
+             s0=None, y=ptr + 0x600000, sT=None)
+    p.update(over)
+    return (p["r"], p["w"], p["k"], p["v"], p["a"], p["b"], p["s0"], p["y"], p["sT"], B, T, H, D, offs, io, wd, None)
+
+
+def test_forward_rejects_bad_arguments(wk):
+    call = wk._binding.raw_call_forward
+    assert call(*_fwd(D=32)) == -2  # head size
+    assert call(*_fwd(B=0)) == -1
+    assert call(*_fwd(T=-1)) == -1
+    assert call(*_fwd(H=0)) == -1
+    assert call(*_fwd(io=7)) == -1  # dtype code
+    assert call(*_fwd(wd=3)) == -1
+    assert call(*_fwd(r=None)) == -1  # null input
+    assert call(*_fwd(y=None)) == -1  # null output
+    assert call(*_fwd(k=0x1008 + 0x200000)) == -3  # misaligned
+    assert call(*_fwd(sT=0x7000008)) == -3
+    assert call(*_fwd(y=0x1000)) == -1  # y aliases r
+    assert call(*_fwd(sT=0x1000 + 0x600000)) == -1  # sT overlaps y
+    # sT overlapping s0 without being the same buffer
+    assert call(*_fwd(s0=0x9000000, sT=0x9000000 + 4096)) == -1
+
+
+def test_decode_rejects_bad_arguments(wk):
+    call = wk._binding.raw_call_decode
+    base = [0x1000 + i * 0x100000 for i in range(9)]
+
+    def args(**over):
+        a = list(base)
+        for k_, v_ in over.items():
+            a[int(k_[1:])] = v_
+        return tuple(a) + (2, 3, 64, 1, 1, None)
+
+    assert call(*(args()[:-4] + (32, 1, 1, None))) == -2
+    assert call(*args(p0=None)) == -1
+    assert call(*args(p8=None)) == -1
+    assert call(*args(p3=0x1004 + 0x300000)) == -3
+    assert call(*args(p7=0x1000)) == -1  # y aliases r
+    # partial overlap of s_in and s_out
+    assert call(*args(p6=0x9000000, p8=0x9000000 + 256)) == -1
+
+
+def test_oracle_and_library_share_no_code():
+    """The oracle neither includes nor loads anything from the CUDA package, and
+    the CUDA sources never mention the oracle."""
+    osrc = open(os.path.join(ROOT, "oracle", "wkv7_oracle.c")).read()
+    assert "#include \"" not in osrc
+    opy = open(os.path.join(ROOT, "oracle", "__init__.py")).read()
+    assert "linear_recurrent_lm_wkv7_b200" not in opy
+    csrc = os.path.join(ROOT, "linear_recurrent_lm_wkv7_b200", "csrc")
+    for f in os.listdir(csrc):
+        assert "oracle" not in open(os.path.join(csrc, f)).read().lower(), f
+    for f in ("__init__.py", "_binding.py", "build.py"):
+        assert "oracle" not in open(os.path.join(ROOT, "linear_recurrent_lm_wkv7_b200", f)).read(), f
