@@ -41,6 +41,8 @@ struct DecodeArgs {
 };
 
 cudaError_t launch_prefill(const PrefillArgs& p, int io_dtype, int w_dtype, cudaStream_t stream);
+// warp-specialised kernel for bf16 inputs (wkv7_prefill_pipe.cu)
+cudaError_t launch_prefill_pipe(const PrefillArgs& p, int w_dtype, cudaStream_t stream);
 cudaError_t launch_decode(const DecodeArgs& p, int io_dtype, int w_dtype, cudaStream_t stream);
 cudaError_t launch_expire_wait(int spins, int* status, cudaStream_t stream);
 

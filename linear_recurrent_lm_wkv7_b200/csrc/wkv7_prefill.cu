@@ -39,6 +39,11 @@
 // MN-major B operands (rows = tokens / keys, as they arrive) for bf16; for tf32
 // they are stored transposed, K-major, because kind::tf32 with an MN-major
 // SWIZZLE_128B operand does not produce the product (measured on B200).
+#include <cuda.h>
+
+#include <cstring>
+
+#include "prefill_common.cuh"
 #include "sm100_ptx.cuh"
 #include "wkv7_internal.cuh"
 
@@ -54,100 +59,6 @@ constexpr uint32_t COL_O = 0;    // TMEM columns of OUT (64): reuses G columns 0
 constexpr uint32_t TMEM_COLS = 256;
 constexpr uint64_t WAIT_LIMIT_NS = 1000000000ull;  // 1 s: far above any legitimate wait
 
-template <bool TF32>
-struct OpType {
-    static constexpr uint32_t EB = TF32 ? 4 : 2;       // bytes per operand element
-    static constexpr uint32_t FMT = TF32 ? 2 : 1;      // instruction-descriptor format
-    static constexpr uint32_t KSTEP = TF32 ? 8 : 16;   // K per tcgen05.mma
-    static constexpr uint32_t KSTEPS = 64 / KSTEP;     // MMAs per K = 64
-    static constexpr uint32_t TILE64 = 64 * 64 * EB;   // 64 rows x 64 elements
-    static constexpr uint32_t TILE128 = 128 * 64 * EB; // 128 rows x 64 elements
-};
-
-__device__ __forceinline__ float round_tf32(float x) {
-    uint32_t u;
-    asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(u) : "f"(x));
-    return __uint_as_float(u);
-}
-
-// element (row, col) of a swizzled operand tile with R rows
-template <bool TF32>
-__device__ __forceinline__ void st_op(uint8_t* tile, uint32_t R, uint32_t row, uint32_t col, float x) {
-    if constexpr (TF32) {
-        *reinterpret_cast<float*>(tile + swz(row, col * 4, R)) = round_tf32(x);
-    } else {
-        *reinterpret_cast<__nv_bfloat16*>(tile + swz(row, col * 2, R)) = __float2bfloat16_rn(x);
-    }
-}
-template <bool TF32>
-__device__ __forceinline__ float ld_op(const uint8_t* tile, uint32_t R, uint32_t row, uint32_t col) {
-    if constexpr (TF32) {
-        return *reinterpret_cast<const float*>(tile + swz(row, col * 4, R));
-    } else {
-        return __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(tile + swz(row, col * 2, R)));
-    }
-}
-// 32 consecutive elements [c0, c0+32) of one row, written with 16-byte stores
-template <bool TF32>
-__device__ __forceinline__ void st_op_row32(uint8_t* tile, uint32_t R, uint32_t row, uint32_t c0, const float* x) {
-    if constexpr (TF32) {
-#pragma unroll
-        for (int q = 0; q < 8; ++q) {
-            float4 v = make_float4(round_tf32(x[4 * q]), round_tf32(x[4 * q + 1]), round_tf32(x[4 * q + 2]),
-                                   round_tf32(x[4 * q + 3]));
-            *reinterpret_cast<float4*>(tile + swz(row, (c0 + 4 * q) * 4, R)) = v;
-        }
-    } else {
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-            uint4 v;
-            uint32_t* w = reinterpret_cast<uint32_t*>(&v);
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                __nv_bfloat162 p = __floats2bfloat162_rn(x[8 * q + 2 * e], x[8 * q + 2 * e + 1]);
-                w[e] = *reinterpret_cast<uint32_t*>(&p);
-            }
-            *reinterpret_cast<uint4*>(tile + swz(row, (c0 + 8 * q) * 2, R)) = v;
-        }
-    }
-}
-template <bool TF32>
-__device__ __forceinline__ void ld_op_row32(const uint8_t* tile, uint32_t R, uint32_t row, uint32_t c0, float* x) {
-    if constexpr (TF32) {
-#pragma unroll
-        for (int q = 0; q < 8; ++q) {
-            const float4 v = *reinterpret_cast<const float4*>(tile + swz(row, (c0 + 4 * q) * 4, R));
-            x[4 * q] = v.x; x[4 * q + 1] = v.y; x[4 * q + 2] = v.z; x[4 * q + 3] = v.w;
-        }
-    } else {
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-            const uint4 v = *reinterpret_cast<const uint4*>(tile + swz(row, (c0 + 8 * q) * 2, R));
-            const uint32_t* w = reinterpret_cast<const uint32_t*>(&v);
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[e]));
-                x[8 * q + 2 * e] = f.x;
-                x[8 * q + 2 * e + 1] = f.y;
-            }
-        }
-    }
-}
-
-// Descriptor of K-step s of a K-major operand tile with R rows (K = 64 elements).
-template <bool TF32>
-__device__ __forceinline__ uint64_t kmajor_desc(const uint8_t* tile, uint32_t R, uint32_t s) {
-    const uint32_t kbyte = s * 32u;  // 16 bf16 or 8 tf32 per step
-    const uint32_t addr = smem_u32(tile) + (kbyte >> 7) * (R << 7) + (kbyte & 127u);
-    return sdesc_sw128(addr, 16, 1024);
-}
-// Descriptor of K-step s of an MN-major operand tile whose rows are K (R rows).
-template <bool TF32>
-__device__ __forceinline__ uint64_t mnmajor_desc(const uint8_t* tile, uint32_t R, uint32_t s) {
-    const uint32_t addr = smem_u32(tile) + s * OpType<TF32>::KSTEP * 128u;
-    return sdesc_sw128(addr, R * 128u, 1024);
-}
-
 struct Smem {
     uint8_t* RA;   // [Rt ; At]            128 x 64, K-major over key channels
     uint8_t* BK;   // [Bt ; Kt]            128 x 64, K-major over key channels   (then [W | Z])
@@ -158,24 +69,39 @@ struct Smem {
     float* NAB;    // Nab fp32             64 x NSTRIDE                           (then AS)
     float* MAK;    // Mak fp32             64 x NSTRIDE
     uint8_t* AS;   // [R' ; Bh^T W]        128 x 64, K-major over key channels    (aliases NAB, MAK)
-    uint8_t* V;    // V: bf16 64 tokens x 64 values (MN-major); tf32 64 values x 64 tokens (K-major)
+    uint8_t* V[2]; // V: bf16 64 tokens x 64 values (MN-major, two TMA slots); tf32 64 values x 64 tokens (K-major)
     uint8_t* S;    // S^T: bf16 64 keys x 64 values (MN-major); tf32 64 values x 64 keys (K-major)
+    uint8_t* raw;  // bf16 only: TMA staging of r, k, a, b (64 x 64 each, row-major) and w_log
     float* gammaL; // Gamma_L per key channel
     float* red;    // per-half products of w (2 x 64)
     uint64_t* bar; // MMA completion barrier
+    uint64_t* raw_bar; // TMA completion barrier (bf16 only)
     uint32_t* tmem_slot;
 };
 
-template <bool TF32>
+// TMA descriptors of the token-major inputs, each viewed as [tokens][H][64]
+// with a box of 64 tokens x 1 head x 64 channels.
+struct TmaMaps {
+    CUtensorMap r, k, a, b, wl, v;
+};
+
+// Bytes of the raw staging area (bf16 inputs): r, k, a, b tiles + the w_log tile.
+template <bool TF32, uint32_t WB>
+__host__ __device__ constexpr uint32_t raw_bytes() {
+    return TF32 ? 0u : 4u * 64u * 64u * 2u + 64u * 64u * WB;
+}
+
+template <bool TF32, uint32_t WB>
 __host__ __device__ constexpr uint32_t smem_bytes_needed() {
     using O = OpType<TF32>;
     constexpr uint32_t solver = 2u * 64u * NSTRIDE * 4u;
     constexpr uint32_t r4 = ((solver > O::TILE128 ? solver : O::TILE128) + 1023u) & ~1023u;
-    return 1024u /* alignment slack */ + 3u * O::TILE128 + O::TILE64 + r4 + 2u * O::TILE64 + 64u * 4u +
-           128u * 4u + 64u;
+    constexpr uint32_t nv = TF32 ? 1u : 2u;
+    return 1024u /* alignment slack */ + 3u * O::TILE128 + O::TILE64 + r4 + (nv + 1u) * O::TILE64 +
+           raw_bytes<TF32, WB>() + 64u * 4u + 128u * 4u + 64u;
 }
 
-template <bool TF32>
+template <bool TF32, uint32_t WB>
 __device__ __forceinline__ Smem carve(uint8_t* raw) {
     using O = OpType<TF32>;
     constexpr uint32_t solver = 2u * 64u * NSTRIDE * 4u;
@@ -187,13 +113,31 @@ __device__ __forceinline__ Smem carve(uint8_t* raw) {
     s.BH = p; s.AQ = p; p += O::TILE128;
     s.KH = p; p += O::TILE64;
     s.NAB = reinterpret_cast<float*>(p); s.MAK = s.NAB + 64 * NSTRIDE; s.AS = p; p += r4;
-    s.V = p; p += O::TILE64;
+    s.V[0] = p; p += O::TILE64;
+    if constexpr (!TF32) { s.V[1] = p; p += O::TILE64; } else { s.V[1] = s.V[0]; }
     s.S = p; p += O::TILE64;
+    s.raw = p; p += raw_bytes<TF32, WB>();
     s.gammaL = reinterpret_cast<float*>(p); p += 64 * 4;
     s.red = reinterpret_cast<float*>(p); p += 128 * 4;
     s.bar = reinterpret_cast<uint64_t*>(p); p += 8;
+    s.raw_bar = reinterpret_cast<uint64_t*>(p); p += 8;
     s.tmem_slot = reinterpret_cast<uint32_t*>(p);
     return s;
+}
+
+// Issues the TMA loads of chunk tokens [row0, row0 + 64) of head h: raw r, k,
+// a, b, w_log tiles and the (swizzled) V tile.  One thread.
+template <uint32_t WB>
+__device__ __forceinline__ void issue_chunk_loads(const TmaMaps& m, const Smem& sm, uint8_t* vdst, int h, long row0) {
+    constexpr uint32_t tile = 64u * 64u * 2u;
+    mbar_arrive_expect_tx(sm.raw_bar, 5u * tile + 64u * 64u * WB);
+    const int t0 = static_cast<int>(row0);
+    tma_load_3d(sm.raw + 0 * tile, &m.r, sm.raw_bar, 0, h, t0);
+    tma_load_3d(sm.raw + 1 * tile, &m.k, sm.raw_bar, 0, h, t0);
+    tma_load_3d(sm.raw + 2 * tile, &m.a, sm.raw_bar, 0, h, t0);
+    tma_load_3d(sm.raw + 3 * tile, &m.b, sm.raw_bar, 0, h, t0);
+    tma_load_3d(sm.raw + 4 * tile, &m.wl, sm.raw_bar, 0, h, t0);
+    tma_load_3d(vdst, &m.v, sm.raw_bar, 0, h, t0);
 }
 
 // Row jj of S^T (key channel jj, all 64 value channels) into the S operand tile.
@@ -251,10 +195,12 @@ __global__ void __launch_bounds__(NT, 1)
     wkv7_prefill_kernel(const IO* __restrict__ r, const WT* __restrict__ wl, const IO* __restrict__ k,
                         const IO* __restrict__ v, const IO* __restrict__ a, const IO* __restrict__ b,
                         const float* s0, IO* __restrict__ y, float* sT, int T, int H,
-                        const int32_t* __restrict__ seq_offsets, int* status) {
+                        const int32_t* __restrict__ seq_offsets, int* status,
+                        const __grid_constant__ TmaMaps maps) {
     using O = OpType<TF32>;
+    constexpr uint32_t WB = sizeof(WT);
     extern __shared__ uint8_t smem_raw[];
-    const Smem sm = carve<TF32>(smem_raw);
+    const Smem sm = carve<TF32, WB>(smem_raw);
     const int tid = threadIdx.x;
     const int warp = tid >> 5;
 
@@ -284,9 +230,14 @@ __global__ void __launch_bounds__(NT, 1)
     const long sbase = (static_cast<long>(n) * H + h) * kHead * kHead;
 
     // ---- set-up: barrier, TMEM
+    const int nchunks = static_cast<int>((len + L - 1) / L);
     if (tid == 0) {
         mbar_init(sm.bar, 1);
+        mbar_init(sm.raw_bar, 1);
         fence_mbar_init();
+        if constexpr (!TF32) {
+            if (nchunks > 0) issue_chunk_loads<WB>(maps, sm, sm.V[0], h, tb);
+        }
     }
     if (warp == 0) {
         tmem_alloc(sm.tmem_slot, TMEM_COLS);
@@ -308,22 +259,34 @@ __global__ void __launch_bounds__(NT, 1)
     }
 
     bool ok = true;
-    uint32_t phase = 0;
-    const int nchunks = static_cast<int>((len + L - 1) / L);
+    uint32_t phase = 0;          // parity of the next MMA completion
+    bool mma_pending = false;    // an MMA commit not yet waited for
+    int tma_issued = (!TF32 && nchunks > 0) ? 1 : 0;  // chunks whose TMA loads were issued
+    int tma_consumed = 0;                              // chunks whose TMA loads were waited for
     for (int c = 0; c < nchunks && ok; ++c) {
         const long row0 = tb + static_cast<long>(c) * L;  // first token of the chunk
         const int nv = static_cast<int>(len - static_cast<long>(c) * L < L ? len - static_cast<long>(c) * L : L);
 
         // ---- p1: decay products and scaled operand tiles.  Thread (j, half).
+        if constexpr (!TF32) {
+            ok = __syncthreads_and(mbar_wait(sm.raw_bar, static_cast<uint32_t>(c) & 1u, WAIT_LIMIT_NS));
+            if (!ok) break;
+            tma_consumed = c + 1;
+        }
         {
             const int j = tid & 63, hf = tid >> 6;
+            const __nv_bfloat16* raw16 = reinterpret_cast<const __nv_bfloat16*>(sm.raw);
+            const WT* rawl = reinterpret_cast<const WT*>(sm.raw + 4 * 64 * 64 * 2);
             float cp[32];
             float prod = 1.f;
 #pragma unroll
             for (int q = 0; q < 32; ++q) {
                 const int t = hf * 32 + q;
                 float w = 1.f;
-                if (t < nv) w = expf(-expf(to_f32(wl[(row0 + t) * tstride + hoff + j])));
+                if (t < nv) {
+                    const float l = TF32 ? to_f32(wl[(row0 + t) * tstride + hoff + j]) : to_f32(rawl[t * 64 + j]);
+                    w = expf(-expf(l));
+                }
                 prod *= w;
                 cp[q] = prod;
             }
@@ -334,34 +297,50 @@ __global__ void __launch_bounds__(NT, 1)
             if (hf == 0) sm.gammaL[j] = GL;
             float gprev = pre;
 #pragma unroll
-            for (int q = 0; q < 32; ++q) {
-                const int t = hf * 32 + q;
-                const float G = pre * cp[q];
-                const float inv = 1.f / G;
-                float rr = 0.f, kk = 0.f, aa = 0.f, bb = 0.f;
-                if (t < nv) {
-                    const long off = (row0 + t) * tstride + hoff + j;
-                    rr = to_f32(r[off]);
-                    kk = to_f32(k[off]);
-                    aa = to_f32(a[off]);
-                    bb = to_f32(b[off]);
+            for (int g = 0; g < 4; ++g) {
+                // batches of 8 tokens: all loads of a batch are issued before its stores
+                float rr[8], kk[8], aa[8], bb[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    const int t = hf * 32 + g * 8 + e;
+                    rr[e] = kk[e] = aa[e] = bb[e] = 0.f;
+                    if (t < nv) {
+                        if constexpr (TF32) {
+                            const long off = (row0 + t) * tstride + hoff + j;
+                            rr[e] = to_f32(r[off]);
+                            kk[e] = to_f32(k[off]);
+                            aa[e] = to_f32(a[off]);
+                            bb[e] = to_f32(b[off]);
+                        } else {
+                            rr[e] = to_f32(raw16[0 * 4096 + t * 64 + j]);
+                            kk[e] = to_f32(raw16[1 * 4096 + t * 64 + j]);
+                            aa[e] = to_f32(raw16[2 * 4096 + t * 64 + j]);
+                            bb[e] = to_f32(raw16[3 * 4096 + t * 64 + j]);
+                        }
+                    }
                 }
-                const float invL = inv * GL;
-                st_op<TF32>(sm.RA, 128, t, j, rr * G);
-                st_op<TF32>(sm.RA, 128, 64 + t, j, aa * gprev);
-                st_op<TF32>(sm.BK, 128, t, j, bb * inv);
-                st_op<TF32>(sm.BK, 128, 64 + t, j, kk * inv);
-                st_op<TF32>(sm.BH, 128, 64 + j, t, bb * invL);
-                st_op<TF32>(sm.KH, 64, j, t, kk * invL);
-                gprev = G;
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    const int t = hf * 32 + g * 8 + e;
+                    const float G = pre * cp[g * 8 + e];
+                    const float inv = 1.f / G;
+                    const float invL = inv * GL;
+                    st_op<TF32>(sm.RA, 128, t, j, rr[e] * G);
+                    st_op<TF32>(sm.RA, 128, 64 + t, j, aa[e] * gprev);
+                    st_op<TF32>(sm.BK, 128, t, j, bb[e] * inv);
+                    st_op<TF32>(sm.BK, 128, 64 + t, j, kk[e] * inv);
+                    st_op<TF32>(sm.BH, 128, 64 + j, t, bb[e] * invL);
+                    st_op<TF32>(sm.KH, 64, j, t, kk[e] * invL);
+                    gprev = G;
+                }
             }
-            load_v_tile<IO, TF32>(v, row0, tstride, hoff, nv, sm.V, tid);
+            if constexpr (TF32) load_v_tile<IO, TF32>(v, row0, tstride, hoff, nv, sm.V[0], tid);
         }
         fence_proxy_async_smem();
         tc_fence_before();
         __syncthreads();
 
-        // ---- G = [Rt; At] [Bt; Kt]^T
+        // ---- G = [Rt; At] [Bt; Kt]^T; then prefetch the next chunk's inputs
         if (tid == 0) {
             tc_fence_after();
             constexpr uint32_t idesc = idesc_f32acc(O::FMT, 128, 128, 0, 0);
@@ -370,9 +349,17 @@ __global__ void __launch_bounds__(NT, 1)
                 mma_ss<TF32>(tmem + COL_G, kmajor_desc<TF32>(sm.RA, 128, s), kmajor_desc<TF32>(sm.BK, 128, s), idesc,
                              s > 0);
             mma_commit(sm.bar);
+            if constexpr (!TF32) {
+                // the raw tiles were consumed by p1 (fenced above); the other V slot
+                // was last read by the previous chunk's OUT product, which has completed
+                if (c + 1 < nchunks) issue_chunk_loads<WB>(maps, sm, sm.V[(c + 1) & 1], h, row0 + L);
+            }
         }
+        if (!TF32 && c + 1 < nchunks) tma_issued = c + 2;
+        mma_pending = true;
         ok = __syncthreads_and(mbar_wait(sm.bar, phase, WAIT_LIMIT_NS));
         if (!ok) break;
+        mma_pending = false;
         phase ^= 1u;
         tc_fence_after();
 
@@ -446,8 +433,10 @@ __global__ void __launch_bounds__(NT, 1)
                              idesc, s > 0);
             mma_commit(sm.bar);
         }
+        mma_pending = true;
         ok = __syncthreads_and(mbar_wait(sm.bar, phase, WAIT_LIMIT_NS));
         if (!ok) break;
+        mma_pending = false;
         phase ^= 1u;
         tc_fence_after();
 
@@ -499,7 +488,7 @@ __global__ void __launch_bounds__(NT, 1)
             constexpr uint32_t idesc = idesc_f32acc(O::FMT, 128, 64, 0, TF32 ? 0 : 1);
 #pragma unroll
             for (uint32_t s = 0; s < O::KSTEPS; ++s) {
-                const uint64_t bd = TF32 ? kmajor_desc<TF32>(sm.V, 64, s) : mnmajor_desc<TF32>(sm.V, 64, s);
+                const uint64_t bd = TF32 ? kmajor_desc<TF32>(sm.V[0], 64, s) : mnmajor_desc<TF32>(sm.V[c & 1], 64, s);
                 mma_ss<TF32>(tmem + COL_O, kmajor_desc<TF32>(sm.AQ, 128, s), bd, idesc, s > 0);
             }
 #pragma unroll
@@ -509,8 +498,10 @@ __global__ void __launch_bounds__(NT, 1)
             }
             mma_commit(sm.bar);
         }
+        mma_pending = true;
         ok = __syncthreads_and(mbar_wait(sm.bar, phase, WAIT_LIMIT_NS));
         if (!ok) break;
+        mma_pending = false;
         phase ^= 1u;
         tc_fence_after();
 
@@ -560,8 +551,11 @@ __global__ void __launch_bounds__(NT, 1)
 
     if (!ok) {
         if (tid == 0) report_status(status, WKV7_ERR_DEVICE_TIMEOUT);
-        // let any MMA still in flight finish (bounded) before TMEM is released
-        mbar_wait(sm.bar, phase, WAIT_LIMIT_NS);
+        // let MMAs and TMA loads still in flight finish (bounded) before the
+        // block releases TMEM and its shared memory
+        if (mma_pending) mbar_wait(sm.bar, phase, WAIT_LIMIT_NS);
+        for (int ci = tma_consumed; ci < tma_issued; ++ci)
+            mbar_wait(sm.raw_bar, static_cast<uint32_t>(ci) & 1u, WAIT_LIMIT_NS);
     } else if (sT && tid >= 64) {
 #pragma unroll
         for (int i = 0; i < 64; ++i) sT[sbase + i * kHead + jj] = S[i];
@@ -574,9 +568,54 @@ __global__ void __launch_bounds__(NT, 1)
     }
 }
 
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    if (!fn) {
+        void* f = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(f);
+    }
+    return fn;
+}
+
+// [ntok][H][64] tensor of `esize`-byte elements, box 64 x 1 x 64.
+bool make_token_map(CUtensorMap* m, const void* base, CUtensorMapDataType dt, uint64_t esize, uint64_t H,
+                    uint64_t ntok, CUtensorMapSwizzle sw) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    const cuuint64_t dims[3] = {64, H, ntok};
+    const cuuint64_t strides[2] = {64 * esize, H * 64 * esize};
+    const cuuint32_t box[3] = {64, 1, 64};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    return fn(m, dt, 3, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 template <typename IO, typename WT, bool TF32>
 cudaError_t launch_typed(const PrefillArgs& p, cudaStream_t stream) {
-    constexpr uint32_t smem = smem_bytes_needed<TF32>();
+    constexpr uint32_t smem = smem_bytes_needed<TF32, sizeof(WT)>();
+    TmaMaps maps;
+    memset(&maps, 0, sizeof(maps));
+    if constexpr (!TF32) {
+        const uint64_t ntok = p.seq_offsets ? static_cast<uint64_t>(p.T) : static_cast<uint64_t>(p.B) * p.T;
+        const CUtensorMapDataType bf = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+        const CUtensorMapDataType wdt =
+            sizeof(WT) == 4 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+        const CUtensorMapSwizzle none = CU_TENSOR_MAP_SWIZZLE_NONE;
+        if (!make_token_map(&maps.r, p.r, bf, 2, p.H, ntok, none) ||
+            !make_token_map(&maps.k, p.k, bf, 2, p.H, ntok, none) ||
+            !make_token_map(&maps.a, p.a, bf, 2, p.H, ntok, none) ||
+            !make_token_map(&maps.b, p.b, bf, 2, p.H, ntok, none) ||
+            !make_token_map(&maps.wl, p.w_log, wdt, sizeof(WT), p.H, ntok, none) ||
+            !make_token_map(&maps.v, p.v, bf, 2, p.H, ntok, CU_TENSOR_MAP_SWIZZLE_128B))
+            return cudaErrorInvalidValue;
+    }
     auto kern = wkv7_prefill_kernel<IO, WT, TF32>;
     static unsigned long long configured = 0;  // one bit per device ordinal
     int dev = 0;
@@ -592,7 +631,7 @@ cudaError_t launch_typed(const PrefillArgs& p, cudaStream_t stream) {
     kern<<<static_cast<unsigned>(units), NT, smem, stream>>>(
         static_cast<const IO*>(p.r), static_cast<const WT*>(p.w_log), static_cast<const IO*>(p.k),
         static_cast<const IO*>(p.v), static_cast<const IO*>(p.a), static_cast<const IO*>(p.b), p.s0,
-        static_cast<IO*>(p.y), p.sT, p.T, p.H, p.seq_offsets, p.status);
+        static_cast<IO*>(p.y), p.sT, p.T, p.H, p.seq_offsets, p.status, maps);
     return cudaGetLastError();
 }
 
@@ -609,10 +648,7 @@ __global__ void expire_wait_kernel(int spins, int* status) {
 }  // namespace
 
 cudaError_t launch_prefill(const PrefillArgs& p, int io_dtype, int w_dtype, cudaStream_t stream) {
-    if (io_dtype == WKV7_BF16) {
-        return w_dtype == WKV7_BF16 ? launch_typed<__nv_bfloat16, __nv_bfloat16, false>(p, stream)
-                                    : launch_typed<__nv_bfloat16, float, false>(p, stream);
-    }
+    if (io_dtype == WKV7_BF16) return launch_prefill_pipe(p, w_dtype, stream);
     return w_dtype == WKV7_BF16 ? launch_typed<float, __nv_bfloat16, true>(p, stream)
                                 : launch_typed<float, float, true>(p, stream);
 }

@@ -1,0 +1,638 @@
+// wkv7_prefill_pipe.cu — warp-specialised chunked WKV-7 prefill for bf16 inputs.
+//
+// Same chunk algebra as wkv7_prefill.cu (derived from the generalized delta
+// rule of "RWKV-7 Goose: Expressive Dynamic State Evolution", section
+// "Generalized Delta rule", with the argument roles of the hxa07D WKV call):
+// per 64-token chunk with start state S0 and Gamma_t = prod_{s<=t} w_s,
+//   Y     = (Rt + Mrb W) S0^T + (Mrk + Mrb Z) V
+//   S_L^T = Gamma_L (.) S0^T  + (Bh^T W) S0^T + (Kh^T + Bh^T Z) V
+// with [W | Z] = T [At | Mak] and T = (I - Nab)^{-1}.  T is formed explicitly
+// in fp32 on the CUDA cores (32 x 32 diagonal blocks by substitution, the
+// off-diagonal block as T_hi Nab_hl T_lo) and folded into tensor-core products:
+//   G   = [Rt; At] [Bt; Kt]^T                        (Mrb | Mrk over Nab | Mak)
+//   Q   = [Mrb; Bh^T] T
+//   P   = Q [At | Mak]                               (Mrb W | Mrb Z over Bh^T W | Bh^T Z)
+//   OUT = [Mrb Z; Bh^T Z] V + [Mrk; Kh^T] V + [Rt + Mrb W; Bh^T W] S0^T
+//                                                    (Y over S_L^T - Gamma_L (.) S0^T)
+// Only the last product depends on the state.
+//
+// Block of 384 threads, one (sequence, head) unit:
+//   warps 0-3  prep group 0: chunks 0, 2, 4, ...   (everything up to OUT without S0)
+//   warps 4-7  prep group 1: chunks 1, 3, 5, ...
+//   warps 8-11 serial group: for every chunk in order, the S0-dependent product,
+//              the y rows and the fp32 state update (state held in registers
+//              of the threads owning TMEM lanes 64..127, one key channel each).
+// The two prep groups overlap each other's latencies and run ahead of the
+// serial group; each owns its shared-memory tiles and TMEM columns, except the
+// [R'; Bh^T W] tile that the serial group reads, which is shared.
+// Synchronisation: a prep group hands a chunk to the serial group through
+// `ready[g]` (MMA commit + release arrive); the serial group releases the
+// shared tile (and the group's OUT columns) through `free_` after each chunk.
+// All waits are bounded.
+#include <cstring>
+
+#include "prefill_common.cuh"
+#include "sm100_ptx.cuh"
+#include "wkv7_internal.cuh"
+
+namespace wkv7 {
+namespace {
+
+constexpr int L = 64;
+constexpr int NTHR = 384;
+constexpr uint32_t GROUP = 128;
+constexpr uint64_t WAIT_NS = 1000000000ull;  // 1 s
+
+// per prep-group shared-memory tiles (bytes)
+constexpr uint32_t OFF_RAM = 0;        // Rt (rows 0-63) | At (rows 64-127) | Mak (64 tokens x 64), 24 KB
+constexpr uint32_t OFF_BK = 24576;     // [Bt; Kt] 16 KB, then T fp32 (64 x 64, column-swizzled)
+constexpr uint32_t OFF_BH = 40960;     // [Mrb; Bh^T] 16 KB, then [Mrb Z; Bh^T Z]
+constexpr uint32_t OFF_MK = 57344;     // [Mrk; Kh^T] 16 KB, K-major over tokens
+constexpr uint32_t OFF_NQ = 73728;     // Nab^T fp32 16 KB, then X (32 x 32 fp32) + T bf16 at +8 KB, then Q bf16
+constexpr uint32_t OFF_V = 90112;      // V 8 KB (MN-major)
+constexpr uint32_t GROUP_TILES = 98304;
+constexpr uint32_t OFF_AS = 2 * GROUP_TILES;          // [R'; Bh^T W] 16 KB, shared by both groups
+constexpr uint32_t OFF_S = OFF_AS + 16384;            // S^T bf16, 8 KB (serial group)
+constexpr uint32_t OFF_GAMMA = OFF_S + 8192;          // Gamma_L [2 groups][2 slots][64] fp32
+constexpr uint32_t OFF_RED = OFF_GAMMA + 2 * 2 * 64 * 4;  // block products [2 groups][4][64] fp32
+constexpr uint32_t OFF_BAR = OFF_RED + 2 * 4 * 64 * 4;
+constexpr uint32_t SMEM_USED = OFF_BAR + 8 * 8 + 16;
+constexpr uint32_t SMEM_BYTES = SMEM_USED + 1024;      // alignment slack
+
+// TMEM columns
+constexpr uint32_t TM_GP = 0;    // + 256 g: G, then P (128 columns)
+constexpr uint32_t TM_Q = 128;   // + 256 g: Q (64 columns)
+constexpr uint32_t TM_OUT = 192; // + 256 g: OUT (64 columns)
+constexpr uint32_t TMEM_COLS = 512;
+
+constexpr uint32_t ID_G16 = idesc_f32acc(1, 128, 128, 0, 0);  // K-major A and B, N = 128
+constexpr uint32_t ID_KM128 = idesc_f32acc(1, 128, 128, 0, 1); // B MN-major, N = 128
+constexpr uint32_t ID_KM64 = idesc_f32acc(1, 128, 64, 0, 1);   // B MN-major, N = 64
+
+// fp32 64 x 64 matrix with its 4-column groups XOR-permuted by row (bank spread)
+__device__ __forceinline__ uint32_t tf_idx(uint32_t row, uint32_t col) {
+    return row * 64u + (col ^ ((row & 7u) << 2));
+}
+
+__device__ __forceinline__ float2 unpack_bf16x2(uint32_t u) { return make_float2(bf16lo_to_f32(u), bf16hi_to_f32(u)); }
+
+template <typename WT>
+__device__ __forceinline__ float2 load_pair(const WT* p);
+template <>
+__device__ __forceinline__ float2 load_pair<float>(const float* p) {
+    return __ldg(reinterpret_cast<const float2*>(p));
+}
+template <>
+__device__ __forceinline__ float2 load_pair<__nv_bfloat16>(const __nv_bfloat16* p) {
+    return unpack_bf16x2(__ldg(reinterpret_cast<const unsigned int*>(p)));
+}
+__device__ __forceinline__ uint32_t load_u32(const __nv_bfloat16* p) {
+    return __ldg(reinterpret_cast<const unsigned int*>(p));
+}
+
+struct Bars {
+    uint64_t* mma;    // [2] prep-group MMA completions (G, Q, P)
+    uint64_t* ready;  // [2] OUT-pre complete and chunk tiles published (count 2)
+    uint64_t* free_;  // serial group done with a chunk (shared tile and OUT columns reusable)
+    uint64_t* ser;    // serial MMA completion
+    uint32_t* tmem_slot;
+};
+
+template <typename WT>
+__global__ void __launch_bounds__(NTHR, 1)
+    wkv7_prefill_pipe_kernel(const __nv_bfloat16* __restrict__ r, const WT* __restrict__ wl,
+                             const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restrict__ v,
+                             const __nv_bfloat16* __restrict__ a, const __nv_bfloat16* __restrict__ b,
+                             const float* s0, __nv_bfloat16* __restrict__ y, float* sT, int T, int H,
+                             const int32_t* __restrict__ seq_offsets, int* status) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023u) & ~uintptr_t(1023));
+    const int tid = threadIdx.x;
+    const int warp = tid >> 5;
+    Bars bars;
+    {
+        uint64_t* p = reinterpret_cast<uint64_t*>(sm + OFF_BAR);
+        bars.mma = p;
+        bars.ready = p + 2;
+        bars.free_ = p + 4;
+        bars.ser = p + 6;
+        bars.tmem_slot = reinterpret_cast<uint32_t*>(p + 8);
+    }
+
+    // ---- the unit and its tokens
+    const int unit = blockIdx.x;
+    const int n = unit / H, h = unit % H;
+    long tb = 0, len = 0;
+    if (seq_offsets) {
+        const long o0 = seq_offsets[n], o1 = seq_offsets[n + 1];
+        if (o0 < 0 || o1 < o0 || o1 > T) {
+            if (tid == 0) report_status(status, WKV7_ERR_DEVICE_BOUNDS);
+            return;
+        }
+        tb = o0;
+        len = o1 - o0;
+    } else {
+        tb = static_cast<long>(n) * T;
+        len = T;
+    }
+    const long tstride = static_cast<long>(H) * kHead;
+    const long hoff = static_cast<long>(h) * kHead;
+    const long sbase = (static_cast<long>(n) * H + h) * kHead * kHead;
+    const int nchunks = static_cast<int>((len + L - 1) / L);
+
+    if (tid == 0) {
+        for (int g = 0; g < 2; ++g) {
+            mbar_init(&bars.mma[g], 1);
+            mbar_init(&bars.ready[g], 2);
+        }
+        mbar_init(bars.free_, 1);
+        mbar_init(bars.ser, 1);
+        fence_mbar_init();
+    }
+    if (warp == 0) {
+        tmem_alloc(bars.tmem_slot, TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *bars.tmem_slot;
+    const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    bool ok = true;
+
+    if (warp < 8) {
+        // =========================================================== prep groups
+        const int g = warp >> 2;
+        const int tg = tid & 127;
+        const uint32_t bar_id = 1 + g;
+        uint8_t* gt = sm + g * GROUP_TILES;
+        uint8_t* RAM = gt + OFF_RAM;
+        uint8_t* BK = gt + OFF_BK;
+        uint8_t* BH = gt + OFF_BH;
+        uint8_t* MK = gt + OFF_MK;
+        float* Tf = reinterpret_cast<float*>(gt + OFF_BK);
+        float* Nt = reinterpret_cast<float*>(gt + OFF_NQ);
+        float* Xs = Nt;
+        uint8_t* Tb = gt + OFF_NQ + 8192;
+        uint8_t* Qt = gt + OFF_NQ;
+        uint8_t* AS = sm + OFF_AS;
+        uint8_t* Vt = gt + OFF_V;
+        float* gam = reinterpret_cast<float*>(sm + OFF_GAMMA) + g * 128;
+        float* red = reinterpret_cast<float*>(sm + OFF_RED) + g * 256;
+        const uint32_t tm_gp = tmem + 256u * g + TM_GP;
+        const uint32_t tm_q = tmem + 256u * g + TM_Q;
+        const uint32_t tm_out = tmem + 256u * g + TM_OUT;
+        uint32_t mma_phase = 0;
+        bool mma_pending = false;
+        int issued_out = 0;  // OUT-pre commits issued by this group
+
+        for (int c = g; c < nchunks; c += 2) {
+            const int kk_ = c >> 1;
+            const long row0 = tb + static_cast<long>(c) * L;
+            const int nv = static_cast<int>(len - static_cast<long>(c) * L < L ? len - static_cast<long>(c) * L : L);
+
+            // ---- p1: decay products and the scaled operand tiles.  Thread (jp, tq):
+            // key channels 2jp, 2jp+1 of tokens 16tq .. 16tq+15.  Global loads come
+            // in two batches (decay logits with the first 8 tokens, then the last 8),
+            // each issued before any shared-memory store.
+            const int jp = tg & 31, tq = tg >> 5, j0 = 2 * jp;
+            float2 cw[16];
+            uint32_t rr[8], kv[8], av[8], bv[8], vv[8];
+            auto load_batch = [&](int e0) {
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    const int t = 16 * tq + e0 + e;
+                    if (t < nv) {
+                        const long off = (row0 + t) * tstride + hoff + j0;
+                        rr[e] = load_u32(r + off);
+                        kv[e] = load_u32(k + off);
+                        av[e] = load_u32(a + off);
+                        bv[e] = load_u32(b + off);
+                        vv[e] = load_u32(v + off);
+                    } else {
+                        rr[e] = kv[e] = av[e] = bv[e] = vv[e] = 0u;
+                    }
+                }
+            };
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {
+                const int t = 16 * tq + e;
+                cw[e] = (t < nv) ? load_pair<WT>(wl + (row0 + t) * tstride + hoff + j0) : make_float2(-INFINITY, -INFINITY);
+            }
+            load_batch(0);
+            float p0 = 1.f, p1 = 1.f;
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {
+                p0 *= __expf(-__expf(cw[e].x));
+                p1 *= __expf(-__expf(cw[e].y));
+                cw[e] = make_float2(p0, p1);  // cumulative product inside the 16-token block
+            }
+            // the previous reads of this group's V, BH and MK tiles (OUT of chunk c-2) must be complete
+            bool w_ok = true;
+            if (kk_ >= 1 && tg == 0) w_ok = mbar_wait(&bars.ready[g], static_cast<uint32_t>(kk_ - 1) & 1u, WAIT_NS);
+            red[tq * 64 + j0] = p0;
+            red[tq * 64 + j0 + 1] = p1;
+            ok = group_sync_and(bar_id, GROUP, w_ok);
+            if (!ok) break;
+            float pre0 = 1.f, pre1 = 1.f, GL0 = 1.f, GL1 = 1.f;
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const float x0 = red[q * 64 + j0], x1 = red[q * 64 + j0 + 1];
+                if (q < tq) { pre0 *= x0; pre1 *= x1; }
+                GL0 *= x0;
+                GL1 *= x1;
+            }
+            if (tq == 3) {
+                gam[(kk_ & 1) * 64 + j0] = GL0;
+                gam[(kk_ & 1) * 64 + j0 + 1] = GL1;
+            }
+            float gp0 = pre0, gp1 = pre1;
+            const uint32_t cb = static_cast<uint32_t>(j0) * 2u;
+#pragma unroll
+            for (int half = 0; half < 2; ++half) {
+                if (half == 1) load_batch(8);
+                uint32_t bh0[4], bh1[4], kh0[4], kh1[4];  // 8 tokens of Bh^T / Kh^T rows j0, j0+1
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    const int t = 16 * tq + 8 * half + e;
+                    const float G0 = pre0 * cw[8 * half + e].x, G1 = pre1 * cw[8 * half + e].y;
+                    const float i0 = __frcp_rn(G0), i1 = __frcp_rn(G1);
+                    const float l0 = i0 * GL0, l1 = i1 * GL1;
+                    const float2 rf = unpack_bf16x2(rr[e]), kf = unpack_bf16x2(kv[e]);
+                    const float2 af = unpack_bf16x2(av[e]), bf = unpack_bf16x2(bv[e]);
+                    *reinterpret_cast<uint32_t*>(RAM + swz(t, cb, 128)) = pack_bf16x2(rf.x * G0, rf.y * G1);
+                    *reinterpret_cast<uint32_t*>(RAM + swz(64 + t, cb, 128)) = pack_bf16x2(af.x * gp0, af.y * gp1);
+                    *reinterpret_cast<uint32_t*>(BK + swz(t, cb, 128)) = pack_bf16x2(bf.x * i0, bf.y * i1);
+                    *reinterpret_cast<uint32_t*>(BK + swz(64 + t, cb, 128)) = pack_bf16x2(kf.x * i0, kf.y * i1);
+                    *reinterpret_cast<uint32_t*>(Vt + swz(t, cb, 64)) = vv[e];
+                    const float b0 = bf.x * l0, b1 = bf.y * l1, k0 = kf.x * l0, k1 = kf.y * l1;
+                    if ((e & 1) == 0) {
+                        bh0[e >> 1] = __float_as_uint(b0);
+                        bh1[e >> 1] = __float_as_uint(b1);
+                        kh0[e >> 1] = __float_as_uint(k0);
+                        kh1[e >> 1] = __float_as_uint(k1);
+                    } else {
+                        bh0[e >> 1] = pack_bf16x2(__uint_as_float(bh0[e >> 1]), b0);
+                        bh1[e >> 1] = pack_bf16x2(__uint_as_float(bh1[e >> 1]), b1);
+                        kh0[e >> 1] = pack_bf16x2(__uint_as_float(kh0[e >> 1]), k0);
+                        kh1[e >> 1] = pack_bf16x2(__uint_as_float(kh1[e >> 1]), k1);
+                    }
+                    gp0 = G0;
+                    gp1 = G1;
+                }
+                const uint32_t tb8 = static_cast<uint32_t>(16 * tq + 8 * half) * 2u;  // byte of the first token
+                *reinterpret_cast<uint4*>(BH + swz(64 + j0, tb8, 128)) = make_uint4(bh0[0], bh0[1], bh0[2], bh0[3]);
+                *reinterpret_cast<uint4*>(BH + swz(64 + j0 + 1, tb8, 128)) = make_uint4(bh1[0], bh1[1], bh1[2], bh1[3]);
+                *reinterpret_cast<uint4*>(MK + swz(64 + j0, tb8, 128)) = make_uint4(kh0[0], kh0[1], kh0[2], kh0[3]);
+                *reinterpret_cast<uint4*>(MK + swz(64 + j0 + 1, tb8, 128)) = make_uint4(kh1[0], kh1[1], kh1[2], kh1[3]);
+            }
+            fence_proxy_async_smem();
+            tc_fence_before();
+            group_sync(bar_id, GROUP);
+
+            // ---- G = [Rt; At] [Bt; Kt]^T
+            if (tg == 0) {
+                tc_fence_after();
+#pragma unroll
+                for (uint32_t s = 0; s < 4; ++s)
+                    mma_ss<false>(tm_gp, kmajor_desc<false>(RAM, 128, s), kmajor_desc<false>(BK, 128, s), ID_G16, s > 0);
+                mma_commit(&bars.mma[g]);
+            }
+            mma_pending = true;
+            ok = group_sync_and(bar_id, GROUP, mbar_wait(&bars.mma[g], mma_phase, WAIT_NS));
+            if (!ok) break;
+            mma_pending = false;
+            mma_phase ^= 1u;
+            tc_fence_after();
+
+            // ---- masks: Mrb -> BH rows 0..63, Mrk -> MK rows 0..63 (incl. diagonal);
+            //      Nab -> Nab^T fp32 and Mak -> MN-major tile next to At (strict)
+            {
+                float x[32];
+                if (tg < 64) {
+                    const int t = tg;
+#pragma unroll
+                    for (int qq = 0; qq < 4; ++qq) {
+                        tmem_load32(tm_gp + lane_base + 32 * qq, x);
+#pragma unroll
+                        for (int i = 0; i < 32; ++i)
+                            if (32 * (qq & 1) + i > t) x[i] = 0.f;
+                        st_op_row32<false>(qq < 2 ? BH : MK, 128, t, 32 * (qq & 1), x);
+                    }
+                } else {
+                    const int t = tg - 64;
+#pragma unroll
+                    for (int qq = 0; qq < 2; ++qq) {
+                        tmem_load32(tm_gp + lane_base + 32 * qq, x);
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) Nt[(32 * qq + i) * 64 + t] = (32 * qq + i < t) ? x[i] : 0.f;
+                    }
+#pragma unroll
+                    for (int qq = 0; qq < 2; ++qq) {
+                        tmem_load32(tm_gp + lane_base + 64 + 32 * qq, x);
+#pragma unroll
+                        for (int i = 0; i < 32; ++i)
+                            if (32 * qq + i >= t) x[i] = 0.f;
+                        st_op_row32<false>(RAM + 16384, 64, t, 32 * qq, x);
+                    }
+                }
+            }
+            fence_proxy_async_smem();
+            tc_fence_before();
+            group_sync(bar_id, GROUP);
+
+            // ---- T = (I - Nab)^{-1}: 32 x 32 diagonal blocks by right-looking substitution
+            if (tg < 64) {
+                const int blk = (tg >> 5) * 32, col = tg & 31;
+                float acc[32];
+#pragma unroll
+                for (int i = 0; i < 32; ++i) acc[i] = (i == col) ? 1.f : 0.f;
+#pragma unroll
+                for (int t = 0; t < 31; ++t) {
+                    const float xt = acc[t];
+                    const float* nrow = Nt + (blk + t) * 64 + blk;  // column blk+t of Nab
+#pragma unroll
+                    for (int i = t + 1; i < 32; ++i) acc[i] = fmaf(nrow[i], xt, acc[i]);
+                }
+#pragma unroll
+                for (int i = 0; i < 32; ++i) Tf[tf_idx(blk + i, blk + col)] = acc[i];
+                if (blk == 0) {
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) Tf[tf_idx(i, 32 + col)] = 0.f;
+                }
+            }
+            group_sync(bar_id, GROUP);
+            // off-diagonal block: T_hl = T_hi (N_hl T_lo)
+            {
+                const int rr2 = tg >> 2, cq = tg & 3;
+                float xo[8];
+#pragma unroll
+                for (int i = 0; i < 8; ++i) xo[i] = 0.f;
+#pragma unroll 8
+                for (int kk2 = 0; kk2 < 32; ++kk2) {
+                    const float nvv = Nt[kk2 * 64 + 32 + rr2];  // N[32 + rr2][kk2]
+                    const float4 t0 = *reinterpret_cast<const float4*>(Tf + tf_idx(kk2, 8 * cq));
+                    const float4 t1 = *reinterpret_cast<const float4*>(Tf + tf_idx(kk2, 8 * cq + 4));
+                    xo[0] = fmaf(nvv, t0.x, xo[0]); xo[1] = fmaf(nvv, t0.y, xo[1]);
+                    xo[2] = fmaf(nvv, t0.z, xo[2]); xo[3] = fmaf(nvv, t0.w, xo[3]);
+                    xo[4] = fmaf(nvv, t1.x, xo[4]); xo[5] = fmaf(nvv, t1.y, xo[5]);
+                    xo[6] = fmaf(nvv, t1.z, xo[6]); xo[7] = fmaf(nvv, t1.w, xo[7]);
+                }
+                group_sync(bar_id, GROUP);  // every thread has finished reading Nab^T
+                *reinterpret_cast<float4*>(Xs + rr2 * 32 + 8 * cq) = make_float4(xo[0], xo[1], xo[2], xo[3]);
+                *reinterpret_cast<float4*>(Xs + rr2 * 32 + 8 * cq + 4) = make_float4(xo[4], xo[5], xo[6], xo[7]);
+                group_sync(bar_id, GROUP);
+#pragma unroll
+                for (int i = 0; i < 8; ++i) xo[i] = 0.f;
+#pragma unroll 8
+                for (int kk2 = 0; kk2 < 32; ++kk2) {
+                    const float th = Tf[tf_idx(32 + rr2, 32 + kk2)];  // T_hi[rr2][kk2]
+                    const float4 x0 = *reinterpret_cast<const float4*>(Xs + kk2 * 32 + 8 * cq);
+                    const float4 x1 = *reinterpret_cast<const float4*>(Xs + kk2 * 32 + 8 * cq + 4);
+                    xo[0] = fmaf(th, x0.x, xo[0]); xo[1] = fmaf(th, x0.y, xo[1]);
+                    xo[2] = fmaf(th, x0.z, xo[2]); xo[3] = fmaf(th, x0.w, xo[3]);
+                    xo[4] = fmaf(th, x1.x, xo[4]); xo[5] = fmaf(th, x1.y, xo[5]);
+                    xo[6] = fmaf(th, x1.z, xo[6]); xo[7] = fmaf(th, x1.w, xo[7]);
+                }
+                *reinterpret_cast<float4*>(Tf + tf_idx(32 + rr2, 8 * cq)) = make_float4(xo[0], xo[1], xo[2], xo[3]);
+                *reinterpret_cast<float4*>(Tf + tf_idx(32 + rr2, 8 * cq + 4)) = make_float4(xo[4], xo[5], xo[6], xo[7]);
+            }
+            group_sync(bar_id, GROUP);
+            // T -> bf16, MN-major (rows i, columns j)
+#pragma unroll
+            for (int m = 0; m < 4; ++m) {
+                const int qd = tg + 128 * m;
+                const int row = qd >> 3, ch = qd & 7;
+                const float4 f0 = *reinterpret_cast<const float4*>(Tf + tf_idx(row, 8 * ch));
+                const float4 f1 = *reinterpret_cast<const float4*>(Tf + tf_idx(row, 8 * ch + 4));
+                *reinterpret_cast<uint4*>(Tb + swz(row, ch * 16, 64)) =
+                    make_uint4(pack_bf16x2(f0.x, f0.y), pack_bf16x2(f0.z, f0.w), pack_bf16x2(f1.x, f1.y),
+                               pack_bf16x2(f1.z, f1.w));
+            }
+            fence_proxy_async_smem();
+            group_sync(bar_id, GROUP);
+
+            // ---- Q = [Mrb; Bh^T] T
+            if (tg == 0) {
+                tc_fence_after();
+#pragma unroll
+                for (uint32_t s = 0; s < 4; ++s)
+                    mma_ss<false>(tm_q, kmajor_desc<false>(BH, 128, s), mnmajor_desc<false>(Tb, 64, s), ID_KM64, s > 0);
+                mma_commit(&bars.mma[g]);
+            }
+            mma_pending = true;
+            ok = group_sync_and(bar_id, GROUP, mbar_wait(&bars.mma[g], mma_phase, WAIT_NS));
+            if (!ok) break;
+            mma_pending = false;
+            mma_phase ^= 1u;
+            tc_fence_after();
+            {
+                float x[32];
+#pragma unroll
+                for (int qq = 0; qq < 2; ++qq) {
+                    tmem_load32(tm_q + lane_base + 32 * qq, x);
+                    st_op_row32<false>(Qt, 128, tg, 32 * qq, x);
+                }
+            }
+            fence_proxy_async_smem();
+            tc_fence_before();
+            group_sync(bar_id, GROUP);
+
+            // ---- P = Q [At | Mak]
+            if (tg == 0) {
+                tc_fence_after();
+#pragma unroll
+                for (uint32_t s = 0; s < 4; ++s)
+                    mma_ss<false>(tm_gp, kmajor_desc<false>(Qt, 128, s), mnmajor_desc<false>(RAM + 8192, 64, s),
+                                  ID_KM128, s > 0);
+                mma_commit(&bars.mma[g]);
+            }
+            // the shared [R'; Bh^T W] tile and this group's OUT columns are free once
+            // the serial group is done with chunk c-1
+            mma_pending = true;
+            {
+                bool w1 = mbar_wait(&bars.mma[g], mma_phase, WAIT_NS);
+                if (c >= 1) w1 = w1 && mbar_wait(bars.free_, static_cast<uint32_t>(c - 1) & 1u, WAIT_NS);
+                ok = group_sync_and(bar_id, GROUP, w1);
+            }
+            if (!ok) break;
+            mma_pending = false;
+            mma_phase ^= 1u;
+            tc_fence_after();
+            {
+                float x[32];
+                const int row = tg;  // lanes 0..63: token rows (R' = Rt + Mrb W, Mrb Z); 64..127: key rows
+#pragma unroll
+                for (int q = 0; q < 2; ++q) {
+                    tmem_load32(tm_gp + lane_base + 32 * q, x);
+                    if (tg < 64) {
+                        float rt[32];
+                        ld_op_row32<false>(RAM, 128, row, 32 * q, rt);
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) x[i] += rt[i];
+                    }
+                    st_op_row32<false>(AS, 128, row, 32 * q, x);
+                }
+#pragma unroll
+                for (int q = 0; q < 2; ++q) {
+                    tmem_load32(tm_gp + lane_base + 64 + 32 * q, x);
+                    st_op_row32<false>(BH, 128, row, 32 * q, x);
+                }
+            }
+            fence_proxy_async_smem();
+            tc_fence_before();
+            group_sync(bar_id, GROUP);
+
+            // ---- OUT = [Mrb Z; Bh^T Z] V + [Mrk; Kh^T] V   (the serial group adds [R'; Bh^T W] S0^T)
+            if (tg == 0) {
+                tc_fence_after();
+#pragma unroll
+                for (uint32_t s = 0; s < 4; ++s)
+                    mma_ss<false>(tm_out, kmajor_desc<false>(BH, 128, s), mnmajor_desc<false>(Vt, 64, s), ID_KM64, s > 0);
+#pragma unroll
+                for (uint32_t s = 0; s < 4; ++s)
+                    mma_ss<false>(tm_out, kmajor_desc<false>(MK, 128, s), mnmajor_desc<false>(Vt, 64, s), ID_KM64, 1);
+                mma_commit(&bars.ready[g]);
+                mbar_arrive(&bars.ready[g]);  // this chunk's [R'; Bh^T W] and Gamma_L are published
+            }
+            ++issued_out;
+        }
+        if (!ok && tg == 0) report_status(status, WKV7_ERR_DEVICE_TIMEOUT);
+        // drain: an unwaited G/Q/P product, and the last OUT-pre product
+        if (mma_pending) mbar_wait(&bars.mma[g], mma_phase, WAIT_NS);
+        if (issued_out > 0) mbar_wait(&bars.ready[g], static_cast<uint32_t>(issued_out - 1) & 1u, WAIT_NS);
+    } else {
+        // =========================================================== serial group
+        const int ts = tid - 256;
+        const uint32_t bar_id = 3;
+        uint8_t* St = sm + OFF_S;
+        const float* gam_all = reinterpret_cast<const float*>(sm + OFF_GAMMA);
+        float S[64];
+        const int x = ts - 64;  // key channel owned by lanes 64..127
+        if (ts >= 64) {
+#pragma unroll
+            for (int i = 0; i < 64; ++i) S[i] = s0 ? s0[sbase + i * kHead + x] : 0.f;
+            st_op_row32<false>(St, 64, x, 0, S);
+            st_op_row32<false>(St, 64, x, 32, S + 32);
+        }
+        fence_proxy_async_smem();
+        group_sync(bar_id, GROUP);
+        uint32_t ser_phase = 0;
+        bool ser_pending = false;
+        for (int c = 0; c < nchunks; ++c) {
+            const int g = c & 1, kk_ = c >> 1;
+            const long row0 = tb + static_cast<long>(c) * L;
+            const int nv = static_cast<int>(len - static_cast<long>(c) * L < L ? len - static_cast<long>(c) * L : L);
+            const uint32_t tm_out = tmem + 256u * g + TM_OUT;
+            uint8_t* AS = sm + OFF_AS;
+            if (c + 2 < nchunks) {
+                // L2 line hints for the rows a prep group will load two chunks ahead
+                const long rows2 = row0 + 2 * L;
+                const int nv2 = static_cast<int>(len - static_cast<long>(c + 2) * L < L ? len - static_cast<long>(c + 2) * L : L);
+                const int row = ts & 63;
+                if (row < nv2) {
+                    const long off = (rows2 + row) * tstride + hoff;
+                    if (ts < 64) {
+                        prefetch_line_l2(r + off);
+                        prefetch_line_l2(k + off);
+                        prefetch_line_l2(a + off);
+                        prefetch_line_l2(wl + off);
+                    } else {
+                        prefetch_line_l2(b + off);
+                        prefetch_line_l2(v + off);
+                        prefetch_line_l2(wl + off + 32);
+                    }
+                }
+            }
+            ok = group_sync_and(bar_id, GROUP, mbar_wait(&bars.ready[g], static_cast<uint32_t>(kk_) & 1u, WAIT_NS));
+            if (!ok) break;
+            tc_fence_after();
+            if (ts == 0) {
+#pragma unroll
+                for (uint32_t s = 0; s < 4; ++s)
+                    mma_ss<false>(tm_out, kmajor_desc<false>(AS, 128, s), mnmajor_desc<false>(St, 64, s), ID_KM64, 1);
+                mma_commit(bars.ser);
+            }
+            ser_pending = true;
+            ok = group_sync_and(bar_id, GROUP, mbar_wait(bars.ser, ser_phase, WAIT_NS));
+            if (!ok) break;
+            ser_pending = false;
+            ser_phase ^= 1u;
+            tc_fence_after();
+            float o[32];
+            if (ts < 64) {
+                const int t = ts;
+#pragma unroll
+                for (int q = 0; q < 2; ++q) {
+                    tmem_load32(tm_out + lane_base + 32 * q, o);
+                    if (t < nv) {
+                        __nv_bfloat16* dst = y + (row0 + t) * tstride + hoff + 32 * q;
+#pragma unroll
+                        for (int i = 0; i < 32; i += 8)
+                            *reinterpret_cast<uint4*>(dst + i) =
+                                make_uint4(pack_bf16x2(o[i], o[i + 1]), pack_bf16x2(o[i + 2], o[i + 3]),
+                                           pack_bf16x2(o[i + 4], o[i + 5]), pack_bf16x2(o[i + 6], o[i + 7]));
+                    }
+                }
+            } else {
+                const float GL = gam_all[g * 128 + (kk_ & 1) * 64 + x];
+#pragma unroll
+                for (int q = 0; q < 2; ++q) {
+                    tmem_load32(tm_out + lane_base + 32 * q, o);
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) S[32 * q + i] = fmaf(GL, S[32 * q + i], o[i]);
+                }
+                st_op_row32<false>(St, 64, x, 0, S);
+                st_op_row32<false>(St, 64, x, 32, S + 32);
+            }
+            fence_proxy_async_smem();
+            tc_fence_before();
+            group_sync(bar_id, GROUP);
+            if (ts == 0) mbar_arrive(bars.free_);
+        }
+        if (!ok) {
+            if (ts == 0) report_status(status, WKV7_ERR_DEVICE_TIMEOUT);
+            if (ser_pending) mbar_wait(bars.ser, ser_phase, WAIT_NS);
+        } else if (sT && ts >= 64) {
+#pragma unroll
+            for (int i = 0; i < 64; ++i) sT[sbase + i * kHead + x] = S[i];
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem, TMEM_COLS);
+    }
+}
+
+template <typename WT>
+cudaError_t launch_pipe_typed(const PrefillArgs& p, cudaStream_t stream) {
+    auto kern = wkv7_prefill_pipe_kernel<WT>;
+    static unsigned long long configured = 0;
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    const unsigned long long bit = 1ull << (dev & 63);
+    if (!(configured & bit)) {
+        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+        if (e != cudaSuccess) return e;
+        configured |= bit;
+    }
+    const long units = static_cast<long>(p.B) * p.H;
+    kern<<<static_cast<unsigned>(units), NTHR, SMEM_BYTES, stream>>>(
+        static_cast<const __nv_bfloat16*>(p.r), static_cast<const WT*>(p.w_log),
+        static_cast<const __nv_bfloat16*>(p.k), static_cast<const __nv_bfloat16*>(p.v),
+        static_cast<const __nv_bfloat16*>(p.a), static_cast<const __nv_bfloat16*>(p.b), p.s0,
+        static_cast<__nv_bfloat16*>(p.y), p.sT, p.T, p.H, p.seq_offsets, p.status);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_prefill_pipe(const PrefillArgs& p, int w_dtype, cudaStream_t stream) {
+    return w_dtype == WKV7_BF16 ? launch_pipe_typed<__nv_bfloat16>(p, stream) : launch_pipe_typed<float>(p, stream);
+}
+
+}  // namespace wkv7
