@@ -186,40 +186,47 @@ __global__ void __launch_bounds__(NTHR, 1)
         bool mma_pending = false;
         int issued_out = 0;  // OUT-pre commits issued by this group
 
+        // p1 work split: thread (jp, tq) owns key channels 2jp, 2jp+1 of tokens
+        // 16tq .. 16tq+15.  Global loads come in two batches (decay logits with the
+        // first 8 tokens, then the last 8), each issued before any shared-memory store.
+        const int jp = tg & 31, tq = tg >> 5, j0 = 2 * jp;
+        float2 cw[16];
+        uint32_t rr[8], kv[8], av[8], bv[8], vv[8];
+        auto load_batch = [&](long row0b, int nvb, int e0) {
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                const int t = 16 * tq + e0 + e;
+                if (t < nvb) {
+                    const long off = (row0b + t) * tstride + hoff + j0;
+                    rr[e] = load_u32(r + off);
+                    kv[e] = load_u32(k + off);
+                    av[e] = load_u32(a + off);
+                    bv[e] = load_u32(b + off);
+                    vv[e] = load_u32(v + off);
+                } else {
+                    rr[e] = kv[e] = av[e] = bv[e] = vv[e] = 0u;
+                }
+            }
+        };
+        auto load_head = [&](int cc) {  // decay logits + first 8 tokens of chunk cc
+            const long row0b = tb + static_cast<long>(cc) * L;
+            const int nvb = static_cast<int>(len - static_cast<long>(cc) * L < L ? len - static_cast<long>(cc) * L : L);
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {
+                const int t = 16 * tq + e;
+                cw[e] = (t < nvb) ? load_pair<WT>(wl + (row0b + t) * tstride + hoff + j0)
+                                  : make_float2(-INFINITY, -INFINITY);
+            }
+            load_batch(row0b, nvb, 0);
+        };
+
         for (int c = g; c < nchunks; c += 2) {
             const int kk_ = c >> 1;
             const long row0 = tb + static_cast<long>(c) * L;
             const int nv = static_cast<int>(len - static_cast<long>(c) * L < L ? len - static_cast<long>(c) * L : L);
 
-            // ---- p1: decay products and the scaled operand tiles.  Thread (jp, tq):
-            // key channels 2jp, 2jp+1 of tokens 16tq .. 16tq+15.  Global loads come
-            // in two batches (decay logits with the first 8 tokens, then the last 8),
-            // each issued before any shared-memory store.
-            const int jp = tg & 31, tq = tg >> 5, j0 = 2 * jp;
-            float2 cw[16];
-            uint32_t rr[8], kv[8], av[8], bv[8], vv[8];
-            auto load_batch = [&](int e0) {
-#pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    const int t = 16 * tq + e0 + e;
-                    if (t < nv) {
-                        const long off = (row0 + t) * tstride + hoff + j0;
-                        rr[e] = load_u32(r + off);
-                        kv[e] = load_u32(k + off);
-                        av[e] = load_u32(a + off);
-                        bv[e] = load_u32(b + off);
-                        vv[e] = load_u32(v + off);
-                    } else {
-                        rr[e] = kv[e] = av[e] = bv[e] = vv[e] = 0u;
-                    }
-                }
-            };
-#pragma unroll
-            for (int e = 0; e < 16; ++e) {
-                const int t = 16 * tq + e;
-                cw[e] = (t < nv) ? load_pair<WT>(wl + (row0 + t) * tstride + hoff + j0) : make_float2(-INFINITY, -INFINITY);
-            }
-            load_batch(0);
+            // ---- p1: decay products and the scaled operand tiles
+            load_head(c);
             float p0 = 1.f, p1 = 1.f;
 #pragma unroll
             for (int e = 0; e < 16; ++e) {
@@ -250,13 +257,13 @@ __global__ void __launch_bounds__(NTHR, 1)
             const uint32_t cb = static_cast<uint32_t>(j0) * 2u;
 #pragma unroll
             for (int half = 0; half < 2; ++half) {
-                if (half == 1) load_batch(8);
+                if (half == 1) load_batch(row0, nv, 8);
                 uint32_t bh0[4], bh1[4], kh0[4], kh1[4];  // 8 tokens of Bh^T / Kh^T rows j0, j0+1
 #pragma unroll
                 for (int e = 0; e < 8; ++e) {
                     const int t = 16 * tq + 8 * half + e;
                     const float G0 = pre0 * cw[8 * half + e].x, G1 = pre1 * cw[8 * half + e].y;
-                    const float i0 = __frcp_rn(G0), i1 = __frcp_rn(G1);
+                    const float i0 = __fdividef(1.f, G0), i1 = __fdividef(1.f, G1);
                     const float l0 = i0 * GL0, l1 = i1 * GL1;
                     const float2 rf = unpack_bf16x2(rr[e]), kf = unpack_bf16x2(kv[e]);
                     const float2 af = unpack_bf16x2(av[e]), bf = unpack_bf16x2(bv[e]);
