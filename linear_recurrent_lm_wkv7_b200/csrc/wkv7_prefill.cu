@@ -44,6 +44,7 @@
 #include <cstring>
 
 #include "prefill_common.cuh"
+#include "tma_host.cuh"
 #include "sm100_ptx.cuh"
 #include "wkv7_internal.cuh"
 
@@ -79,11 +80,6 @@ struct Smem {
     uint32_t* tmem_slot;
 };
 
-// TMA descriptors of the token-major inputs, each viewed as [tokens][H][64]
-// with a box of 64 tokens x 1 head x 64 channels.
-struct TmaMaps {
-    CUtensorMap r, k, a, b, wl, v;
-};
 
 // Bytes of the raw staging area (bf16 inputs): r, k, a, b tiles + the w_log tile.
 template <bool TF32, uint32_t WB>
@@ -568,52 +564,14 @@ __global__ void __launch_bounds__(NT, 1)
     }
 }
 
-using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
-                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
-                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn encode_fn() {
-    static EncodeTiledFn fn = nullptr;
-    if (!fn) {
-        void* f = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<EncodeTiledFn>(f);
-    }
-    return fn;
-}
-
-// [ntok][H][64] tensor of `esize`-byte elements, box 64 x 1 x 64.
-bool make_token_map(CUtensorMap* m, const void* base, CUtensorMapDataType dt, uint64_t esize, uint64_t H,
-                    uint64_t ntok, CUtensorMapSwizzle sw) {
-    EncodeTiledFn fn = encode_fn();
-    if (!fn) return false;
-    const cuuint64_t dims[3] = {64, H, ntok};
-    const cuuint64_t strides[2] = {64 * esize, H * 64 * esize};
-    const cuuint32_t box[3] = {64, 1, 64};
-    const cuuint32_t estr[3] = {1, 1, 1};
-    return fn(m, dt, 3, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
-              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 template <typename IO, typename WT, bool TF32>
 cudaError_t launch_typed(const PrefillArgs& p, cudaStream_t stream) {
     constexpr uint32_t smem = smem_bytes_needed<TF32, sizeof(WT)>();
-    TmaMaps maps;
+    TmaMaps maps;  // unused by the fp32 path
     memset(&maps, 0, sizeof(maps));
     if constexpr (!TF32) {
         const uint64_t ntok = p.seq_offsets ? static_cast<uint64_t>(p.T) : static_cast<uint64_t>(p.B) * p.T;
-        const CUtensorMapDataType bf = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
-        const CUtensorMapDataType wdt =
-            sizeof(WT) == 4 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
-        const CUtensorMapSwizzle none = CU_TENSOR_MAP_SWIZZLE_NONE;
-        if (!make_token_map(&maps.r, p.r, bf, 2, p.H, ntok, none) ||
-            !make_token_map(&maps.k, p.k, bf, 2, p.H, ntok, none) ||
-            !make_token_map(&maps.a, p.a, bf, 2, p.H, ntok, none) ||
-            !make_token_map(&maps.b, p.b, bf, 2, p.H, ntok, none) ||
-            !make_token_map(&maps.wl, p.w_log, wdt, sizeof(WT), p.H, ntok, none) ||
-            !make_token_map(&maps.v, p.v, bf, 2, p.H, ntok, CU_TENSOR_MAP_SWIZZLE_128B))
+        if (!make_prefill_maps(&maps, p.r, p.w_log, p.k, p.v, p.a, p.b, p.H, ntok, sizeof(WT)))
             return cudaErrorInvalidValue;
     }
     auto kern = wkv7_prefill_kernel<IO, WT, TF32>;

@@ -28,11 +28,17 @@
 // Synchronisation: a prep group hands a chunk to the serial group through
 // `ready[g]` (MMA commit + release arrive); the serial group releases the
 // shared tile (and the group's OUT columns) through `free_` after each chunk.
-// All waits are bounded.
+// Inputs arrive by TMA into tiles of the group that are dead at that point of
+// the previous chunk: w_log of chunk c + 2 into BK once T is built, r and k into
+// NQ once P has consumed Q, a and b into RAM once the conversion has read Rt; V
+// goes straight into the group's MN-major V tile once the previous OUT product
+// has read it.  Waits are polled by one thread while the others sleep on the
+// group's named barrier; every wait is bounded.
 #include <cstring>
 
 #include "prefill_common.cuh"
 #include "sm100_ptx.cuh"
+#include "tma_host.cuh"
 #include "wkv7_internal.cuh"
 
 namespace wkv7 {
@@ -56,7 +62,9 @@ constexpr uint32_t OFF_S = OFF_AS + 16384;            // S^T bf16, 8 KB (serial 
 constexpr uint32_t OFF_GAMMA = OFF_S + 8192;          // Gamma_L [2 groups][2 slots][64] fp32
 constexpr uint32_t OFF_RED = OFF_GAMMA + 2 * 2 * 64 * 4;  // block products [2 groups][4][64] fp32
 constexpr uint32_t OFF_BAR = OFF_RED + 2 * 4 * 64 * 4;
-constexpr uint32_t SMEM_USED = OFF_BAR + 8 * 8 + 16;
+constexpr uint32_t SMEM_USED = OFF_BAR + 14 * 8 + 16;
+// raw TMA staging inside a group's tiles (dead at the time of the load)
+constexpr uint32_t RAW_R = OFF_NQ, RAW_K = OFF_NQ + 8192, RAW_A = OFF_RAM, RAW_B = OFF_RAM + 8192, RAW_L = OFF_BK;
 constexpr uint32_t SMEM_BYTES = SMEM_USED + 1024;      // alignment slack
 
 // TMEM columns
@@ -76,25 +84,15 @@ __device__ __forceinline__ uint32_t tf_idx(uint32_t row, uint32_t col) {
 
 __device__ __forceinline__ float2 unpack_bf16x2(uint32_t u) { return make_float2(bf16lo_to_f32(u), bf16hi_to_f32(u)); }
 
-template <typename WT>
-__device__ __forceinline__ float2 load_pair(const WT* p);
-template <>
-__device__ __forceinline__ float2 load_pair<float>(const float* p) {
-    return __ldg(reinterpret_cast<const float2*>(p));
-}
-template <>
-__device__ __forceinline__ float2 load_pair<__nv_bfloat16>(const __nv_bfloat16* p) {
-    return unpack_bf16x2(__ldg(reinterpret_cast<const unsigned int*>(p)));
-}
-__device__ __forceinline__ uint32_t load_u32(const __nv_bfloat16* p) {
-    return __ldg(reinterpret_cast<const unsigned int*>(p));
-}
-
 struct Bars {
     uint64_t* mma;    // [2] prep-group MMA completions (G, Q, P)
     uint64_t* ready;  // [2] OUT-pre complete and chunk tiles published (count 2)
     uint64_t* free_;  // serial group done with a chunk (shared tile and OUT columns reusable)
     uint64_t* ser;    // serial MMA completion
+    uint64_t* rl;     // [2] TMA of a group's raw w_log tile
+    uint64_t* rrk;    // [2] TMA of a group's raw r, k tiles
+    uint64_t* rab;    // [2] TMA of a group's raw a, b tiles
+    uint64_t* vld;    // [2] TMA of a group's V tile
     uint32_t* tmem_slot;
 };
 
@@ -104,7 +102,8 @@ __global__ void __launch_bounds__(NTHR, 1)
                              const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restrict__ v,
                              const __nv_bfloat16* __restrict__ a, const __nv_bfloat16* __restrict__ b,
                              const float* s0, __nv_bfloat16* __restrict__ y, float* sT, int T, int H,
-                             const int32_t* __restrict__ seq_offsets, int* status) {
+                             const int32_t* __restrict__ seq_offsets, int* status,
+                             const __grid_constant__ TmaMaps maps) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023u) & ~uintptr_t(1023));
     const int tid = threadIdx.x;
@@ -114,9 +113,13 @@ __global__ void __launch_bounds__(NTHR, 1)
         uint64_t* p = reinterpret_cast<uint64_t*>(sm + OFF_BAR);
         bars.mma = p;
         bars.ready = p + 2;
-        bars.free_ = p + 4;
-        bars.ser = p + 6;
-        bars.tmem_slot = reinterpret_cast<uint32_t*>(p + 8);
+        bars.free_ = p + 4;  // one barrier
+        bars.ser = p + 5;
+        bars.rl = p + 6;
+        bars.rrk = p + 8;
+        bars.rab = p + 10;
+        bars.vld = p + 12;
+        bars.tmem_slot = reinterpret_cast<uint32_t*>(p + 14);
     }
 
     // ---- the unit and its tokens
@@ -144,6 +147,10 @@ __global__ void __launch_bounds__(NTHR, 1)
         for (int g = 0; g < 2; ++g) {
             mbar_init(&bars.mma[g], 1);
             mbar_init(&bars.ready[g], 2);
+            mbar_init(&bars.rl[g], 1);
+            mbar_init(&bars.rrk[g], 1);
+            mbar_init(&bars.rab[g], 1);
+            mbar_init(&bars.vld[g], 1);
         }
         mbar_init(bars.free_, 1);
         mbar_init(bars.ser, 1);
@@ -185,48 +192,78 @@ __global__ void __launch_bounds__(NTHR, 1)
         uint32_t mma_phase = 0;
         bool mma_pending = false;
         int issued_out = 0;  // OUT-pre commits issued by this group
+        int raw_issued = 0, raw_done = 0, v_issued = 0, v_done = 0;  // TMA loads (chunks) of this group
+        constexpr uint32_t WB = sizeof(WT);
+        // one thread each; `which`: 0 = w_log, 1 = r and k, 2 = a and b
+        auto issue_raw = [&](int cc, int which) {
+            const int t0 = static_cast<int>(tb + static_cast<long>(cc) * L);
+            if (which == 0) {
+                mbar_arrive_expect_tx(&bars.rl[g], 4096u * WB);
+                tma_load_3d(gt + RAW_L, &maps.wl, &bars.rl[g], 0, h, t0);
+            } else if (which == 1) {
+                mbar_arrive_expect_tx(&bars.rrk[g], 2u * 8192u);
+                tma_load_3d(gt + RAW_R, &maps.r, &bars.rrk[g], 0, h, t0);
+                tma_load_3d(gt + RAW_K, &maps.k, &bars.rrk[g], 0, h, t0);
+            } else {
+                mbar_arrive_expect_tx(&bars.rab[g], 2u * 8192u);
+                tma_load_3d(gt + RAW_A, &maps.a, &bars.rab[g], 0, h, t0);
+                tma_load_3d(gt + RAW_B, &maps.b, &bars.rab[g], 0, h, t0);
+            }
+        };
+        auto issue_v = [&](int cc) {  // one thread
+            mbar_arrive_expect_tx(&bars.vld[g], 8192u);
+            tma_load_3d(Vt, &maps.v, &bars.vld[g], 0, h, static_cast<int>(tb + static_cast<long>(cc) * L));
+        };
+        if (g < nchunks) {
+            if (tg == 0) {
+                issue_raw(g, 0);
+                issue_raw(g, 1);
+                issue_raw(g, 2);
+                issue_v(g);
+            }
+            raw_issued = v_issued = 1;
+        }
 
-        // p1 work split: thread (jp, tq) owns key channels 2jp, 2jp+1 of tokens
-        // 16tq .. 16tq+15.  Global loads come in two batches (decay logits with the
-        // first 8 tokens, then the last 8), each issued before any shared-memory store.
+        // p1 work split: thread (jp, tq) owns key channels 2jp, 2jp+1 of tokens 16tq .. 16tq+15
         const int jp = tg & 31, tq = tg >> 5, j0 = 2 * jp;
-        float2 cw[16];
-        uint32_t rr[8], kv[8], av[8], bv[8], vv[8];
-        auto load_batch = [&](long row0b, int nvb, int e0) {
-#pragma unroll
-            for (int e = 0; e < 8; ++e) {
-                const int t = 16 * tq + e0 + e;
-                if (t < nvb) {
-                    const long off = (row0b + t) * tstride + hoff + j0;
-                    rr[e] = load_u32(r + off);
-                    kv[e] = load_u32(k + off);
-                    av[e] = load_u32(a + off);
-                    bv[e] = load_u32(b + off);
-                    vv[e] = load_u32(v + off);
-                } else {
-                    rr[e] = kv[e] = av[e] = bv[e] = vv[e] = 0u;
-                }
-            }
-        };
-        auto load_head = [&](int cc) {  // decay logits + first 8 tokens of chunk cc
-            const long row0b = tb + static_cast<long>(cc) * L;
-            const int nvb = static_cast<int>(len - static_cast<long>(cc) * L < L ? len - static_cast<long>(cc) * L : L);
-#pragma unroll
-            for (int e = 0; e < 16; ++e) {
-                const int t = 16 * tq + e;
-                cw[e] = (t < nvb) ? load_pair<WT>(wl + (row0b + t) * tstride + hoff + j0)
-                                  : make_float2(-INFINITY, -INFINITY);
-            }
-            load_batch(row0b, nvb, 0);
-        };
+        const WT* rawl = reinterpret_cast<const WT*>(gt + RAW_L);
+        const uint32_t* rawr = reinterpret_cast<const uint32_t*>(gt + RAW_R);
+        const uint32_t* rawk = reinterpret_cast<const uint32_t*>(gt + RAW_K);
+        const uint32_t* rawa = reinterpret_cast<const uint32_t*>(gt + RAW_A);
+        const uint32_t* rawb = reinterpret_cast<const uint32_t*>(gt + RAW_B);
 
         for (int c = g; c < nchunks; c += 2) {
             const int kk_ = c >> 1;
-            const long row0 = tb + static_cast<long>(c) * L;
             const int nv = static_cast<int>(len - static_cast<long>(c) * L < L ? len - static_cast<long>(c) * L : L);
 
             // ---- p1: decay products and the scaled operand tiles
-            load_head(c);
+            {
+                // the previous OUT product of this group (chunk c-2) must have read V, BH and MK
+                bool w_ok = true;
+                if (kk_ >= 1 && tg == 0) {
+                    w_ok = mbar_wait(&bars.ready[g], static_cast<uint32_t>(kk_ - 1) & 1u, WAIT_NS);
+                    if (w_ok) issue_v(c);
+                }
+                if (kk_ >= 1) ++v_issued;
+                if (tg == 0) w_ok = w_ok && mbar_wait(&bars.rl[g], static_cast<uint32_t>(kk_) & 1u, WAIT_NS);
+                ok = group_sync_and(bar_id, GROUP, w_ok);
+                if (!ok) break;
+            }
+            float2 cw[16];
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {
+                const int t = 16 * tq + e;
+                if (t < nv) {
+                    if constexpr (sizeof(WT) == 4) {
+                        cw[e] = *reinterpret_cast<const float2*>(rawl + t * 64 + j0);
+                    } else {
+                        const uint32_t u = *reinterpret_cast<const uint32_t*>(rawl + t * 64 + j0);
+                        cw[e] = make_float2(bf16lo_to_f32(u), bf16hi_to_f32(u));
+                    }
+                } else {
+                    cw[e] = make_float2(-INFINITY, -INFINITY);
+                }
+            }
             float p0 = 1.f, p1 = 1.f;
 #pragma unroll
             for (int e = 0; e < 16; ++e) {
@@ -234,13 +271,18 @@ __global__ void __launch_bounds__(NTHR, 1)
                 p1 *= __expf(-__expf(cw[e].y));
                 cw[e] = make_float2(p0, p1);  // cumulative product inside the 16-token block
             }
-            // the previous reads of this group's V, BH and MK tiles (OUT of chunk c-2) must be complete
-            bool w_ok = true;
-            if (kk_ >= 1 && tg == 0) w_ok = mbar_wait(&bars.ready[g], static_cast<uint32_t>(kk_ - 1) & 1u, WAIT_NS);
             red[tq * 64 + j0] = p0;
             red[tq * 64 + j0 + 1] = p1;
-            ok = group_sync_and(bar_id, GROUP, w_ok);
-            if (!ok) break;
+            {
+                // every raw w_log read is done once all threads pass this barrier (BK is rewritten below)
+                bool w_ok = true;
+                if (tg == 0)
+                    w_ok = mbar_wait(&bars.rrk[g], static_cast<uint32_t>(kk_) & 1u, WAIT_NS) &&
+                           mbar_wait(&bars.rab[g], static_cast<uint32_t>(kk_) & 1u, WAIT_NS);
+                ok = group_sync_and(bar_id, GROUP, w_ok);
+                if (!ok) break;
+                ++raw_done;
+            }
             float pre0 = 1.f, pre1 = 1.f, GL0 = 1.f, GL1 = 1.f;
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
@@ -255,9 +297,20 @@ __global__ void __launch_bounds__(NTHR, 1)
             }
             float gp0 = pre0, gp1 = pre1;
             const uint32_t cb = static_cast<uint32_t>(j0) * 2u;
+            uint32_t rr[8], kv[8], av[8], bv[8];
 #pragma unroll
             for (int half = 0; half < 2; ++half) {
-                if (half == 1) load_batch(row0, nv, 8);
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    const int t = 16 * tq + 8 * half + e;
+                    const int idx = t * 32 + jp;  // 32-bit word of (t, j0)
+                    const bool in = t < nv;
+                    rr[e] = in ? rawr[idx] : 0u;
+                    kv[e] = in ? rawk[idx] : 0u;
+                    av[e] = in ? rawa[idx] : 0u;
+                    bv[e] = in ? rawb[idx] : 0u;
+                }
+                __syncwarp();  // this warp's raw rows are read before its tiles overwrite them
                 uint32_t bh0[4], bh1[4], kh0[4], kh1[4];  // 8 tokens of Bh^T / Kh^T rows j0, j0+1
 #pragma unroll
                 for (int e = 0; e < 8; ++e) {
@@ -271,7 +324,6 @@ __global__ void __launch_bounds__(NTHR, 1)
                     *reinterpret_cast<uint32_t*>(RAM + swz(64 + t, cb, 128)) = pack_bf16x2(af.x * gp0, af.y * gp1);
                     *reinterpret_cast<uint32_t*>(BK + swz(t, cb, 128)) = pack_bf16x2(bf.x * i0, bf.y * i1);
                     *reinterpret_cast<uint32_t*>(BK + swz(64 + t, cb, 128)) = pack_bf16x2(kf.x * i0, kf.y * i1);
-                    *reinterpret_cast<uint32_t*>(Vt + swz(t, cb, 64)) = vv[e];
                     const float b0 = bf.x * l0, b1 = bf.y * l1, k0 = kf.x * l0, k1 = kf.y * l1;
                     if ((e & 1) == 0) {
                         bh0[e >> 1] = __float_as_uint(b0);
@@ -306,7 +358,7 @@ __global__ void __launch_bounds__(NTHR, 1)
                 mma_commit(&bars.mma[g]);
             }
             mma_pending = true;
-            ok = group_sync_and(bar_id, GROUP, mbar_wait(&bars.mma[g], mma_phase, WAIT_NS));
+            ok = group_sync_and(bar_id, GROUP, tg == 0 ? mbar_wait(&bars.mma[g], mma_phase, WAIT_NS) : true);
             if (!ok) break;
             mma_pending = false;
             mma_phase ^= 1u;
@@ -357,9 +409,15 @@ __global__ void __launch_bounds__(NTHR, 1)
 #pragma unroll
                 for (int t = 0; t < 31; ++t) {
                     const float xt = acc[t];
-                    const float* nrow = Nt + (blk + t) * 64 + blk;  // column blk+t of Nab
+                    const float4* nrow = reinterpret_cast<const float4*>(Nt + (blk + t) * 64 + blk);  // column blk+t of Nab
 #pragma unroll
-                    for (int i = t + 1; i < 32; ++i) acc[i] = fmaf(nrow[i], xt, acc[i]);
+                    for (int q4 = (t + 1) >> 2; q4 < 8; ++q4) {
+                        const float4 n4 = nrow[q4];
+                        if (4 * q4 + 0 > t) acc[4 * q4 + 0] = fmaf(n4.x, xt, acc[4 * q4 + 0]);
+                        if (4 * q4 + 1 > t) acc[4 * q4 + 1] = fmaf(n4.y, xt, acc[4 * q4 + 1]);
+                        if (4 * q4 + 2 > t) acc[4 * q4 + 2] = fmaf(n4.z, xt, acc[4 * q4 + 2]);
+                        if (4 * q4 + 3 > t) acc[4 * q4 + 3] = fmaf(n4.w, xt, acc[4 * q4 + 3]);
+                    }
                 }
 #pragma unroll
                 for (int i = 0; i < 32; ++i) Tf[tf_idx(blk + i, blk + col)] = acc[i];
@@ -418,6 +476,11 @@ __global__ void __launch_bounds__(NTHR, 1)
             }
             fence_proxy_async_smem();
             group_sync(bar_id, GROUP);
+            // BK (the fp32 T) is dead: load the w_log tile of this group's next chunk
+            if (c + 2 < nchunks) {
+                if (tg == 0) issue_raw(c + 2, 0);
+                ++raw_issued;  // counted at the first of the chunk's three raw loads
+            }
 
             // ---- Q = [Mrb; Bh^T] T
             if (tg == 0) {
@@ -428,7 +491,7 @@ __global__ void __launch_bounds__(NTHR, 1)
                 mma_commit(&bars.mma[g]);
             }
             mma_pending = true;
-            ok = group_sync_and(bar_id, GROUP, mbar_wait(&bars.mma[g], mma_phase, WAIT_NS));
+            ok = group_sync_and(bar_id, GROUP, tg == 0 ? mbar_wait(&bars.mma[g], mma_phase, WAIT_NS) : true);
             if (!ok) break;
             mma_pending = false;
             mma_phase ^= 1u;
@@ -458,14 +521,19 @@ __global__ void __launch_bounds__(NTHR, 1)
             // the serial group is done with chunk c-1
             mma_pending = true;
             {
-                bool w1 = mbar_wait(&bars.mma[g], mma_phase, WAIT_NS);
-                if (c >= 1) w1 = w1 && mbar_wait(bars.free_, static_cast<uint32_t>(c - 1) & 1u, WAIT_NS);
+                bool w1 = true;
+                if (tg == 0) {
+                    w1 = mbar_wait(&bars.mma[g], mma_phase, WAIT_NS);
+                    if (c >= 1) w1 = w1 && mbar_wait(bars.free_, static_cast<uint32_t>(c - 1) & 1u, WAIT_NS);
+                }
                 ok = group_sync_and(bar_id, GROUP, w1);
             }
             if (!ok) break;
             mma_pending = false;
             mma_phase ^= 1u;
             tc_fence_after();
+            // NQ (Q) has been consumed by P: load r and k of this group's next chunk
+            if (c + 2 < nchunks && tg == 0) issue_raw(c + 2, 1);
             {
                 float x[32];
                 const int row = tg;  // lanes 0..63: token rows (R' = Rt + Mrb W, Mrb Z); 64..127: key rows
@@ -490,7 +558,15 @@ __global__ void __launch_bounds__(NTHR, 1)
             tc_fence_before();
             group_sync(bar_id, GROUP);
 
+            // RAM (Rt, At, Mak) is dead: load a and b of this group's next chunk
+            if (c + 2 < nchunks && tg == 0) issue_raw(c + 2, 2);
             // ---- OUT = [Mrb Z; Bh^T Z] V + [Mrk; Kh^T] V   (the serial group adds [R'; Bh^T W] S0^T)
+            {
+                const bool vok = (tg == 0) ? mbar_wait(&bars.vld[g], static_cast<uint32_t>(kk_) & 1u, WAIT_NS) : true;
+                ok = group_sync_and(bar_id, GROUP, vok);
+                if (!ok) break;
+                ++v_done;
+            }
             if (tg == 0) {
                 tc_fence_after();
 #pragma unroll
@@ -506,8 +582,17 @@ __global__ void __launch_bounds__(NTHR, 1)
         }
         if (!ok && tg == 0) report_status(status, WKV7_ERR_DEVICE_TIMEOUT);
         // drain: an unwaited G/Q/P product, and the last OUT-pre product
-        if (mma_pending) mbar_wait(&bars.mma[g], mma_phase, WAIT_NS);
-        if (issued_out > 0) mbar_wait(&bars.ready[g], static_cast<uint32_t>(issued_out - 1) & 1u, WAIT_NS);
+        if (tg == 0) {
+            if (mma_pending) mbar_wait(&bars.mma[g], mma_phase, WAIT_NS);
+            if (issued_out > 0) mbar_wait(&bars.ready[g], static_cast<uint32_t>(issued_out - 1) & 1u, WAIT_NS);
+            // a chunk's raw loads are issued in three batches; wait for every one that may be in flight
+            for (int i = raw_done; i < raw_issued; ++i) {
+                mbar_wait(&bars.rl[g], static_cast<uint32_t>(i) & 1u, WAIT_NS);
+                mbar_wait(&bars.rrk[g], static_cast<uint32_t>(i) & 1u, WAIT_NS);
+                mbar_wait(&bars.rab[g], static_cast<uint32_t>(i) & 1u, WAIT_NS);
+            }
+            for (int i = v_done; i < v_issued; ++i) mbar_wait(&bars.vld[g], static_cast<uint32_t>(i) & 1u, WAIT_NS);
+        }
     } else {
         // =========================================================== serial group
         const int ts = tid - 256;
@@ -532,26 +617,8 @@ __global__ void __launch_bounds__(NTHR, 1)
             const int nv = static_cast<int>(len - static_cast<long>(c) * L < L ? len - static_cast<long>(c) * L : L);
             const uint32_t tm_out = tmem + 256u * g + TM_OUT;
             uint8_t* AS = sm + OFF_AS;
-            if (c + 2 < nchunks) {
-                // L2 line hints for the rows a prep group will load two chunks ahead
-                const long rows2 = row0 + 2 * L;
-                const int nv2 = static_cast<int>(len - static_cast<long>(c + 2) * L < L ? len - static_cast<long>(c + 2) * L : L);
-                const int row = ts & 63;
-                if (row < nv2) {
-                    const long off = (rows2 + row) * tstride + hoff;
-                    if (ts < 64) {
-                        prefetch_line_l2(r + off);
-                        prefetch_line_l2(k + off);
-                        prefetch_line_l2(a + off);
-                        prefetch_line_l2(wl + off);
-                    } else {
-                        prefetch_line_l2(b + off);
-                        prefetch_line_l2(v + off);
-                        prefetch_line_l2(wl + off + 32);
-                    }
-                }
-            }
-            ok = group_sync_and(bar_id, GROUP, mbar_wait(&bars.ready[g], static_cast<uint32_t>(kk_) & 1u, WAIT_NS));
+            ok = group_sync_and(bar_id, GROUP,
+                                ts == 0 ? mbar_wait(&bars.ready[g], static_cast<uint32_t>(kk_) & 1u, WAIT_NS) : true);
             if (!ok) break;
             tc_fence_after();
             if (ts == 0) {
@@ -561,7 +628,7 @@ __global__ void __launch_bounds__(NTHR, 1)
                 mma_commit(bars.ser);
             }
             ser_pending = true;
-            ok = group_sync_and(bar_id, GROUP, mbar_wait(bars.ser, ser_phase, WAIT_NS));
+            ok = group_sync_and(bar_id, GROUP, ts == 0 ? mbar_wait(bars.ser, ser_phase, WAIT_NS) : true);
             if (!ok) break;
             ser_pending = false;
             ser_phase ^= 1u;
@@ -599,7 +666,7 @@ __global__ void __launch_bounds__(NTHR, 1)
         }
         if (!ok) {
             if (ts == 0) report_status(status, WKV7_ERR_DEVICE_TIMEOUT);
-            if (ser_pending) mbar_wait(bars.ser, ser_phase, WAIT_NS);
+            if (ser_pending && ts == 0) mbar_wait(bars.ser, ser_phase, WAIT_NS);
         } else if (sT && ts >= 64) {
 #pragma unroll
             for (int i = 0; i < 64; ++i) sT[sbase + i * kHead + x] = S[i];
@@ -627,12 +694,15 @@ cudaError_t launch_pipe_typed(const PrefillArgs& p, cudaStream_t stream) {
         if (e != cudaSuccess) return e;
         configured |= bit;
     }
+    TmaMaps maps;
+    const uint64_t ntok = p.seq_offsets ? static_cast<uint64_t>(p.T) : static_cast<uint64_t>(p.B) * p.T;
+    if (!make_prefill_maps(&maps, p.r, p.w_log, p.k, p.v, p.a, p.b, p.H, ntok, sizeof(WT))) return cudaErrorInvalidValue;
     const long units = static_cast<long>(p.B) * p.H;
     kern<<<static_cast<unsigned>(units), NTHR, SMEM_BYTES, stream>>>(
         static_cast<const __nv_bfloat16*>(p.r), static_cast<const WT*>(p.w_log),
         static_cast<const __nv_bfloat16*>(p.k), static_cast<const __nv_bfloat16*>(p.v),
         static_cast<const __nv_bfloat16*>(p.a), static_cast<const __nv_bfloat16*>(p.b), p.s0,
-        static_cast<__nv_bfloat16*>(p.y), p.sT, p.T, p.H, p.seq_offsets, p.status);
+        static_cast<__nv_bfloat16*>(p.y), p.sT, p.T, p.H, p.seq_offsets, p.status, maps);
     return cudaGetLastError();
 }
 
