@@ -7,8 +7,9 @@
 //   Y     = (Rt + Mrb W) S0^T + (Mrk + Mrb Z) V
 //   S_L^T = Gamma_L (.) S0^T  + (Bh^T W) S0^T + (Kh^T + Bh^T Z) V
 // with [W | Z] = T [At | Mak] and T = (I - Nab)^{-1}.  T is formed explicitly
-// in fp32 on the CUDA cores (32 x 32 diagonal blocks by substitution, the
-// off-diagonal block as T_hi Nab_hl T_lo) and folded into tensor-core products:
+// in fp32 (16 x 16 diagonal blocks by substitution on the CUDA cores, the
+// blocks below them by warp-level tf32 tensor-core products) and folded into
+// tcgen05 products:
 //   G   = [Rt; At] [Bt; Kt]^T                        (Mrb | Mrk over Nab | Mak)
 //   Q   = [Mrb; Bh^T] T
 //   P   = Q [At | Mak]                               (Mrb W | Mrb Z over Bh^T W | Bh^T Z)
@@ -51,10 +52,10 @@ constexpr uint64_t WAIT_NS = 1000000000ull;  // 1 s
 
 // per prep-group shared-memory tiles (bytes)
 constexpr uint32_t OFF_RAM = 0;        // Rt (rows 0-63) | At (rows 64-127) | Mak (64 tokens x 64), 24 KB
-constexpr uint32_t OFF_BK = 24576;     // [Bt; Kt] 16 KB, then T fp32 (64 x 64, column-swizzled)
+constexpr uint32_t OFF_BK = 24576;     // raw w_log (16 KB), then T fp32 (64 x 64, tf_idx layout)
 constexpr uint32_t OFF_BH = 40960;     // [Mrb; Bh^T] 16 KB, then [Mrb Z; Bh^T Z]
 constexpr uint32_t OFF_MK = 57344;     // [Mrk; Kh^T] 16 KB, K-major over tokens
-constexpr uint32_t OFF_NQ = 73728;     // Nab^T fp32 16 KB, then X (32 x 32 fp32) + T bf16 at +8 KB, then Q bf16
+constexpr uint32_t OFF_NQ = 73728;     // raw r, k -> [Bt; Kt] 16 KB, then Nab fp32, then T bf16 at +8 KB, then Q bf16
 constexpr uint32_t OFF_V = 90112;      // V 8 KB (MN-major)
 constexpr uint32_t GROUP_TILES = 98304;
 constexpr uint32_t OFF_AS = 2 * GROUP_TILES;          // [R'; Bh^T W] 16 KB, shared by both groups
@@ -82,7 +83,45 @@ __device__ __forceinline__ uint32_t tf_idx(uint32_t row, uint32_t col) {
     return row * 64u + (col ^ ((row & 7u) << 2));
 }
 
+// Warp-level tf32 tensor-core product on fp32 matrices held in the tf_idx layout.
+// m16n8k8 fragments: lane = 4 gq + t4; A (16 x 8) holds rows gq, gq + 8 and
+// columns t4, t4 + 4; B (8 x 8) rows t4, t4 + 4 and column gq; C (16 x 8) rows
+// gq, gq + 8 and columns 2 t4, 2 t4 + 1.  Stored values are already tf32.
+__device__ __forceinline__ void frag_a_tf32(const float* M, int r0, int c0, int gq, int t4, uint32_t (&a)[4]) {
+    a[0] = __float_as_uint(M[tf_idx(r0 + gq, c0 + t4)]);
+    a[1] = __float_as_uint(M[tf_idx(r0 + gq + 8, c0 + t4)]);
+    a[2] = __float_as_uint(M[tf_idx(r0 + gq, c0 + t4 + 4)]);
+    a[3] = __float_as_uint(M[tf_idx(r0 + gq + 8, c0 + t4 + 4)]);
+}
+__device__ __forceinline__ void frag_b_tf32(const float* M, int k0, int n0, int gq, int t4, uint32_t (&b)[2]) {
+    b[0] = __float_as_uint(M[tf_idx(k0 + t4, n0 + gq)]);
+    b[1] = __float_as_uint(M[tf_idx(k0 + t4 + 4, n0 + gq)]);
+}
+__device__ __forceinline__ void frag_c_store_tf32(float* M, int r0, int n0, int gq, int t4, const float (&d)[4]) {
+    *reinterpret_cast<float2*>(M + tf_idx(r0 + gq, n0 + 2 * t4)) = make_float2(round_tf32(d[0]), round_tf32(d[1]));
+    *reinterpret_cast<float2*>(M + tf_idx(r0 + gq + 8, n0 + 2 * t4)) = make_float2(round_tf32(d[2]), round_tf32(d[3]));
+}
+__device__ __forceinline__ void mma_tf32_16x8x8(float (&d)[4], const uint32_t (&a)[4], const uint32_t (&b)[2]) {
+    asm("mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+        "{%0, %1, %2, %3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
+}
+
 __device__ __forceinline__ float2 unpack_bf16x2(uint32_t u) { return make_float2(bf16lo_to_f32(u), bf16hi_to_f32(u)); }
+
+// w_log of key channels j, j + 1 (element index i of the raw tile) as floats
+__device__ __forceinline__ float2 ld_wlog2(const float* p, int i) { return *reinterpret_cast<const float2*>(p + i); }
+__device__ __forceinline__ float2 ld_wlog2(const __nv_bfloat16* p, int i) {
+    const uint32_t u = *reinterpret_cast<const uint32_t*>(p + i);
+    return make_float2(bf16lo_to_f32(u), bf16hi_to_f32(u));
+}
+template <typename WT>
+__device__ __forceinline__ WT neg_inf_of();
+template <>
+__device__ __forceinline__ float neg_inf_of<float>() { return -INFINITY; }
+template <>
+__device__ __forceinline__ __nv_bfloat16 neg_inf_of<__nv_bfloat16>() { return __ushort_as_bfloat16(0xFF80u); }
 
 struct Bars {
     uint64_t* mma;    // [2] prep-group MMA completions (G, Q, P)
@@ -174,12 +213,10 @@ __global__ void __launch_bounds__(NTHR, 1)
         const uint32_t bar_id = 1 + g;
         uint8_t* gt = sm + g * GROUP_TILES;
         uint8_t* RAM = gt + OFF_RAM;
-        uint8_t* BK = gt + OFF_BK;
         uint8_t* BH = gt + OFF_BH;
         uint8_t* MK = gt + OFF_MK;
         float* Tf = reinterpret_cast<float*>(gt + OFF_BK);
-        float* Nt = reinterpret_cast<float*>(gt + OFF_NQ);
-        float* Xs = Nt;
+        float* Nr = reinterpret_cast<float*>(gt + OFF_NQ);
         uint8_t* Tb = gt + OFF_NQ + 8192;
         uint8_t* Qt = gt + OFF_NQ;
         uint8_t* AS = sm + OFF_AS;
@@ -227,6 +264,8 @@ __global__ void __launch_bounds__(NTHR, 1)
         // p1 work split: thread (jp, tq) owns key channels 2jp, 2jp+1 of tokens 16tq .. 16tq+15
         const int jp = tg & 31, tq = tg >> 5, j0 = 2 * jp;
         const WT* rawl = reinterpret_cast<const WT*>(gt + RAW_L);
+        WT* rawl_w = reinterpret_cast<WT*>(gt + RAW_L);
+        uint8_t* BKt = gt + OFF_NQ;  // [Bt; Kt], written over the raw r, k rows
         const uint32_t* rawr = reinterpret_cast<const uint32_t*>(gt + RAW_R);
         const uint32_t* rawk = reinterpret_cast<const uint32_t*>(gt + RAW_K);
         const uint32_t* rawa = reinterpret_cast<const uint32_t*>(gt + RAW_A);
@@ -249,32 +288,23 @@ __global__ void __launch_bounds__(NTHR, 1)
                 ok = group_sync_and(bar_id, GROUP, w_ok);
                 if (!ok) break;
             }
-            float2 cw[16];
-#pragma unroll
-            for (int e = 0; e < 16; ++e) {
-                const int t = 16 * tq + e;
-                if (t < nv) {
-                    if constexpr (sizeof(WT) == 4) {
-                        cw[e] = *reinterpret_cast<const float2*>(rawl + t * 64 + j0);
-                    } else {
-                        const uint32_t u = *reinterpret_cast<const uint32_t*>(rawl + t * 64 + j0);
-                        cw[e] = make_float2(bf16lo_to_f32(u), bf16hi_to_f32(u));
-                    }
-                } else {
-                    cw[e] = make_float2(-INFINITY, -INFINITY);
-                }
+            const bool ragged = nv < L;  // group-uniform
+            if (ragged) {
+                // tokens past the end of the sequence are identity steps: w_log = -inf (w = 1)
+                for (int i = nv * 64 + tg; i < L * 64; i += static_cast<int>(GROUP)) rawl_w[i] = neg_inf_of<WT>();
+                group_sync(bar_id, GROUP);
             }
+            // pass 1: product of w over this thread's 16 tokens, per key channel
             float p0 = 1.f, p1 = 1.f;
-#pragma unroll
+#pragma unroll 4
             for (int e = 0; e < 16; ++e) {
-                p0 *= __expf(-__expf(cw[e].x));
-                p1 *= __expf(-__expf(cw[e].y));
-                cw[e] = make_float2(p0, p1);  // cumulative product inside the 16-token block
+                const float2 lv = ld_wlog2(rawl, (16 * tq + e) * 64 + j0);
+                p0 *= __expf(-__expf(lv.x));
+                p1 *= __expf(-__expf(lv.y));
             }
             red[tq * 64 + j0] = p0;
             red[tq * 64 + j0 + 1] = p1;
             {
-                // every raw w_log read is done once all threads pass this barrier (BK is rewritten below)
                 bool w_ok = true;
                 if (tg == 0)
                     w_ok = mbar_wait(&bars.rrk[g], static_cast<uint32_t>(kk_) & 1u, WAIT_NS) &&
@@ -282,6 +312,17 @@ __global__ void __launch_bounds__(NTHR, 1)
                 ok = group_sync_and(bar_id, GROUP, w_ok);
                 if (!ok) break;
                 ++raw_done;
+            }
+            if (ragged) {
+                // ... and r = k = a = b = 0
+                const int nrow = L - nv;
+                for (int i = tg; i < 4 * nrow * 8; i += static_cast<int>(GROUP)) {
+                    const int tile = i / (nrow * 8), rem = i - tile * nrow * 8;
+                    const uint32_t off = tile == 0 ? RAW_R : tile == 1 ? RAW_K : tile == 2 ? RAW_A : RAW_B;
+                    *reinterpret_cast<uint4*>(gt + off + (nv + (rem >> 3)) * 128 + (rem & 7) * 16) =
+                        make_uint4(0u, 0u, 0u, 0u);
+                }
+                group_sync(bar_id, GROUP);
             }
             float pre0 = 1.f, pre1 = 1.f, GL0 = 1.f, GL1 = 1.f;
 #pragma unroll
@@ -295,55 +336,62 @@ __global__ void __launch_bounds__(NTHR, 1)
                 gam[(kk_ & 1) * 64 + j0] = GL0;
                 gam[(kk_ & 1) * 64 + j0 + 1] = GL1;
             }
-            float gp0 = pre0, gp1 = pre1;
-            const uint32_t cb = static_cast<uint32_t>(j0) * 2u;
-            uint32_t rr[8], kv[8], av[8], bv[8];
+            // pass 2, eight tokens at a time: Gamma_t again from w, then
+            //   Rt = r Gamma_t, At = a Gamma_{t-1}, Bt = b / Gamma_t, Kt = k / Gamma_t  (token rows)
+            //   Bh^T, Kh^T = (b, k) Gamma_L / Gamma_t                                    (key rows)
+            // Rt and At overwrite the raw a, b rows of the same tokens in RAM, Bt and Kt the raw r, k
+            // rows in NQ; each warp owns its 16 token rows and reads them before writing.
+            {
+                float gp0 = pre0, gp1 = pre1;  // Gamma_{t-1}
+                const uint32_t cb = static_cast<uint32_t>(j0) * 2u;
+#pragma unroll 1
+                for (int half = 0; half < 2; ++half) {
+                    const int t0 = 16 * tq + 8 * half;
+                    uint32_t rr[8], kv[8], av[8], bv[8];
 #pragma unroll
-            for (int half = 0; half < 2; ++half) {
-#pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    const int t = 16 * tq + 8 * half + e;
-                    const int idx = t * 32 + jp;  // 32-bit word of (t, j0)
-                    const bool in = t < nv;
-                    rr[e] = in ? rawr[idx] : 0u;
-                    kv[e] = in ? rawk[idx] : 0u;
-                    av[e] = in ? rawa[idx] : 0u;
-                    bv[e] = in ? rawb[idx] : 0u;
-                }
-                __syncwarp();  // this warp's raw rows are read before its tiles overwrite them
-                uint32_t bh0[4], bh1[4], kh0[4], kh1[4];  // 8 tokens of Bh^T / Kh^T rows j0, j0+1
-#pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    const int t = 16 * tq + 8 * half + e;
-                    const float G0 = pre0 * cw[8 * half + e].x, G1 = pre1 * cw[8 * half + e].y;
-                    const float i0 = __fdividef(1.f, G0), i1 = __fdividef(1.f, G1);
-                    const float l0 = i0 * GL0, l1 = i1 * GL1;
-                    const float2 rf = unpack_bf16x2(rr[e]), kf = unpack_bf16x2(kv[e]);
-                    const float2 af = unpack_bf16x2(av[e]), bf = unpack_bf16x2(bv[e]);
-                    *reinterpret_cast<uint32_t*>(RAM + swz(t, cb, 128)) = pack_bf16x2(rf.x * G0, rf.y * G1);
-                    *reinterpret_cast<uint32_t*>(RAM + swz(64 + t, cb, 128)) = pack_bf16x2(af.x * gp0, af.y * gp1);
-                    *reinterpret_cast<uint32_t*>(BK + swz(t, cb, 128)) = pack_bf16x2(bf.x * i0, bf.y * i1);
-                    *reinterpret_cast<uint32_t*>(BK + swz(64 + t, cb, 128)) = pack_bf16x2(kf.x * i0, kf.y * i1);
-                    const float b0 = bf.x * l0, b1 = bf.y * l1, k0 = kf.x * l0, k1 = kf.y * l1;
-                    if ((e & 1) == 0) {
-                        bh0[e >> 1] = __float_as_uint(b0);
-                        bh1[e >> 1] = __float_as_uint(b1);
-                        kh0[e >> 1] = __float_as_uint(k0);
-                        kh1[e >> 1] = __float_as_uint(k1);
-                    } else {
-                        bh0[e >> 1] = pack_bf16x2(__uint_as_float(bh0[e >> 1]), b0);
-                        bh1[e >> 1] = pack_bf16x2(__uint_as_float(bh1[e >> 1]), b1);
-                        kh0[e >> 1] = pack_bf16x2(__uint_as_float(kh0[e >> 1]), k0);
-                        kh1[e >> 1] = pack_bf16x2(__uint_as_float(kh1[e >> 1]), k1);
+                    for (int e = 0; e < 8; ++e) {
+                        const int idx = (t0 + e) * 32 + jp;  // 32-bit word of (t, j0)
+                        rr[e] = rawr[idx];
+                        kv[e] = rawk[idx];
+                        av[e] = rawa[idx];
+                        bv[e] = rawb[idx];
                     }
-                    gp0 = G0;
-                    gp1 = G1;
+                    __syncwarp();
+                    uint32_t bh0[4], bh1[4], kh0[4], kh1[4];  // 8 tokens of Bh^T / Kh^T rows j0, j0 + 1
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        const int t = t0 + e;
+                        const float2 lv = ld_wlog2(rawl, t * 64 + j0);
+                        const float G0 = gp0 * __expf(-__expf(lv.x)), G1 = gp1 * __expf(-__expf(lv.y));
+                        const float i0 = __fdividef(1.f, G0), i1 = __fdividef(1.f, G1);
+                        const float l0 = i0 * GL0, l1 = i1 * GL1;
+                        const float2 rf = unpack_bf16x2(rr[e]), kf = unpack_bf16x2(kv[e]);
+                        const float2 af = unpack_bf16x2(av[e]), bf = unpack_bf16x2(bv[e]);
+                        *reinterpret_cast<uint32_t*>(RAM + swz(t, cb, 128)) = pack_bf16x2(rf.x * G0, rf.y * G1);
+                        *reinterpret_cast<uint32_t*>(RAM + swz(64 + t, cb, 128)) = pack_bf16x2(af.x * gp0, af.y * gp1);
+                        *reinterpret_cast<uint32_t*>(BKt + swz(t, cb, 128)) = pack_bf16x2(bf.x * i0, bf.y * i1);
+                        *reinterpret_cast<uint32_t*>(BKt + swz(64 + t, cb, 128)) = pack_bf16x2(kf.x * i0, kf.y * i1);
+                        const float b0 = bf.x * l0, b1 = bf.y * l1, k0 = kf.x * l0, k1 = kf.y * l1;
+                        if ((e & 1) == 0) {
+                            bh0[e >> 1] = __float_as_uint(b0);
+                            bh1[e >> 1] = __float_as_uint(b1);
+                            kh0[e >> 1] = __float_as_uint(k0);
+                            kh1[e >> 1] = __float_as_uint(k1);
+                        } else {
+                            bh0[e >> 1] = pack_bf16x2(__uint_as_float(bh0[e >> 1]), b0);
+                            bh1[e >> 1] = pack_bf16x2(__uint_as_float(bh1[e >> 1]), b1);
+                            kh0[e >> 1] = pack_bf16x2(__uint_as_float(kh0[e >> 1]), k0);
+                            kh1[e >> 1] = pack_bf16x2(__uint_as_float(kh1[e >> 1]), k1);
+                        }
+                        gp0 = G0;
+                        gp1 = G1;
+                    }
+                    const uint32_t tb8 = static_cast<uint32_t>(t0) * 2u;  // byte of the first token
+                    *reinterpret_cast<uint4*>(BH + swz(64 + j0, tb8, 128)) = make_uint4(bh0[0], bh0[1], bh0[2], bh0[3]);
+                    *reinterpret_cast<uint4*>(BH + swz(64 + j0 + 1, tb8, 128)) = make_uint4(bh1[0], bh1[1], bh1[2], bh1[3]);
+                    *reinterpret_cast<uint4*>(MK + swz(64 + j0, tb8, 128)) = make_uint4(kh0[0], kh0[1], kh0[2], kh0[3]);
+                    *reinterpret_cast<uint4*>(MK + swz(64 + j0 + 1, tb8, 128)) = make_uint4(kh1[0], kh1[1], kh1[2], kh1[3]);
                 }
-                const uint32_t tb8 = static_cast<uint32_t>(16 * tq + 8 * half) * 2u;  // byte of the first token
-                *reinterpret_cast<uint4*>(BH + swz(64 + j0, tb8, 128)) = make_uint4(bh0[0], bh0[1], bh0[2], bh0[3]);
-                *reinterpret_cast<uint4*>(BH + swz(64 + j0 + 1, tb8, 128)) = make_uint4(bh1[0], bh1[1], bh1[2], bh1[3]);
-                *reinterpret_cast<uint4*>(MK + swz(64 + j0, tb8, 128)) = make_uint4(kh0[0], kh0[1], kh0[2], kh0[3]);
-                *reinterpret_cast<uint4*>(MK + swz(64 + j0 + 1, tb8, 128)) = make_uint4(kh1[0], kh1[1], kh1[2], kh1[3]);
             }
             fence_proxy_async_smem();
             tc_fence_before();
@@ -354,7 +402,7 @@ __global__ void __launch_bounds__(NTHR, 1)
                 tc_fence_after();
 #pragma unroll
                 for (uint32_t s = 0; s < 4; ++s)
-                    mma_ss<false>(tm_gp, kmajor_desc<false>(RAM, 128, s), kmajor_desc<false>(BK, 128, s), ID_G16, s > 0);
+                    mma_ss<false>(tm_gp, kmajor_desc<false>(RAM, 128, s), kmajor_desc<false>(BKt, 128, s), ID_G16, s > 0);
                 mma_commit(&bars.mma[g]);
             }
             mma_pending = true;
@@ -364,35 +412,28 @@ __global__ void __launch_bounds__(NTHR, 1)
             mma_phase ^= 1u;
             tc_fence_after();
 
-            // ---- masks: Mrb -> BH rows 0..63, Mrk -> MK rows 0..63 (incl. diagonal);
-            //      Nab -> Nab^T fp32 and Mak -> MN-major tile next to At (strict)
+            // ---- masks.  Lanes 0..63 hold token rows of G: Mrb -> BH rows 0..63 and Mrk -> MK
+            //      rows 0..63 (columns up to the diagonal).  Lanes 64..127 hold At rows: Nab ->
+            //      fp32 row-major Nr and Mak -> the MN-major tile next to At (strictly lower).
             {
-                float x[32];
-                if (tg < 64) {
-                    const int t = tg;
+                const bool tok = tg < 64;
+                const int t = tok ? tg : tg - 64;
+#pragma unroll 1
+                for (int qq = 0; qq < 4; ++qq) {
+                    float x[32];
+                    tmem_load32(tm_gp + lane_base + 32 * qq, x);
+                    const int c0 = 32 * (qq & 1);
+                    const int lim = t - c0 - (tok ? 0 : 1);  // columns c0 + i with i <= lim are kept
 #pragma unroll
-                    for (int qq = 0; qq < 4; ++qq) {
-                        tmem_load32(tm_gp + lane_base + 32 * qq, x);
+                    for (int i = 0; i < 32; ++i)
+                        if (i > lim) x[i] = 0.f;
+                    if (!tok && qq < 2) {
 #pragma unroll
-                        for (int i = 0; i < 32; ++i)
-                            if (32 * (qq & 1) + i > t) x[i] = 0.f;
-                        st_op_row32<false>(qq < 2 ? BH : MK, 128, t, 32 * (qq & 1), x);
-                    }
-                } else {
-                    const int t = tg - 64;
-#pragma unroll
-                    for (int qq = 0; qq < 2; ++qq) {
-                        tmem_load32(tm_gp + lane_base + 32 * qq, x);
-#pragma unroll
-                        for (int i = 0; i < 32; ++i) Nt[(32 * qq + i) * 64 + t] = (32 * qq + i < t) ? x[i] : 0.f;
-                    }
-#pragma unroll
-                    for (int qq = 0; qq < 2; ++qq) {
-                        tmem_load32(tm_gp + lane_base + 64 + 32 * qq, x);
-#pragma unroll
-                        for (int i = 0; i < 32; ++i)
-                            if (32 * qq + i >= t) x[i] = 0.f;
-                        st_op_row32<false>(RAM + 16384, 64, t, 32 * qq, x);
+                        for (int i = 0; i < 32; i += 4)
+                            *reinterpret_cast<float4*>(Nr + tf_idx(t, c0 + i)) = make_float4(
+                                round_tf32(x[i]), round_tf32(x[i + 1]), round_tf32(x[i + 2]), round_tf32(x[i + 3]));
+                    } else {
+                        st_op_row32<false>(tok ? (qq < 2 ? BH : MK) : RAM + 16384, 128, t, c0, x);
                     }
                 }
             }
@@ -400,79 +441,114 @@ __global__ void __launch_bounds__(NTHR, 1)
             tc_fence_before();
             group_sync(bar_id, GROUP);
 
-            // ---- T = (I - Nab)^{-1}: 32 x 32 diagonal blocks by right-looking substitution
-            if (tg < 64) {
-                const int blk = (tg >> 5) * 32, col = tg & 31;
-                float acc[32];
+            // ---- T = (I - Nab)^{-1} in fp32 (tf32-rounded), built in 16 x 16 blocks:
+            //  (1) the diagonal blocks D_b = (I - Nab_bb)^{-1}: one warp per block, lane c (mod 16)
+            //      computes column c by forward substitution over the rows of Nab;
+            //  (2) T_{b+1,b} = D_{b+1} (Nab_{b+1,b} D_b) for b = 0, 2;
+            //  (3) T_hl = T_hi (Nab_hl T_lo) for the 32 x 32 halves.
+            //  Steps (2) and (3) are warp-level tf32 tensor-core products (m16n8k8); their
+            //  intermediate products live in the upper-right 32 x 32 quadrant of Tf, which is
+            //  zero in T and written as zeros by the bf16 conversion.
+            {
+                const int w = tg >> 5, lane = tg & 31, gq = lane >> 2, t4 = lane & 3;
+                {
+                    const int c = lane & 15, r0 = 16 * w;
+                    float x[16];
 #pragma unroll
-                for (int i = 0; i < 32; ++i) acc[i] = (i == col) ? 1.f : 0.f;
+                    for (int i = 0; i < 16; ++i) {
+                        float p = (i == c) ? 1.f : 0.f;
 #pragma unroll
-                for (int t = 0; t < 31; ++t) {
-                    const float xt = acc[t];
-                    const float4* nrow = reinterpret_cast<const float4*>(Nt + (blk + t) * 64 + blk);  // column blk+t of Nab
+                        for (int q = 0; q < i; q += 4) {
+                            const float4 n4 = *reinterpret_cast<const float4*>(Nr + tf_idx(r0 + i, r0 + q));
+                            p = fmaf(n4.x, x[q], p);
+                            if (q + 1 < i) p = fmaf(n4.y, x[q + 1], p);
+                            if (q + 2 < i) p = fmaf(n4.z, x[q + 2], p);
+                            if (q + 3 < i) p = fmaf(n4.w, x[q + 3], p);
+                        }
+                        x[i] = p;
+                    }
+                    if (lane < 16) {
 #pragma unroll
-                    for (int q4 = (t + 1) >> 2; q4 < 8; ++q4) {
-                        const float4 n4 = nrow[q4];
-                        if (4 * q4 + 0 > t) acc[4 * q4 + 0] = fmaf(n4.x, xt, acc[4 * q4 + 0]);
-                        if (4 * q4 + 1 > t) acc[4 * q4 + 1] = fmaf(n4.y, xt, acc[4 * q4 + 1]);
-                        if (4 * q4 + 2 > t) acc[4 * q4 + 2] = fmaf(n4.z, xt, acc[4 * q4 + 2]);
-                        if (4 * q4 + 3 > t) acc[4 * q4 + 3] = fmaf(n4.w, xt, acc[4 * q4 + 3]);
+                        for (int i = 0; i < 16; ++i) Tf[tf_idx(r0 + i, r0 + c)] = round_tf32(x[i]);
                     }
                 }
-#pragma unroll
-                for (int i = 0; i < 32; ++i) Tf[tf_idx(blk + i, blk + col)] = acc[i];
-                if (blk == 0) {
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) Tf[tf_idx(i, 32 + col)] = 0.f;
-                }
-            }
-            group_sync(bar_id, GROUP);
-            // off-diagonal block: T_hl = T_hi (N_hl T_lo)
-            {
-                const int rr2 = tg >> 2, cq = tg & 3;
-                float xo[8];
-#pragma unroll
-                for (int i = 0; i < 8; ++i) xo[i] = 0.f;
-#pragma unroll 8
-                for (int kk2 = 0; kk2 < 32; ++kk2) {
-                    const float nvv = Nt[kk2 * 64 + 32 + rr2];  // N[32 + rr2][kk2]
-                    const float4 t0 = *reinterpret_cast<const float4*>(Tf + tf_idx(kk2, 8 * cq));
-                    const float4 t1 = *reinterpret_cast<const float4*>(Tf + tf_idx(kk2, 8 * cq + 4));
-                    xo[0] = fmaf(nvv, t0.x, xo[0]); xo[1] = fmaf(nvv, t0.y, xo[1]);
-                    xo[2] = fmaf(nvv, t0.z, xo[2]); xo[3] = fmaf(nvv, t0.w, xo[3]);
-                    xo[4] = fmaf(nvv, t1.x, xo[4]); xo[5] = fmaf(nvv, t1.y, xo[5]);
-                    xo[6] = fmaf(nvv, t1.z, xo[6]); xo[7] = fmaf(nvv, t1.w, xo[7]);
-                }
-                group_sync(bar_id, GROUP);  // every thread has finished reading Nab^T
-                *reinterpret_cast<float4*>(Xs + rr2 * 32 + 8 * cq) = make_float4(xo[0], xo[1], xo[2], xo[3]);
-                *reinterpret_cast<float4*>(Xs + rr2 * 32 + 8 * cq + 4) = make_float4(xo[4], xo[5], xo[6], xo[7]);
                 group_sync(bar_id, GROUP);
+                const int bb = 2 * (w >> 1), mt = w >> 1, np = w & 1;
+                {
+                    // Y_b = Nab_{b+1,b} D_b -> scratch rows 8b .. 8b+15, columns 32 .. 47
+                    float d[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-                for (int i = 0; i < 8; ++i) xo[i] = 0.f;
-#pragma unroll 8
-                for (int kk2 = 0; kk2 < 32; ++kk2) {
-                    const float th = Tf[tf_idx(32 + rr2, 32 + kk2)];  // T_hi[rr2][kk2]
-                    const float4 x0 = *reinterpret_cast<const float4*>(Xs + kk2 * 32 + 8 * cq);
-                    const float4 x1 = *reinterpret_cast<const float4*>(Xs + kk2 * 32 + 8 * cq + 4);
-                    xo[0] = fmaf(th, x0.x, xo[0]); xo[1] = fmaf(th, x0.y, xo[1]);
-                    xo[2] = fmaf(th, x0.z, xo[2]); xo[3] = fmaf(th, x0.w, xo[3]);
-                    xo[4] = fmaf(th, x1.x, xo[4]); xo[5] = fmaf(th, x1.y, xo[5]);
-                    xo[6] = fmaf(th, x1.z, xo[6]); xo[7] = fmaf(th, x1.w, xo[7]);
+                    for (int ks = 0; ks < 2; ++ks) {
+                        uint32_t af[4], bf[2];
+                        frag_a_tf32(Nr, 16 * (bb + 1), 16 * bb + 8 * ks, gq, t4, af);
+                        frag_b_tf32(Tf, 16 * bb + 8 * ks, 16 * bb + 8 * np, gq, t4, bf);
+                        mma_tf32_16x8x8(d, af, bf);
+                    }
+                    frag_c_store_tf32(Tf, 8 * bb, 32 + 8 * np, gq, t4, d);
                 }
-                *reinterpret_cast<float4*>(Tf + tf_idx(32 + rr2, 8 * cq)) = make_float4(xo[0], xo[1], xo[2], xo[3]);
-                *reinterpret_cast<float4*>(Tf + tf_idx(32 + rr2, 8 * cq + 4)) = make_float4(xo[4], xo[5], xo[6], xo[7]);
+                group_sync(bar_id, GROUP);
+                {
+                    // T_{b+1,b} = D_{b+1} Y_b
+                    float d[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                    for (int ks = 0; ks < 2; ++ks) {
+                        uint32_t af[4], bf[2];
+                        frag_a_tf32(Tf, 16 * (bb + 1), 16 * (bb + 1) + 8 * ks, gq, t4, af);
+                        frag_b_tf32(Tf, 8 * bb + 8 * ks, 32 + 8 * np, gq, t4, bf);
+                        mma_tf32_16x8x8(d, af, bf);
+                    }
+                    frag_c_store_tf32(Tf, 16 * (bb + 1), 16 * bb + 8 * np, gq, t4, d);
+                }
+                group_sync(bar_id, GROUP);
+                {
+                    // X = Nab_hl T_lo -> scratch rows 0 .. 31, columns 32 .. 63.  T_lo is zero in
+                    // rows 0 .. 15 of columns 16 .. 31, so those n-tiles start at k = 16.
+                    float d0[4] = {0.f, 0.f, 0.f, 0.f}, d1[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                    for (int ks = 0; ks < 4; ++ks) {
+                        if (np == 1 && ks < 2) continue;
+                        uint32_t af[4], b0[2], b1[2];
+                        frag_a_tf32(Nr, 32 + 16 * mt, 8 * ks, gq, t4, af);
+                        frag_b_tf32(Tf, 8 * ks, 16 * np, gq, t4, b0);
+                        frag_b_tf32(Tf, 8 * ks, 16 * np + 8, gq, t4, b1);
+                        mma_tf32_16x8x8(d0, af, b0);
+                        mma_tf32_16x8x8(d1, af, b1);
+                    }
+                    frag_c_store_tf32(Tf, 16 * mt, 32 + 16 * np, gq, t4, d0);
+                    frag_c_store_tf32(Tf, 16 * mt, 32 + 16 * np + 8, gq, t4, d1);
+                }
+                group_sync(bar_id, GROUP);
+                {
+                    // T_hl = T_hi X.  Rows 32 .. 47 of T_hi are zero beyond column 47.
+                    float d0[4] = {0.f, 0.f, 0.f, 0.f}, d1[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                    for (int ks = 0; ks < 4; ++ks) {
+                        if (mt == 0 && ks >= 2) continue;
+                        uint32_t af[4], b0[2], b1[2];
+                        frag_a_tf32(Tf, 32 + 16 * mt, 32 + 8 * ks, gq, t4, af);
+                        frag_b_tf32(Tf, 8 * ks, 32 + 16 * np, gq, t4, b0);
+                        frag_b_tf32(Tf, 8 * ks, 32 + 16 * np + 8, gq, t4, b1);
+                        mma_tf32_16x8x8(d0, af, b0);
+                        mma_tf32_16x8x8(d1, af, b1);
+                    }
+                    frag_c_store_tf32(Tf, 32 + 16 * mt, 16 * np, gq, t4, d0);
+                    frag_c_store_tf32(Tf, 32 + 16 * mt, 16 * np + 8, gq, t4, d1);
+                }
             }
             group_sync(bar_id, GROUP);
-            // T -> bf16, MN-major (rows i, columns j)
+            // T -> bf16, MN-major (rows i, columns j); blocks above the diagonal are zero
 #pragma unroll
             for (int m = 0; m < 4; ++m) {
                 const int qd = tg + 128 * m;
                 const int row = qd >> 3, ch = qd & 7;
-                const float4 f0 = *reinterpret_cast<const float4*>(Tf + tf_idx(row, 8 * ch));
-                const float4 f1 = *reinterpret_cast<const float4*>(Tf + tf_idx(row, 8 * ch + 4));
-                *reinterpret_cast<uint4*>(Tb + swz(row, ch * 16, 64)) =
-                    make_uint4(pack_bf16x2(f0.x, f0.y), pack_bf16x2(f0.z, f0.w), pack_bf16x2(f1.x, f1.y),
-                               pack_bf16x2(f1.z, f1.w));
+                uint4 val = make_uint4(0u, 0u, 0u, 0u);
+                if ((ch >> 1) <= (row >> 4)) {
+                    const float4 f0 = *reinterpret_cast<const float4*>(Tf + tf_idx(row, 8 * ch));
+                    const float4 f1 = *reinterpret_cast<const float4*>(Tf + tf_idx(row, 8 * ch + 4));
+                    val = make_uint4(pack_bf16x2(f0.x, f0.y), pack_bf16x2(f0.z, f0.w), pack_bf16x2(f1.x, f1.y),
+                                     pack_bf16x2(f1.z, f1.w));
+                }
+                *reinterpret_cast<uint4*>(Tb + swz(row, ch * 16, 64)) = val;
             }
             fence_proxy_async_smem();
             group_sync(bar_id, GROUP);
