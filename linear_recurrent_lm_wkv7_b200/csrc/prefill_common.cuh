@@ -92,6 +92,25 @@ __device__ __forceinline__ void ld_op_row32(const uint8_t* tile, uint32_t R, uin
     }
 }
 
+// 16 consecutive bf16 elements [c0, c0+16) of one row (two 16-byte accesses)
+__device__ __forceinline__ void st_bf16_row16(uint8_t* tile, uint32_t R, uint32_t row, uint32_t c0, const float* x) {
+#pragma unroll
+    for (int q = 0; q < 2; ++q)
+        *reinterpret_cast<uint4*>(tile + swz(row, (c0 + 8 * q) * 2, R)) =
+            make_uint4(pack_bf16x2(x[8 * q], x[8 * q + 1]), pack_bf16x2(x[8 * q + 2], x[8 * q + 3]),
+                       pack_bf16x2(x[8 * q + 4], x[8 * q + 5]), pack_bf16x2(x[8 * q + 6], x[8 * q + 7]));
+}
+__device__ __forceinline__ void ld_bf16_row16(const uint8_t* tile, uint32_t R, uint32_t row, uint32_t c0, float* x) {
+#pragma unroll
+    for (int q = 0; q < 2; ++q) {
+        const uint4 v = *reinterpret_cast<const uint4*>(tile + swz(row, (c0 + 8 * q) * 2, R));
+        x[8 * q + 0] = bf16lo_to_f32(v.x); x[8 * q + 1] = bf16hi_to_f32(v.x);
+        x[8 * q + 2] = bf16lo_to_f32(v.y); x[8 * q + 3] = bf16hi_to_f32(v.y);
+        x[8 * q + 4] = bf16lo_to_f32(v.z); x[8 * q + 5] = bf16hi_to_f32(v.z);
+        x[8 * q + 6] = bf16lo_to_f32(v.w); x[8 * q + 7] = bf16hi_to_f32(v.w);
+    }
+}
+
 // Descriptor of K-step s of a K-major operand tile with R rows (K = 64 elements).
 template <bool TF32>
 __device__ __forceinline__ uint64_t kmajor_desc(const uint8_t* tile, uint32_t R, uint32_t s) {

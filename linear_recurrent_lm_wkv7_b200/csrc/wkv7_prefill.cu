@@ -102,7 +102,7 @@ __device__ __forceinline__ Smem carve(uint8_t* raw) {
     using O = OpType<TF32>;
     constexpr uint32_t solver = 2u * 64u * NSTRIDE * 4u;
     constexpr uint32_t r4 = ((solver > O::TILE128 ? solver : O::TILE128) + 1023u) & ~1023u;
-    uint8_t* p = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(raw) + 1023u) & ~uintptr_t(1023));
+    uint8_t* p = raw + ((1024u - (smem_u32(raw) & 1023u)) & 1023u);  // stays in the shared address space
     Smem s;
     s.RA = p; p += O::TILE128;
     s.BK = p; s.WZ = p; p += O::TILE128;
@@ -195,7 +195,7 @@ __global__ void __launch_bounds__(NT, 1)
                         const __grid_constant__ TmaMaps maps) {
     using O = OpType<TF32>;
     constexpr uint32_t WB = sizeof(WT);
-    extern __shared__ uint8_t smem_raw[];
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
     const Smem sm = carve<TF32, WB>(smem_raw);
     const int tid = threadIdx.x;
     const int warp = tid >> 5;

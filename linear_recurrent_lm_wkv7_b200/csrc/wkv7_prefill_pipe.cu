@@ -108,6 +108,24 @@ __device__ __forceinline__ void mma_tf32_16x8x8(float (&d)[4], const uint32_t (&
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
 }
 
+// C[cr + 0..15][cc + 0..15] = sum over k-steps ks in [ks0, ks1) of
+//   A[ar + 0..15][ac + 8 ks + 0..7] * B[bk + 8 ks + 0..7][bn + 0..15]   (one warp)
+__device__ __forceinline__ void tf32_tile16(const float* A, int ar, int ac, const float* B, int bk, int bn, int ks0,
+                                            int ks1, float* C, int cr, int cc, int gq, int t4) {
+    float d0[4] = {0.f, 0.f, 0.f, 0.f}, d1[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 1
+    for (int ks = ks0; ks < ks1; ++ks) {
+        uint32_t af[4], b0[2], b1[2];
+        frag_a_tf32(A, ar, ac + 8 * ks, gq, t4, af);
+        frag_b_tf32(B, bk + 8 * ks, bn, gq, t4, b0);
+        frag_b_tf32(B, bk + 8 * ks, bn + 8, gq, t4, b1);
+        mma_tf32_16x8x8(d0, af, b0);
+        mma_tf32_16x8x8(d1, af, b1);
+    }
+    frag_c_store_tf32(C, cr, cc, gq, t4, d0);
+    frag_c_store_tf32(C, cr, cc + 8, gq, t4, d1);
+}
+
 __device__ __forceinline__ float2 unpack_bf16x2(uint32_t u) { return make_float2(bf16lo_to_f32(u), bf16hi_to_f32(u)); }
 
 // w_log of key channels j, j + 1 (element index i of the raw tile) as floats
@@ -143,8 +161,10 @@ __global__ void __launch_bounds__(NTHR, 1)
                              const float* s0, __nv_bfloat16* __restrict__ y, float* sT, int T, int H,
                              const int32_t* __restrict__ seq_offsets, int* status,
                              const __grid_constant__ TmaMaps maps) {
-    extern __shared__ uint8_t smem_raw[];
-    uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023u) & ~uintptr_t(1023));
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    // 1024-byte aligned base, derived from the shared array so that every tile pointer
+    // stays in the shared address space (32-bit addressing)
+    uint8_t* sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     const int tid = threadIdx.x;
     const int warp = tid >> 5;
     Bars bars;
@@ -473,67 +493,20 @@ __global__ void __launch_bounds__(NTHR, 1)
                     }
                 }
                 group_sync(bar_id, GROUP);
-                const int bb = 2 * (w >> 1), mt = w >> 1, np = w & 1;
-                {
-                    // Y_b = Nab_{b+1,b} D_b -> scratch rows 8b .. 8b+15, columns 32 .. 47
-                    float d[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-                    for (int ks = 0; ks < 2; ++ks) {
-                        uint32_t af[4], bf[2];
-                        frag_a_tf32(Nr, 16 * (bb + 1), 16 * bb + 8 * ks, gq, t4, af);
-                        frag_b_tf32(Tf, 16 * bb + 8 * ks, 16 * bb + 8 * np, gq, t4, bf);
-                        mma_tf32_16x8x8(d, af, bf);
-                    }
-                    frag_c_store_tf32(Tf, 8 * bb, 32 + 8 * np, gq, t4, d);
-                }
+                const int mt = w >> 1, np = w & 1;
+                // Y_b = Nab_{b+1,b} D_b (b = 2w, warps 0-1) -> scratch rows 8b .. 8b+15, columns 32 .. 47
+                if (w < 2) tf32_tile16(Nr, 16 * (2 * w + 1), 32 * w, Tf, 32 * w, 32 * w, 0, 2, Tf, 16 * w, 32, gq, t4);
                 group_sync(bar_id, GROUP);
-                {
-                    // T_{b+1,b} = D_{b+1} Y_b
-                    float d[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-                    for (int ks = 0; ks < 2; ++ks) {
-                        uint32_t af[4], bf[2];
-                        frag_a_tf32(Tf, 16 * (bb + 1), 16 * (bb + 1) + 8 * ks, gq, t4, af);
-                        frag_b_tf32(Tf, 8 * bb + 8 * ks, 32 + 8 * np, gq, t4, bf);
-                        mma_tf32_16x8x8(d, af, bf);
-                    }
-                    frag_c_store_tf32(Tf, 16 * (bb + 1), 16 * bb + 8 * np, gq, t4, d);
-                }
+                // T_{b+1,b} = D_{b+1} Y_b
+                if (w < 2)
+                    tf32_tile16(Tf, 16 * (2 * w + 1), 16 * (2 * w + 1), Tf, 16 * w, 32, 0, 2, Tf, 16 * (2 * w + 1), 32 * w, gq, t4);
                 group_sync(bar_id, GROUP);
-                {
-                    // X = Nab_hl T_lo -> scratch rows 0 .. 31, columns 32 .. 63.  T_lo is zero in
-                    // rows 0 .. 15 of columns 16 .. 31, so those n-tiles start at k = 16.
-                    float d0[4] = {0.f, 0.f, 0.f, 0.f}, d1[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-                    for (int ks = 0; ks < 4; ++ks) {
-                        if (np == 1 && ks < 2) continue;
-                        uint32_t af[4], b0[2], b1[2];
-                        frag_a_tf32(Nr, 32 + 16 * mt, 8 * ks, gq, t4, af);
-                        frag_b_tf32(Tf, 8 * ks, 16 * np, gq, t4, b0);
-                        frag_b_tf32(Tf, 8 * ks, 16 * np + 8, gq, t4, b1);
-                        mma_tf32_16x8x8(d0, af, b0);
-                        mma_tf32_16x8x8(d1, af, b1);
-                    }
-                    frag_c_store_tf32(Tf, 16 * mt, 32 + 16 * np, gq, t4, d0);
-                    frag_c_store_tf32(Tf, 16 * mt, 32 + 16 * np + 8, gq, t4, d1);
-                }
+                // X = Nab_hl T_lo -> scratch rows 0 .. 31, columns 32 .. 63 (T_lo is zero in rows
+                // 0 .. 15 of columns 16 .. 31, so those columns start at k = 16)
+                tf32_tile16(Nr, 32 + 16 * mt, 0, Tf, 0, 16 * np, np ? 2 : 0, 4, Tf, 16 * mt, 32 + 16 * np, gq, t4);
                 group_sync(bar_id, GROUP);
-                {
-                    // T_hl = T_hi X.  Rows 32 .. 47 of T_hi are zero beyond column 47.
-                    float d0[4] = {0.f, 0.f, 0.f, 0.f}, d1[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-                    for (int ks = 0; ks < 4; ++ks) {
-                        if (mt == 0 && ks >= 2) continue;
-                        uint32_t af[4], b0[2], b1[2];
-                        frag_a_tf32(Tf, 32 + 16 * mt, 32 + 8 * ks, gq, t4, af);
-                        frag_b_tf32(Tf, 8 * ks, 32 + 16 * np, gq, t4, b0);
-                        frag_b_tf32(Tf, 8 * ks, 32 + 16 * np + 8, gq, t4, b1);
-                        mma_tf32_16x8x8(d0, af, b0);
-                        mma_tf32_16x8x8(d1, af, b1);
-                    }
-                    frag_c_store_tf32(Tf, 32 + 16 * mt, 16 * np, gq, t4, d0);
-                    frag_c_store_tf32(Tf, 32 + 16 * mt, 16 * np + 8, gq, t4, d1);
-                }
+                // T_hl = T_hi X (rows 32 .. 47 of T_hi are zero beyond column 47)
+                tf32_tile16(Tf, 32 + 16 * mt, 32, Tf, 0, 32 + 16 * np, 0, mt ? 4 : 2, Tf, 32 + 16 * mt, 16 * np, gq, t4);
             }
             group_sync(bar_id, GROUP);
             // T -> bf16, MN-major (rows i, columns j); blocks above the diagonal are zero
@@ -611,23 +584,21 @@ __global__ void __launch_bounds__(NTHR, 1)
             // NQ (Q) has been consumed by P: load r and k of this group's next chunk
             if (c + 2 < nchunks && tg == 0) issue_raw(c + 2, 1);
             {
-                float x[32];
-                const int row = tg;  // lanes 0..63: token rows (R' = Rt + Mrb W, Mrb Z); 64..127: key rows
-#pragma unroll
-                for (int q = 0; q < 2; ++q) {
+                // P columns 0..63 -> AS (token rows get Rt added: R' = Rt + Mrb W; key rows Bh^T W),
+                // columns 64..127 -> BH ([Mrb Z; Bh^T Z])
+                const int row = tg;
+#pragma unroll 1
+                for (int q = 0; q < 4; ++q) {
+                    float x[32];
                     tmem_load32(tm_gp + lane_base + 32 * q, x);
-                    if (tg < 64) {
+                    const int c0 = 32 * (q & 1);
+                    if (q < 2 && tg < 64) {
                         float rt[32];
-                        ld_op_row32<false>(RAM, 128, row, 32 * q, rt);
+                        ld_op_row32<false>(RAM, 128, row, c0, rt);
 #pragma unroll
                         for (int i = 0; i < 32; ++i) x[i] += rt[i];
                     }
-                    st_op_row32<false>(AS, 128, row, 32 * q, x);
-                }
-#pragma unroll
-                for (int q = 0; q < 2; ++q) {
-                    tmem_load32(tm_gp + lane_base + 64 + 32 * q, x);
-                    st_op_row32<false>(BH, 128, row, 32 * q, x);
+                    st_op_row32<false>(q < 2 ? AS : BH, 128, row, c0, x);
                 }
             }
             fence_proxy_async_smem();
@@ -712,7 +683,7 @@ __global__ void __launch_bounds__(NTHR, 1)
             float o[32];
             if (ts < 64) {
                 const int t = ts;
-#pragma unroll
+#pragma unroll 1
                 for (int q = 0; q < 2; ++q) {
                     tmem_load32(tm_out + lane_base + 32 * q, o);
                     if (t < nv) {
