@@ -134,6 +134,12 @@ __device__ __forceinline__ float2 ld_wlog2(const __nv_bfloat16* p, int i) {
     const uint32_t u = *reinterpret_cast<const uint32_t*>(p + i);
     return make_float2(bf16lo_to_f32(u), bf16hi_to_f32(u));
 }
+// w = exp(-exp(w_log)) for two key channels
+__device__ __forceinline__ float2 decay2(float2 lv) {
+    return make_float2(__expf(-__expf(lv.x)), __expf(-__expf(lv.y)));
+}
+__device__ __forceinline__ uint32_t pack2(float2 v) { return pack_bf16x2(v.x, v.y); }
+
 template <typename WT>
 __device__ __forceinline__ WT neg_inf_of();
 template <>
@@ -314,16 +320,17 @@ __global__ void __launch_bounds__(NTHR, 1)
                 for (int i = nv * 64 + tg; i < L * 64; i += static_cast<int>(GROUP)) rawl_w[i] = neg_inf_of<WT>();
                 group_sync(bar_id, GROUP);
             }
-            // pass 1: product of w over this thread's 16 tokens, per key channel
-            float p0 = 1.f, p1 = 1.f;
+            // pass 1: product of w over this thread's 16 tokens, per key channel.  With fp32
+            // w_log the running products overwrite the thread's own w_log elements.
+            float2 pw = make_float2(1.f, 1.f);
 #pragma unroll 4
             for (int e = 0; e < 16; ++e) {
-                const float2 lv = ld_wlog2(rawl, (16 * tq + e) * 64 + j0);
-                p0 *= __expf(-__expf(lv.x));
-                p1 *= __expf(-__expf(lv.y));
+                const int i = (16 * tq + e) * 64 + j0;
+                pw = __fmul2_rn(pw, decay2(ld_wlog2(rawl, i)));
+                if constexpr (sizeof(WT) == 4) *reinterpret_cast<float2*>(rawl_w + i) = pw;
             }
-            red[tq * 64 + j0] = p0;
-            red[tq * 64 + j0 + 1] = p1;
+            red[tq * 64 + j0] = pw.x;
+            red[tq * 64 + j0 + 1] = pw.y;
             {
                 bool w_ok = true;
                 if (tg == 0)
@@ -356,13 +363,15 @@ __global__ void __launch_bounds__(NTHR, 1)
                 gam[(kk_ & 1) * 64 + j0] = GL0;
                 gam[(kk_ & 1) * 64 + j0 + 1] = GL1;
             }
-            // pass 2, eight tokens at a time: Gamma_t again from w, then
+            // pass 2, eight tokens at a time: Gamma_t (from the stored running products, or
+            // from w again for bf16 w_log), then
             //   Rt = r Gamma_t, At = a Gamma_{t-1}, Bt = b / Gamma_t, Kt = k / Gamma_t  (token rows)
             //   Bh^T, Kh^T = (b, k) Gamma_L / Gamma_t                                    (key rows)
             // Rt and At overwrite the raw a, b rows of the same tokens in RAM, Bt and Kt the raw r, k
             // rows in NQ; each warp owns its 16 token rows and reads them before writing.
             {
-                float gp0 = pre0, gp1 = pre1;  // Gamma_{t-1}
+                const float2 pre = make_float2(pre0, pre1), GL = make_float2(GL0, GL1);
+                float2 gp = pre;  // Gamma_{t-1}
                 const uint32_t cb = static_cast<uint32_t>(j0) * 2u;
 #pragma unroll 1
                 for (int half = 0; half < 2; ++half) {
@@ -381,30 +390,33 @@ __global__ void __launch_bounds__(NTHR, 1)
 #pragma unroll
                     for (int e = 0; e < 8; ++e) {
                         const int t = t0 + e;
-                        const float2 lv = ld_wlog2(rawl, t * 64 + j0);
-                        const float G0 = gp0 * __expf(-__expf(lv.x)), G1 = gp1 * __expf(-__expf(lv.y));
-                        const float i0 = __fdividef(1.f, G0), i1 = __fdividef(1.f, G1);
-                        const float l0 = i0 * GL0, l1 = i1 * GL1;
+                        float2 G;  // Gamma_t
+                        if constexpr (sizeof(WT) == 4) {
+                            G = __fmul2_rn(pre, *reinterpret_cast<const float2*>(rawl + t * 64 + j0));
+                        } else {
+                            G = __fmul2_rn(gp, decay2(ld_wlog2(rawl, t * 64 + j0)));
+                        }
+                        const float2 iv = make_float2(__fdividef(1.f, G.x), __fdividef(1.f, G.y));
+                        const float2 l = __fmul2_rn(iv, GL);
                         const float2 rf = unpack_bf16x2(rr[e]), kf = unpack_bf16x2(kv[e]);
                         const float2 af = unpack_bf16x2(av[e]), bf = unpack_bf16x2(bv[e]);
-                        *reinterpret_cast<uint32_t*>(RAM + swz(t, cb, 128)) = pack_bf16x2(rf.x * G0, rf.y * G1);
-                        *reinterpret_cast<uint32_t*>(RAM + swz(64 + t, cb, 128)) = pack_bf16x2(af.x * gp0, af.y * gp1);
-                        *reinterpret_cast<uint32_t*>(BKt + swz(t, cb, 128)) = pack_bf16x2(bf.x * i0, bf.y * i1);
-                        *reinterpret_cast<uint32_t*>(BKt + swz(64 + t, cb, 128)) = pack_bf16x2(kf.x * i0, kf.y * i1);
-                        const float b0 = bf.x * l0, b1 = bf.y * l1, k0 = kf.x * l0, k1 = kf.y * l1;
+                        *reinterpret_cast<uint32_t*>(RAM + swz(t, cb, 128)) = pack2(__fmul2_rn(rf, G));
+                        *reinterpret_cast<uint32_t*>(RAM + swz(64 + t, cb, 128)) = pack2(__fmul2_rn(af, gp));
+                        *reinterpret_cast<uint32_t*>(BKt + swz(t, cb, 128)) = pack2(__fmul2_rn(bf, iv));
+                        *reinterpret_cast<uint32_t*>(BKt + swz(64 + t, cb, 128)) = pack2(__fmul2_rn(kf, iv));
+                        const float2 bhv = __fmul2_rn(bf, l), khv = __fmul2_rn(kf, l);
                         if ((e & 1) == 0) {
-                            bh0[e >> 1] = __float_as_uint(b0);
-                            bh1[e >> 1] = __float_as_uint(b1);
-                            kh0[e >> 1] = __float_as_uint(k0);
-                            kh1[e >> 1] = __float_as_uint(k1);
+                            bh0[e >> 1] = __float_as_uint(bhv.x);
+                            bh1[e >> 1] = __float_as_uint(bhv.y);
+                            kh0[e >> 1] = __float_as_uint(khv.x);
+                            kh1[e >> 1] = __float_as_uint(khv.y);
                         } else {
-                            bh0[e >> 1] = pack_bf16x2(__uint_as_float(bh0[e >> 1]), b0);
-                            bh1[e >> 1] = pack_bf16x2(__uint_as_float(bh1[e >> 1]), b1);
-                            kh0[e >> 1] = pack_bf16x2(__uint_as_float(kh0[e >> 1]), k0);
-                            kh1[e >> 1] = pack_bf16x2(__uint_as_float(kh1[e >> 1]), k1);
+                            bh0[e >> 1] = pack_bf16x2(__uint_as_float(bh0[e >> 1]), bhv.x);
+                            bh1[e >> 1] = pack_bf16x2(__uint_as_float(bh1[e >> 1]), bhv.y);
+                            kh0[e >> 1] = pack_bf16x2(__uint_as_float(kh0[e >> 1]), khv.x);
+                            kh1[e >> 1] = pack_bf16x2(__uint_as_float(kh1[e >> 1]), khv.y);
                         }
-                        gp0 = G0;
-                        gp1 = G1;
+                        gp = G;
                     }
                     const uint32_t tb8 = static_cast<uint32_t>(t0) * 2u;  // byte of the first token
                     *reinterpret_cast<uint4*>(BH + swz(64 + j0, tb8, 128)) = make_uint4(bh0[0], bh0[1], bh0[2], bh0[3]);
