@@ -55,7 +55,7 @@ constexpr uint32_t OFF_RAM = 0;        // Rt (rows 0-63) | At (rows 64-127) | Ma
 constexpr uint32_t OFF_BK = 24576;     // raw w_log (16 KB), then T fp32 (64 x 64, tf_idx layout)
 constexpr uint32_t OFF_BH = 40960;     // [Mrb; Bh^T] 16 KB, then [Mrb Z; Bh^T Z]
 constexpr uint32_t OFF_MK = 57344;     // [Mrk; Kh^T] 16 KB, K-major over tokens
-constexpr uint32_t OFF_NQ = 73728;     // raw r, k -> [Bt; Kt] 16 KB, then Nab fp32, then T bf16 at +8 KB, then Q bf16
+constexpr uint32_t OFF_NQ = 73728;     // raw r, k -> [Bt; Kt] 16 KB, then Nab fp32, then T bf16 (first 8 KB), then Q bf16
 constexpr uint32_t OFF_V = 90112;      // V 8 KB (MN-major)
 constexpr uint32_t GROUP_TILES = 98304;
 constexpr uint32_t OFF_AS = 2 * GROUP_TILES;          // [R'; Bh^T W] 16 KB, shared by both groups
@@ -110,8 +110,9 @@ __device__ __forceinline__ void mma_tf32_16x8x8(float (&d)[4], const uint32_t (&
 
 // C[cr + 0..15][cc + 0..15] = sum over k-steps ks in [ks0, ks1) of
 //   A[ar + 0..15][ac + 8 ks + 0..7] * B[bk + 8 ks + 0..7][bn + 0..15]   (one warp)
+// written to C (tf32, tf_idx layout) and/or to Cb (bf16, 128-byte swizzled rows); either may be null.
 __device__ __forceinline__ void tf32_tile16(const float* A, int ar, int ac, const float* B, int bk, int bn, int ks0,
-                                            int ks1, float* C, int cr, int cc, int gq, int t4) {
+                                            int ks1, float* C, uint8_t* Cb, int cr, int cc, int gq, int t4) {
     float d0[4] = {0.f, 0.f, 0.f, 0.f}, d1[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll 1
     for (int ks = ks0; ks < ks1; ++ks) {
@@ -122,8 +123,16 @@ __device__ __forceinline__ void tf32_tile16(const float* A, int ar, int ac, cons
         mma_tf32_16x8x8(d0, af, b0);
         mma_tf32_16x8x8(d1, af, b1);
     }
-    frag_c_store_tf32(C, cr, cc, gq, t4, d0);
-    frag_c_store_tf32(C, cr, cc + 8, gq, t4, d1);
+    if (C) {
+        frag_c_store_tf32(C, cr, cc, gq, t4, d0);
+        frag_c_store_tf32(C, cr, cc + 8, gq, t4, d1);
+    }
+    if (Cb) {
+        *reinterpret_cast<uint32_t*>(Cb + swz(cr + gq, 2 * (cc + 2 * t4), 64)) = pack_bf16x2(d0[0], d0[1]);
+        *reinterpret_cast<uint32_t*>(Cb + swz(cr + gq + 8, 2 * (cc + 2 * t4), 64)) = pack_bf16x2(d0[2], d0[3]);
+        *reinterpret_cast<uint32_t*>(Cb + swz(cr + gq, 2 * (cc + 8 + 2 * t4), 64)) = pack_bf16x2(d1[0], d1[1]);
+        *reinterpret_cast<uint32_t*>(Cb + swz(cr + gq + 8, 2 * (cc + 8 + 2 * t4), 64)) = pack_bf16x2(d1[2], d1[3]);
+    }
 }
 
 __device__ __forceinline__ float2 unpack_bf16x2(uint32_t u) { return make_float2(bf16lo_to_f32(u), bf16hi_to_f32(u)); }
@@ -243,7 +252,7 @@ __global__ void __launch_bounds__(NTHR, 1)
         uint8_t* MK = gt + OFF_MK;
         float* Tf = reinterpret_cast<float*>(gt + OFF_BK);
         float* Nr = reinterpret_cast<float*>(gt + OFF_NQ);
-        uint8_t* Tb = gt + OFF_NQ + 8192;
+        uint8_t* Tb = gt + OFF_NQ;  // bf16 T, over the rows of Nab no longer read
         uint8_t* Qt = gt + OFF_NQ;
         uint8_t* AS = sm + OFF_AS;
         uint8_t* Vt = gt + OFF_V;
@@ -474,13 +483,15 @@ __global__ void __launch_bounds__(NTHR, 1)
             group_sync(bar_id, GROUP);
 
             // ---- T = (I - Nab)^{-1} in fp32 (tf32-rounded), built in 16 x 16 blocks:
-            //  (1) the diagonal blocks D_b = (I - Nab_bb)^{-1}: one warp per block, lane c (mod 16)
-            //      computes column c by forward substitution over the rows of Nab;
-            //  (2) T_{b+1,b} = D_{b+1} (Nab_{b+1,b} D_b) for b = 0, 2;
+            //  (1) the diagonal blocks D_b = (I - Nab_bb)^{-1}: warp b, lane c (mod 16) computes
+            //      column c by forward substitution over the rows of Nab;
+            //  (2) T_{b+1,b} = D_{b+1} (Nab_{b+1,b} D_b) for b = 0, 2 (the inner product by warp b
+            //      straight after its own block);
             //  (3) T_hl = T_hi (Nab_hl T_lo) for the 32 x 32 halves.
             //  Steps (2) and (3) are warp-level tf32 tensor-core products (m16n8k8); their
-            //  intermediate products live in the upper-right 32 x 32 quadrant of Tf, which is
-            //  zero in T and written as zeros by the bf16 conversion.
+            //  intermediate products live in the upper-right 32 x 32 quadrant of Tf, which is zero
+            //  in T.  T goes to the bf16 MN-major tile Tb as its blocks are final (Tb covers the
+            //  first 8 KB of NQ, whose rows of Nab are no longer read from step (2) on).
             {
                 const int w = tg >> 5, lane = tg & 31, gq = lane >> 2, t4 = lane & 3;
                 {
@@ -504,36 +515,56 @@ __global__ void __launch_bounds__(NTHR, 1)
                         for (int i = 0; i < 16; ++i) Tf[tf_idx(r0 + i, r0 + c)] = round_tf32(x[i]);
                     }
                 }
+                if ((w & 1) == 0) {
+                    // Y_w = Nab_{w+1,w} D_w -> scratch rows 8w .. 8w+15, columns 32 .. 47
+                    __syncwarp();
+                    tf32_tile16(Nr, 16 * (w + 1), 16 * w, Tf, 16 * w, 16 * w, 0, 2, Tf, nullptr, 8 * w, 32, gq, t4);
+                }
+                group_sync(bar_id, GROUP);
+                if (w & 1) {
+                    // T_{w,w-1} = D_w Y_{w-1} -> Tf and Tb
+                    tf32_tile16(Tf, 16 * w, 16 * w, Tf, 8 * (w - 1), 32, 0, 2, Tf, Tb, 16 * w, 16 * (w - 1), gq, t4);
+                } else {
+                    const int i0 = (w >> 1) * 32 + lane;  // 0 .. 63 over warps 0 and 2
+                    // diagonal blocks -> Tb (64 rows x two 8-column chunks)
+#pragma unroll
+                    for (int m = 0; m < 2; ++m) {
+                        const int q = i0 + 64 * m;
+                        const int row = q >> 1, ch = 2 * (row >> 4) + (q & 1);
+                        const float4 f0 = *reinterpret_cast<const float4*>(Tf + tf_idx(row, 8 * ch));
+                        const float4 f1 = *reinterpret_cast<const float4*>(Tf + tf_idx(row, 8 * ch + 4));
+                        *reinterpret_cast<uint4*>(Tb + swz(row, ch * 16, 64)) =
+                            make_uint4(pack_bf16x2(f0.x, f0.y), pack_bf16x2(f0.z, f0.w), pack_bf16x2(f1.x, f1.y),
+                                       pack_bf16x2(f1.z, f1.w));
+                    }
+                    // blocks above the diagonal are zero: rows 0-15 chunks 2-7, rows 16-31 chunks
+                    // 4-7, rows 32-47 chunks 6-7 (192 chunks)
+#pragma unroll
+                    for (int m = 0; m < 3; ++m) {
+                        const int q = i0 + 64 * m;
+                        int row, ch;
+                        if (q < 96) {
+                            row = q / 6;
+                            ch = 2 + q % 6;
+                        } else if (q < 160) {
+                            row = 16 + ((q - 96) >> 2);
+                            ch = 4 + ((q - 96) & 3);
+                        } else {
+                            row = 32 + ((q - 160) >> 1);
+                            ch = 6 + ((q - 160) & 1);
+                        }
+                        *reinterpret_cast<uint4*>(Tb + swz(row, ch * 16, 64)) = make_uint4(0u, 0u, 0u, 0u);
+                    }
+                }
                 group_sync(bar_id, GROUP);
                 const int mt = w >> 1, np = w & 1;
-                // Y_b = Nab_{b+1,b} D_b (b = 2w, warps 0-1) -> scratch rows 8b .. 8b+15, columns 32 .. 47
-                if (w < 2) tf32_tile16(Nr, 16 * (2 * w + 1), 32 * w, Tf, 32 * w, 32 * w, 0, 2, Tf, 16 * w, 32, gq, t4);
-                group_sync(bar_id, GROUP);
-                // T_{b+1,b} = D_{b+1} Y_b
-                if (w < 2)
-                    tf32_tile16(Tf, 16 * (2 * w + 1), 16 * (2 * w + 1), Tf, 16 * w, 32, 0, 2, Tf, 16 * (2 * w + 1), 32 * w, gq, t4);
-                group_sync(bar_id, GROUP);
                 // X = Nab_hl T_lo -> scratch rows 0 .. 31, columns 32 .. 63 (T_lo is zero in rows
                 // 0 .. 15 of columns 16 .. 31, so those columns start at k = 16)
-                tf32_tile16(Nr, 32 + 16 * mt, 0, Tf, 0, 16 * np, np ? 2 : 0, 4, Tf, 16 * mt, 32 + 16 * np, gq, t4);
+                tf32_tile16(Nr, 32 + 16 * mt, 0, Tf, 0, 16 * np, np ? 2 : 0, 4, Tf, nullptr, 16 * mt, 32 + 16 * np, gq, t4);
                 group_sync(bar_id, GROUP);
-                // T_hl = T_hi X (rows 32 .. 47 of T_hi are zero beyond column 47)
-                tf32_tile16(Tf, 32 + 16 * mt, 32, Tf, 0, 32 + 16 * np, 0, mt ? 4 : 2, Tf, 32 + 16 * mt, 16 * np, gq, t4);
-            }
-            group_sync(bar_id, GROUP);
-            // T -> bf16, MN-major (rows i, columns j); blocks above the diagonal are zero
-#pragma unroll
-            for (int m = 0; m < 4; ++m) {
-                const int qd = tg + 128 * m;
-                const int row = qd >> 3, ch = qd & 7;
-                uint4 val = make_uint4(0u, 0u, 0u, 0u);
-                if ((ch >> 1) <= (row >> 4)) {
-                    const float4 f0 = *reinterpret_cast<const float4*>(Tf + tf_idx(row, 8 * ch));
-                    const float4 f1 = *reinterpret_cast<const float4*>(Tf + tf_idx(row, 8 * ch + 4));
-                    val = make_uint4(pack_bf16x2(f0.x, f0.y), pack_bf16x2(f0.z, f0.w), pack_bf16x2(f1.x, f1.y),
-                                     pack_bf16x2(f1.z, f1.w));
-                }
-                *reinterpret_cast<uint4*>(Tb + swz(row, ch * 16, 64)) = val;
+                // T_hl = T_hi X -> Tb (rows 32 .. 47 of T_hi are zero beyond column 47)
+                tf32_tile16(Tf, 32 + 16 * mt, 32, Tf, 0, 32 + 16 * np, 0, mt ? 4 : 2, nullptr, Tb, 32 + 16 * mt, 16 * np,
+                            gq, t4);
             }
             fence_proxy_async_smem();
             group_sync(bar_id, GROUP);
