@@ -296,6 +296,12 @@ __global__ void __launch_bounds__(NTHR, 1)
             raw_issued = v_issued = 1;
         }
 
+        // matrix descriptors of K-step 0; K-step s adds 2 s (K-major) or 128 s (MN-major)
+        const uint64_t dRAM = kmajor_desc<false>(RAM, 128, 0), dBKt = kmajor_desc<false>(gt + OFF_NQ, 128, 0);
+        const uint64_t dBH = kmajor_desc<false>(BH, 128, 0), dMK = kmajor_desc<false>(MK, 128, 0);
+        const uint64_t dQt = kmajor_desc<false>(Qt, 128, 0);
+        const uint64_t dTb = mnmajor_desc<false>(Tb, 64, 0), dAZ = mnmajor_desc<false>(RAM + 8192, 64, 0);
+        const uint64_t dV = mnmajor_desc<false>(Vt, 64, 0);
         // p1 work split: thread (jp, tq) owns key channels 2jp, 2jp+1 of tokens 16tq .. 16tq+15
         const int jp = tg & 31, tq = tg >> 5, j0 = 2 * jp;
         const WT* rawl = reinterpret_cast<const WT*>(gt + RAW_L);
@@ -312,14 +318,7 @@ __global__ void __launch_bounds__(NTHR, 1)
 
             // ---- p1: decay products and the scaled operand tiles
             {
-                // the previous OUT product of this group (chunk c-2) must have read V, BH and MK
-                bool w_ok = true;
-                if (kk_ >= 1 && tg == 0) {
-                    w_ok = mbar_wait(&bars.ready[g], static_cast<uint32_t>(kk_ - 1) & 1u, WAIT_NS);
-                    if (w_ok) issue_v(c);
-                }
-                if (kk_ >= 1) ++v_issued;
-                if (tg == 0) w_ok = w_ok && mbar_wait(&bars.rl[g], static_cast<uint32_t>(kk_) & 1u, WAIT_NS);
+                const bool w_ok = (tg == 0) ? mbar_wait(&bars.rl[g], static_cast<uint32_t>(kk_) & 1u, WAIT_NS) : true;
                 ok = group_sync_and(bar_id, GROUP, w_ok);
                 if (!ok) break;
             }
@@ -341,10 +340,18 @@ __global__ void __launch_bounds__(NTHR, 1)
             red[tq * 64 + j0] = pw.x;
             red[tq * 64 + j0 + 1] = pw.y;
             {
+                // pass 2 rewrites BH and MK and V is reloaded: the previous OUT product of this
+                // group (chunk c-2) must have read them
                 bool w_ok = true;
-                if (tg == 0)
-                    w_ok = mbar_wait(&bars.rrk[g], static_cast<uint32_t>(kk_) & 1u, WAIT_NS) &&
+                if (tg == 0) {
+                    if (kk_ >= 1) {
+                        w_ok = mbar_wait(&bars.ready[g], static_cast<uint32_t>(kk_ - 1) & 1u, WAIT_NS);
+                        if (w_ok) issue_v(c);
+                    }
+                    w_ok = w_ok && mbar_wait(&bars.rrk[g], static_cast<uint32_t>(kk_) & 1u, WAIT_NS) &&
                            mbar_wait(&bars.rab[g], static_cast<uint32_t>(kk_) & 1u, WAIT_NS);
+                }
+                if (kk_ >= 1) ++v_issued;
                 ok = group_sync_and(bar_id, GROUP, w_ok);
                 if (!ok) break;
                 ++raw_done;
@@ -443,7 +450,7 @@ __global__ void __launch_bounds__(NTHR, 1)
                 tc_fence_after();
 #pragma unroll
                 for (uint32_t s = 0; s < 4; ++s)
-                    mma_ss<false>(tm_gp, kmajor_desc<false>(RAM, 128, s), kmajor_desc<false>(BKt, 128, s), ID_G16, s > 0);
+                    mma_ss<false>(tm_gp, dRAM + 2 * s, dBKt + 2 * s, ID_G16, s > 0);
                 mma_commit(&bars.mma[g]);
             }
             mma_pending = true;
@@ -579,7 +586,7 @@ __global__ void __launch_bounds__(NTHR, 1)
                 tc_fence_after();
 #pragma unroll
                 for (uint32_t s = 0; s < 4; ++s)
-                    mma_ss<false>(tm_q, kmajor_desc<false>(BH, 128, s), mnmajor_desc<false>(Tb, 64, s), ID_KM64, s > 0);
+                    mma_ss<false>(tm_q, dBH + 2 * s, dTb + 128 * s, ID_KM64, s > 0);
                 mma_commit(&bars.mma[g]);
             }
             mma_pending = true;
@@ -605,8 +612,7 @@ __global__ void __launch_bounds__(NTHR, 1)
                 tc_fence_after();
 #pragma unroll
                 for (uint32_t s = 0; s < 4; ++s)
-                    mma_ss<false>(tm_gp, kmajor_desc<false>(Qt, 128, s), mnmajor_desc<false>(RAM + 8192, 64, s),
-                                  ID_KM128, s > 0);
+                    mma_ss<false>(tm_gp, dQt + 2 * s, dAZ + 128 * s, ID_KM128, s > 0);
                 mma_commit(&bars.mma[g]);
             }
             // the shared [R'; Bh^T W] tile and this group's OUT columns are free once
@@ -661,10 +667,10 @@ __global__ void __launch_bounds__(NTHR, 1)
                 tc_fence_after();
 #pragma unroll
                 for (uint32_t s = 0; s < 4; ++s)
-                    mma_ss<false>(tm_out, kmajor_desc<false>(BH, 128, s), mnmajor_desc<false>(Vt, 64, s), ID_KM64, s > 0);
+                    mma_ss<false>(tm_out, dBH + 2 * s, dV + 128 * s, ID_KM64, s > 0);
 #pragma unroll
                 for (uint32_t s = 0; s < 4; ++s)
-                    mma_ss<false>(tm_out, kmajor_desc<false>(MK, 128, s), mnmajor_desc<false>(Vt, 64, s), ID_KM64, 1);
+                    mma_ss<false>(tm_out, dMK + 2 * s, dV + 128 * s, ID_KM64, 1);
                 mma_commit(&bars.ready[g]);
                 mbar_arrive(&bars.ready[g]);  // this chunk's [R'; Bh^T W] and Gamma_L are published
             }
@@ -689,6 +695,7 @@ __global__ void __launch_bounds__(NTHR, 1)
         const uint32_t bar_id = 3;
         uint8_t* St = sm + OFF_S;
         const float* gam_all = reinterpret_cast<const float*>(sm + OFF_GAMMA);
+        const uint64_t dAS = kmajor_desc<false>(sm + OFF_AS, 128, 0), dSt = mnmajor_desc<false>(St, 64, 0);
         float S[64];
         const int x = ts - 64;  // key channel owned by lanes 64..127
         if (ts >= 64) {
@@ -714,7 +721,7 @@ __global__ void __launch_bounds__(NTHR, 1)
             if (ts == 0) {
 #pragma unroll
                 for (uint32_t s = 0; s < 4; ++s)
-                    mma_ss<false>(tm_out, kmajor_desc<false>(AS, 128, s), mnmajor_desc<false>(St, 64, s), ID_KM64, 1);
+                    mma_ss<false>(tm_out, dAS + 2 * s, dSt + 128 * s, ID_KM64, 1);
                 mma_commit(bars.ser);
             }
             ser_pending = true;
