@@ -28,7 +28,9 @@
 // [R'; Bh^T W] tile that the serial group reads, which is shared.
 // Synchronisation: a prep group hands a chunk to the serial group through
 // `ready[g]` (MMA commit + release arrive); the serial group releases the
-// shared tile (and the group's OUT columns) through `free_` after each chunk.
+// shared tile (and the group's OUT columns) through `freeg[g]`, one barrier per
+// prep group so that no waiter can be two phases behind (a parity wait would
+// then return on the wrong phase).
 // Inputs arrive by TMA into tiles of the group that are dead at that point of
 // the previous chunk: w_log of chunk c + 2 into BK once T is built, r and k into
 // NQ once P has consumed Q, a and b into RAM once the conversion has read Rt; V
@@ -63,7 +65,7 @@ constexpr uint32_t OFF_S = OFF_AS + 16384;            // S^T bf16, 8 KB (serial 
 constexpr uint32_t OFF_GAMMA = OFF_S + 8192;          // Gamma_L [2 groups][2 slots][64] fp32
 constexpr uint32_t OFF_RED = OFF_GAMMA + 2 * 2 * 64 * 4;  // block products [2 groups][4][64] fp32
 constexpr uint32_t OFF_BAR = OFF_RED + 2 * 4 * 64 * 4;
-constexpr uint32_t SMEM_USED = OFF_BAR + 14 * 8 + 16;
+constexpr uint32_t SMEM_USED = OFF_BAR + 16 * 8 + 16;
 // raw TMA staging inside a group's tiles (dead at the time of the load)
 constexpr uint32_t RAW_R = OFF_NQ, RAW_K = OFF_NQ + 8192, RAW_A = OFF_RAM, RAW_B = OFF_RAM + 8192, RAW_L = OFF_BK;
 constexpr uint32_t SMEM_BYTES = SMEM_USED + 1024;      // alignment slack
@@ -159,7 +161,7 @@ __device__ __forceinline__ __nv_bfloat16 neg_inf_of<__nv_bfloat16>() { return __
 struct Bars {
     uint64_t* mma;    // [2] prep-group MMA completions (G, Q, P)
     uint64_t* ready;  // [2] OUT-pre complete and chunk tiles published (count 2)
-    uint64_t* free_;  // serial group done with a chunk (shared tile and OUT columns reusable)
+    uint64_t* freeg;  // [2] serial group done with a chunk of prep group g (shared tile, OUT columns)
     uint64_t* ser;    // serial MMA completion
     uint64_t* rl;     // [2] TMA of a group's raw w_log tile
     uint64_t* rrk;    // [2] TMA of a group's raw r, k tiles
@@ -187,13 +189,13 @@ __global__ void __launch_bounds__(NTHR, 1)
         uint64_t* p = reinterpret_cast<uint64_t*>(sm + OFF_BAR);
         bars.mma = p;
         bars.ready = p + 2;
-        bars.free_ = p + 4;  // one barrier
-        bars.ser = p + 5;
+        bars.ser = p + 4;
         bars.rl = p + 6;
         bars.rrk = p + 8;
         bars.rab = p + 10;
         bars.vld = p + 12;
-        bars.tmem_slot = reinterpret_cast<uint32_t*>(p + 14);
+        bars.freeg = p + 14;
+        bars.tmem_slot = reinterpret_cast<uint32_t*>(p + 16);
     }
 
     // ---- the unit and its tokens
@@ -225,8 +227,8 @@ __global__ void __launch_bounds__(NTHR, 1)
             mbar_init(&bars.rrk[g], 1);
             mbar_init(&bars.rab[g], 1);
             mbar_init(&bars.vld[g], 1);
+            mbar_init(&bars.freeg[g], 1);
         }
-        mbar_init(bars.free_, 1);
         mbar_init(bars.ser, 1);
         fence_mbar_init();
     }
@@ -622,7 +624,9 @@ __global__ void __launch_bounds__(NTHR, 1)
                 bool w1 = true;
                 if (tg == 0) {
                     w1 = mbar_wait(&bars.mma[g], mma_phase, WAIT_NS);
-                    if (c >= 1) w1 = w1 && mbar_wait(bars.free_, static_cast<uint32_t>(c - 1) & 1u, WAIT_NS);
+                    // chunk c - 1 belongs to the other group; it is that group's ((c - 1) >> 1)-th
+                    if (c >= 1)
+                        w1 = w1 && mbar_wait(&bars.freeg[(c - 1) & 1], static_cast<uint32_t>((c - 1) >> 1) & 1u, WAIT_NS);
                 }
                 ok = group_sync_and(bar_id, GROUP, w1);
             }
@@ -759,7 +763,7 @@ __global__ void __launch_bounds__(NTHR, 1)
             fence_proxy_async_smem();
             tc_fence_before();
             group_sync(bar_id, GROUP);
-            if (ts == 0) mbar_arrive(bars.free_);
+            if (ts == 0) mbar_arrive(&bars.freeg[g]);
         }
         if (!ok) {
             if (ts == 0) report_status(status, WKV7_ERR_DEVICE_TIMEOUT);
