@@ -44,6 +44,8 @@ def _load():
         lib.wkv7_oracle_forward.restype = ctypes.c_int
         lib.wkv7_oracle_decode_step.argtypes = [dp] * 9 + [ctypes.c_int] * 4
         lib.wkv7_oracle_decode_step.restype = ctypes.c_int
+        lib.wkv7_oracle_gate.argtypes = [dp] * 7 + [ctypes.c_long, ctypes.c_int, ctypes.c_int]
+        lib.wkv7_oracle_gate.restype = ctypes.c_int
         _lib = lib
     return _lib
 
@@ -114,3 +116,29 @@ def decode_step(r, w_log, k, v, a, b, s_in, n_threads=None):
     if rc != 0:
         raise RuntimeError(f"wkv7_oracle_decode_step failed with status {rc}")
     return y, s_out
+
+
+def gate(y, r, k, v, rk, g):
+    """Gated read-out z = (y / sqrt(D) + (sum_d r k rk) v) * g.  y, r, k, v, g
+    share one shape [..., H, D]; rk is [H, D].  Returns z as a float64 array."""
+    lib = _load()
+    y, r, k, v, g = (_f64(t) for t in (y, r, k, v, g))
+    rk = _f64(rk)
+    for t in (r, k, v, g):
+        if t.shape != y.shape:
+            raise ValueError("input shapes differ")
+    H, D = y.shape[-2], y.shape[-1]
+    if rk.shape != (H, D):
+        raise ValueError("rk must be [H, D]")
+    ntok = int(np.prod(y.shape[:-2])) if y.ndim > 2 else 1
+    z = np.empty_like(y)
+    rc = lib.wkv7_oracle_gate(_ptr(y), _ptr(r), _ptr(k), _ptr(v), _ptr(rk), _ptr(g), _ptr(z), ntok, H, D)
+    if rc != 0:
+        raise RuntimeError(f"wkv7_oracle_gate failed with status {rc}")
+    return z
+
+
+def forward_gated(r, w_log, k, v, a, b, rk, g, s0=None, seq_offsets=None, n_threads=None):
+    """The recurrence followed by the gated read-out.  Returns ``(z, sT)``."""
+    y, sT = forward(r, w_log, k, v, a, b, s0, seq_offsets, n_threads)
+    return gate(y, r, k, v, rk, g), sT

@@ -32,6 +32,17 @@
  *    variable length and padding"; here sequences are given by offsets into a
  *    packed token axis and each sequence starts from its own initial state.
  *
+ * Gated read-out (wkv7_oracle_gate), the steps the hxa07D forward listing
+ * applies to the WKV result before its output projection ("RWKV hxa07D
+ * architecture explainer", forward listing after the WKV call, and its section
+ * 9 on the scaling, the r-k-v term and the output gate):
+ *
+ *   u     = sum_d r_d k_d rk[h][d]                              (per token, head)
+ *   z_i   = (y_i / sqrt(D) + u v_i) g_i
+ *
+ * with y the recurrence output above, r, k, v the same inputs, rk a per-head
+ * vector and g the gate.
+ *
  * Layouts (all double, contiguous, the fastest index last):
  *  dense  (seq_offsets == NULL): r, w_log, k, v, a, b, y are [B][T][H][D]
  *  packed (seq_offsets != NULL): they are [T][H][D] with T the packed length and
@@ -188,4 +199,23 @@ int wkv7_oracle_decode_step(const double *r, const double *w_log, const double *
     /* a dense call with T = 1 whose initial and final state are the same buffer */
     return wkv7_oracle_forward(r, w_log, k, v, a, b, s_out, y, s_out, B, 1, H, D, NULL,
                                n_threads);
+}
+
+/*
+ * Gated read-out over `ntok` tokens of H heads: y, r, k, v, g, z are
+ * [ntok][H][D]; rk is [H][D].  z may alias y.  Returns 0, or -1 on bad sizes.
+ */
+int wkv7_oracle_gate(const double *y, const double *r, const double *k, const double *v,
+                     const double *rk, const double *g, double *z, long ntok, int H, int D) {
+    if (ntok < 0 || H <= 0 || D <= 0) return -1;
+    const double scale = 1.0 / sqrt((double)D);
+    for (long t = 0; t < ntok; ++t) {
+        for (int h = 0; h < H; ++h) {
+            const long base = (t * H + h) * (long)D;
+            double u = 0.0;
+            for (int d = 0; d < D; ++d) u += r[base + d] * k[base + d] * rk[(long)h * D + d];
+            for (int i = 0; i < D; ++i) z[base + i] = (y[base + i] * scale + u * v[base + i]) * g[base + i];
+        }
+    }
+    return 0;
 }

@@ -267,3 +267,33 @@ def test_invalid_arguments_rejected(oracle_mod):
         oracle_mod.forward(*flat, None, seq_offsets=np.array([0, 5], dtype=np.int32))
     with pytest.raises(RuntimeError):
         oracle_mod.forward(*flat, None, seq_offsets=np.array([0, 3, 2, 4], dtype=np.int32))
+
+
+def test_gated_readout_first_token_closed_form(oracle_mod):
+    """Gated read-out at the first token from a zero state: S_1 = v_1 k_1^T, so
+    y_1 = v_1 (k_1 . r_1) and z_1 = (v_1 (k_1 . r_1) / sqrt(D) + (sum_d r k rk) v_1) g_1.
+    Written from the closed form, not from the oracle's y; catches a missing
+    1/sqrt(D), an rk indexed by the wrong head, or the gate applied to one term
+    only."""
+    rng = np.random.default_rng(21)
+    B, T, H, D = 3, 1, 4, 64
+    r, w_log, k, v, a, b, _ = _rand_inputs(rng, B, T, H, D)
+    rk = rng.standard_normal((H, D))
+    g = rng.standard_normal((B, T, H, D))
+    z, _ = oracle_mod.forward_gated(r, w_log, k, v, a, b, rk, g)
+    kr = (k * r).sum(-1, keepdims=True)
+    u = (r * k * rk[None, None]).sum(-1, keepdims=True)
+    np.testing.assert_allclose(z, (v * kr / np.sqrt(D) + u * v) * g, rtol=0, atol=1e-12)
+
+
+def test_gated_readout_special_cases(oracle_mod):
+    """rk = 0 and g = 1 leave z = y / sqrt(D) (a plain rescaling of the
+    recurrence output); g = 0 gives z = 0 exactly."""
+    rng = np.random.default_rng(22)
+    B, T, H, D = 2, 9, 2, 64
+    r, w_log, k, v, a, b, S0 = _rand_inputs(rng, B, T, H, D)
+    y, _ = oracle_mod.forward(r, w_log, k, v, a, b, S0)
+    z, _ = oracle_mod.forward_gated(r, w_log, k, v, a, b, np.zeros((H, D)), np.ones_like(r), S0)
+    np.testing.assert_allclose(z, y / 8.0, rtol=1e-15, atol=0)
+    z0, _ = oracle_mod.forward_gated(r, w_log, k, v, a, b, rng.standard_normal((H, D)), np.zeros_like(r), S0)
+    assert np.all(z0 == 0.0)
