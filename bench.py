@@ -7,7 +7,9 @@ B4 T1024 H32 D64 prefill (bf16 inputs, fp32 decay logits, zero initial state),
 timed with CUDA events per launch on the launching stream, L2 flushed (a
 256 MB write) between timed launches.  `e2e` is the same metric through the
 public API from pinned host buffers (host->device copies of the inputs and
-device->host copies of y and sT inside the timed region).  `decode` reports
+device->host copies of y and sT inside the timed region).  `gated` times the
+same prefill with the gated read-out (wkv7_forward_gated, z instead of y; the
+gate adds its bf16 bytes to the roofline).  `decode` reports
 the B256 H40 decode step with the fp32 state carried through 128 steps.
 Multi-GPU: every rank runs the same per-GPU workload on its own device
 (independent (sequence, head) units, no collective on the data path); the job
@@ -248,6 +250,30 @@ def run_ours(args):
     achieved = bytes_alg / (ms * 1e-3) / 1e9
     flops = prefill_flops(B * T * H)
 
+    # ---------------- the same prefill with the gated read-out (wkv7_forward_gated)
+    rk_h, gate_h = W.make_gate(tuple(dev["r"].shape), H, D, io="bf16", seed=2 + 1000 * rank)
+    rk_d, gate_d = rk_h.cuda(), gate_h.cuda()
+    z = torch.empty_like(dev["r"])
+
+    def gstep():
+        wk.wkv7_forward_gated(dev["r"], dev["w_log"], dev["k"], dev["v"], dev["a"], dev["b"], None, rk_d, gate_d, z,
+                              sT, B, T, H, D, None, stream)
+
+    for _ in range(max(3, args.warmup)):
+        gstep()
+    torch.cuda.synchronize()
+    gtimes = time_launches(gstep, args.steps, stream, flush)
+    if wk.wkv7_get_device_status() != 0:
+        raise RuntimeError("device status set during the gated run")
+    gms = sum(gtimes) / len(gtimes)
+    if world > 1:
+        t = torch.tensor([gms], device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        gms = float(t.item())
+    gbytes = bytes_alg + B * T * H * D * 2 + H * D * 4  # + the bf16 gate and r_k
+    gach = gbytes / (gms * 1e-3) / 1e9
+    del z, gate_d
+
     # ---------------- end to end through the public API from pinned host memory
     y_h = torch.empty(y.shape, dtype=y.dtype).pin_memory()
     sT_h = torch.empty(sT.shape, dtype=sT.dtype).pin_memory()
@@ -322,6 +348,10 @@ def run_ours(args):
                     "ms_per_step": e2e_ms},
             "gpu_launches": args.steps,
             "clocks": clocks,
+            "gated": {"workload": PREFILL_WORKLOAD, "tokens_per_s": world * tokens / (gms * 1e-3),
+                      "ms_per_step": gms,
+                      "roofline": {"bound": "hbm", "achieved": gach, "peak": hbm_peak, "unit": "GB/s",
+                                   "frac": gach / hbm_peak, "algorithmic_bytes_per_launch": gbytes}},
             "decode": {"workload": DECODE_WORKLOAD, "B": dB, "H": dH, "steps_per_s": 1000.0 / dms,
                        "tokens_per_s": world * dB / (dms * 1e-3), "ms_per_step": dms,
                        "roofline": {"bound": "hbm", "achieved": dach, "peak": hbm_peak, "unit": "GB/s",

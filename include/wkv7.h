@@ -90,6 +90,28 @@ int wkv7_forward(const void* r, const void* w_log, const void* k, const void* v,
                  int io_dtype, int w_dtype, void* stream);
 
 /*
+ * wkv7_forward_gated — wkv7_forward followed by the read-out that the forward
+ * listing of "RWKV hxa07D architecture explainer" (zenn.dev/openmose) applies
+ * to the WKV result before its output projection (the lines after the WKV call;
+ * section 9 of that page: scaling, the r-k-v term, the output gate):
+ *
+ *     u_t = sum_d r_t[d] k_t[d] r_k[h][d]
+ *     z_t = (y_t / sqrt(D) + u_t v_t) (.) g_t          (per sequence, token, head)
+ *
+ * with y_t the WKV output of wkv7_forward, which is not written.
+ *   r_k : [H][D] fp32 per-head weights (DEVICE).
+ *   g   : gate, same shape and dtype code as r (DEVICE).
+ *   z   : output, same shape and dtype code as r; must not overlap any input.
+ * Every other argument, layout and rule as in wkv7_forward.  With bf16 inputs
+ * the read-out is applied to the output rows inside the prefill kernel; with
+ * fp32 inputs it runs as a second pass over z.
+ */
+int wkv7_forward_gated(const void* r, const void* w_log, const void* k, const void* v,
+                       const void* a, const void* b, const float* s0, const float* r_k,
+                       const void* g, void* z, float* sT, int B, int T, int H, int D,
+                       const int32_t* seq_offsets, int io_dtype, int w_dtype, void* stream);
+
+/*
  * wkv7_decode_step — one token per sequence (RNN mode).
  *   r, w_log, k, v, a, b, y : [B][H][D]
  *   s_in, s_out            : [B][H][D][D] fp32; s_in == s_out (in place) is

@@ -3,8 +3,8 @@ decode step behind a C ABI (``include/wkv7.h``, ``libwkv7.so``).
 
 The Python layer only marshals arguments to the CUDA library; importing the
 package loads ``libwkv7.so`` and fails loudly if it has not been built.
-Convenience wrappers ``forward`` and ``decode_step`` allocate outputs with
-torch and call the C entry points.
+Convenience wrappers ``forward``, ``forward_gated`` and ``decode_step``
+allocate outputs with torch and call the C entry points.
 """
 from __future__ import annotations
 
@@ -19,6 +19,7 @@ from ._binding import (  # noqa: F401
     wkv7_debug_expire_wait,
     wkv7_decode_step,
     wkv7_forward,
+    wkv7_forward_gated,
     wkv7_get_device_status,
     wkv7_status_string,
     wkv7_version,
@@ -42,6 +43,23 @@ def forward(r, w_log, k, v, a, b, s0=None, seq_offsets=None, want_state=True, st
     sT = torch.empty((B, H, D, D), dtype=torch.float32, device=r.device) if want_state else None
     wkv7_forward(r, w_log, k, v, a, b, s0, y, sT, B, T, H, D, seq_offsets, stream)
     return y, sT
+
+
+def forward_gated(r, w_log, k, v, a, b, r_k, g, s0=None, seq_offsets=None, want_state=True, stream=None):
+    """Chunked prefill with the gated read-out z = (y / sqrt(D) + (sum r k r_k) v) * g.
+    ``r_k`` is [H, D] fp32, ``g`` has the shape and dtype of ``r``.  Returns
+    ``(z, sT)``."""
+    import torch
+
+    if seq_offsets is not None:
+        T, H, D = r.shape
+        B = seq_offsets.numel() - 1
+    else:
+        B, T, H, D = r.shape
+    z = torch.empty_like(r)
+    sT = torch.empty((B, H, D, D), dtype=torch.float32, device=r.device) if want_state else None
+    wkv7_forward_gated(r, w_log, k, v, a, b, s0, r_k, g, z, sT, B, T, H, D, seq_offsets, stream)
+    return z, sT
 
 
 def decode_step(r, w_log, k, v, a, b, state, y=None, stream=None):

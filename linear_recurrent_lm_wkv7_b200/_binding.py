@@ -27,6 +27,7 @@ STATUS = {
 # every symbol include/wkv7.h declares
 EXPORTS = (
     "wkv7_forward",
+    "wkv7_forward_gated",
     "wkv7_decode_step",
     "wkv7_status_string",
     "wkv7_get_device_status",
@@ -54,6 +55,8 @@ def _lib():
         vp, i = ctypes.c_void_p, ctypes.c_int
         lib.wkv7_forward.argtypes = [vp] * 9 + [i] * 4 + [vp, i, i, vp]
         lib.wkv7_forward.restype = i
+        lib.wkv7_forward_gated.argtypes = [vp] * 11 + [i] * 4 + [vp, i, i, vp]
+        lib.wkv7_forward_gated.restype = i
         lib.wkv7_decode_step.argtypes = [vp] * 9 + [i] * 3 + [i, i, vp]
         lib.wkv7_decode_step.restype = i
         lib.wkv7_status_string.argtypes = [i]
@@ -106,6 +109,15 @@ def wkv7_forward(r, w_log, k, v, a, b, s0, y, sT, B, T, H, D, seq_offsets=None, 
         raise Wkv7Error(st, "wkv7_forward")
 
 
+def wkv7_forward_gated(r, w_log, k, v, a, b, s0, r_k, g, z, sT, B, T, H, D, seq_offsets=None, stream=None):
+    """Enqueue the prefill with the gated read-out (see include/wkv7.h)."""
+    st = _lib().wkv7_forward_gated(_ptr(r), _ptr(w_log), _ptr(k), _ptr(v), _ptr(a), _ptr(b), _ptr(s0), _ptr(r_k),
+                                   _ptr(g), _ptr(z), _ptr(sT), int(B), int(T), int(H), int(D), _ptr(seq_offsets),
+                                   _dtype_code(r), _dtype_code(w_log), _stream(stream))
+    if st != 0:
+        raise Wkv7Error(st, "wkv7_forward_gated")
+
+
 def wkv7_decode_step(r, w_log, k, v, a, b, s_in, y, s_out, B, H, D, stream=None):
     """Enqueue one decoding step (see include/wkv7.h)."""
     st = _lib().wkv7_decode_step(_ptr(r), _ptr(w_log), _ptr(k), _ptr(v), _ptr(a), _ptr(b), _ptr(s_in), _ptr(y),
@@ -136,6 +148,10 @@ def wkv7_version() -> int:
 def raw_call_forward(*args):
     """Direct C call with raw integer pointers (used by host-validation tests)."""
     return int(_lib().wkv7_forward(*args))
+
+
+def raw_call_forward_gated(*args):
+    return int(_lib().wkv7_forward_gated(*args))
 
 
 def raw_call_decode(*args):

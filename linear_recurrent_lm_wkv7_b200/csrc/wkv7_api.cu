@@ -83,15 +83,18 @@ const char* wkv7_status_string(int status) {
     }
 }
 
-int wkv7_forward(const void* r, const void* w_log, const void* k, const void* v, const void* a, const void* b,
-                 const float* s0, void* y, float* sT, int B, int T, int H, int D, const int32_t* seq_offsets,
-                 int io_dtype, int w_dtype, void* stream) {
+// wkv7_forward and wkv7_forward_gated; rk and g are null for the former.
+static int forward_impl(const void* r, const void* w_log, const void* k, const void* v, const void* a, const void* b,
+                        const float* s0, const float* rk, const void* g, void* y, float* sT, int B, int T, int H,
+                        int D, const int32_t* seq_offsets, int io_dtype, int w_dtype, void* stream) {
+    const bool gated = rk != nullptr;
     // ---- host-side validation; nothing is launched on failure
     if (B <= 0 || T < 0 || H <= 0 || D <= 0) return WKV7_ERR_INVALID_ARG;
     if (!dtype_ok(io_dtype) || !dtype_ok(w_dtype)) return WKV7_ERR_INVALID_ARG;
     if (D != wkv7::kHead) return WKV7_ERR_UNSUPPORTED;
     if (T > 0 && (!r || !w_log || !k || !v || !a || !b || !y)) return WKV7_ERR_INVALID_ARG;
-    const void* ptrs[] = {r, w_log, k, v, a, b, s0, y, sT, seq_offsets};
+    if (gated && T > 0 && !g) return WKV7_ERR_INVALID_ARG;
+    const void* ptrs[] = {r, w_log, k, v, a, b, s0, y, sT, seq_offsets, rk, g};
     for (const void* p : ptrs)
         if (p && !aligned16(p)) return WKV7_ERR_MISALIGNED;
     const long tokens = seq_offsets ? static_cast<long>(T) : static_cast<long>(B) * T;
@@ -103,6 +106,11 @@ int wkv7_forward(const void* r, const void* w_log, const void* k, const void* v,
         if (overlaps(y, n_act * io_b, p, n_act * io_b)) return WKV7_ERR_INVALID_ARG;
     if (overlaps(y, n_act * io_b, w_log, n_act * w_b) || overlaps(y, n_act * io_b, s0, n_state * 4) ||
         overlaps(y, n_act * io_b, sT, n_state * 4))
+        return WKV7_ERR_INVALID_ARG;
+    if (gated && (overlaps(y, n_act * io_b, g, n_act * io_b) ||
+                  overlaps(y, n_act * io_b, rk, static_cast<size_t>(H) * D * 4) ||
+                  overlaps(sT, n_state * 4, g, n_act * io_b) ||
+                  overlaps(sT, n_state * 4, rk, static_cast<size_t>(H) * D * 4)))
         return WKV7_ERR_INVALID_ARG;
     // sT == s0 is allowed: each (sequence, head) block reads its own initial state
     // before it writes its own final state.  Any other overlap is rejected.
@@ -126,8 +134,33 @@ int wkv7_forward(const void* r, const void* w_log, const void* k, const void* v,
     int* status = nullptr;
     if (status_ptr(&status) != WKV7_OK) return WKV7_ERR_CUDA;
     wkv7::PrefillArgs p{r, w_log, k, v, a, b, s0, y, sT, B, T, H, seq_offsets, status};
-    return wkv7::launch_prefill(p, io_dtype, w_dtype, st) == cudaSuccess ? WKV7_OK : WKV7_ERR_CUDA;
+    if (gated) {
+        p.rk = rk;
+        p.g = g;
+    }
+    if (wkv7::launch_prefill(p, io_dtype, w_dtype, st) != cudaSuccess) return WKV7_ERR_CUDA;
+    // the bf16 kernel writes the gated rows directly; the fp32 path applies the read-out in place
+    if (gated && io_dtype == WKV7_F32 &&
+        wkv7::launch_gate(y, r, k, v, rk, g, tokens, H, io_dtype, st) != cudaSuccess)
+        return WKV7_ERR_CUDA;
+    return WKV7_OK;
 }
+
+int wkv7_forward(const void* r, const void* w_log, const void* k, const void* v, const void* a, const void* b,
+                 const float* s0, void* y, float* sT, int B, int T, int H, int D, const int32_t* seq_offsets,
+                 int io_dtype, int w_dtype, void* stream) {
+    return forward_impl(r, w_log, k, v, a, b, s0, nullptr, nullptr, y, sT, B, T, H, D, seq_offsets, io_dtype,
+                        w_dtype, stream);
+}
+
+int wkv7_forward_gated(const void* r, const void* w_log, const void* k, const void* v, const void* a,
+                       const void* b, const float* s0, const float* r_k, const void* g, void* z, float* sT, int B,
+                       int T, int H, int D, const int32_t* seq_offsets, int io_dtype, int w_dtype, void* stream) {
+    if (!r_k) return WKV7_ERR_INVALID_ARG;
+    return forward_impl(r, w_log, k, v, a, b, s0, r_k, g, z, sT, B, T, H, D, seq_offsets, io_dtype, w_dtype,
+                        stream);
+}
+
 
 int wkv7_decode_step(const void* r, const void* w_log, const void* k, const void* v, const void* a, const void* b,
                      const float* s_in, void* y, float* s_out, int B, int H, int D, int io_dtype, int w_dtype,

@@ -1,5 +1,5 @@
 // wkv7_internal.cuh — launch interface between the C-ABI layer (wkv7_api.cu)
-// and the kernels (wkv7_decode.cu, wkv7_prefill.cu).  Not part of the ABI.
+// and the kernels (wkv7_decode.cu, wkv7_prefill*.cu, wkv7_gate.cu).  Not part of the ABI.
 #pragma once
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -25,6 +25,9 @@ struct PrefillArgs {
     int B, T, H;
     const int32_t* seq_offsets;
     int* status;  // device status word of the current device
+    // gated read-out (wkv7_forward_gated): y then holds z; both null otherwise
+    const float* rk = nullptr;  // [H][D] fp32
+    const void* g = nullptr;    // gate, same layout and dtype as r
 };
 
 struct DecodeArgs {
@@ -44,6 +47,9 @@ cudaError_t launch_prefill(const PrefillArgs& p, int io_dtype, int w_dtype, cuda
 // warp-specialised kernel for bf16 inputs (wkv7_prefill_pipe.cu)
 cudaError_t launch_prefill_pipe(const PrefillArgs& p, int w_dtype, cudaStream_t stream);
 cudaError_t launch_decode(const DecodeArgs& p, int io_dtype, int w_dtype, cudaStream_t stream);
+// z <- (z / sqrt(D) + (sum_d r k rk) v) * g in place over ntok x H rows (wkv7_gate.cu)
+cudaError_t launch_gate(void* z, const void* r, const void* k, const void* v, const float* rk, const void* g,
+                        long ntok, int H, int io_dtype, cudaStream_t stream);
 cudaError_t launch_expire_wait(int spins, int* status, cudaStream_t stream);
 
 // Records the first device-side error of a call sequence (first writer wins).

@@ -64,7 +64,8 @@ constexpr uint32_t OFF_AS = 2 * GROUP_TILES;          // [R'; Bh^T W] 16 KB, sha
 constexpr uint32_t OFF_S = OFF_AS + 16384;            // S^T bf16, 8 KB (serial group)
 constexpr uint32_t OFF_GAMMA = OFF_S + 8192;          // Gamma_L [2 groups][2 slots][64] fp32
 constexpr uint32_t OFF_RED = OFF_GAMMA + 2 * 2 * 64 * 4;  // block products [2 groups][4][64] fp32
-constexpr uint32_t OFF_BAR = OFF_RED + 2 * 4 * 64 * 4;
+constexpr uint32_t OFF_U = OFF_RED + 2 * 4 * 64 * 4;    // gated read-out: u [2 groups][2 slots][64] fp32
+constexpr uint32_t OFF_BAR = OFF_U + 2 * 2 * 64 * 4;
 constexpr uint32_t SMEM_USED = OFF_BAR + 16 * 8 + 16;
 // raw TMA staging inside a group's tiles (dead at the time of the load)
 constexpr uint32_t RAW_R = OFF_NQ, RAW_K = OFF_NQ + 8192, RAW_A = OFF_RAM, RAW_B = OFF_RAM + 8192, RAW_L = OFF_BK;
@@ -170,13 +171,16 @@ struct Bars {
     uint32_t* tmem_slot;
 };
 
-template <typename WT>
+// GATED: the output rows are z = (y / sqrt(D) + u v) (.) g with u = sum_d r k rk
+// (the read-out of wkv7_forward_gated) instead of y.
+template <typename WT, bool GATED>
 __global__ void __launch_bounds__(NTHR, 1)
     wkv7_prefill_pipe_kernel(const __nv_bfloat16* __restrict__ r, const WT* __restrict__ wl,
                              const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restrict__ v,
                              const __nv_bfloat16* __restrict__ a, const __nv_bfloat16* __restrict__ b,
                              const float* s0, __nv_bfloat16* __restrict__ y, float* sT, int T, int H,
                              const int32_t* __restrict__ seq_offsets, int* status,
+                             const float* __restrict__ rk, const __nv_bfloat16* __restrict__ gte,
                              const __grid_constant__ TmaMaps maps) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     // 1024-byte aligned base, derived from the shared array so that every tile pointer
@@ -306,6 +310,8 @@ __global__ void __launch_bounds__(NTHR, 1)
         const uint64_t dV = mnmajor_desc<false>(Vt, 64, 0);
         // p1 work split: thread (jp, tq) owns key channels 2jp, 2jp+1 of tokens 16tq .. 16tq+15
         const int jp = tg & 31, tq = tg >> 5, j0 = 2 * jp;
+        float2 rkv = make_float2(0.f, 0.f);  // rk of key channels j0, j0 + 1 (gated read-out)
+        if constexpr (GATED) rkv = make_float2(rk[h * kHead + j0], rk[h * kHead + j0 + 1]);
         const WT* rawl = reinterpret_cast<const WT*>(gt + RAW_L);
         WT* rawl_w = reinterpret_cast<WT*>(gt + RAW_L);
         uint8_t* BKt = gt + OFF_NQ;  // [Bt; Kt], written over the raw r, k rows
@@ -405,6 +411,7 @@ __global__ void __launch_bounds__(NTHR, 1)
                     }
                     __syncwarp();
                     uint32_t bh0[4], bh1[4], kh0[4], kh1[4];  // 8 tokens of Bh^T / Kh^T rows j0, j0 + 1
+                    float pd[8];                              // this thread's part of u for 8 tokens
 #pragma unroll
                     for (int e = 0; e < 8; ++e) {
                         const int t = t0 + e;
@@ -418,6 +425,7 @@ __global__ void __launch_bounds__(NTHR, 1)
                         const float2 l = __fmul2_rn(iv, GL);
                         const float2 rf = unpack_bf16x2(rr[e]), kf = unpack_bf16x2(kv[e]);
                         const float2 af = unpack_bf16x2(av[e]), bf = unpack_bf16x2(bv[e]);
+                        if constexpr (GATED) pd[e] = rf.x * kf.x * rkv.x + rf.y * kf.y * rkv.y;
                         *reinterpret_cast<uint32_t*>(RAM + swz(t, cb, 128)) = pack2(__fmul2_rn(rf, G));
                         *reinterpret_cast<uint32_t*>(RAM + swz(64 + t, cb, 128)) = pack2(__fmul2_rn(af, gp));
                         *reinterpret_cast<uint32_t*>(BKt + swz(t, cb, 128)) = pack2(__fmul2_rn(bf, iv));
@@ -435,6 +443,24 @@ __global__ void __launch_bounds__(NTHR, 1)
                             kh1[e >> 1] = pack_bf16x2(__uint_as_float(kh1[e >> 1]), khv.y);
                         }
                         gp = G;
+                    }
+                    if constexpr (GATED) {
+                        // u of the 8 tokens: the warp's 32 lanes cover the 64 key channels.  A
+                        // reduce-scatter over lane bits 4, 3, 2 leaves token (lane >> 2) & 7 in
+                        // lanes 4m .. 4m + 3, and two more steps complete the sum.
+                        const bool b4 = (jp & 16) != 0, b3 = (jp & 8) != 0, b2 = (jp & 4) != 0;
+                        float q4[4], q2[2];
+#pragma unroll
+                        for (int i = 0; i < 4; ++i)
+                            q4[i] = (b4 ? pd[4 + i] : pd[i]) + __shfl_xor_sync(0xffffffffu, b4 ? pd[i] : pd[4 + i], 16);
+#pragma unroll
+                        for (int i = 0; i < 2; ++i)
+                            q2[i] = (b3 ? q4[2 + i] : q4[i]) + __shfl_xor_sync(0xffffffffu, b3 ? q4[i] : q4[2 + i], 8);
+                        float q1 = (b2 ? q2[1] : q2[0]) + __shfl_xor_sync(0xffffffffu, b2 ? q2[0] : q2[1], 4);
+                        q1 += __shfl_xor_sync(0xffffffffu, q1, 2);
+                        q1 += __shfl_xor_sync(0xffffffffu, q1, 1);
+                        if ((jp & 3) == 0)
+                            reinterpret_cast<float*>(sm + OFF_U)[g * 128 + (kk_ & 1) * 64 + t0 + ((jp >> 2) & 7)] = q1;
                     }
                     const uint32_t tb8 = static_cast<uint32_t>(t0) * 2u;  // byte of the first token
                     *reinterpret_cast<uint4*>(BH + swz(64 + j0, tb8, 128)) = make_uint4(bh0[0], bh0[1], bh0[2], bh0[3]);
@@ -717,7 +743,18 @@ __global__ void __launch_bounds__(NTHR, 1)
             const long row0 = tb + static_cast<long>(c) * L;
             const int nv = static_cast<int>(len - static_cast<long>(c) * L < L ? len - static_cast<long>(c) * L : L);
             const uint32_t tm_out = tmem + 256u * g + TM_OUT;
-            uint8_t* AS = sm + OFF_AS;
+            // gated read-out: this token row's v and g, fetched before waiting for the chunk
+            uint4 vpre[8], gpre[8];
+            if constexpr (GATED) {
+                if (ts < nv) {
+                    const long off = (row0 + ts) * tstride + hoff;
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                        vpre[i] = *reinterpret_cast<const uint4*>(v + off + 8 * i);
+                        gpre[i] = *reinterpret_cast<const uint4*>(gte + off + 8 * i);
+                    }
+                }
+            }
             ok = group_sync_and(bar_id, GROUP,
                                 ts == 0 ? mbar_wait(&bars.ready[g], static_cast<uint32_t>(kk_) & 1u, WAIT_NS) : true);
             if (!ok) break;
@@ -737,11 +774,28 @@ __global__ void __launch_bounds__(NTHR, 1)
             float o[32];
             if (ts < 64) {
                 const int t = ts;
-#pragma unroll 1
+                float uu = 0.f;
+                if constexpr (GATED) uu = reinterpret_cast<const float*>(sm + OFF_U)[g * 128 + (kk_ & 1) * 64 + t];
+#pragma unroll(GATED ? 2 : 1)
                 for (int q = 0; q < 2; ++q) {
                     tmem_load32(tm_out + lane_base + 32 * q, o);
                     if (t < nv) {
-                        __nv_bfloat16* dst = y + (row0 + t) * tstride + hoff + 32 * q;
+                        const long off = (row0 + t) * tstride + hoff + 32 * q;
+                        if constexpr (GATED) {
+                            // z = (y / sqrt(D) + u v) (.) g, with v and g of this token row
+#pragma unroll
+                            for (int i = 0; i < 32; i += 8) {
+                                const uint4 vq = vpre[4 * q + i / 8], gq4 = gpre[4 * q + i / 8];
+                                const uint32_t vw[4] = {vq.x, vq.y, vq.z, vq.w}, gw[4] = {gq4.x, gq4.y, gq4.z, gq4.w};
+#pragma unroll
+                                for (int m = 0; m < 4; ++m) {
+                                    const float2 vf = unpack_bf16x2(vw[m]), gf = unpack_bf16x2(gw[m]);
+                                    o[i + 2 * m] = (o[i + 2 * m] * 0.125f + uu * vf.x) * gf.x;
+                                    o[i + 2 * m + 1] = (o[i + 2 * m + 1] * 0.125f + uu * vf.y) * gf.y;
+                                }
+                            }
+                        }
+                        __nv_bfloat16* dst = y + off;
 #pragma unroll
                         for (int i = 0; i < 32; i += 8)
                             *reinterpret_cast<uint4*>(dst + i) =
@@ -782,9 +836,9 @@ __global__ void __launch_bounds__(NTHR, 1)
     }
 }
 
-template <typename WT>
+template <typename WT, bool GATED>
 cudaError_t launch_pipe_typed(const PrefillArgs& p, cudaStream_t stream) {
-    auto kern = wkv7_prefill_pipe_kernel<WT>;
+    auto kern = wkv7_prefill_pipe_kernel<WT, GATED>;
     static unsigned long long configured = 0;
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
@@ -803,14 +857,19 @@ cudaError_t launch_pipe_typed(const PrefillArgs& p, cudaStream_t stream) {
         static_cast<const __nv_bfloat16*>(p.r), static_cast<const WT*>(p.w_log),
         static_cast<const __nv_bfloat16*>(p.k), static_cast<const __nv_bfloat16*>(p.v),
         static_cast<const __nv_bfloat16*>(p.a), static_cast<const __nv_bfloat16*>(p.b), p.s0,
-        static_cast<__nv_bfloat16*>(p.y), p.sT, p.T, p.H, p.seq_offsets, p.status, maps);
+        static_cast<__nv_bfloat16*>(p.y), p.sT, p.T, p.H, p.seq_offsets, p.status, p.rk,
+        static_cast<const __nv_bfloat16*>(p.g), maps);
     return cudaGetLastError();
 }
 
 }  // namespace
 
 cudaError_t launch_prefill_pipe(const PrefillArgs& p, int w_dtype, cudaStream_t stream) {
-    return w_dtype == WKV7_BF16 ? launch_pipe_typed<__nv_bfloat16>(p, stream) : launch_pipe_typed<float>(p, stream);
+    if (p.rk)
+        return w_dtype == WKV7_BF16 ? launch_pipe_typed<__nv_bfloat16, true>(p, stream)
+                                    : launch_pipe_typed<float, true>(p, stream);
+    return w_dtype == WKV7_BF16 ? launch_pipe_typed<__nv_bfloat16, false>(p, stream)
+                                : launch_pipe_typed<float, false>(p, stream);
 }
 
 }  // namespace wkv7

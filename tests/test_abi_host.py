@@ -92,3 +92,24 @@ def test_oracle_and_library_share_no_code():
         assert "oracle" not in open(os.path.join(csrc, f)).read().lower(), f
     for f in ("__init__.py", "_binding.py", "build.py"):
         assert "oracle" not in open(os.path.join(ROOT, "linear_recurrent_lm_wkv7_b200", f)).read(), f
+
+
+# argument tuple for wkv7_forward_gated: 11 pointers, B, T, H, D, offsets, io, w, stream
+def _fwd_gated(ptr=0x1000, B=1, T=8, H=1, D=64, offs=None, io=1, wd=0, **over):
+    p = dict(r=ptr, w=ptr + 0x100000, k=ptr + 0x200000, v=ptr + 0x300000, a=ptr + 0x400000, b=ptr + 0x500000,
+             s0=None, rk=ptr + 0x700000, g=ptr + 0x800000, z=ptr + 0x600000, sT=None)
+    p.update(over)
+    return (p["r"], p["w"], p["k"], p["v"], p["a"], p["b"], p["s0"], p["rk"], p["g"], p["z"], p["sT"], B, T, H, D,
+            offs, io, wd, None)
+
+
+def test_forward_gated_rejects_bad_arguments(wk):
+    call = wk._binding.raw_call_forward_gated
+    assert call(*_fwd_gated(rk=None)) == -1  # r_k is required
+    assert call(*_fwd_gated(g=None)) == -1  # so is the gate
+    assert call(*_fwd_gated(D=32)) == -2
+    assert call(*_fwd_gated(g=0x1008 + 0x800000)) == -3  # misaligned gate
+    assert call(*_fwd_gated(rk=0x1004 + 0x700000)) == -3  # misaligned r_k
+    assert call(*_fwd_gated(z=0x1000 + 0x800000)) == -1  # z aliases g
+    assert call(*_fwd_gated(z=0x1000 + 0x700000)) == -1  # z overlaps r_k
+    assert call(*_fwd_gated(z=0x1000)) == -1  # z aliases r

@@ -14,6 +14,8 @@ order r, k, v, kappa, a_lr logit, decay logit, s0):
 * log_neglog_w = -softplus(-z) - 0.5 with z ~ N(mu_z, 1), so that
   w = exp(-exp(log_neglog_w)) lies in (exp(-exp(-0.5)), 1) ~= (0.545, 1)
 * s0 ~ N(0, s0_std^2) in fp32 when an initial state is requested
+* gated read-out (make_gate, its own generator): r_k ~ N(0, rk_std^2) [H, D]
+  fp32, gate g ~ N(0, 1) in the io dtype
 * packed batches: lengths ~ U{len_lo..len_hi} and pad counts ~ U{0..pad_hi};
   pad tokens carry log_neglog_w = -inf (w = 1) and k = v = a = b = 0, so they
   leave the state unchanged; r stays drawn at pads.
@@ -107,6 +109,15 @@ def make_packed(lengths, pads, H, D=64, io="bf16", wdt="f32", s0_std=0.1, mu_z=0
     seq_offsets = torch.tensor(offs, dtype=torch.int32)
     return PrefillInputs(r, w_log, k, v, a, b, s0, seq_offsets, B, T_total, H, D, io, wdt,
                          sum(lengths), lengths, pads)
+
+
+def make_gate(shape, H, D=64, io="bf16", rk_std=0.5, seed=0):
+    """Inputs of the gated read-out: per-head weights r_k [H, D] fp32 ~ N(0, rk_std^2)
+    and a gate of the given activation shape ~ N(0, 1), rounded to the io dtype."""
+    g = torch.Generator().manual_seed(seed)
+    rk = (torch.randn((H, D), generator=g) * rk_std).contiguous()
+    gate = torch.randn(tuple(shape), generator=g).to(_DT[io]).contiguous()
+    return rk, gate
 
 
 def draw_lengths(n_seq, len_lo, len_hi, pad_hi, seed):
