@@ -187,8 +187,10 @@ int wkv7_decode_step(const void* r, const void* w_log, const void* k, const void
 
     int dev_ok = cached_device_check();
     if (dev_ok != WKV7_OK) return dev_ok;
+    int* status = nullptr;
+    if (status_ptr(&status) != WKV7_OK) return WKV7_ERR_CUDA;
     wkv7::DecodeArgs p{r, w_log, k, v, a, b, s_in, y, s_out, B, H};
-    return wkv7::launch_decode(p, io_dtype, w_dtype, static_cast<cudaStream_t>(stream)) == cudaSuccess
+    return wkv7::launch_decode(p, io_dtype, w_dtype, status, static_cast<cudaStream_t>(stream)) == cudaSuccess
                ? WKV7_OK
                : WKV7_ERR_CUDA;
 }

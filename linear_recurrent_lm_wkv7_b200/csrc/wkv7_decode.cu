@@ -8,31 +8,45 @@
 //   S_ij <- S_ij w_j + sa_i b_j + v_i k_j (w_j = exp(-exp(w_log_j)))
 //   y_i  = sum_j S_ij r_j                 (updated state)
 //
-// Mapping: one 256-thread block per unit.  A thread owns 4 consecutive key
-// columns (one 16-byte vector) of 4 value rows spaced 16 apart; 16 threads
-// cover one row, so both row reductions are 4 xor-shuffles inside a 16-lane
-// group.  All four 16-byte state loads are issued before any arithmetic, the
-// state is read and written with streaming (evict-first) accesses, and a block
-// moves 32 KB of state, so an SM keeps ~128 KB of loads in flight.
+// Streaming: a persistent grid of two 256-thread blocks per SM.  A block walks
+// over units u = blockIdx.x, blockIdx.x + gridDim.x, ... through a ring of four
+// shared-memory stages.  Each stage receives one unit's 16 KB state and its six
+// input rows by untiled bulk copies (one mbarrier per stage); the block updates
+// the state in place in shared memory and writes it back with one bulk store,
+// while the copies for the next three units are in flight.  A stage is
+// refilled only after the bulk store that reads it has finished reading.
+//
+// Thread mapping inside a unit: a thread owns 4 consecutive key columns (one
+// 16-byte vector) of 4 value rows spaced 16 apart; 16 threads cover one row,
+// so both row reductions are 4 xor-shuffles inside a 16-lane group.
+#include "sm100_ptx.cuh"
 #include "wkv7_internal.cuh"
 
 namespace wkv7 {
 namespace {
 
+constexpr int NST = 4;                        // pipeline stages per block
+constexpr uint32_t ST_STATE = kHead * kHead * 4;  // 16 KB fp32 state
+constexpr uint32_t ST_BYTES = ST_STATE + 2048;    // + six input rows (at most 6 x 256 B)
+constexpr uint32_t SMEM_BYTES = NST * ST_BYTES + NST * 8;
+constexpr uint64_t WAIT_NS = 1000000000ull;  // 1 s
+
 template <typename T>
-__device__ __forceinline__ void load4(const T* p, float (&o)[4]);
+__device__ __forceinline__ void lds4(const uint8_t* p, float (&o)[4]);
 template <>
-__device__ __forceinline__ void load4<float>(const float* p, float (&o)[4]) {
-    const float4 x = __ldg(reinterpret_cast<const float4*>(p));
+__device__ __forceinline__ void lds4<float>(const uint8_t* p, float (&o)[4]) {
+    const float4 x = *reinterpret_cast<const float4*>(p);
     o[0] = x.x; o[1] = x.y; o[2] = x.z; o[3] = x.w;
 }
 template <>
-__device__ __forceinline__ void load4<__nv_bfloat16>(const __nv_bfloat16* p, float (&o)[4]) {
-    const uint2 x = __ldg(reinterpret_cast<const uint2*>(p));
-    const __nv_bfloat162 lo = *reinterpret_cast<const __nv_bfloat162*>(&x.x);
-    const __nv_bfloat162 hi = *reinterpret_cast<const __nv_bfloat162*>(&x.y);
-    const float2 fl = __bfloat1622float2(lo), fh = __bfloat1622float2(hi);
-    o[0] = fl.x; o[1] = fl.y; o[2] = fh.x; o[3] = fh.y;
+__device__ __forceinline__ void lds4<__nv_bfloat16>(const uint8_t* p, float (&o)[4]) {
+    const uint2 x = *reinterpret_cast<const uint2*>(p);
+    o[0] = __uint_as_float(x.x << 16); o[1] = __uint_as_float(x.x & 0xFFFF0000u);
+    o[2] = __uint_as_float(x.y << 16); o[3] = __uint_as_float(x.y & 0xFFFF0000u);
+}
+template <typename T>
+__device__ __forceinline__ float lds1(const uint8_t* p, int i) {
+    return to_f32(reinterpret_cast<const T*>(p)[i]);
 }
 
 __device__ __forceinline__ float sum16(float x) {
@@ -44,71 +58,135 @@ __device__ __forceinline__ float sum16(float x) {
 }
 
 template <typename IO, typename WT>
-__global__ void __launch_bounds__(256) wkv7_decode_kernel(const IO* __restrict__ r, const WT* __restrict__ wl,
-                                                          const IO* __restrict__ k, const IO* __restrict__ v,
-                                                          const IO* __restrict__ a, const IO* __restrict__ b,
-                                                          const float* s_in, IO* __restrict__ y, float* s_out) {
-    const long unit = blockIdx.x;
+__global__ void __launch_bounds__(256, 2)
+    wkv7_decode_kernel(const IO* __restrict__ r, const WT* __restrict__ wl, const IO* __restrict__ k,
+                       const IO* __restrict__ v, const IO* __restrict__ a, const IO* __restrict__ b,
+                       const float* s_in, IO* __restrict__ y, float* s_out, long units, int* status) {
+    extern __shared__ __align__(128) uint8_t smem[];
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + NST * ST_BYTES);
     const int tid = threadIdx.x;
     const int cg = tid & 15;  // key columns 4*cg .. 4*cg+3
     const int rg = tid >> 4;  // value rows rg, rg+16, rg+32, rg+48
-    const long vbase = unit * kHead;
-    const long sbase = unit * kHead * kHead;
+    constexpr uint32_t IOB = sizeof(IO) * kHead, WB = sizeof(WT) * kHead;
+    constexpr uint32_t O_R = ST_STATE, O_K = O_R + IOB, O_V = O_K + IOB, O_A = O_V + IOB, O_B = O_A + IOB,
+                       O_W = O_B + IOB;
+    const uint32_t tx = (s_in ? ST_STATE : 0u) + 5u * IOB + WB;
 
-    float4 s[4];
-    if (s_in) {
-#pragma unroll
-        for (int q = 0; q < 4; ++q)
-            s[q] = __ldcs(reinterpret_cast<const float4*>(s_in + sbase + (rg + 16 * q) * kHead + 4 * cg));
-    } else {
-#pragma unroll
-        for (int q = 0; q < 4; ++q) s[q] = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (tid == 0) {
+        for (int i = 0; i < NST; ++i) mbar_init(&full[i], 1);
+        fence_mbar_init();
     }
-    float wv[4], av[4], bv[4], kv[4], rv[4];
-    load4(wl + vbase + 4 * cg, wv);
-    load4(a + vbase + 4 * cg, av);
-    load4(b + vbase + 4 * cg, bv);
-    load4(k + vbase + 4 * cg, kv);
-    load4(r + vbase + 4 * cg, rv);
-#pragma unroll
-    for (int c = 0; c < 4; ++c) wv[c] = expf(-expf(wv[c]));
-    float vrow[4];
-#pragma unroll
-    for (int q = 0; q < 4; ++q) vrow[q] = to_f32(v[vbase + rg + 16 * q]);
+    __syncthreads();
 
+    const long first = blockIdx.x, stride = gridDim.x;
+    const long nmine = first < units ? (units - first + stride - 1) / stride : 0;
+    long n_issued = 0;  // thread 0: units whose copies were issued
+    auto issue = [&](long j) {
+        const long u = first + j * stride;
+        uint8_t* base = smem + (j % NST) * ST_BYTES;
+        uint64_t* bar = &full[j % NST];
+        mbar_arrive_expect_tx(bar, tx);
+        if (s_in) bulk_load(base, s_in + u * (kHead * kHead), ST_STATE, bar);
+        bulk_load(base + O_R, r + u * kHead, IOB, bar);
+        bulk_load(base + O_K, k + u * kHead, IOB, bar);
+        bulk_load(base + O_V, v + u * kHead, IOB, bar);
+        bulk_load(base + O_A, a + u * kHead, IOB, bar);
+        bulk_load(base + O_B, b + u * kHead, IOB, bar);
+        bulk_load(base + O_W, wl + u * kHead, WB, bar);
+        ++n_issued;
+    };
+    if (tid == 0)
+        for (long j = 0; j < NST && j < nmine; ++j) issue(j);
+
+    long j = 0;
+    bool ok = true;
+    for (; j < nmine; ++j) {
+        const long u = first + j * stride;
+        uint8_t* base = smem + (j % NST) * ST_BYTES;
+        const bool w_ok = mbar_wait(&full[j % NST], static_cast<uint32_t>(j / NST) & 1u, WAIT_NS);
+        if (!__syncthreads_and(w_ok)) {
+            ok = false;
+            break;
+        }
+        float wv[4], av[4], bv[4], kv[4], rv[4], vrow[4];
+        lds4<WT>(base + O_W + 4 * cg * sizeof(WT), wv);
+        lds4<IO>(base + O_A + 4 * cg * sizeof(IO), av);
+        lds4<IO>(base + O_B + 4 * cg * sizeof(IO), bv);
+        lds4<IO>(base + O_K + 4 * cg * sizeof(IO), kv);
+        lds4<IO>(base + O_R + 4 * cg * sizeof(IO), rv);
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
-        float4 x = s[q];
-        const float sa = sum16(x.x * av[0] + x.y * av[1] + x.z * av[2] + x.w * av[3]);
-        const float vi = vrow[q];
-        x.x = fmaf(x.x, wv[0], fmaf(sa, bv[0], vi * kv[0]));
-        x.y = fmaf(x.y, wv[1], fmaf(sa, bv[1], vi * kv[1]));
-        x.z = fmaf(x.z, wv[2], fmaf(sa, bv[2], vi * kv[2]));
-        x.w = fmaf(x.w, wv[3], fmaf(sa, bv[3], vi * kv[3]));
-        const float yi = sum16(x.x * rv[0] + x.y * rv[1] + x.z * rv[2] + x.w * rv[3]);
-        __stcs(reinterpret_cast<float4*>(s_out + sbase + (rg + 16 * q) * kHead + 4 * cg), x);
-        if (cg == 0) y[vbase + rg + 16 * q] = from_f32<IO>(yi);
+        for (int q = 0; q < 4; ++q) vrow[q] = lds1<IO>(base + O_V, rg + 16 * q);
+#pragma unroll
+        for (int c = 0; c < 4; ++c) wv[c] = expf(-expf(wv[c]));
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            float4* sp = reinterpret_cast<float4*>(base + ((rg + 16 * q) * kHead + 4 * cg) * 4);
+            float4 x = s_in ? *sp : make_float4(0.f, 0.f, 0.f, 0.f);
+            const float sa = sum16(x.x * av[0] + x.y * av[1] + x.z * av[2] + x.w * av[3]);
+            const float vi = vrow[q];
+            x.x = fmaf(x.x, wv[0], fmaf(sa, bv[0], vi * kv[0]));
+            x.y = fmaf(x.y, wv[1], fmaf(sa, bv[1], vi * kv[1]));
+            x.z = fmaf(x.z, wv[2], fmaf(sa, bv[2], vi * kv[2]));
+            x.w = fmaf(x.w, wv[3], fmaf(sa, bv[3], vi * kv[3]));
+            const float yi = sum16(x.x * rv[0] + x.y * rv[1] + x.z * rv[2] + x.w * rv[3]);
+            *sp = x;
+            if (cg == 0) y[u * kHead + rg + 16 * q] = from_f32<IO>(yi);
+        }
+        fence_proxy_async_smem();  // the updated state is read by the bulk store (async proxy)
+        __syncthreads();
+        if (tid == 0) {
+            bulk_store(s_out + u * (kHead * kHead), base, ST_STATE);
+            bulk_commit();
+            if (j >= 1) {
+                bulk_wait_read<1>();  // unit j-1's store has finished reading its stage
+                if (j - 1 + NST < nmine) issue(j - 1 + NST);
+            }
+        }
+    }
+    if (tid == 0) {
+        if (!ok) {
+            report_status(status, WKV7_ERR_DEVICE_TIMEOUT);
+            for (long m = j; m < n_issued; ++m)  // copies still landing in shared memory
+                mbar_wait(&full[m % NST], static_cast<uint32_t>(m / NST) & 1u, WAIT_NS);
+        }
+        bulk_wait_all();  // every state store has completed
     }
 }
 
 template <typename IO, typename WT>
-cudaError_t launch_typed(const DecodeArgs& p, cudaStream_t stream) {
+cudaError_t launch_typed(const DecodeArgs& p, int* status, cudaStream_t stream) {
+    auto kern = wkv7_decode_kernel<IO, WT>;
+    static unsigned long long configured = 0;
+    static int sm_count[64] = {};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    const unsigned long long bit = 1ull << (dev & 63);
+    if (!(configured & bit)) {
+        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+        if (e != cudaSuccess) return e;
+        e = cudaDeviceGetAttribute(&sm_count[dev & 63], cudaDevAttrMultiProcessorCount, dev);
+        if (e != cudaSuccess) return e;
+        configured |= bit;
+    }
     const long units = static_cast<long>(p.B) * p.H;
-    wkv7_decode_kernel<IO, WT><<<static_cast<unsigned>(units), 256, 0, stream>>>(
+    const long grid = units < 2L * sm_count[dev & 63] ? units : 2L * sm_count[dev & 63];
+    kern<<<static_cast<unsigned>(grid), 256, SMEM_BYTES, stream>>>(
         static_cast<const IO*>(p.r), static_cast<const WT*>(p.w_log), static_cast<const IO*>(p.k),
         static_cast<const IO*>(p.v), static_cast<const IO*>(p.a), static_cast<const IO*>(p.b), p.s_in,
-        static_cast<IO*>(p.y), p.s_out);
+        static_cast<IO*>(p.y), p.s_out, units, status);
     return cudaGetLastError();
 }
 
 }  // namespace
 
-cudaError_t launch_decode(const DecodeArgs& p, int io_dtype, int w_dtype, cudaStream_t stream) {
+cudaError_t launch_decode(const DecodeArgs& p, int io_dtype, int w_dtype, int* status, cudaStream_t stream) {
     if (io_dtype == WKV7_BF16) {
-        return w_dtype == WKV7_BF16 ? launch_typed<__nv_bfloat16, __nv_bfloat16>(p, stream)
-                                    : launch_typed<__nv_bfloat16, float>(p, stream);
+        return w_dtype == WKV7_BF16 ? launch_typed<__nv_bfloat16, __nv_bfloat16>(p, status, stream)
+                                    : launch_typed<__nv_bfloat16, float>(p, status, stream);
     }
-    return w_dtype == WKV7_BF16 ? launch_typed<float, __nv_bfloat16>(p, stream) : launch_typed<float, float>(p, stream);
+    return w_dtype == WKV7_BF16 ? launch_typed<float, __nv_bfloat16>(p, status, stream)
+                                : launch_typed<float, float>(p, status, stream);
 }
 
 }  // namespace wkv7

@@ -46,7 +46,7 @@ struct DecodeArgs {
 cudaError_t launch_prefill(const PrefillArgs& p, int io_dtype, int w_dtype, cudaStream_t stream);
 // warp-specialised kernel for bf16 inputs (wkv7_prefill_pipe.cu)
 cudaError_t launch_prefill_pipe(const PrefillArgs& p, int w_dtype, cudaStream_t stream);
-cudaError_t launch_decode(const DecodeArgs& p, int io_dtype, int w_dtype, cudaStream_t stream);
+cudaError_t launch_decode(const DecodeArgs& p, int io_dtype, int w_dtype, int* status, cudaStream_t stream);
 // z <- (z / sqrt(D) + (sum_d r k rk) v) * g in place over ntok x H rows (wkv7_gate.cu)
 cudaError_t launch_gate(void* z, const void* r, const void* k, const void* v, const float* rk, const void* g,
                         long ntok, int H, int io_dtype, cudaStream_t stream);
