@@ -46,6 +46,8 @@ def _load():
         lib.wkv7_oracle_decode_step.restype = ctypes.c_int
         lib.wkv7_oracle_gate.argtypes = [dp] * 7 + [ctypes.c_long, ctypes.c_int, ctypes.c_int]
         lib.wkv7_oracle_gate.restype = ctypes.c_int
+        lib.wkv7_oracle_prologue.argtypes = [dp] * 8 + [ctypes.c_long, ctypes.c_int, ctypes.c_int, ctypes.c_int]
+        lib.wkv7_oracle_prologue.restype = ctypes.c_int
         _lib = lib
     return _lib
 
@@ -142,3 +144,45 @@ def forward_gated(r, w_log, k, v, a, b, rk, g, s0=None, seq_offsets=None, n_thre
     """The recurrence followed by the gated read-out.  Returns ``(z, sT)``."""
     y, sT = forward(r, w_log, k, v, a, b, s0, seq_offsets, n_threads)
     return gate(y, r, k, v, rk, g), sT
+
+
+def prologue(k, v, w_log, a_lr):
+    """The steps between the projections and the WKV call: k, v [..., H_kv, D] of
+    the kv heads, w_log and a_lr [..., H, D].  Returns ``(k', v_rep, a, b)``, each
+    [..., H, D] float64: k' = k (1 - w + a_lr), v_rep the kv head's v,
+    a = -kk and b = kk a_lr with kk = k / max(||k||, 1e-12)."""
+    lib = _load()
+    k, v, w_log, a_lr = (_f64(t) for t in (k, v, w_log, a_lr))
+    if k.shape != v.shape or w_log.shape != a_lr.shape or k.shape[:-2] != w_log.shape[:-2]:
+        raise ValueError("input shapes differ")
+    H, D = w_log.shape[-2], w_log.shape[-1]
+    H_kv = k.shape[-2]
+    if k.shape[-1] != D or H % H_kv != 0:
+        raise ValueError("H must be a multiple of H_kv and the head sizes must match")
+    ntok = int(np.prod(w_log.shape[:-2])) if w_log.ndim > 2 else 1
+    outs = [np.empty(w_log.shape, dtype=np.float64) for _ in range(4)]
+    rc = lib.wkv7_oracle_prologue(_ptr(k), _ptr(v), _ptr(w_log), _ptr(a_lr), *(_ptr(o) for o in outs), ntok, H,
+                                  H_kv, D)
+    if rc != 0:
+        raise RuntimeError(f"wkv7_oracle_prologue failed with status {rc}")
+    return tuple(outs)
+
+
+def forward_fused(r, w_log, k, v, a_lr, s0=None, seq_offsets=None, rk=None, g=None, n_threads=None):
+    """Prologue, recurrence and (when rk and g are given) the gated read-out.
+    Returns ``(y or z, sT)``."""
+    kp, vr, a, b = prologue(k, v, w_log, a_lr)
+    y, sT = forward(r, w_log, kp, vr, a, b, s0, seq_offsets, n_threads)
+    if rk is None and g is None:
+        return y, sT
+    return gate(y, r, kp, vr, rk, g), sT
+
+
+def decode_step_fused(r, w_log, k, v, a_lr, s_in, rk=None, g=None, n_threads=None):
+    """One decode step with the prologue (and the gated read-out when rk and g
+    are given).  Returns ``(y or z, s_out)``."""
+    kp, vr, a, b = prologue(k, v, w_log, a_lr)
+    y, s_out = decode_step(r, w_log, kp, vr, a, b, s_in, n_threads)
+    if rk is None and g is None:
+        return y, s_out
+    return gate(y, r, kp, vr, rk, g), s_out

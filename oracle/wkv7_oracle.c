@@ -43,6 +43,20 @@
  * with y the recurrence output above, r, k, v the same inputs, rk a per-head
  * vector and g the gate.
  *
+ * Prologue (wkv7_oracle_prologue), the steps the same forward listing takes
+ * between the projections and the WKV call, with the key and value projections
+ * producing H_kv heads that are shared by H / H_kv consecutive query heads
+ * (the listing's repeat of k/v heads when n_kv_heads < n_heads):
+ *
+ *   k, v  = the key and value rows of kv head h / (H / H_kv)
+ *   w_d   = exp(-exp(l_d))
+ *   kk    = k / max(||k||_2, 1e-12)                 (normalise over the head)
+ *   k'    = k (1 - w + a_lr)                        (the key handed to the call)
+ *   a     = -kk,  b = kk a_lr                       (the pair handed to the call)
+ *
+ * with a_lr the per-channel in-context learning rate (the listing's sigmoid
+ * output "a").  The gated read-out after a prologue uses k' and the repeated v.
+ *
  * Layouts (all double, contiguous, the fastest index last):
  *  dense  (seq_offsets == NULL): r, w_log, k, v, a, b, y are [B][T][H][D]
  *  packed (seq_offsets != NULL): they are [T][H][D] with T the packed length and
@@ -215,6 +229,34 @@ int wkv7_oracle_gate(const double *y, const double *r, const double *k, const do
             double u = 0.0;
             for (int d = 0; d < D; ++d) u += r[base + d] * k[base + d] * rk[(long)h * D + d];
             for (int i = 0; i < D; ++i) z[base + i] = (y[base + i] * scale + u * v[base + i]) * g[base + i];
+        }
+    }
+    return 0;
+}
+
+/* The prologue above, per token and head.  k, v: [ntok][H_kv][D]; w_log, a_lr
+ * and the outputs k_out, v_out, a_out, b_out: [ntok][H][D]. */
+int wkv7_oracle_prologue(const double *k, const double *v, const double *w_log, const double *a_lr,
+                         double *k_out, double *v_out, double *a_out, double *b_out, long ntok, int H, int H_kv,
+                         int D) {
+    if (ntok < 0 || H <= 0 || H_kv <= 0 || D <= 0 || H % H_kv != 0) return -1;
+    const int rep = H / H_kv;
+    for (long t = 0; t < ntok; ++t) {
+        for (int h = 0; h < H; ++h) {
+            const long src = (t * H_kv + h / rep) * (long)D;
+            const long dst = (t * H + h) * (long)D;
+            double ss = 0.0;
+            for (int d = 0; d < D; ++d) ss += k[src + d] * k[src + d];
+            const double nrm = sqrt(ss);
+            const double den = nrm > 1e-12 ? nrm : 1e-12;
+            for (int d = 0; d < D; ++d) {
+                const double w = exp(-exp(w_log[dst + d]));
+                const double kk = k[src + d] / den;
+                k_out[dst + d] = k[src + d] * (1.0 - w + a_lr[dst + d]);
+                v_out[dst + d] = v[src + d];
+                a_out[dst + d] = -kk;
+                b_out[dst + d] = kk * a_lr[dst + d];
+            }
         }
     }
     return 0;

@@ -297,3 +297,105 @@ def test_gated_readout_special_cases(oracle_mod):
     np.testing.assert_allclose(z, y / 8.0, rtol=1e-15, atol=0)
     z0, _ = oracle_mod.forward_gated(r, w_log, k, v, a, b, rng.standard_normal((H, D)), np.zeros_like(r), S0)
     assert np.all(z0 == 0.0)
+
+
+def _fused_inputs(rng, B, T, H, H_kv, D):
+    r = rng.standard_normal((B, T, H, D))
+    k, v = (rng.standard_normal((B, T, H_kv, D)) for _ in range(2))
+    a_lr = 1.0 / (1.0 + np.exp(-rng.standard_normal((B, T, H, D))))
+    w_log = -np.log1p(np.exp(-rng.standard_normal((B, T, H, D)))) - 0.5
+    return r, w_log, k, v, a_lr
+
+
+def test_prologue_full_removal_writes_value_at_normalised_key(oracle_mod):
+    """a_lr = 1 and w = 1 (l = -inf) make the step S <- S (I - kk kk^T) + v k^T with
+    kk = k / ||k||: a delta-rule write with unit learning rate, after which
+    S kk = ||k|| v whatever S was.  Checked step by step from random states with
+    H_kv < H; catches an unnormalised or squared-norm kk, a = +kk, b without
+    a_lr, or the key scaled by (1 - w) alone."""
+    rng = np.random.default_rng(31)
+    B, H, H_kv, D = 3, 4, 2, 64
+    s = rng.standard_normal((B, H, D, D)) * 0.5
+    for step in range(5):
+        r, _, k, v, _ = (x[:, 0] for x in _fused_inputs(rng, B, 1, H, H_kv, D))
+        w_log = np.full((B, H, D), -np.inf)
+        a_lr = np.ones((B, H, D))
+        _, s = oracle_mod.decode_step_fused(r, w_log, k, v, a_lr, s)
+        for h in range(H):
+            kh, vh = k[:, h // 2], v[:, h // 2]
+            nrm = np.linalg.norm(kh, axis=-1)
+            got = np.einsum("bij,bj->bi", s[:, h], kh / nrm[:, None])
+            np.testing.assert_allclose(got, nrm[:, None] * vh, rtol=0, atol=1e-10)
+
+
+def test_prologue_no_removal_is_a_decayed_sum(oracle_mod):
+    """a_lr = 0 removes the rank-one term and scales the key by (1 - w): with a
+    per-channel decay constant over time and a zero start,
+    S_T[i, j] = sum_t v_t[i] k_t[j] (1 - w_j) w_j^(T-1-t).  The kv heads are
+    repeated with numpy.repeat; catches a wrong (1 - w + a_lr) factor or the
+    decay applied to the new token's own write."""
+    rng = np.random.default_rng(32)
+    B, T, H, H_kv, D = 2, 7, 4, 2, 64
+    r, _, k, v, _ = _fused_inputs(rng, B, T, H, H_kv, D)
+    wl_h = -np.log1p(np.exp(-rng.standard_normal((H, D)))) - 0.5
+    w_log = np.broadcast_to(wl_h, (B, T, H, D)).copy()
+    a_lr = np.zeros((B, T, H, D))
+    _, sT = oracle_mod.forward_fused(r, w_log, k, v, a_lr)
+    w = np.exp(-np.exp(wl_h))
+    kr, vr = np.repeat(k, 2, axis=2), np.repeat(v, 2, axis=2)
+    pw = np.stack([w ** (T - 1 - t) for t in range(T)])  # [T, H, D]
+    expect = np.einsum("bthi,bthj,hj,thj->bhij", vr, kr, 1.0 - w, pw)
+    np.testing.assert_allclose(sT, expect, rtol=1e-12, atol=1e-12)
+
+
+def test_prologue_kv_heads_match_explicit_repeat(oracle_mod):
+    """H_kv = H / 4 kv heads give exactly the result of the same inputs with
+    each kv head repeated for its 4 query heads (numpy.repeat, the listing's
+    repeat of k/v heads); catches a kv index of h % H_kv instead of h // 4.
+    Also on the gated read-out, which must use the prologue's scaled key."""
+    rng = np.random.default_rng(33)
+    B, T, H, H_kv, D = 2, 9, 8, 2, 64
+    r, w_log, k, v, a_lr = _fused_inputs(rng, B, T, H, H_kv, D)
+    s0 = rng.standard_normal((B, H, D, D)) * 0.2
+    rk = rng.standard_normal((H, D))
+    g = rng.standard_normal((B, T, H, D))
+    y1, s1 = oracle_mod.forward_fused(r, w_log, k, v, a_lr, s0)
+    y2, s2 = oracle_mod.forward_fused(r, w_log, np.repeat(k, 4, axis=2), np.repeat(v, 4, axis=2), a_lr, s0)
+    np.testing.assert_array_equal(y1, y2)
+    np.testing.assert_array_equal(s1, s2)
+    z1, _ = oracle_mod.forward_fused(r, w_log, k, v, a_lr, s0, rk=rk, g=g)
+    z2, _ = oracle_mod.forward_fused(r, w_log, np.repeat(k, 4, axis=2), np.repeat(v, 4, axis=2), a_lr, s0, rk=rk, g=g)
+    np.testing.assert_array_equal(z1, z2)
+
+
+def test_prologue_gate_uses_scaled_key(oracle_mod):
+    """w = 1 and a_lr = 0 scale the key to k (1 - 1 + 0) = 0, so nothing is
+    written, the state stays S0, y_t = S0 r_t and the r-k-rk term vanishes:
+    z_t = (S0 r_t / sqrt(D)) g_t.  Catches the read-out using the raw key."""
+    rng = np.random.default_rng(34)
+    B, T, H, H_kv, D = 2, 5, 2, 1, 64
+    r, _, k, v, _ = _fused_inputs(rng, B, T, H, H_kv, D)
+    w_log = np.full((B, T, H, D), -np.inf)
+    a_lr = np.zeros((B, T, H, D))
+    s0 = rng.standard_normal((B, H, D, D)) * 0.3
+    rk = rng.standard_normal((H, D))
+    g = rng.standard_normal((B, T, H, D))
+    z, sT = oracle_mod.forward_fused(r, w_log, k, v, a_lr, s0, rk=rk, g=g)
+    np.testing.assert_array_equal(sT, s0)
+    y = np.einsum("bhij,bthj->bthi", s0, r)
+    np.testing.assert_allclose(z, y / np.sqrt(D) * g, rtol=1e-13, atol=1e-13)
+
+
+def test_prologue_zero_key_is_identity_step(oracle_mod):
+    """A zero key row (a pad token) normalises to kk = 0 (the 1e-12 floor on the
+    norm, no division by zero), so with v = 0 and w = 1 the step leaves the state
+    unchanged."""
+    rng = np.random.default_rng(35)
+    B, H, D = 2, 2, 64
+    s = rng.standard_normal((B, H, D, D))
+    r = rng.standard_normal((B, H, D))
+    zero = np.zeros((B, 1, D))
+    a_lr = rng.uniform(0.1, 0.9, (B, H, D))
+    y, s1 = oracle_mod.decode_step_fused(r, np.full((B, H, D), -np.inf), zero, zero, a_lr, s)
+    np.testing.assert_array_equal(s1, s)
+    assert np.all(np.isfinite(y))

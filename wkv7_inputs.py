@@ -16,6 +16,11 @@ order r, k, v, kappa, a_lr logit, decay logit, s0):
 * s0 ~ N(0, s0_std^2) in fp32 when an initial state is requested
 * gated read-out (make_gate, its own generator): r_k ~ N(0, rk_std^2) [H, D]
   fp32, gate g ~ N(0, 1) in the io dtype
+* fused prologue (make_fused, its own generator; draw order r, k, v, a_lr logit,
+  decay logit, s0): r ~ N(0, 1) [.., H, D]; raw k, v ~ N(0, 1) over the H_kv
+  kv heads [.., H_kv, D]; a_lr = sigmoid(N(0, 1)) [.., H, D]; log_neglog_w as
+  above.  The prologue (normalised kk, a, b and the scaled key) happens inside
+  the path under test.
 * packed batches: lengths ~ U{len_lo..len_hi} and pad counts ~ U{0..pad_hi};
   pad tokens carry log_neglog_w = -inf (w = 1) and k = v = a = b = 0, so they
   leave the state unchanged; r stays drawn at pads.
@@ -118,6 +123,67 @@ def make_gate(shape, H, D=64, io="bf16", rk_std=0.5, seed=0):
     rk = (torch.randn((H, D), generator=g) * rk_std).contiguous()
     gate = torch.randn(tuple(shape), generator=g).to(_DT[io]).contiguous()
     return rk, gate
+
+
+@dataclass
+class FusedInputs:
+    r: torch.Tensor
+    w_log: torch.Tensor
+    k: torch.Tensor  # [.., H_kv, D]
+    v: torch.Tensor  # [.., H_kv, D]
+    a_lr: torch.Tensor
+    s0: Optional[torch.Tensor]
+    seq_offsets: Optional[torch.Tensor]
+    B: int
+    T: int
+    H: int
+    H_kv: int
+    D: int
+    io: str
+    wdt: str
+    n_real_tokens: int
+
+    def tensors(self):
+        return dict(r=self.r, w_log=self.w_log, k=self.k, v=self.v, a_lr=self.a_lr)
+
+
+def make_fused(B, T, H, H_kv, D=64, io="bf16", wdt="f32", s0_std=None, mu_z=0.0, seed=0, lengths=None, pads=None):
+    """Inputs of the fused-prologue path.  Dense [B, T, .., D] when ``lengths`` is
+    None, else packed [T_total, .., D] with sequence n holding lengths[n] real
+    tokens followed by pads[n] pad tokens (w_log = -inf, k = v = 0)."""
+    g = torch.Generator().manual_seed(seed)
+    seq_offsets = None
+    if lengths is None:
+        lead = (B, T)
+        n_real = B * T
+    else:
+        offs = [0]
+        for l, p_ in zip(lengths, pads):
+            offs.append(offs[-1] + int(l) + int(p_))
+        B, T = len(lengths), offs[-1]
+        lead = (T,)
+        n_real = int(sum(lengths))
+        seq_offsets = torch.tensor(offs, dtype=torch.int32)
+    r = torch.randn(lead + (H, D), generator=g)
+    k = torch.randn(lead + (H_kv, D), generator=g)
+    v = torch.randn(lead + (H_kv, D), generator=g)
+    a_lr = torch.sigmoid(torch.randn(lead + (H, D), generator=g))
+    z = torch.randn(lead + (H, D), generator=g) + mu_z
+    w_log = -torch.nn.functional.softplus(-z) - 0.5
+    s0 = None
+    if s0_std is not None:
+        s0 = (torch.randn((B, H, D, D), generator=g) * s0_std).contiguous()
+    if lengths is not None:
+        pad_mask = torch.zeros(T, dtype=torch.bool)
+        for n in range(B):
+            pad_mask[offs[n] + int(lengths[n]): offs[n + 1]] = True
+        if bool(pad_mask.any()):
+            w_log[pad_mask] = float("-inf")
+            k[pad_mask] = 0
+            v[pad_mask] = 0
+    cast = lambda t, d: t.to(_DT[d]).contiguous()
+    return FusedInputs(cast(r, io), cast(w_log, wdt), cast(k, io), cast(v, io), cast(a_lr, io), s0, seq_offsets,
+                       B, T, H, H_kv, D, io, wdt, n_real)
 
 
 def draw_lengths(n_seq, len_lo, len_hi, pad_hi, seed):
