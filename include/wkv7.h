@@ -112,6 +112,37 @@ int wkv7_forward_gated(const void* r, const void* w_log, const void* k, const vo
                        const int32_t* seq_offsets, int io_dtype, int w_dtype, void* stream);
 
 /*
+ * wkv7_forward_fused — the prologue that the forward listing of "RWKV hxa07D
+ * architecture explainer" (zenn.dev/openmose) runs between its projections and
+ * the WKV call, fused into the prefill, then the recurrence of wkv7_forward and,
+ * optionally, the read-out of wkv7_forward_gated.  Per token and head, with k
+ * and v taken from kv head h / (H / H_kv) (the listing's repeat of k/v heads when
+ * there are fewer kv heads than heads, done by indexing instead of a copy):
+ *
+ *     w  = exp(-exp(w_log))
+ *     kk = k / max(||k||_2, 1e-12)        (normalised over the head)
+ *     k' = k (1 - w + a_lr),   a = -kk,   b = kk (.) a_lr
+ *
+ * and the recurrence runs on (r, w_log, k', v, a, b).  No a, b, k' or repeated
+ * k, v is materialised.
+ *   k, v : [.., H_kv][D] rows of the kv heads (layouts as in wkv7_forward with
+ *          H_kv in place of H); H must be a multiple of H_kv (H_kv == H: no
+ *          sharing).
+ *   a_lr : in-context learning rate, same shape and dtype code as r.
+ *   r_k, g : both NULL (out = y, the WKV output) or both given (out = z of
+ *          wkv7_forward_gated, whose r-k-v term then uses k' and the kv head's v).
+ * r, w_log, s0, sT, seq_offsets, the dtype codes and the rules on overlap and
+ * T == 0 as in wkv7_forward; `out` must not overlap any input.  Pad tokens of a
+ * packed batch carry w_log = -inf and k = v = 0 (kk is then 0).  With bf16
+ * inputs everything runs inside the prefill kernel; with fp32 inputs the
+ * read-out (when asked for) is a second pass over out.
+ */
+int wkv7_forward_fused(const void* r, const void* w_log, const void* k, const void* v,
+                       const void* a_lr, const float* s0, const float* r_k, const void* g,
+                       void* out, float* sT, int B, int T, int H, int H_kv, int D,
+                       const int32_t* seq_offsets, int io_dtype, int w_dtype, void* stream);
+
+/*
  * wkv7_decode_step — one token per sequence (RNN mode).
  *   r, w_log, k, v, a, b, y : [B][H][D]
  *   s_in, s_out            : [B][H][D][D] fp32; s_in == s_out (in place) is
@@ -122,6 +153,22 @@ int wkv7_forward_gated(const void* r, const void* w_log, const void* k, const vo
 int wkv7_decode_step(const void* r, const void* w_log, const void* k, const void* v,
                      const void* a, const void* b, const float* s_in, void* y, float* s_out,
                      int B, int H, int D, int io_dtype, int w_dtype, void* stream);
+
+/*
+ * wkv7_decode_step_fused — one token per sequence with the prologue of
+ * wkv7_forward_fused (kk, a = -kk, b = kk a_lr and the key scaled by
+ * (1 - w + a_lr) formed inside the kernel; k and v from kv head h / (H / H_kv))
+ * and, when r_k and g are both given, the gated read-out of wkv7_forward_gated
+ * (whose r-k-v term uses the scaled key) written to `out` instead of y.
+ *   r, w_log, a_lr, g, out : [B][H][D];  k, v : [B][H_kv][D];  r_k : [H][D] fp32
+ *   s_in, s_out            : as in wkv7_decode_step.
+ * H must be a multiple of H_kv; r_k and g are both NULL or both given; `out`
+ * must not overlap any input.
+ */
+int wkv7_decode_step_fused(const void* r, const void* w_log, const void* k, const void* v,
+                           const void* a_lr, const float* s_in, const float* r_k, const void* g,
+                           void* out, float* s_out, int B, int H, int H_kv, int D,
+                           int io_dtype, int w_dtype, void* stream);
 
 /* Human-readable text for a status code (static storage, never NULL). */
 const char* wkv7_status_string(int status);

@@ -3,8 +3,9 @@ decode step behind a C ABI (``include/wkv7.h``, ``libwkv7.so``).
 
 The Python layer only marshals arguments to the CUDA library; importing the
 package loads ``libwkv7.so`` and fails loudly if it has not been built.
-Convenience wrappers ``forward``, ``forward_gated`` and ``decode_step``
-allocate outputs with torch and call the C entry points.
+Convenience wrappers ``forward``, ``forward_gated``, ``forward_fused``,
+``decode_step`` and ``decode_step_fused`` allocate outputs with torch and call
+the C entry points.
 """
 from __future__ import annotations
 
@@ -18,7 +19,9 @@ from ._binding import (  # noqa: F401
     _lib,
     wkv7_debug_expire_wait,
     wkv7_decode_step,
+    wkv7_decode_step_fused,
     wkv7_forward,
+    wkv7_forward_fused,
     wkv7_forward_gated,
     wkv7_get_device_status,
     wkv7_status_string,
@@ -60,6 +63,38 @@ def forward_gated(r, w_log, k, v, a, b, r_k, g, s0=None, seq_offsets=None, want_
     sT = torch.empty((B, H, D, D), dtype=torch.float32, device=r.device) if want_state else None
     wkv7_forward_gated(r, w_log, k, v, a, b, s0, r_k, g, z, sT, B, T, H, D, seq_offsets, stream)
     return z, sT
+
+
+def forward_fused(r, w_log, k, v, a_lr, s0=None, seq_offsets=None, r_k=None, g=None, want_state=True, stream=None):
+    """Chunked prefill with the fused prologue: ``k`` and ``v`` are the raw rows
+    of the kv heads ([.., H_kv, D]), ``a_lr`` the in-context learning rate; the
+    kernel forms kk, a = -kk, b = kk a_lr and k (1 - w + a_lr) itself.  With
+    ``r_k`` and ``g`` the output is the gated read-out z.  Returns ``(y or z, sT)``."""
+    import torch
+
+    if seq_offsets is not None:
+        T, H, D = r.shape
+        B = seq_offsets.numel() - 1
+    else:
+        B, T, H, D = r.shape
+    H_kv = k.shape[-2]
+    out = torch.empty_like(r)
+    sT = torch.empty((B, H, D, D), dtype=torch.float32, device=r.device) if want_state else None
+    wkv7_forward_fused(r, w_log, k, v, a_lr, s0, r_k, g, out, sT, B, T, H, H_kv, D, seq_offsets, stream)
+    return out, sT
+
+
+def decode_step_fused(r, w_log, k, v, a_lr, state, r_k=None, g=None, out=None, stream=None):
+    """One decoding step with the fused prologue (and the gated read-out when
+    ``r_k`` and ``g`` are given), updating ``state`` in place.  ``k``, ``v`` are
+    [B, H_kv, D].  Returns the output rows [B, H, D]."""
+    import torch
+
+    B, H, D = r.shape
+    if out is None:
+        out = torch.empty_like(r)
+    wkv7_decode_step_fused(r, w_log, k, v, a_lr, state, r_k, g, out, state, B, H, k.shape[-2], D, stream)
+    return out
 
 
 def decode_step(r, w_log, k, v, a, b, state, y=None, stream=None):

@@ -28,7 +28,9 @@ STATUS = {
 EXPORTS = (
     "wkv7_forward",
     "wkv7_forward_gated",
+    "wkv7_forward_fused",
     "wkv7_decode_step",
+    "wkv7_decode_step_fused",
     "wkv7_status_string",
     "wkv7_get_device_status",
     "wkv7_debug_expire_wait",
@@ -57,6 +59,10 @@ def _lib():
         lib.wkv7_forward.restype = i
         lib.wkv7_forward_gated.argtypes = [vp] * 11 + [i] * 4 + [vp, i, i, vp]
         lib.wkv7_forward_gated.restype = i
+        lib.wkv7_forward_fused.argtypes = [vp] * 10 + [i] * 5 + [vp, i, i, vp]
+        lib.wkv7_forward_fused.restype = i
+        lib.wkv7_decode_step_fused.argtypes = [vp] * 10 + [i] * 4 + [i, i, vp]
+        lib.wkv7_decode_step_fused.restype = i
         lib.wkv7_decode_step.argtypes = [vp] * 9 + [i] * 3 + [i, i, vp]
         lib.wkv7_decode_step.restype = i
         lib.wkv7_status_string.argtypes = [i]
@@ -118,6 +124,26 @@ def wkv7_forward_gated(r, w_log, k, v, a, b, s0, r_k, g, z, sT, B, T, H, D, seq_
         raise Wkv7Error(st, "wkv7_forward_gated")
 
 
+def wkv7_forward_fused(r, w_log, k, v, a_lr, s0, r_k, g, out, sT, B, T, H, H_kv, D, seq_offsets=None, stream=None):
+    """Enqueue the prefill with the fused prologue (and the gated read-out when
+    r_k and g are given); see include/wkv7.h."""
+    st = _lib().wkv7_forward_fused(_ptr(r), _ptr(w_log), _ptr(k), _ptr(v), _ptr(a_lr), _ptr(s0), _ptr(r_k), _ptr(g),
+                                   _ptr(out), _ptr(sT), int(B), int(T), int(H), int(H_kv), int(D), _ptr(seq_offsets),
+                                   _dtype_code(r), _dtype_code(w_log), _stream(stream))
+    if st != 0:
+        raise Wkv7Error(st, "wkv7_forward_fused")
+
+
+def wkv7_decode_step_fused(r, w_log, k, v, a_lr, s_in, r_k, g, out, s_out, B, H, H_kv, D, stream=None):
+    """Enqueue one decoding step with the fused prologue (and the gated read-out
+    when r_k and g are given); see include/wkv7.h."""
+    st = _lib().wkv7_decode_step_fused(_ptr(r), _ptr(w_log), _ptr(k), _ptr(v), _ptr(a_lr), _ptr(s_in), _ptr(r_k),
+                                       _ptr(g), _ptr(out), _ptr(s_out), int(B), int(H), int(H_kv), int(D),
+                                       _dtype_code(r), _dtype_code(w_log), _stream(stream))
+    if st != 0:
+        raise Wkv7Error(st, "wkv7_decode_step_fused")
+
+
 def wkv7_decode_step(r, w_log, k, v, a, b, s_in, y, s_out, B, H, D, stream=None):
     """Enqueue one decoding step (see include/wkv7.h)."""
     st = _lib().wkv7_decode_step(_ptr(r), _ptr(w_log), _ptr(k), _ptr(v), _ptr(a), _ptr(b), _ptr(s_in), _ptr(y),
@@ -152,6 +178,14 @@ def raw_call_forward(*args):
 
 def raw_call_forward_gated(*args):
     return int(_lib().wkv7_forward_gated(*args))
+
+
+def raw_call_forward_fused(*args):
+    return int(_lib().wkv7_forward_fused(*args))
+
+
+def raw_call_decode_fused(*args):
+    return int(_lib().wkv7_decode_step_fused(*args))
 
 
 def raw_call_decode(*args):

@@ -44,17 +44,19 @@ inline bool make_token_map(CUtensorMap* m, const void* base, CUtensorMapDataType
               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// Maps for bf16 r, k, a, b (no swizzle), w_log of `wbytes`-byte elements (no
-// swizzle) and bf16 v (128-byte swizzle: the MN-major operand layout).
+// Maps for bf16 r, a, b over H heads, bf16 k over H_kv heads (no swizzle), w_log of
+// `wbytes`-byte elements over H heads (no swizzle) and bf16 v over H_kv heads
+// (128-byte swizzle: the MN-major operand layout).  b may be null (no map).
 inline bool make_prefill_maps(TmaMaps* m, const void* r, const void* wl, const void* k, const void* v, const void* a,
-                              const void* b, uint64_t H, uint64_t ntok, uint32_t wbytes) {
+                              const void* b, uint64_t H, uint64_t H_kv, uint64_t ntok, uint32_t wbytes) {
     const CUtensorMapDataType bf = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
     const CUtensorMapDataType wdt = wbytes == 4 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
     const CUtensorMapSwizzle none = CU_TENSOR_MAP_SWIZZLE_NONE;
-    return make_token_map(&m->r, r, bf, 2, H, ntok, none) && make_token_map(&m->k, k, bf, 2, H, ntok, none) &&
-           make_token_map(&m->a, a, bf, 2, H, ntok, none) && make_token_map(&m->b, b, bf, 2, H, ntok, none) &&
+    return make_token_map(&m->r, r, bf, 2, H, ntok, none) && make_token_map(&m->k, k, bf, 2, H_kv, ntok, none) &&
+           make_token_map(&m->a, a, bf, 2, H, ntok, none) &&
+           (b == nullptr || make_token_map(&m->b, b, bf, 2, H, ntok, none)) &&
            make_token_map(&m->wl, wl, wdt, wbytes, H, ntok, none) &&
-           make_token_map(&m->v, v, bf, 2, H, ntok, CU_TENSOR_MAP_SWIZZLE_128B);
+           make_token_map(&m->v, v, bf, 2, H_kv, ntok, CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
 }  // namespace wkv7

@@ -83,27 +83,35 @@ const char* wkv7_status_string(int status) {
     }
 }
 
-// wkv7_forward and wkv7_forward_gated; rk and g are null for the former.
+// wkv7_forward, wkv7_forward_gated and wkv7_forward_fused; rk and g are null
+// without the gated read-out.  With `prologue`, `a` is a_lr, b is unused and k,
+// v have H_kv heads; otherwise H_kv is H.
 static int forward_impl(const void* r, const void* w_log, const void* k, const void* v, const void* a, const void* b,
                         const float* s0, const float* rk, const void* g, void* y, float* sT, int B, int T, int H,
-                        int D, const int32_t* seq_offsets, int io_dtype, int w_dtype, void* stream) {
+                        int D, const int32_t* seq_offsets, int io_dtype, int w_dtype, void* stream,
+                        bool prologue = false, int H_kv = 0) {
     const bool gated = rk != nullptr;
+    if (!prologue) H_kv = H;
     // ---- host-side validation; nothing is launched on failure
     if (B <= 0 || T < 0 || H <= 0 || D <= 0) return WKV7_ERR_INVALID_ARG;
+    if (H_kv <= 0 || H % H_kv != 0) return WKV7_ERR_INVALID_ARG;
     if (!dtype_ok(io_dtype) || !dtype_ok(w_dtype)) return WKV7_ERR_INVALID_ARG;
     if (D != wkv7::kHead) return WKV7_ERR_UNSUPPORTED;
-    if (T > 0 && (!r || !w_log || !k || !v || !a || !b || !y)) return WKV7_ERR_INVALID_ARG;
+    if (T > 0 && (!r || !w_log || !k || !v || !a || (!prologue && !b) || !y)) return WKV7_ERR_INVALID_ARG;
     if (gated && T > 0 && !g) return WKV7_ERR_INVALID_ARG;
+    if (prologue) b = nullptr;
     const void* ptrs[] = {r, w_log, k, v, a, b, s0, y, sT, seq_offsets, rk, g};
     for (const void* p : ptrs)
         if (p && !aligned16(p)) return WKV7_ERR_MISALIGNED;
     const long tokens = seq_offsets ? static_cast<long>(T) : static_cast<long>(B) * T;
     const size_t n_act = static_cast<size_t>(tokens) * H * D;
+    const size_t n_kv = static_cast<size_t>(tokens) * H_kv * D;  // k and v
     const size_t n_state = static_cast<size_t>(B) * H * D * D;
     const size_t io_b = dtype_bytes(io_dtype), w_b = dtype_bytes(w_dtype);
     const void* ins[] = {r, k, v, a, b};
-    for (const void* p : ins)
-        if (overlaps(y, n_act * io_b, p, n_act * io_b)) return WKV7_ERR_INVALID_ARG;
+    const size_t in_n[] = {n_act, n_kv, n_kv, n_act, n_act};
+    for (int i = 0; i < 5; ++i)
+        if (overlaps(y, n_act * io_b, ins[i], in_n[i] * io_b)) return WKV7_ERR_INVALID_ARG;
     if (overlaps(y, n_act * io_b, w_log, n_act * w_b) || overlaps(y, n_act * io_b, s0, n_state * 4) ||
         overlaps(y, n_act * io_b, sT, n_state * 4))
         return WKV7_ERR_INVALID_ARG;
@@ -116,8 +124,8 @@ static int forward_impl(const void* r, const void* w_log, const void* k, const v
     // before it writes its own final state.  Any other overlap is rejected.
     if (sT && sT != s0 && overlaps(sT, n_state * 4, s0, n_state * 4)) return WKV7_ERR_INVALID_ARG;
     if (n_act > 0) {
-        for (const void* p : ins)
-            if (overlaps(sT, n_state * 4, p, n_act * io_b)) return WKV7_ERR_INVALID_ARG;
+        for (int i = 0; i < 5; ++i)
+            if (overlaps(sT, n_state * 4, ins[i], in_n[i] * io_b)) return WKV7_ERR_INVALID_ARG;
         if (overlaps(sT, n_state * 4, w_log, n_act * w_b)) return WKV7_ERR_INVALID_ARG;
     }
 
@@ -138,10 +146,13 @@ static int forward_impl(const void* r, const void* w_log, const void* k, const v
         p.rk = rk;
         p.g = g;
     }
+    p.prologue = prologue;
+    p.H_kv = H_kv;
     if (wkv7::launch_prefill(p, io_dtype, w_dtype, st) != cudaSuccess) return WKV7_ERR_CUDA;
     // the bf16 kernel writes the gated rows directly; the fp32 path applies the read-out in place
     if (gated && io_dtype == WKV7_F32 &&
-        wkv7::launch_gate(y, r, k, v, rk, g, tokens, H, io_dtype, st) != cudaSuccess)
+        wkv7::launch_gate(y, r, k, v, rk, g, tokens, H, io_dtype, st, prologue ? w_log : nullptr,
+                          prologue ? a : nullptr, H_kv, w_dtype) != cudaSuccess)
         return WKV7_ERR_CUDA;
     return WKV7_OK;
 }
@@ -161,27 +172,44 @@ int wkv7_forward_gated(const void* r, const void* w_log, const void* k, const vo
                         stream);
 }
 
+int wkv7_forward_fused(const void* r, const void* w_log, const void* k, const void* v, const void* a_lr,
+                       const float* s0, const float* r_k, const void* g, void* out, float* sT, int B, int T, int H,
+                       int H_kv, int D, const int32_t* seq_offsets, int io_dtype, int w_dtype, void* stream) {
+    if ((r_k == nullptr) != (g == nullptr)) return WKV7_ERR_INVALID_ARG;
+    return forward_impl(r, w_log, k, v, a_lr, nullptr, s0, r_k, g, out, sT, B, T, H, D, seq_offsets, io_dtype,
+                        w_dtype, stream, true, H_kv);
+}
 
-int wkv7_decode_step(const void* r, const void* w_log, const void* k, const void* v, const void* a, const void* b,
-                     const float* s_in, void* y, float* s_out, int B, int H, int D, int io_dtype, int w_dtype,
-                     void* stream) {
-    if (B <= 0 || H <= 0 || D <= 0) return WKV7_ERR_INVALID_ARG;
+
+// wkv7_decode_step and wkv7_decode_step_fused (`prologue`: a is a_lr, b unused,
+// k and v have H_kv heads; rk and g both null or both given).
+static int decode_impl(const void* r, const void* w_log, const void* k, const void* v, const void* a, const void* b,
+                       const float* s_in, const float* rk, const void* g, void* y, float* s_out, int B, int H,
+                       int H_kv, int D, int io_dtype, int w_dtype, void* stream, bool prologue) {
+    if (!prologue) H_kv = H;
+    if (B <= 0 || H <= 0 || D <= 0 || H_kv <= 0 || H % H_kv != 0) return WKV7_ERR_INVALID_ARG;
     if (!dtype_ok(io_dtype) || !dtype_ok(w_dtype)) return WKV7_ERR_INVALID_ARG;
     if (D != wkv7::kHead) return WKV7_ERR_UNSUPPORTED;
-    if (!r || !w_log || !k || !v || !a || !b || !y || !s_out) return WKV7_ERR_INVALID_ARG;
-    const void* ptrs[] = {r, w_log, k, v, a, b, s_in, y, s_out};
+    if (!r || !w_log || !k || !v || !a || (!prologue && !b) || !y || !s_out) return WKV7_ERR_INVALID_ARG;
+    if ((rk == nullptr) != (g == nullptr)) return WKV7_ERR_INVALID_ARG;
+    if (prologue) b = nullptr;
+    const void* ptrs[] = {r, w_log, k, v, a, b, s_in, y, s_out, rk, g};
     for (const void* p : ptrs)
         if (p && !aligned16(p)) return WKV7_ERR_MISALIGNED;
     const size_t n_act = static_cast<size_t>(B) * H * D;
+    const size_t n_kv = static_cast<size_t>(B) * H_kv * D;
     const size_t n_state = static_cast<size_t>(B) * H * D * D;
     const size_t io_b = dtype_bytes(io_dtype), w_b = dtype_bytes(w_dtype);
-    const void* ins[] = {r, k, v, a, b};
-    for (const void* p : ins) {
-        if (overlaps(y, n_act * io_b, p, n_act * io_b)) return WKV7_ERR_INVALID_ARG;
-        if (overlaps(s_out, n_state * 4, p, n_act * io_b)) return WKV7_ERR_INVALID_ARG;
+    const void* ins[] = {r, k, v, a, b, g};
+    const size_t in_n[] = {n_act, n_kv, n_kv, n_act, n_act, n_act};
+    for (int i = 0; i < 6; ++i) {
+        if (overlaps(y, n_act * io_b, ins[i], in_n[i] * io_b)) return WKV7_ERR_INVALID_ARG;
+        if (overlaps(s_out, n_state * 4, ins[i], in_n[i] * io_b)) return WKV7_ERR_INVALID_ARG;
     }
+    const size_t rk_b = static_cast<size_t>(H) * D * 4;
     if (overlaps(y, n_act * io_b, w_log, n_act * w_b) || overlaps(y, n_act * io_b, s_in, n_state * 4) ||
-        overlaps(y, n_act * io_b, s_out, n_state * 4) || overlaps(s_out, n_state * 4, w_log, n_act * w_b))
+        overlaps(y, n_act * io_b, s_out, n_state * 4) || overlaps(s_out, n_state * 4, w_log, n_act * w_b) ||
+        overlaps(y, n_act * io_b, rk, rk_b) || overlaps(s_out, n_state * 4, rk, rk_b))
         return WKV7_ERR_INVALID_ARG;
     if (s_in && s_in != s_out && overlaps(s_in, n_state * 4, s_out, n_state * 4)) return WKV7_ERR_INVALID_ARG;
 
@@ -190,9 +218,27 @@ int wkv7_decode_step(const void* r, const void* w_log, const void* k, const void
     int* status = nullptr;
     if (status_ptr(&status) != WKV7_OK) return WKV7_ERR_CUDA;
     wkv7::DecodeArgs p{r, w_log, k, v, a, b, s_in, y, s_out, B, H};
+    p.prologue = prologue;
+    p.H_kv = H_kv;
+    p.rk = rk;
+    p.g = g;
     return wkv7::launch_decode(p, io_dtype, w_dtype, status, static_cast<cudaStream_t>(stream)) == cudaSuccess
                ? WKV7_OK
                : WKV7_ERR_CUDA;
+}
+
+int wkv7_decode_step(const void* r, const void* w_log, const void* k, const void* v, const void* a, const void* b,
+                     const float* s_in, void* y, float* s_out, int B, int H, int D, int io_dtype, int w_dtype,
+                     void* stream) {
+    return decode_impl(r, w_log, k, v, a, b, s_in, nullptr, nullptr, y, s_out, B, H, H, D, io_dtype, w_dtype, stream,
+                       false);
+}
+
+int wkv7_decode_step_fused(const void* r, const void* w_log, const void* k, const void* v, const void* a_lr,
+                           const float* s_in, const float* r_k, const void* g, void* out, float* s_out, int B, int H,
+                           int H_kv, int D, int io_dtype, int w_dtype, void* stream) {
+    return decode_impl(r, w_log, k, v, a_lr, nullptr, s_in, r_k, g, out, s_out, B, H, H_kv, D, io_dtype, w_dtype,
+                       stream, true);
 }
 
 int wkv7_get_device_status(void* stream) {

@@ -19,6 +19,15 @@
 // Thread mapping inside a unit: a thread owns 4 consecutive key columns (one
 // 16-byte vector) of 4 value rows spaced 16 apart; 16 threads cover one row,
 // so both row reductions are 4 xor-shuffles inside a 16-lane group.
+//
+// PRO (wkv7_decode_step_fused): the prologue of the WKV call on the raw inputs
+// ("RWKV hxa07D architecture explainer", forward listing before the WKV call):
+// k and v are rows of kv head h / (H / H_kv), the `a` row carries a_lr, and
+//   kk = k / max(||k||, 1e-12),  a = -kk,  b = kk a_lr,  k <- k (1 - w + a_lr)
+// (the norm is one more 16-lane reduction); `b` is not read.  GATED: the output
+// row is z = (y / sqrt(D) + u v) (.) g with u = sum_d r k rk (k the scaled key),
+// the read-out the same listing applies after the call; r_k and g rows join the
+// stage's inputs.
 #include "sm100_ptx.cuh"
 #include "wkv7_internal.cuh"
 
@@ -27,7 +36,7 @@ namespace {
 
 constexpr int NST = 4;                        // pipeline stages per block
 constexpr uint32_t ST_STATE = kHead * kHead * 4;  // 16 KB fp32 state
-constexpr uint32_t ST_BYTES = ST_STATE + 2048;    // + six input rows (at most 6 x 256 B)
+constexpr uint32_t ST_BYTES = ST_STATE + 2048;    // + input rows (at most 8 x 256 B)
 constexpr uint32_t SMEM_BYTES = NST * ST_BYTES + NST * 8;
 constexpr uint64_t WAIT_NS = 1000000000ull;  // 1 s
 
@@ -57,11 +66,12 @@ __device__ __forceinline__ float sum16(float x) {
     return x;
 }
 
-template <typename IO, typename WT>
+template <typename IO, typename WT, bool PRO, bool GATED>
 __global__ void __launch_bounds__(256, 2)
     wkv7_decode_kernel(const IO* __restrict__ r, const WT* __restrict__ wl, const IO* __restrict__ k,
                        const IO* __restrict__ v, const IO* __restrict__ a, const IO* __restrict__ b,
-                       const float* s_in, IO* __restrict__ y, float* s_out, long units, int* status) {
+                       const float* s_in, IO* __restrict__ y, float* s_out, long units, int* status, int H,
+                       int H_kv, const float* __restrict__ rk, const IO* __restrict__ gte) {
     extern __shared__ __align__(128) uint8_t smem[];
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + NST * ST_BYTES);
     const int tid = threadIdx.x;
@@ -69,8 +79,9 @@ __global__ void __launch_bounds__(256, 2)
     const int rg = tid >> 4;  // value rows rg, rg+16, rg+32, rg+48
     constexpr uint32_t IOB = sizeof(IO) * kHead, WB = sizeof(WT) * kHead;
     constexpr uint32_t O_R = ST_STATE, O_K = O_R + IOB, O_V = O_K + IOB, O_A = O_V + IOB, O_B = O_A + IOB,
-                       O_W = O_B + IOB;
-    const uint32_t tx = (s_in ? ST_STATE : 0u) + 5u * IOB + WB;
+                       O_W = O_B + IOB, O_RK = O_W + WB, O_G = O_RK + kHead * 4;
+    static_assert(O_G + IOB <= ST_BYTES, "stage inputs overflow");
+    const uint32_t tx = (s_in ? ST_STATE : 0u) + (PRO ? 4u : 5u) * IOB + WB + (GATED ? kHead * 4u + IOB : 0u);
 
     if (tid == 0) {
         for (int i = 0; i < NST; ++i) mbar_init(&full[i], 1);
@@ -86,13 +97,19 @@ __global__ void __launch_bounds__(256, 2)
         uint8_t* base = smem + (j % NST) * ST_BYTES;
         uint64_t* bar = &full[j % NST];
         mbar_arrive_expect_tx(bar, tx);
+        // row of k and v: the unit's own, or its kv head's
+        const long ukv = PRO ? (u / H) * H_kv + (u % H) / (H / H_kv) : u;
         if (s_in) bulk_load(base, s_in + u * (kHead * kHead), ST_STATE, bar);
         bulk_load(base + O_R, r + u * kHead, IOB, bar);
-        bulk_load(base + O_K, k + u * kHead, IOB, bar);
-        bulk_load(base + O_V, v + u * kHead, IOB, bar);
+        bulk_load(base + O_K, k + ukv * kHead, IOB, bar);
+        bulk_load(base + O_V, v + ukv * kHead, IOB, bar);
         bulk_load(base + O_A, a + u * kHead, IOB, bar);
-        bulk_load(base + O_B, b + u * kHead, IOB, bar);
+        if constexpr (!PRO) bulk_load(base + O_B, b + u * kHead, IOB, bar);
         bulk_load(base + O_W, wl + u * kHead, WB, bar);
+        if constexpr (GATED) {
+            bulk_load(base + O_RK, rk + (u % H) * kHead, kHead * 4, bar);
+            bulk_load(base + O_G, gte + u * kHead, IOB, bar);
+        }
         ++n_issued;
     };
     if (tid == 0)
@@ -111,13 +128,32 @@ __global__ void __launch_bounds__(256, 2)
         float wv[4], av[4], bv[4], kv[4], rv[4], vrow[4];
         lds4<WT>(base + O_W + 4 * cg * sizeof(WT), wv);
         lds4<IO>(base + O_A + 4 * cg * sizeof(IO), av);
-        lds4<IO>(base + O_B + 4 * cg * sizeof(IO), bv);
+        if constexpr (!PRO) lds4<IO>(base + O_B + 4 * cg * sizeof(IO), bv);
         lds4<IO>(base + O_K + 4 * cg * sizeof(IO), kv);
         lds4<IO>(base + O_R + 4 * cg * sizeof(IO), rv);
 #pragma unroll
         for (int q = 0; q < 4; ++q) vrow[q] = lds1<IO>(base + O_V, rg + 16 * q);
 #pragma unroll
         for (int c = 0; c < 4; ++c) wv[c] = expf(-expf(wv[c]));
+        if constexpr (PRO) {
+            // av holds a_lr: form kk, a, b and the scaled key
+            const float inv =
+                1.f / fmaxf(sqrtf(sum16(kv[0] * kv[0] + kv[1] * kv[1] + kv[2] * kv[2] + kv[3] * kv[3])), 1e-12f);
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                const float kn = kv[c] * inv, alr = av[c];
+                bv[c] = kn * alr;
+                av[c] = -kn;
+                kv[c] *= 1.f - wv[c] + alr;
+            }
+        }
+        float uu = 0.f;  // gated read-out: u = sum_d r k rk
+        if constexpr (GATED) {
+            float rkv[4];
+            lds4<float>(base + O_RK + 16 * cg, rkv);
+            uu = sum16(rv[0] * kv[0] * rkv[0] + rv[1] * kv[1] * rkv[1] + rv[2] * kv[2] * rkv[2] +
+                       rv[3] * kv[3] * rkv[3]);
+        }
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
             float4* sp = reinterpret_cast<float4*>(base + ((rg + 16 * q) * kHead + 4 * cg) * 4);
@@ -128,7 +164,8 @@ __global__ void __launch_bounds__(256, 2)
             x.y = fmaf(x.y, wv[1], fmaf(sa, bv[1], vi * kv[1]));
             x.z = fmaf(x.z, wv[2], fmaf(sa, bv[2], vi * kv[2]));
             x.w = fmaf(x.w, wv[3], fmaf(sa, bv[3], vi * kv[3]));
-            const float yi = sum16(x.x * rv[0] + x.y * rv[1] + x.z * rv[2] + x.w * rv[3]);
+            float yi = sum16(x.x * rv[0] + x.y * rv[1] + x.z * rv[2] + x.w * rv[3]);
+            if constexpr (GATED) yi = (yi * 0.125f + uu * vi) * lds1<IO>(base + O_G, rg + 16 * q);
             *sp = x;
             if (cg == 0) y[u * kHead + rg + 16 * q] = from_f32<IO>(yi);
         }
@@ -153,9 +190,9 @@ __global__ void __launch_bounds__(256, 2)
     }
 }
 
-template <typename IO, typename WT>
+template <typename IO, typename WT, bool PRO, bool GATED>
 cudaError_t launch_typed(const DecodeArgs& p, int* status, cudaStream_t stream) {
-    auto kern = wkv7_decode_kernel<IO, WT>;
+    auto kern = wkv7_decode_kernel<IO, WT, PRO, GATED>;
     static unsigned long long configured = 0;
     static int sm_count[64] = {};
     int dev = 0;
@@ -174,19 +211,27 @@ cudaError_t launch_typed(const DecodeArgs& p, int* status, cudaStream_t stream) 
     kern<<<static_cast<unsigned>(grid), 256, SMEM_BYTES, stream>>>(
         static_cast<const IO*>(p.r), static_cast<const WT*>(p.w_log), static_cast<const IO*>(p.k),
         static_cast<const IO*>(p.v), static_cast<const IO*>(p.a), static_cast<const IO*>(p.b), p.s_in,
-        static_cast<IO*>(p.y), p.s_out, units, status);
+        static_cast<IO*>(p.y), p.s_out, units, status, p.H, PRO ? p.H_kv : p.H, p.rk,
+        static_cast<const IO*>(p.g));
     return cudaGetLastError();
+}
+
+template <typename IO, typename WT>
+cudaError_t launch_io(const DecodeArgs& p, int* status, cudaStream_t stream) {
+    if (!p.prologue) return launch_typed<IO, WT, false, false>(p, status, stream);
+    return p.rk ? launch_typed<IO, WT, true, true>(p, status, stream)
+                : launch_typed<IO, WT, true, false>(p, status, stream);
 }
 
 }  // namespace
 
 cudaError_t launch_decode(const DecodeArgs& p, int io_dtype, int w_dtype, int* status, cudaStream_t stream) {
     if (io_dtype == WKV7_BF16) {
-        return w_dtype == WKV7_BF16 ? launch_typed<__nv_bfloat16, __nv_bfloat16>(p, status, stream)
-                                    : launch_typed<__nv_bfloat16, float>(p, status, stream);
+        return w_dtype == WKV7_BF16 ? launch_io<__nv_bfloat16, __nv_bfloat16>(p, status, stream)
+                                    : launch_io<__nv_bfloat16, float>(p, status, stream);
     }
-    return w_dtype == WKV7_BF16 ? launch_typed<float, __nv_bfloat16>(p, status, stream)
-                                : launch_typed<float, float>(p, status, stream);
+    return w_dtype == WKV7_BF16 ? launch_io<float, __nv_bfloat16>(p, status, stream)
+                                : launch_io<float, float>(p, status, stream);
 }
 
 }  // namespace wkv7

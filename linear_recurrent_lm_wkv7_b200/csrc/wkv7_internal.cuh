@@ -28,6 +28,10 @@ struct PrefillArgs {
     // gated read-out (wkv7_forward_gated): y then holds z; both null otherwise
     const float* rk = nullptr;  // [H][D] fp32
     const void* g = nullptr;    // gate, same layout and dtype as r
+    // fused prologue (wkv7_forward_fused): a holds a_lr, b is unused, k and v
+    // have H_kv heads; the kernels form kk, a, b and the scaled key themselves
+    bool prologue = false;
+    int H_kv = 0;
 };
 
 struct DecodeArgs {
@@ -41,15 +45,24 @@ struct DecodeArgs {
     void* y;
     float* s_out;
     int B, H;
+    // fused prologue (wkv7_decode_step_fused): a holds a_lr, b is unused, k and v
+    // have H_kv heads; rk and g (both or neither) add the gated read-out
+    bool prologue = false;
+    int H_kv = 0;
+    const float* rk = nullptr;
+    const void* g = nullptr;
 };
 
 cudaError_t launch_prefill(const PrefillArgs& p, int io_dtype, int w_dtype, cudaStream_t stream);
 // warp-specialised kernel for bf16 inputs (wkv7_prefill_pipe.cu)
 cudaError_t launch_prefill_pipe(const PrefillArgs& p, int w_dtype, cudaStream_t stream);
 cudaError_t launch_decode(const DecodeArgs& p, int io_dtype, int w_dtype, int* status, cudaStream_t stream);
-// z <- (z / sqrt(D) + (sum_d r k rk) v) * g in place over ntok x H rows (wkv7_gate.cu)
+// z <- (z / sqrt(D) + (sum_d r k rk) v) * g in place over ntok x H rows (wkv7_gate.cu).
+// With a_lr non-null (after the fused prologue) the key is k (1 - w + a_lr) with
+// w = exp(-exp(w_log)), and k, v are rows of kv head h / (H / H_kv).
 cudaError_t launch_gate(void* z, const void* r, const void* k, const void* v, const float* rk, const void* g,
-                        long ntok, int H, int io_dtype, cudaStream_t stream);
+                        long ntok, int H, int io_dtype, cudaStream_t stream, const void* w_log = nullptr,
+                        const void* a_lr = nullptr, int H_kv = 0, int w_dtype = WKV7_F32);
 cudaError_t launch_expire_wait(int spins, int* status, cudaStream_t stream);
 
 // Records the first device-side error of a call sequence (first writer wins).

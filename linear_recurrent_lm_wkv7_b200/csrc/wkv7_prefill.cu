@@ -74,7 +74,7 @@ struct Smem {
     uint8_t* S;    // S^T: bf16 64 keys x 64 values (MN-major); tf32 64 values x 64 keys (K-major)
     uint8_t* raw;  // bf16 only: TMA staging of r, k, a, b (64 x 64 each, row-major) and w_log
     float* gammaL; // Gamma_L per key channel
-    float* red;    // per-half products of w (2 x 64)
+    float* red;    // per-half products of w (2 x 64), then (prologue) 1 / ||k_t|| per token (64)
     uint64_t* bar; // MMA completion barrier
     uint64_t* raw_bar; // TMA completion barrier (bf16 only)
     uint32_t* tmem_slot;
@@ -94,7 +94,7 @@ __host__ __device__ constexpr uint32_t smem_bytes_needed() {
     constexpr uint32_t r4 = ((solver > O::TILE128 ? solver : O::TILE128) + 1023u) & ~1023u;
     constexpr uint32_t nv = TF32 ? 1u : 2u;
     return 1024u /* alignment slack */ + 3u * O::TILE128 + O::TILE64 + r4 + (nv + 1u) * O::TILE64 +
-           raw_bytes<TF32, WB>() + 64u * 4u + 128u * 4u + 64u;
+           raw_bytes<TF32, WB>() + 64u * 4u + 192u * 4u + 64u;
 }
 
 template <bool TF32, uint32_t WB>
@@ -114,7 +114,7 @@ __device__ __forceinline__ Smem carve(uint8_t* raw) {
     s.S = p; p += O::TILE64;
     s.raw = p; p += raw_bytes<TF32, WB>();
     s.gammaL = reinterpret_cast<float*>(p); p += 64 * 4;
-    s.red = reinterpret_cast<float*>(p); p += 128 * 4;
+    s.red = reinterpret_cast<float*>(p); p += 192 * 4;
     s.bar = reinterpret_cast<uint64_t*>(p); p += 8;
     s.raw_bar = reinterpret_cast<uint64_t*>(p); p += 8;
     s.tmem_slot = reinterpret_cast<uint32_t*>(p);
@@ -186,13 +186,19 @@ __device__ __forceinline__ void load_v_tile(const IO* __restrict__ v, long row0,
     }
 }
 
-template <typename IO, typename WT, bool TF32>
+// PRO (fp32 inputs only): the prologue of the WKV call is applied to the raw
+// inputs in the element-wise stage (wkv7_forward_fused): k and v are rows of kv
+// head h / (H / H_kv), `a` carries a_lr, and per token
+//   kk = k / max(||k||, 1e-12),  a = -kk,  b = kk a_lr,  k <- k (1 - w + a_lr);
+// `b` is not read.
+template <typename IO, typename WT, bool TF32, bool PRO>
 __global__ void __launch_bounds__(NT, 1)
     wkv7_prefill_kernel(const IO* __restrict__ r, const WT* __restrict__ wl, const IO* __restrict__ k,
                         const IO* __restrict__ v, const IO* __restrict__ a, const IO* __restrict__ b,
                         const float* s0, IO* __restrict__ y, float* sT, int T, int H,
-                        const int32_t* __restrict__ seq_offsets, int* status,
+                        const int32_t* __restrict__ seq_offsets, int* status, int H_kv,
                         const __grid_constant__ TmaMaps maps) {
+    static_assert(TF32 || !PRO, "the prologue is fused into the fp32 path only");
     using O = OpType<TF32>;
     constexpr uint32_t WB = sizeof(WT);
     extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -223,6 +229,8 @@ __global__ void __launch_bounds__(NT, 1)
     }
     const long tstride = static_cast<long>(H) * kHead;  // elements between consecutive tokens
     const long hoff = static_cast<long>(h) * kHead;
+    const long tstride_kv = PRO ? static_cast<long>(H_kv) * kHead : tstride;  // k and v rows
+    const long hoff_kv = PRO ? static_cast<long>(h / (H / H_kv)) * kHead : hoff;
     const long sbase = (static_cast<long>(n) * H + h) * kHead * kHead;
 
     // ---- set-up: barrier, TMEM
@@ -287,6 +295,21 @@ __global__ void __launch_bounds__(NT, 1)
                 cp[q] = prod;
             }
             sm.red[hf * 64 + j] = prod;
+            if constexpr (PRO) {
+                // 1 / max(||k_t||, 1e-12) of token t = tid / 2: each thread of the pair sums 32 channels
+                const int t = tid >> 1, c0 = (tid & 1) * 32;
+                float ss = 0.f;
+                if (t < nv) {
+                    const IO* kr = k + (row0 + t) * tstride_kv + hoff_kv + c0;
+#pragma unroll 8
+                    for (int i = 0; i < 32; ++i) {
+                        const float x = to_f32(kr[i]);
+                        ss = fmaf(x, x, ss);
+                    }
+                }
+                ss += __shfl_xor_sync(0xffffffffu, ss, 1);
+                if ((tid & 1) == 0) sm.red[128 + t] = 1.f / fmaxf(sqrtf(ss), 1e-12f);
+            }
             __syncthreads();
             const float pre = hf ? sm.red[j] : 1.f;
             const float GL = sm.red[j] * sm.red[64 + j];
@@ -304,9 +327,13 @@ __global__ void __launch_bounds__(NT, 1)
                         if constexpr (TF32) {
                             const long off = (row0 + t) * tstride + hoff + j;
                             rr[e] = to_f32(r[off]);
-                            kk[e] = to_f32(k[off]);
                             aa[e] = to_f32(a[off]);
-                            bb[e] = to_f32(b[off]);
+                            if constexpr (PRO) {
+                                kk[e] = to_f32(k[(row0 + t) * tstride_kv + hoff_kv + j]);
+                            } else {
+                                kk[e] = to_f32(k[off]);
+                                bb[e] = to_f32(b[off]);
+                            }
                         } else {
                             rr[e] = to_f32(raw16[0 * 4096 + t * 64 + j]);
                             kk[e] = to_f32(raw16[1 * 4096 + t * 64 + j]);
@@ -321,6 +348,12 @@ __global__ void __launch_bounds__(NT, 1)
                     const float G = pre * cp[g * 8 + e];
                     const float inv = 1.f / G;
                     const float invL = inv * GL;
+                    if constexpr (PRO) {
+                        const float w = G / gprev, kn = kk[e] * sm.red[128 + t];  // w_t and kk
+                        bb[e] = kn * aa[e];
+                        kk[e] *= 1.f - w + aa[e];
+                        aa[e] = -kn;
+                    }
                     st_op<TF32>(sm.RA, 128, t, j, rr[e] * G);
                     st_op<TF32>(sm.RA, 128, 64 + t, j, aa[e] * gprev);
                     st_op<TF32>(sm.BK, 128, t, j, bb[e] * inv);
@@ -330,7 +363,7 @@ __global__ void __launch_bounds__(NT, 1)
                     gprev = G;
                 }
             }
-            if constexpr (TF32) load_v_tile<IO, TF32>(v, row0, tstride, hoff, nv, sm.V[0], tid);
+            if constexpr (TF32) load_v_tile<IO, TF32>(v, row0, tstride_kv, hoff_kv, nv, sm.V[0], tid);
         }
         fence_proxy_async_smem();
         tc_fence_before();
@@ -564,17 +597,17 @@ __global__ void __launch_bounds__(NT, 1)
     }
 }
 
-template <typename IO, typename WT, bool TF32>
+template <typename IO, typename WT, bool TF32, bool PRO>
 cudaError_t launch_typed(const PrefillArgs& p, cudaStream_t stream) {
     constexpr uint32_t smem = smem_bytes_needed<TF32, sizeof(WT)>();
     TmaMaps maps;  // unused by the fp32 path
     memset(&maps, 0, sizeof(maps));
     if constexpr (!TF32) {
         const uint64_t ntok = p.seq_offsets ? static_cast<uint64_t>(p.T) : static_cast<uint64_t>(p.B) * p.T;
-        if (!make_prefill_maps(&maps, p.r, p.w_log, p.k, p.v, p.a, p.b, p.H, ntok, sizeof(WT)))
+        if (!make_prefill_maps(&maps, p.r, p.w_log, p.k, p.v, p.a, p.b, p.H, p.H, ntok, sizeof(WT)))
             return cudaErrorInvalidValue;
     }
-    auto kern = wkv7_prefill_kernel<IO, WT, TF32>;
+    auto kern = wkv7_prefill_kernel<IO, WT, TF32, PRO>;
     static unsigned long long configured = 0;  // one bit per device ordinal
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
@@ -589,7 +622,7 @@ cudaError_t launch_typed(const PrefillArgs& p, cudaStream_t stream) {
     kern<<<static_cast<unsigned>(units), NT, smem, stream>>>(
         static_cast<const IO*>(p.r), static_cast<const WT*>(p.w_log), static_cast<const IO*>(p.k),
         static_cast<const IO*>(p.v), static_cast<const IO*>(p.a), static_cast<const IO*>(p.b), p.s0,
-        static_cast<IO*>(p.y), p.sT, p.T, p.H, p.seq_offsets, p.status, maps);
+        static_cast<IO*>(p.y), p.sT, p.T, p.H, p.seq_offsets, p.status, PRO ? p.H_kv : p.H, maps);
     return cudaGetLastError();
 }
 
@@ -607,8 +640,11 @@ __global__ void expire_wait_kernel(int spins, int* status) {
 
 cudaError_t launch_prefill(const PrefillArgs& p, int io_dtype, int w_dtype, cudaStream_t stream) {
     if (io_dtype == WKV7_BF16) return launch_prefill_pipe(p, w_dtype, stream);
-    return w_dtype == WKV7_BF16 ? launch_typed<float, __nv_bfloat16, true>(p, stream)
-                                : launch_typed<float, float, true>(p, stream);
+    if (p.prologue)
+        return w_dtype == WKV7_BF16 ? launch_typed<float, __nv_bfloat16, true, true>(p, stream)
+                                    : launch_typed<float, float, true, true>(p, stream);
+    return w_dtype == WKV7_BF16 ? launch_typed<float, __nv_bfloat16, true, false>(p, stream)
+                                : launch_typed<float, float, true, false>(p, stream);
 }
 
 cudaError_t launch_expire_wait(int spins, int* status, cudaStream_t stream) {

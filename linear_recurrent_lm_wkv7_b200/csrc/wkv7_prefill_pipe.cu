@@ -171,16 +171,40 @@ struct Bars {
     uint32_t* tmem_slot;
 };
 
+// Sum over a warp of 8 per-token partial sums (lane jp holds its share of
+// tokens 0..7): a reduce-scatter over lane bits 4, 3, 2 leaves token
+// (jp >> 2) & 7 in lanes 4m .. 4m + 3, and two more steps complete the sum, so
+// lane 4m returns the total of token m.  9 shuffles for 8 tokens.
+__device__ __forceinline__ float sum8_scatter(const float (&pd)[8], int jp) {
+    const bool b4 = (jp & 16) != 0, b3 = (jp & 8) != 0, b2 = (jp & 4) != 0;
+    float q4[4], q2[2];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+        q4[i] = (b4 ? pd[4 + i] : pd[i]) + __shfl_xor_sync(0xffffffffu, b4 ? pd[i] : pd[4 + i], 16);
+#pragma unroll
+    for (int i = 0; i < 2; ++i)
+        q2[i] = (b3 ? q4[2 + i] : q4[i]) + __shfl_xor_sync(0xffffffffu, b3 ? q4[i] : q4[2 + i], 8);
+    float q1 = (b2 ? q2[1] : q2[0]) + __shfl_xor_sync(0xffffffffu, b2 ? q2[0] : q2[1], 4);
+    q1 += __shfl_xor_sync(0xffffffffu, q1, 2);
+    q1 += __shfl_xor_sync(0xffffffffu, q1, 1);
+    return q1;
+}
+
 // GATED: the output rows are z = (y / sqrt(D) + u v) (.) g with u = sum_d r k rk
 // (the read-out of wkv7_forward_gated) instead of y.
-template <typename WT, bool GATED>
+// PRO: the prologue of the WKV call is applied to the raw inputs in the
+// element-wise stage (wkv7_forward_fused): k and v are rows of kv head
+// h / (H / H_kv), the `a` tile carries a_lr, and per token
+//   kk = k / max(||k||, 1e-12),  a = -kk,  b = kk a_lr,  k <- k (1 - w + a_lr);
+// `b` is not read.
+template <typename WT, bool GATED, bool PRO>
 __global__ void __launch_bounds__(NTHR, 1)
     wkv7_prefill_pipe_kernel(const __nv_bfloat16* __restrict__ r, const WT* __restrict__ wl,
                              const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restrict__ v,
                              const __nv_bfloat16* __restrict__ a, const __nv_bfloat16* __restrict__ b,
                              const float* s0, __nv_bfloat16* __restrict__ y, float* sT, int T, int H,
                              const int32_t* __restrict__ seq_offsets, int* status,
-                             const float* __restrict__ rk, const __nv_bfloat16* __restrict__ gte,
+                             const float* __restrict__ rk, const __nv_bfloat16* __restrict__ gte, int H_kv,
                              const __grid_constant__ TmaMaps maps) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     // 1024-byte aligned base, derived from the shared array so that every tile pointer
@@ -205,6 +229,7 @@ __global__ void __launch_bounds__(NTHR, 1)
     // ---- the unit and its tokens
     const int unit = blockIdx.x;
     const int n = unit / H, h = unit % H;
+    const int hk = PRO ? h / (H / H_kv) : h;  // kv head of k and v
     long tb = 0, len = 0;
     if (seq_offsets) {
         const long o0 = seq_offsets[n], o1 = seq_offsets[n + 1];
@@ -220,6 +245,8 @@ __global__ void __launch_bounds__(NTHR, 1)
     }
     const long tstride = static_cast<long>(H) * kHead;
     const long hoff = static_cast<long>(h) * kHead;
+    const long tstride_kv = static_cast<long>(PRO ? H_kv : H) * kHead;
+    const long hoff_kv = static_cast<long>(hk) * kHead;
     const long sbase = (static_cast<long>(n) * H + h) * kHead * kHead;
     const int nchunks = static_cast<int>((len + L - 1) / L);
 
@@ -281,7 +308,10 @@ __global__ void __launch_bounds__(NTHR, 1)
             } else if (which == 1) {
                 mbar_arrive_expect_tx(&bars.rrk[g], 2u * 8192u);
                 tma_load_3d(gt + RAW_R, &maps.r, &bars.rrk[g], 0, h, t0);
-                tma_load_3d(gt + RAW_K, &maps.k, &bars.rrk[g], 0, h, t0);
+                tma_load_3d(gt + RAW_K, &maps.k, &bars.rrk[g], 0, hk, t0);
+            } else if constexpr (PRO) {
+                mbar_arrive_expect_tx(&bars.rab[g], 8192u);
+                tma_load_3d(gt + RAW_A, &maps.a, &bars.rab[g], 0, h, t0);
             } else {
                 mbar_arrive_expect_tx(&bars.rab[g], 2u * 8192u);
                 tma_load_3d(gt + RAW_A, &maps.a, &bars.rab[g], 0, h, t0);
@@ -290,7 +320,7 @@ __global__ void __launch_bounds__(NTHR, 1)
         };
         auto issue_v = [&](int cc) {  // one thread
             mbar_arrive_expect_tx(&bars.vld[g], 8192u);
-            tma_load_3d(Vt, &maps.v, &bars.vld[g], 0, h, static_cast<int>(tb + static_cast<long>(cc) * L));
+            tma_load_3d(Vt, &maps.v, &bars.vld[g], 0, hk, static_cast<int>(tb + static_cast<long>(cc) * L));
         };
         if (g < nchunks) {
             if (tg == 0) {
@@ -407,24 +437,48 @@ __global__ void __launch_bounds__(NTHR, 1)
                         rr[e] = rawr[idx];
                         kv[e] = rawk[idx];
                         av[e] = rawa[idx];
-                        bv[e] = rawb[idx];
+                        if constexpr (!PRO) bv[e] = rawb[idx];
                     }
                     __syncwarp();
+                    float rn[8];  // prologue: 1 / max(||k_t||, 1e-12) of the 8 tokens, in every lane
+                    if constexpr (PRO) {
+                        float ss[8];
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) {
+                            const float2 kf = unpack_bf16x2(kv[e]);
+                            ss[e] = kf.x * kf.x + kf.y * kf.y;
+                        }
+                        const float inv = 1.f / fmaxf(sqrtf(sum8_scatter(ss, jp)), 1e-12f);
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) rn[e] = __shfl_sync(0xffffffffu, inv, 4 * e);
+                    }
                     uint32_t bh0[4], bh1[4], kh0[4], kh1[4];  // 8 tokens of Bh^T / Kh^T rows j0, j0 + 1
                     float pd[8];                              // this thread's part of u for 8 tokens
 #pragma unroll
                     for (int e = 0; e < 8; ++e) {
                         const int t = t0 + e;
-                        float2 G;  // Gamma_t
+                        float2 G, wv;  // Gamma_t and (prologue) w_t
                         if constexpr (sizeof(WT) == 4) {
                             G = __fmul2_rn(pre, *reinterpret_cast<const float2*>(rawl + t * 64 + j0));
+                            if constexpr (PRO) wv = make_float2(__fdividef(G.x, gp.x), __fdividef(G.y, gp.y));
                         } else {
-                            G = __fmul2_rn(gp, decay2(ld_wlog2(rawl, t * 64 + j0)));
+                            wv = decay2(ld_wlog2(rawl, t * 64 + j0));
+                            G = __fmul2_rn(gp, wv);
                         }
                         const float2 iv = make_float2(__fdividef(1.f, G.x), __fdividef(1.f, G.y));
                         const float2 l = __fmul2_rn(iv, GL);
-                        const float2 rf = unpack_bf16x2(rr[e]), kf = unpack_bf16x2(kv[e]);
-                        const float2 af = unpack_bf16x2(av[e]), bf = unpack_bf16x2(bv[e]);
+                        const float2 rf = unpack_bf16x2(rr[e]);
+                        float2 kf = unpack_bf16x2(kv[e]), af, bf;
+                        if constexpr (PRO) {
+                            const float2 alr = unpack_bf16x2(av[e]);
+                            const float2 kn = make_float2(kf.x * rn[e], kf.y * rn[e]);  // kk
+                            af = make_float2(-kn.x, -kn.y);
+                            bf = __fmul2_rn(kn, alr);
+                            kf = __fmul2_rn(kf, make_float2(1.f - wv.x + alr.x, 1.f - wv.y + alr.y));
+                        } else {
+                            af = unpack_bf16x2(av[e]);
+                            bf = unpack_bf16x2(bv[e]);
+                        }
                         if constexpr (GATED) pd[e] = rf.x * kf.x * rkv.x + rf.y * kf.y * rkv.y;
                         *reinterpret_cast<uint32_t*>(RAM + swz(t, cb, 128)) = pack2(__fmul2_rn(rf, G));
                         *reinterpret_cast<uint32_t*>(RAM + swz(64 + t, cb, 128)) = pack2(__fmul2_rn(af, gp));
@@ -445,20 +499,8 @@ __global__ void __launch_bounds__(NTHR, 1)
                         gp = G;
                     }
                     if constexpr (GATED) {
-                        // u of the 8 tokens: the warp's 32 lanes cover the 64 key channels.  A
-                        // reduce-scatter over lane bits 4, 3, 2 leaves token (lane >> 2) & 7 in
-                        // lanes 4m .. 4m + 3, and two more steps complete the sum.
-                        const bool b4 = (jp & 16) != 0, b3 = (jp & 8) != 0, b2 = (jp & 4) != 0;
-                        float q4[4], q2[2];
-#pragma unroll
-                        for (int i = 0; i < 4; ++i)
-                            q4[i] = (b4 ? pd[4 + i] : pd[i]) + __shfl_xor_sync(0xffffffffu, b4 ? pd[i] : pd[4 + i], 16);
-#pragma unroll
-                        for (int i = 0; i < 2; ++i)
-                            q2[i] = (b3 ? q4[2 + i] : q4[i]) + __shfl_xor_sync(0xffffffffu, b3 ? q4[i] : q4[2 + i], 8);
-                        float q1 = (b2 ? q2[1] : q2[0]) + __shfl_xor_sync(0xffffffffu, b2 ? q2[0] : q2[1], 4);
-                        q1 += __shfl_xor_sync(0xffffffffu, q1, 2);
-                        q1 += __shfl_xor_sync(0xffffffffu, q1, 1);
+                        // u of the 8 tokens: the warp's 32 lanes cover the 64 key channels
+                        const float q1 = sum8_scatter(pd, jp);
                         if ((jp & 3) == 0)
                             reinterpret_cast<float*>(sm + OFF_U)[g * 128 + (kk_ & 1) * 64 + t0 + ((jp >> 2) & 7)] = q1;
                     }
@@ -748,9 +790,10 @@ __global__ void __launch_bounds__(NTHR, 1)
             if constexpr (GATED) {
                 if (ts < nv) {
                     const long off = (row0 + ts) * tstride + hoff;
+                    const long voff = PRO ? (row0 + ts) * tstride_kv + hoff_kv : off;
 #pragma unroll
                     for (int i = 0; i < 8; ++i) {
-                        vpre[i] = *reinterpret_cast<const uint4*>(v + off + 8 * i);
+                        vpre[i] = *reinterpret_cast<const uint4*>(v + voff + 8 * i);
                         gpre[i] = *reinterpret_cast<const uint4*>(gte + off + 8 * i);
                     }
                 }
@@ -836,9 +879,9 @@ __global__ void __launch_bounds__(NTHR, 1)
     }
 }
 
-template <typename WT, bool GATED>
+template <typename WT, bool GATED, bool PRO>
 cudaError_t launch_pipe_typed(const PrefillArgs& p, cudaStream_t stream) {
-    auto kern = wkv7_prefill_pipe_kernel<WT, GATED>;
+    auto kern = wkv7_prefill_pipe_kernel<WT, GATED, PRO>;
     static unsigned long long configured = 0;
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
@@ -851,25 +894,34 @@ cudaError_t launch_pipe_typed(const PrefillArgs& p, cudaStream_t stream) {
     }
     TmaMaps maps;
     const uint64_t ntok = p.seq_offsets ? static_cast<uint64_t>(p.T) : static_cast<uint64_t>(p.B) * p.T;
-    if (!make_prefill_maps(&maps, p.r, p.w_log, p.k, p.v, p.a, p.b, p.H, ntok, sizeof(WT))) return cudaErrorInvalidValue;
+    const int H_kv = PRO ? p.H_kv : p.H;
+    if (!make_prefill_maps(&maps, p.r, p.w_log, p.k, p.v, p.a, PRO ? nullptr : p.b, p.H, H_kv, ntok, sizeof(WT)))
+        return cudaErrorInvalidValue;
     const long units = static_cast<long>(p.B) * p.H;
     kern<<<static_cast<unsigned>(units), NTHR, SMEM_BYTES, stream>>>(
         static_cast<const __nv_bfloat16*>(p.r), static_cast<const WT*>(p.w_log),
         static_cast<const __nv_bfloat16*>(p.k), static_cast<const __nv_bfloat16*>(p.v),
         static_cast<const __nv_bfloat16*>(p.a), static_cast<const __nv_bfloat16*>(p.b), p.s0,
         static_cast<__nv_bfloat16*>(p.y), p.sT, p.T, p.H, p.seq_offsets, p.status, p.rk,
-        static_cast<const __nv_bfloat16*>(p.g), maps);
+        static_cast<const __nv_bfloat16*>(p.g), H_kv, maps);
     return cudaGetLastError();
 }
 
 }  // namespace
 
 cudaError_t launch_prefill_pipe(const PrefillArgs& p, int w_dtype, cudaStream_t stream) {
+    if (p.prologue) {
+        if (p.rk)
+            return w_dtype == WKV7_BF16 ? launch_pipe_typed<__nv_bfloat16, true, true>(p, stream)
+                                        : launch_pipe_typed<float, true, true>(p, stream);
+        return w_dtype == WKV7_BF16 ? launch_pipe_typed<__nv_bfloat16, false, true>(p, stream)
+                                    : launch_pipe_typed<float, false, true>(p, stream);
+    }
     if (p.rk)
-        return w_dtype == WKV7_BF16 ? launch_pipe_typed<__nv_bfloat16, true>(p, stream)
-                                    : launch_pipe_typed<float, true>(p, stream);
-    return w_dtype == WKV7_BF16 ? launch_pipe_typed<__nv_bfloat16, false>(p, stream)
-                                : launch_pipe_typed<float, false>(p, stream);
+        return w_dtype == WKV7_BF16 ? launch_pipe_typed<__nv_bfloat16, true, false>(p, stream)
+                                    : launch_pipe_typed<float, true, false>(p, stream);
+    return w_dtype == WKV7_BF16 ? launch_pipe_typed<__nv_bfloat16, false, false>(p, stream)
+                                : launch_pipe_typed<float, false, false>(p, stream);
 }
 
 }  // namespace wkv7

@@ -113,3 +113,48 @@ def test_forward_gated_rejects_bad_arguments(wk):
     assert call(*_fwd_gated(z=0x1000 + 0x800000)) == -1  # z aliases g
     assert call(*_fwd_gated(z=0x1000 + 0x700000)) == -1  # z overlaps r_k
     assert call(*_fwd_gated(z=0x1000)) == -1  # z aliases r
+
+
+# argument tuple for wkv7_forward_fused: 10 pointers, B, T, H, H_kv, D, offsets, io, w, stream
+def _fwd_fused(ptr=0x1000, B=1, T=8, H=4, H_kv=2, D=64, offs=None, io=1, wd=0, **over):
+    p = dict(r=ptr, w=ptr + 0x100000, k=ptr + 0x200000, v=ptr + 0x300000, alr=ptr + 0x400000, s0=None, rk=None,
+             g=None, out=ptr + 0x600000, sT=None)
+    p.update(over)
+    return (p["r"], p["w"], p["k"], p["v"], p["alr"], p["s0"], p["rk"], p["g"], p["out"], p["sT"], B, T, H, H_kv,
+            D, offs, io, wd, None)
+
+
+def test_forward_fused_rejects_bad_arguments(wk):
+    call = wk._binding.raw_call_forward_fused
+    assert call(*_fwd_fused(H_kv=3)) == -1  # H not a multiple of H_kv
+    assert call(*_fwd_fused(H_kv=0)) == -1
+    assert call(*_fwd_fused(H_kv=8)) == -1  # more kv heads than heads
+    assert call(*_fwd_fused(rk=0x1000 + 0x700000)) == -1  # r_k without g
+    assert call(*_fwd_fused(g=0x1000 + 0x800000)) == -1  # g without r_k
+    assert call(*_fwd_fused(alr=None)) == -1
+    assert call(*_fwd_fused(D=32)) == -2
+    assert call(*_fwd_fused(k=0x1008 + 0x200000)) == -3  # misaligned
+    assert call(*_fwd_fused(out=0x1000 + 0x200000)) == -1  # out aliases k
+    # k holds T * H_kv * D bf16 = 2 KB; out starting 1 KB into it overlaps
+    assert call(*_fwd_fused(out=0x1000 + 0x200000 + 1024)) == -1
+    assert call(*_fwd_fused(sT=0x1000 + 0x300000)) == -1  # sT overlaps v
+
+
+def test_decode_fused_rejects_bad_arguments(wk):
+    call = wk._binding.raw_call_decode_fused
+
+    def args(B=2, H=4, H_kv=2, D=64, **over):
+        p = dict(r=0x1000, w=0x101000, k=0x201000, v=0x301000, alr=0x401000, s_in=None, rk=None, g=None,
+                 out=0x601000, s_out=0x701000)
+        p.update(over)
+        return (p["r"], p["w"], p["k"], p["v"], p["alr"], p["s_in"], p["rk"], p["g"], p["out"], p["s_out"], B, H,
+                H_kv, D, 1, 1, None)
+
+    assert call(*args(H_kv=3)) == -1
+    assert call(*args(rk=0x801000)) == -1  # r_k without g
+    assert call(*args(alr=None)) == -1
+    assert call(*args(s_out=None)) == -1
+    assert call(*args(D=32)) == -2
+    assert call(*args(g=0x901008, rk=0x801000)) == -3  # misaligned gate
+    assert call(*args(out=0x201000)) == -1  # out aliases k
+    assert call(*args(s_out=0x401000)) == -1  # s_out overlaps a_lr
