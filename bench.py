@@ -35,6 +35,7 @@ if ROOT not in sys.path:
 METRIC = "WKV7 prefill tokens/s and decode steps/s on 1 B200; % of roofline"
 PREFILL_WORKLOAD = "prefill_1p5b"
 DECODE_WORKLOAD = "decode_2p9b"
+FUSED_HKV = 8  # kv heads of the fused-prologue measurement (4 query heads per kv head)
 D = 64
 L2_FLUSH_BYTES = 256 << 20
 
@@ -274,7 +275,34 @@ def run_ours(args):
         gms = float(t.item())
     gbytes = bytes_alg + B * T * H * D * 2 + H * D * 4  # + the bf16 gate and r_k
     gach = gbytes / (gms * 1e-3) / 1e9
-    del z, gate_d
+    del z
+
+    # ---------------- the fused layer path (wkv7_forward_fused): raw k, v of FUSED_HKV kv heads
+    # and a_lr in, the prologue and the gated read-out inside the kernel
+    fin = W.make_fused(B, T, H, FUSED_HKV, io="bf16", wdt="f32", seed=3 + 1000 * rank)
+    fd = {k_: v_.cuda() for k_, v_ in fin.tensors().items()}
+    del fin
+    zf = torch.empty_like(dev["r"])
+
+    def fstep():
+        wk.wkv7_forward_fused(fd["r"], fd["w_log"], fd["k"], fd["v"], fd["a_lr"], None, rk_d, gate_d, zf, sT, B, T,
+                              H, FUSED_HKV, D, None, stream)
+
+    for _ in range(max(3, args.warmup)):
+        fstep()
+    torch.cuda.synchronize()
+    ftimes = time_launches(fstep, args.steps, stream, flush)
+    if wk.wkv7_get_device_status() != 0:
+        raise RuntimeError("device status set during the fused run")
+    fms = sum(ftimes) / len(ftimes)
+    if world > 1:
+        t = torch.tensor([fms], device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        fms = float(t.item())
+    # r, a_lr, g, z (bf16) and w_log (fp32) per token-head; k, v (bf16) per token-kv-head; sT; r_k
+    fbytes = B * T * H * D * (2 + 2 + 2 + 2 + 4) + B * T * FUSED_HKV * D * 2 * 2 + B * H * D * D * 4 + H * D * 4
+    fach = fbytes / (fms * 1e-3) / 1e9
+    del zf, fd, gate_d
 
     # ---------------- end to end through the public API from pinned host memory
     y_h = torch.empty(y.shape, dtype=y.dtype).pin_memory()
@@ -364,6 +392,10 @@ def run_ours(args):
                       "ms_per_step": gms,
                       "roofline": {"bound": "hbm", "achieved": gach, "peak": hbm_peak, "unit": "GB/s",
                                    "frac": gach / hbm_peak, "algorithmic_bytes_per_launch": gbytes}},
+            "fused": {"workload": PREFILL_WORKLOAD, "H_kv": FUSED_HKV, "read_out": "gated",
+                      "tokens_per_s": world * tokens / (fms * 1e-3), "ms_per_step": fms,
+                      "roofline": {"bound": "hbm", "achieved": fach, "peak": hbm_peak, "unit": "GB/s",
+                                   "frac": fach / hbm_peak, "algorithmic_bytes_per_launch": fbytes}},
             "decode": {"workload": DECODE_WORKLOAD, "B": dB, "H": dH, "steps_per_s": 1000.0 / dms,
                        "tokens_per_s": world * dB / (dms * 1e-3), "ms_per_step": dms,
                        "timing": f"{nsteps} steps back to back, one event pair around them",
