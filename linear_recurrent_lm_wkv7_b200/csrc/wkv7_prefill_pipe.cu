@@ -111,20 +111,28 @@ __device__ __forceinline__ void mma_tf32_16x8x8(float (&d)[4], const uint32_t (&
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
 }
 
-// C[cr + 0..15][cc + 0..15] = sum over k-steps ks in [ks0, ks1) of
+// C[cr + 0..15][cc + 0..15] = sum over k-steps ks in [ks0, ks1) (0 <= ks0 < ks1 <= 4) of
 //   A[ar + 0..15][ac + 8 ks + 0..7] * B[bk + 8 ks + 0..7][bn + 0..15]   (one warp)
 // written to C (tf32, tf_idx layout) and/or to Cb (bf16, 128-byte swizzled rows); either may be null.
+// All fragments are loaded before the first product, so the loads of the k-steps overlap.
 __device__ __forceinline__ void tf32_tile16(const float* A, int ar, int ac, const float* B, int bk, int bn, int ks0,
                                             int ks1, float* C, uint8_t* Cb, int cr, int cc, int gq, int t4) {
     float d0[4] = {0.f, 0.f, 0.f, 0.f}, d1[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll 1
-    for (int ks = ks0; ks < ks1; ++ks) {
-        uint32_t af[4], b0[2], b1[2];
-        frag_a_tf32(A, ar, ac + 8 * ks, gq, t4, af);
-        frag_b_tf32(B, bk + 8 * ks, bn, gq, t4, b0);
-        frag_b_tf32(B, bk + 8 * ks, bn + 8, gq, t4, b1);
-        mma_tf32_16x8x8(d0, af, b0);
-        mma_tf32_16x8x8(d1, af, b1);
+    uint32_t af[4][4], b0[4][2], b1[4][2];
+#pragma unroll
+    for (int ks = 0; ks < 4; ++ks) {
+        if (ks >= ks0 && ks < ks1) {
+            frag_a_tf32(A, ar, ac + 8 * ks, gq, t4, af[ks]);
+            frag_b_tf32(B, bk + 8 * ks, bn, gq, t4, b0[ks]);
+            frag_b_tf32(B, bk + 8 * ks, bn + 8, gq, t4, b1[ks]);
+        }
+    }
+#pragma unroll
+    for (int ks = 0; ks < 4; ++ks) {
+        if (ks >= ks0 && ks < ks1) {
+            mma_tf32_16x8x8(d0, af[ks], b0[ks]);
+            mma_tf32_16x8x8(d1, af[ks], b1[ks]);
+        }
     }
     if (C) {
         frag_c_store_tf32(C, cr, cc, gq, t4, d0);
