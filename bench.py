@@ -368,6 +368,42 @@ def run_ours(args):
     dbytes = 2 * dB * dH * D * D * 4 + dB * dH * D * (6 * 2 + 2)
     dach = dbytes / (dms * 1e-3) / 1e9
 
+    # ---------------- fused decode step: raw k, v of FUSED_HKV kv heads, a_lr, gated read-out
+    fsteps = []
+    for s_ in range(4):
+        fi = W.make_fused(dB, 1, dH, FUSED_HKV, io=cfg["io"], wdt=cfg["wdt"], seed=cfg["seed"] + 100 * s_)
+        fsteps.append({k_: v_[:, 0].contiguous().cuda() for k_, v_ in fi.tensors().items()})
+    drk, _ = W.make_gate((dB, dH, D), dH, D, io=cfg["io"], seed=cfg["seed"])
+    _, dg = W.make_gate((dB, dH, D), dH, D, io=cfg["io"], seed=cfg["seed"] + 1)
+    drk, dg = drk.cuda(), dg.cuda()
+    fit = {"i": 0}
+
+    def dfstep():
+        d = fsteps[fit["i"] % len(fsteps)]
+        fit["i"] += 1
+        wk.wkv7_decode_step_fused(d["r"], d["w_log"], d["k"], d["v"], d["a_lr"], state, drk, dg, dy, state, dB, dH,
+                                  FUSED_HKV, D, stream)
+
+    for _ in range(max(3, args.warmup)):
+        dfstep()
+    torch.cuda.synchronize()
+    ls.record(stream)
+    for _ in range(nsteps):
+        dfstep()
+    le.record(stream)
+    torch.cuda.synchronize()
+    if wk.wkv7_get_device_status() != 0:
+        raise RuntimeError("device status set during the fused decode run")
+    dfms = ls.elapsed_time(le) / nsteps
+    if world > 1:
+        t = torch.tensor([dfms], device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        dfms = float(t.item())
+    # state in and out; r, w_log, a_lr, g, out per head row; k, v per kv-head row; r_k
+    dfbytes = 2 * dB * dH * D * D * 4 + dB * dH * D * 2 * 5 + dB * FUSED_HKV * D * 2 * 2 + dH * D * 4
+    dfach = dfbytes / (dfms * 1e-3) / 1e9
+    del fsteps
+
     if rank == 0:
         cb = oracle_baseline(budget_s=20.0) if (world == 1 and not args.no_cpu_baseline) else None
         line = {
@@ -402,6 +438,11 @@ def run_ours(args):
                        "ms_per_step_single_launch": dms_launch,
                        "roofline": {"bound": "hbm", "achieved": dach, "peak": hbm_peak, "unit": "GB/s",
                                     "frac": dach / hbm_peak, "algorithmic_bytes_per_launch": dbytes}},
+            "decode_fused": {"workload": DECODE_WORKLOAD, "H_kv": FUSED_HKV, "read_out": "gated",
+                             "steps_per_s": 1000.0 / dfms, "ms_per_step": dfms,
+                             "timing": f"{nsteps} steps back to back, one event pair around them",
+                             "roofline": {"bound": "hbm", "achieved": dfach, "peak": hbm_peak, "unit": "GB/s",
+                                          "frac": dfach / hbm_peak, "algorithmic_bytes_per_launch": dfbytes}},
         }
         print(json.dumps(line), flush=True)
     if world > 1:

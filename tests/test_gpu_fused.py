@@ -146,3 +146,23 @@ def test_fused_decode_matches_fused_prefill(wk):
     assert wk.wkv7_get_device_status() == 0
     assert relerr(yd.float().cpu().numpy(), y.float().cpu().numpy()) <= 2e-2
     assert relerr(state.cpu().numpy(), sT.cpu().numpy()) <= 2e-2
+
+
+def test_fused_decode_full_size(wk, oracle_mod):
+    """The 2.9B-class decode batch (B256 H40) with 8 kv heads and the read-out, two
+    chained steps, in the launch configuration of the benchmark."""
+    B, H, H_kv, D = 256, 40, 8, 64
+    state = W.make_state(B, H, std=0.1, seed=5).cuda()
+    sref = state.double().cpu().numpy()
+    rk, _ = W.make_gate((B, H, D), H, D, io="bf16", seed=6)
+    for step in range(2):
+        inp = W.make_fused(B, 1, H, H_kv, io="bf16", wdt="bf16", seed=2000 + step)
+        t = {n: x[:, 0].contiguous() for n, x in inp.tensors().items()}
+        _, g = W.make_gate((B, H, D), H, D, io="bf16", seed=70 + step)
+        d = {n: x.cuda() for n, x in t.items()}
+        out = wk.decode_step_fused(d["r"], d["w_log"], d["k"], d["v"], d["a_lr"], state, rk.cuda(), g.cuda())
+        assert wk.wkv7_get_device_status() == 0
+        ref, sref = oracle_mod.decode_step_fused(*(f64(t[n]) for n in ("r", "w_log", "k", "v", "a_lr")), sref,
+                                                 f64(rk), f64(g))
+        assert relerr(out.float().cpu().numpy(), ref) <= TOL["bf16"]
+    assert relerr(state.cpu().numpy(), sref) <= TOL["bf16"]
