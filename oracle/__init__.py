@@ -48,6 +48,8 @@ def _load():
         lib.wkv7_oracle_gate.restype = ctypes.c_int
         lib.wkv7_oracle_prologue.argtypes = [dp] * 8 + [ctypes.c_long, ctypes.c_int, ctypes.c_int, ctypes.c_int]
         lib.wkv7_oracle_prologue.restype = ctypes.c_int
+        lib.wkv7_oracle_backward.argtypes = [dp] * 16 + [ctypes.c_int] * 4 + [ip, ctypes.c_int]
+        lib.wkv7_oracle_backward.restype = ctypes.c_int
         _lib = lib
     return _lib
 
@@ -186,3 +188,32 @@ def decode_step_fused(r, w_log, k, v, a_lr, s_in, rk=None, g=None, n_threads=Non
     if rk is None and g is None:
         return y, s_out
     return gate(y, r, kp, vr, rk, g), s_out
+
+
+def backward(r, w_log, k, v, a, b, dy, s0=None, dsT=None, seq_offsets=None, n_threads=None):
+    """Gradient of L = sum <dy, y> + <dsT, sT> with respect to r, w_log, k, v, a, b
+    and s0.  Layouts as for ``forward``.  Returns ``(dr, dw_log, dk, dv, da, db, ds0)``
+    as float64 arrays."""
+    lib = _load()
+    r, w_log, k, v, a, b, dy = (_f64(t) for t in (r, w_log, k, v, a, b, dy))
+    for t in (w_log, k, v, a, b, dy):
+        if t.shape != r.shape:
+            raise ValueError("input shapes differ")
+    if seq_offsets is not None:
+        offs = np.ascontiguousarray(seq_offsets, dtype=np.int32)
+        T, H, D = r.shape
+        B = offs.size - 1
+        offs_p = offs.ctypes.data_as(ctypes.POINTER(ctypes.c_int32))
+    else:
+        B, T, H, D = r.shape
+        offs, offs_p = None, None
+    s0 = _f64(s0) if s0 is not None else None
+    dsT = _f64(dsT) if dsT is not None else None
+    grads = [np.zeros(r.shape, dtype=np.float64) for _ in range(6)]
+    ds0 = np.zeros((B, H, D, D), dtype=np.float64)
+    nt = default_threads() if n_threads is None else n_threads
+    rc = lib.wkv7_oracle_backward(_ptr(r), _ptr(w_log), _ptr(k), _ptr(v), _ptr(a), _ptr(b), _ptr(s0), _ptr(dy),
+                                  _ptr(dsT), *(_ptr(g) for g in grads), _ptr(ds0), B, T, H, D, offs_p, nt)
+    if rc != 0:
+        raise RuntimeError(f"wkv7_oracle_backward failed with status {rc}")
+    return tuple(grads) + (ds0,)

@@ -57,6 +57,23 @@
  * with a_lr the per-channel in-context learning rate (the listing's sigmoid
  * output "a").  The gated read-out after a prologue uses k' and the repeated v.
  *
+ * Backward (wkv7_oracle_backward): the gradient of a scalar loss
+ * L = sum_t <dy_t, y_t> + <dsT, S_T> with respect to every input of the
+ * recurrence above, by the chain rule through each step (the pages print no
+ * backward; this is the derivative of the forward definition).  Writing
+ * G = dL/dS_t and sweeping t = T .. 1 from G = dsT:
+ *
+ *   G    += dy_t r_t^T                      (y_t = S_t r_t)
+ *   dr_t  = S_t^T dy_t
+ *   dv_t  = G k_t,            dk_t = G^T v_t
+ *   q     = G b_t,            p    = S_{t-1} a_t
+ *   da_t  = S_{t-1}^T q,      db_t = G^T p
+ *   dw_t[j] = sum_i G[i][j] S_{t-1}[i][j]
+ *   dl_t[j] = dw_t[j] * (-exp(l_t[j]) w_t[j])   (w = exp(-exp(l)))
+ *   G     <- G diag(w_t) + q a_t^T          (dL/dS_{t-1})
+ *
+ * and ds0 = G at the end.  Every state S_0 .. S_T of the unit is kept.
+ *
  * Layouts (all double, contiguous, the fastest index last):
  *  dense  (seq_offsets == NULL): r, w_log, k, v, a, b, y are [B][T][H][D]
  *  packed (seq_offsets != NULL): they are [T][H][D] with T the packed length and
@@ -260,4 +277,151 @@ int wkv7_oracle_prologue(const double *k, const double *v, const double *w_log, 
         }
     }
     return 0;
+}
+
+typedef struct {
+    const double *r, *w_log, *k, *v, *a, *b, *s0, *dy, *dsT;
+    double *dr, *dw_log, *dk, *dv, *da, *db, *ds0;
+    int B, T, H, D;
+    const int32_t *seq_offsets;
+    long next_unit;
+    pthread_mutex_t lock;
+    int status;
+} oracle_bwd_job;
+
+static int bwd_unit(const oracle_bwd_job *jb, int n, int h) {
+    const int D = jb->D, H = jb->H;
+    long t0, t1;
+    if (jb->seq_offsets) {
+        t0 = jb->seq_offsets[n];
+        t1 = jb->seq_offsets[n + 1];
+    } else {
+        t0 = (long)n * jb->T;
+        t1 = t0 + jb->T;
+    }
+    const long len = t1 - t0, DD = (long)D * D, stride = (long)H * D, hoff = (long)h * D;
+    double *S = (double *)malloc(sizeof(double) * DD * (len + 1)); /* S_0 .. S_len */
+    double *G = (double *)malloc(sizeof(double) * DD);
+    double *w = (double *)malloc(sizeof(double) * D);
+    double *q = (double *)malloc(sizeof(double) * D);
+    double *pv = (double *)malloc(sizeof(double) * D);
+    if (!S || !G || !w || !q || !pv) {
+        free(S); free(G); free(w); free(q); free(pv);
+        return -2;
+    }
+    const long sb = ((long)n * H + h) * DD;
+    if (jb->s0) memcpy(S, jb->s0 + sb, sizeof(double) * DD);
+    else memset(S, 0, sizeof(double) * DD);
+    /* forward, keeping every state */
+    for (long t = 0; t < len; ++t) {
+        const long off = (t0 + t) * stride + hoff;
+        const double *Sp = S + t * DD;
+        double *Sn = S + (t + 1) * DD;
+        for (int j = 0; j < D; ++j) w[j] = exp(-exp(jb->w_log[off + j]));
+        for (int i = 0; i < D; ++i) {
+            double acc = 0.0;
+            for (int j = 0; j < D; ++j) acc += Sp[i * D + j] * jb->a[off + j];
+            pv[i] = acc;
+        }
+        for (int i = 0; i < D; ++i)
+            for (int j = 0; j < D; ++j)
+                Sn[i * D + j] = Sp[i * D + j] * w[j] + pv[i] * jb->b[off + j] + jb->v[off + i] * jb->k[off + j];
+    }
+    /* backward */
+    if (jb->dsT) memcpy(G, jb->dsT + sb, sizeof(double) * DD);
+    else memset(G, 0, sizeof(double) * DD);
+    for (long t = len - 1; t >= 0; --t) {
+        const long off = (t0 + t) * stride + hoff;
+        const double *Sp = S + t * DD, *St = S + (t + 1) * DD;
+        const double *r = jb->r + off, *k = jb->k + off, *v = jb->v + off, *a = jb->a + off, *b = jb->b + off;
+        const double *dy = jb->dy + off, *wl = jb->w_log + off;
+        for (int i = 0; i < D; ++i)
+            for (int j = 0; j < D; ++j) G[i * D + j] += dy[i] * r[j];
+        for (int j = 0; j < D; ++j) {
+            double acc = 0.0;
+            for (int i = 0; i < D; ++i) acc += St[i * D + j] * dy[i];
+            jb->dr[off + j] = acc;
+        }
+        for (int i = 0; i < D; ++i) {
+            double gk = 0.0, gb = 0.0, sa = 0.0;
+            for (int j = 0; j < D; ++j) {
+                gk += G[i * D + j] * k[j];
+                gb += G[i * D + j] * b[j];
+                sa += Sp[i * D + j] * a[j];
+            }
+            jb->dv[off + i] = gk;
+            q[i] = gb;
+            pv[i] = sa;
+        }
+        for (int j = 0; j < D; ++j) {
+            double gv = 0.0, sq = 0.0, gp = 0.0, gs = 0.0;
+            for (int i = 0; i < D; ++i) {
+                gv += G[i * D + j] * v[i];
+                sq += Sp[i * D + j] * q[i];
+                gp += G[i * D + j] * pv[i];
+                gs += G[i * D + j] * Sp[i * D + j];
+            }
+            jb->dk[off + j] = gv;
+            jb->da[off + j] = sq;
+            jb->db[off + j] = gp;
+            w[j] = exp(-exp(wl[j]));
+            jb->dw_log[off + j] = gs * (-exp(wl[j]) * w[j]);
+        }
+        for (int i = 0; i < D; ++i)
+            for (int j = 0; j < D; ++j) G[i * D + j] = G[i * D + j] * w[j] + q[i] * a[j];
+    }
+    memcpy(jb->ds0 + sb, G, sizeof(double) * DD);
+    free(S); free(G); free(w); free(q); free(pv);
+    return 0;
+}
+
+static void *bwd_worker(void *arg) {
+    oracle_bwd_job *jb = (oracle_bwd_job *)arg;
+    const long n_units = (long)jb->B * jb->H;
+    for (;;) {
+        pthread_mutex_lock(&jb->lock);
+        long u = jb->next_unit++;
+        pthread_mutex_unlock(&jb->lock);
+        if (u >= n_units) break;
+        if (bwd_unit(jb, (int)(u / jb->H), (int)(u % jb->H)) != 0) {
+            pthread_mutex_lock(&jb->lock);
+            jb->status = -2;
+            pthread_mutex_unlock(&jb->lock);
+        }
+    }
+    return NULL;
+}
+
+/* Layouts as for wkv7_oracle_forward; dy and the input gradients share the
+ * layout of r, dsT and ds0 that of the states.  s0 == NULL: zero initial state;
+ * dsT == NULL: no gradient on the final state. */
+int wkv7_oracle_backward(const double *r, const double *w_log, const double *k, const double *v, const double *a,
+                         const double *b, const double *s0, const double *dy, const double *dsT, double *dr,
+                         double *dw_log, double *dk, double *dv, double *da, double *db, double *ds0, int B, int T,
+                         int H, int D, const int32_t *seq_offsets, int n_threads) {
+    if (B <= 0 || T < 0 || H <= 0 || D <= 0) return -1;
+    if (seq_offsets) {
+        if (seq_offsets[0] != 0 || seq_offsets[B] != T) return -1;
+        for (int n = 0; n < B; ++n)
+            if (seq_offsets[n + 1] < seq_offsets[n]) return -1;
+    }
+    oracle_bwd_job jb;
+    jb.r = r; jb.w_log = w_log; jb.k = k; jb.v = v; jb.a = a; jb.b = b; jb.s0 = s0; jb.dy = dy; jb.dsT = dsT;
+    jb.dr = dr; jb.dw_log = dw_log; jb.dk = dk; jb.dv = dv; jb.da = da; jb.db = db; jb.ds0 = ds0;
+    jb.B = B; jb.T = T; jb.H = H; jb.D = D; jb.seq_offsets = seq_offsets;
+    jb.next_unit = 0;
+    jb.status = 0;
+    pthread_mutex_init(&jb.lock, NULL);
+    if (n_threads < 1) n_threads = 1;
+    if (n_threads > 256) n_threads = 256;
+    pthread_t tid[256];
+    int started = 0;
+    for (int i = 0; i < n_threads - 1; ++i) {
+        if (pthread_create(&tid[i], NULL, bwd_worker, &jb) != 0) break;
+        ++started;
+    }
+    bwd_worker(&jb);
+    for (int i = 0; i < started; ++i) pthread_join(tid[i], NULL);
+    pthread_mutex_destroy(&jb.lock);
+    return jb.status;
 }

@@ -399,3 +399,71 @@ def test_prologue_zero_key_is_identity_step(oracle_mod):
     y, s1 = oracle_mod.decode_step_fused(r, np.full((B, H, D), -np.inf), zero, zero, a_lr, s)
     np.testing.assert_array_equal(s1, s)
     assert np.all(np.isfinite(y))
+
+
+def _bwd_loss(oracle_mod, args, dy, dsT, offs=None):
+    y, sT = oracle_mod.forward(*args, seq_offsets=offs)
+    return float(np.sum(y * dy) + np.sum(sT * dsT))
+
+
+@pytest.mark.parametrize("packed", [False, True])
+def test_backward_matches_finite_differences(oracle_mod, packed):
+    """The backward's gradients of L = <dy, y> + <dsT, sT> against central
+    differences of the (separately pinned) forward along random directions, for
+    every input: r, w_log, k, v, a, b and s0.  fp64 with eps = 1e-6 leaves a
+    truncation and rounding error near 1e-9, so a dropped term, a wrong sign or
+    a transposed product fails by orders of magnitude."""
+    rng = np.random.default_rng(41 + packed)
+    B, T, H, D = 2, 7, 2, 64
+    r, w_log, k, v, a, b, S0 = _rand_inputs(rng, B, T, H, D)
+    dy = rng.standard_normal((B, T, H, D))
+    dsT = rng.standard_normal((B, H, D, D))
+    offs = None
+    if packed:
+        # sequences of 3 and 11 tokens on one packed axis
+        flat = lambda x: x.reshape(B * T, H, D)
+        r, w_log, k, v, a, b, dy = (flat(x).copy() for x in (r, w_log, k, v, a, b, dy))
+        offs = np.array([0, 3, 14], dtype=np.int32)
+    args = [r, w_log, k, v, a, b, S0]
+    grads = oracle_mod.backward(r, w_log, k, v, a, b, dy, S0, dsT, offs)
+    eps = 1e-6
+    for idx, X in enumerate(args):
+        for _ in range(2):
+            u = rng.standard_normal(X.shape)
+            plus = list(args)
+            minus = list(args)
+            plus[idx] = X + eps * u
+            minus[idx] = X - eps * u
+            fd = (_bwd_loss(oracle_mod, plus, dy, dsT, offs) - _bwd_loss(oracle_mod, minus, dy, dsT, offs)) / (2 * eps)
+            an = float(np.sum(grads[idx] * u))
+            assert abs(fd - an) <= 1e-6 * max(1.0, abs(an)), (idx, fd, an)
+
+
+def test_backward_linear_attention_closed_form(oracle_mod):
+    """a = b = 0 and w = 1 (l = -inf): y_t = S0 r_t + sum_{s<=t} (k_s . r_t) v_s, so
+    dv_s = sum_{t>=s} (r_t . k_s) dy_t + dsT k_s, dk_s = sum_{t>=s} (v_s . dy_t) r_t +
+    dsT^T v_s, dr_t = S_t^T dy_t, ds0 = sum_t dy_t r_t^T + dsT, and the decay logit,
+    a and b get the gradients of their linear terms.  Written with numpy from
+    this closed form."""
+    rng = np.random.default_rng(43)
+    B, T, H, D = 1, 6, 1, 64
+    r, _, k, v, _, _, S0 = _rand_inputs(rng, B, T, H, D)
+    zero = np.zeros((B, T, H, D))
+    w_log = np.full((B, T, H, D), -np.inf)
+    dy = rng.standard_normal((B, T, H, D))
+    dsT = rng.standard_normal((B, H, D, D))
+    dr, dwl, dk, dv, da, db, ds0 = oracle_mod.backward(r, w_log, k, v, zero, zero, dy, S0, dsT)
+    R, K, V, DY = (x[0, :, 0] for x in (r, k, v, dy))
+    mask = np.triu(np.ones((T, T)))  # mask[s, t] = 1 for t >= s
+    RK = (K @ R.T) * mask            # RK[s, t] = k_s . r_t for t >= s
+    VD = (V @ DY.T) * mask           # VD[s, t] = v_s . dy_t for t >= s
+    exp_dv = RK @ DY + K @ dsT[0, 0].T
+    exp_dk = VD @ R + V @ dsT[0, 0]
+    S = S0[0, 0] + np.cumsum(np.einsum("ti,tj->tij", V, K), axis=0)
+    exp_dr = np.einsum("tij,ti->tj", S, DY)
+    exp_ds0 = DY.T @ R + dsT[0, 0]
+    np.testing.assert_allclose(dv[0, :, 0], exp_dv, rtol=1e-10, atol=1e-10)
+    np.testing.assert_allclose(dk[0, :, 0], exp_dk, rtol=1e-10, atol=1e-10)
+    np.testing.assert_allclose(dr[0, :, 0], exp_dr, rtol=1e-10, atol=1e-10)
+    np.testing.assert_allclose(ds0[0, 0], exp_ds0, rtol=1e-10, atol=1e-10)
+    assert np.all(dwl == 0.0)  # w = 1 exactly: dw/dl = -exp(l) w = 0
