@@ -304,6 +304,34 @@ def run_ours(args):
     fach = fbytes / (fms * 1e-3) / 1e9
     del zf, fd, gate_d
 
+    # ---------------- backward of the recurrence (wkv7_backward), same workload
+    dy_h, _ = W.make_upstream(tuple(dev["r"].shape), B, H, D, io="bf16", seed=4 + 1000 * rank, with_dsT=False)
+    dyd = dy_h.cuda()
+    del dy_h
+    bgrads = [torch.empty_like(dev[n]) for n in ("r", "w_log", "k", "v", "a", "b")]
+    bds0 = torch.empty((B, H, D, D), dtype=torch.float32, device="cuda")
+    bws = torch.empty(wk.wkv7_backward_workspace_bytes(B, T, H, D, False) // 4, dtype=torch.float32, device="cuda")
+
+    def bstep():
+        wk.wkv7_backward(dev["r"], dev["w_log"], dev["k"], dev["v"], dev["a"], dev["b"], None, dyd, None,
+                         *bgrads, bds0, bws, B, T, H, D, None, stream)
+
+    for _ in range(3):
+        bstep()
+    torch.cuda.synchronize()
+    btimes = time_launches(bstep, max(3, args.steps // 5), stream, flush)
+    if wk.wkv7_get_device_status() != 0:
+        raise RuntimeError("device status set during the backward run")
+    bms = sum(btimes) / len(btimes)
+    if world > 1:
+        t = torch.tensor([bms], device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        bms = float(t.item())
+    # inputs (r, k, v, a, b, dy bf16; w_log fp32) in, gradients (bf16; dw_log fp32) out, ds0 out
+    bbytes = B * T * H * D * (6 * 2 + 4) + B * T * H * D * (5 * 2 + 4) + B * H * D * D * 4
+    bach = bbytes / (bms * 1e-3) / 1e9
+    del bgrads, bds0, bws, dyd
+
     # ---------------- end to end through the public API from pinned host memory
     y_h = torch.empty(y.shape, dtype=y.dtype).pin_memory()
     sT_h = torch.empty(sT.shape, dtype=sT.dtype).pin_memory()
@@ -432,6 +460,10 @@ def run_ours(args):
                       "tokens_per_s": world * tokens / (fms * 1e-3), "ms_per_step": fms,
                       "roofline": {"bound": "hbm", "achieved": fach, "peak": hbm_peak, "unit": "GB/s",
                                    "frac": fach / hbm_peak, "algorithmic_bytes_per_launch": fbytes}},
+            "backward": {"workload": PREFILL_WORKLOAD, "tokens_per_s": world * tokens / (bms * 1e-3),
+                         "ms_per_step": bms, "form": "recurrent (chunk checkpoints, per-token sweep)",
+                         "roofline": {"bound": "hbm", "achieved": bach, "peak": hbm_peak, "unit": "GB/s",
+                                      "frac": bach / hbm_peak, "algorithmic_bytes_per_launch": bbytes}},
             "decode": {"workload": DECODE_WORKLOAD, "B": dB, "H": dH, "steps_per_s": 1000.0 / dms,
                        "tokens_per_s": world * dB / (dms * 1e-3), "ms_per_step": dms,
                        "timing": f"{nsteps} steps back to back, one event pair around them",

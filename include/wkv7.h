@@ -44,6 +44,7 @@
 #ifndef WKV7_H
 #define WKV7_H
 
+#include <stddef.h>
 #include <stdint.h>
 
 #ifdef __cplusplus
@@ -169,6 +170,34 @@ int wkv7_decode_step_fused(const void* r, const void* w_log, const void* k, cons
                            const void* a_lr, const float* s_in, const float* r_k, const void* g,
                            void* out, float* s_out, int B, int H, int H_kv, int D,
                            int io_dtype, int w_dtype, void* stream);
+
+/*
+ * wkv7_backward — gradient of the recurrence of wkv7_forward (training).  For
+ * the scalar L = sum over tokens of <dy_t, y_t> + <dsT, S_T>, writes
+ * dL/dr, dL/dw_log, dL/dk, dL/dv, dL/da, dL/db and dL/ds0 (the chain rule
+ * through each step of the generalized delta rule of "RWKV-7 Goose: Expressive
+ * Dynamic State Evolution", section "Generalized Delta rule"; the pages print no
+ * backward).
+ *   r .. b, s0, seq_offsets, B, T, H, D, dtype codes : as in wkv7_forward.
+ *   dy  : gradient of y, same shape and dtype code as r.
+ *   dsT : [B][H][D][D] fp32 gradient of the final state, or NULL (zero).
+ *   dr, dk, dv, da, db : outputs, same shape and dtype code as r;
+ *   dw_log : output, same shape and dtype code as w_log; ds0 : [B][H][D][D] fp32
+ *          (written even when s0 is NULL: the gradient of a zero initial state).
+ *   workspace : DEVICE scratch of at least
+ *          wkv7_backward_workspace_bytes(B, T, H, D, seq_offsets != NULL) bytes,
+ *          owned by the caller and not read before it is written.
+ * Every output and the workspace must be disjoint from every input and from
+ * each other.  Recurrent form: one block per (sequence, head) recomputes the
+ * states of each 64-token chunk from checkpoints and sweeps the tokens backward.
+ */
+size_t wkv7_backward_workspace_bytes(int B, int T, int H, int D, int packed);
+int wkv7_backward(const void* r, const void* w_log, const void* k, const void* v,
+                  const void* a, const void* b, const float* s0, const void* dy,
+                  const float* dsT, void* dr, void* dw_log, void* dk, void* dv,
+                  void* da, void* db, float* ds0, void* workspace, size_t workspace_bytes,
+                  int B, int T, int H, int D, const int32_t* seq_offsets,
+                  int io_dtype, int w_dtype, void* stream);
 
 /* Human-readable text for a status code (static storage, never NULL). */
 const char* wkv7_status_string(int status);

@@ -4,8 +4,8 @@ decode step behind a C ABI (``include/wkv7.h``, ``libwkv7.so``).
 The Python layer only marshals arguments to the CUDA library; importing the
 package loads ``libwkv7.so`` and fails loudly if it has not been built.
 Convenience wrappers ``forward``, ``forward_gated``, ``forward_fused``,
-``decode_step`` and ``decode_step_fused`` allocate outputs with torch and call
-the C entry points.
+``decode_step``, ``decode_step_fused`` and ``backward`` allocate outputs with
+torch and call the C entry points.
 """
 from __future__ import annotations
 
@@ -17,6 +17,8 @@ from ._binding import (  # noqa: F401
     WKV7_F32,
     Wkv7Error,
     _lib,
+    wkv7_backward,
+    wkv7_backward_workspace_bytes,
     wkv7_debug_expire_wait,
     wkv7_decode_step,
     wkv7_decode_step_fused,
@@ -95,6 +97,28 @@ def decode_step_fused(r, w_log, k, v, a_lr, state, r_k=None, g=None, out=None, s
         out = torch.empty_like(r)
     wkv7_decode_step_fused(r, w_log, k, v, a_lr, state, r_k, g, out, state, B, H, k.shape[-2], D, stream)
     return out
+
+
+def backward(r, w_log, k, v, a, b, dy, s0=None, dsT=None, seq_offsets=None, workspace=None, stream=None):
+    """Gradient of <dy, y> + <dsT, sT> with respect to r, w_log, k, v, a, b and s0.
+    Layouts as for ``forward``.  ``workspace`` (a device tensor of at least
+    ``wkv7_backward_workspace_bytes`` bytes) is allocated when not given.
+    Returns ``(dr, dw_log, dk, dv, da, db, ds0)``."""
+    import torch
+
+    if seq_offsets is not None:
+        T, H, D = r.shape
+        B = seq_offsets.numel() - 1
+    else:
+        B, T, H, D = r.shape
+    if workspace is None:
+        nbytes = wkv7_backward_workspace_bytes(B, T, H, D, seq_offsets is not None)
+        workspace = torch.empty(nbytes // 4, dtype=torch.float32, device=r.device)
+    grads = [torch.empty_like(x) for x in (r, w_log, k, v, a, b)]
+    ds0 = torch.empty((B, H, D, D), dtype=torch.float32, device=r.device)
+    wkv7_backward(r, w_log, k, v, a, b, s0, dy, dsT, grads[0], grads[1], grads[2], grads[3], grads[4], grads[5], ds0,
+                  workspace, B, T, H, D, seq_offsets, stream)
+    return tuple(grads) + (ds0,)
 
 
 def decode_step(r, w_log, k, v, a, b, state, y=None, stream=None):

@@ -31,6 +31,8 @@ EXPORTS = (
     "wkv7_forward_fused",
     "wkv7_decode_step",
     "wkv7_decode_step_fused",
+    "wkv7_backward",
+    "wkv7_backward_workspace_bytes",
     "wkv7_status_string",
     "wkv7_get_device_status",
     "wkv7_debug_expire_wait",
@@ -63,6 +65,10 @@ def _lib():
         lib.wkv7_forward_fused.restype = i
         lib.wkv7_decode_step_fused.argtypes = [vp] * 10 + [i] * 4 + [i, i, vp]
         lib.wkv7_decode_step_fused.restype = i
+        lib.wkv7_backward.argtypes = [vp] * 17 + [ctypes.c_size_t] + [i] * 4 + [vp, i, i, vp]
+        lib.wkv7_backward.restype = i
+        lib.wkv7_backward_workspace_bytes.argtypes = [i] * 5
+        lib.wkv7_backward_workspace_bytes.restype = ctypes.c_size_t
         lib.wkv7_decode_step.argtypes = [vp] * 9 + [i] * 3 + [i, i, vp]
         lib.wkv7_decode_step.restype = i
         lib.wkv7_status_string.argtypes = [i]
@@ -144,6 +150,22 @@ def wkv7_decode_step_fused(r, w_log, k, v, a_lr, s_in, r_k, g, out, s_out, B, H,
         raise Wkv7Error(st, "wkv7_decode_step_fused")
 
 
+def wkv7_backward_workspace_bytes(B, T, H, D, packed) -> int:
+    return int(_lib().wkv7_backward_workspace_bytes(int(B), int(T), int(H), int(D), 1 if packed else 0))
+
+
+def wkv7_backward(r, w_log, k, v, a, b, s0, dy, dsT, dr, dw_log, dk, dv, da, db, ds0, workspace, B, T, H, D,
+                  seq_offsets=None, stream=None):
+    """Enqueue the backward of the recurrence (see include/wkv7.h)."""
+    nbytes = workspace.numel() * workspace.element_size()
+    st = _lib().wkv7_backward(_ptr(r), _ptr(w_log), _ptr(k), _ptr(v), _ptr(a), _ptr(b), _ptr(s0), _ptr(dy),
+                              _ptr(dsT), _ptr(dr), _ptr(dw_log), _ptr(dk), _ptr(dv), _ptr(da), _ptr(db), _ptr(ds0),
+                              _ptr(workspace), int(nbytes), int(B), int(T), int(H), int(D), _ptr(seq_offsets),
+                              _dtype_code(r), _dtype_code(w_log), _stream(stream))
+    if st != 0:
+        raise Wkv7Error(st, "wkv7_backward")
+
+
 def wkv7_decode_step(r, w_log, k, v, a, b, s_in, y, s_out, B, H, D, stream=None):
     """Enqueue one decoding step (see include/wkv7.h)."""
     st = _lib().wkv7_decode_step(_ptr(r), _ptr(w_log), _ptr(k), _ptr(v), _ptr(a), _ptr(b), _ptr(s_in), _ptr(y),
@@ -186,6 +208,10 @@ def raw_call_forward_fused(*args):
 
 def raw_call_decode_fused(*args):
     return int(_lib().wkv7_decode_step_fused(*args))
+
+
+def raw_call_backward(*args):
+    return int(_lib().wkv7_backward(*args))
 
 
 def raw_call_decode(*args):

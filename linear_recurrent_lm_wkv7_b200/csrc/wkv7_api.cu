@@ -241,6 +241,58 @@ int wkv7_decode_step_fused(const void* r, const void* w_log, const void* k, cons
                        stream, true);
 }
 
+size_t wkv7_backward_workspace_bytes(int B, int T, int H, int D, int packed) {
+    if (B <= 0 || T < 0 || H <= 0 || D != wkv7::kHead) return 0;
+    return wkv7::backward_workspace_floats(B, T, H, packed ? 1 : 0) * sizeof(float);
+}
+
+int wkv7_backward(const void* r, const void* w_log, const void* k, const void* v, const void* a, const void* b,
+                  const float* s0, const void* dy, const float* dsT, void* dr, void* dw_log, void* dk, void* dv,
+                  void* da, void* db, float* ds0, void* workspace, size_t workspace_bytes, int B, int T, int H,
+                  int D, const int32_t* seq_offsets, int io_dtype, int w_dtype, void* stream) {
+    // ---- host-side validation; nothing is launched on failure
+    if (B <= 0 || T < 0 || H <= 0 || D <= 0) return WKV7_ERR_INVALID_ARG;
+    if (!dtype_ok(io_dtype) || !dtype_ok(w_dtype)) return WKV7_ERR_INVALID_ARG;
+    if (D != wkv7::kHead) return WKV7_ERR_UNSUPPORTED;
+    if (!ds0 || !workspace) return WKV7_ERR_INVALID_ARG;
+    if (T > 0 && (!r || !w_log || !k || !v || !a || !b || !dy || !dr || !dw_log || !dk || !dv || !da || !db))
+        return WKV7_ERR_INVALID_ARG;
+    const void* ptrs[] = {r, w_log, k, v, a, b, s0, dy, dsT, dr, dw_log, dk, dv, da, db, ds0, workspace, seq_offsets};
+    for (const void* p : ptrs)
+        if (p && !aligned16(p)) return WKV7_ERR_MISALIGNED;
+    const int packed = seq_offsets ? 1 : 0;
+    if (workspace_bytes < wkv7::backward_workspace_floats(B, T, H, packed) * sizeof(float))
+        return WKV7_ERR_INVALID_ARG;
+    const long tokens = packed ? static_cast<long>(T) : static_cast<long>(B) * T;
+    const size_t n_act = static_cast<size_t>(tokens) * H * D;
+    const size_t n_state = static_cast<size_t>(B) * H * D * D;
+    const size_t io_b = dtype_bytes(io_dtype), w_b = dtype_bytes(w_dtype);
+    // every output (and the workspace) is disjoint from every input and from the others
+    const void* outs[] = {dr, dk, dv, da, db, dw_log, ds0, workspace};
+    const size_t out_b[] = {n_act * io_b, n_act * io_b, n_act * io_b, n_act * io_b,
+                            n_act * io_b, n_act * w_b,  n_state * 4,  workspace_bytes};
+    const void* ins[] = {r, k, v, a, b, dy, w_log, s0, dsT};
+    const size_t in_b[] = {n_act * io_b, n_act * io_b, n_act * io_b, n_act * io_b, n_act * io_b,
+                           n_act * io_b, n_act * w_b,  n_state * 4,  n_state * 4};
+    for (int i = 0; i < 8; ++i) {
+        for (int j = 0; j < 9; ++j)
+            if (overlaps(outs[i], out_b[i], ins[j], in_b[j])) return WKV7_ERR_INVALID_ARG;
+        for (int j = i + 1; j < 8; ++j)
+            if (overlaps(outs[i], out_b[i], outs[j], out_b[j])) return WKV7_ERR_INVALID_ARG;
+    }
+
+    int dev_ok = cached_device_check();
+    if (dev_ok != WKV7_OK) return dev_ok;
+    int* status = nullptr;
+    if (status_ptr(&status) != WKV7_OK) return WKV7_ERR_CUDA;
+    wkv7::BackwardArgs p{r, w_log, k, v, a, b, s0, dy, dsT, dr, dw_log, dk, dv, da, db, ds0,
+                         static_cast<float*>(workspace), B, T, H, seq_offsets,
+                         wkv7::backward_ckpt_chunks(B, T, packed), status};
+    return wkv7::launch_backward(p, io_dtype, w_dtype, static_cast<cudaStream_t>(stream)) == cudaSuccess
+               ? WKV7_OK
+               : WKV7_ERR_CUDA;
+}
+
 int wkv7_get_device_status(void* stream) {
     if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return WKV7_ERR_CUDA;
     int* dptr = nullptr;

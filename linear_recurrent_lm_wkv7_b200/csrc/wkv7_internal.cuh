@@ -53,6 +53,30 @@ struct DecodeArgs {
     const void* g = nullptr;
 };
 
+struct BackwardArgs {
+    const void* r;
+    const void* w_log;
+    const void* k;
+    const void* v;
+    const void* a;
+    const void* b;
+    const float* s0;   // null: zero initial state
+    const void* dy;
+    const float* dsT;  // null: no gradient on the final state
+    void* dr;
+    void* dw_log;
+    void* dk;
+    void* dv;
+    void* da;
+    void* db;
+    float* ds0;
+    float* ws;  // workspace: chunk checkpoints, then one chunk of states per unit
+    int B, T, H;
+    const int32_t* seq_offsets;
+    long ckpt_chunks;  // checkpoint slots per head in the workspace
+    int* status;
+};
+
 cudaError_t launch_prefill(const PrefillArgs& p, int io_dtype, int w_dtype, cudaStream_t stream);
 // warp-specialised kernel for bf16 inputs (wkv7_prefill_pipe.cu)
 cudaError_t launch_prefill_pipe(const PrefillArgs& p, int w_dtype, cudaStream_t stream);
@@ -64,6 +88,10 @@ cudaError_t launch_gate(void* z, const void* r, const void* k, const void* v, co
                         long ntok, int H, int io_dtype, cudaStream_t stream, const void* w_log = nullptr,
                         const void* a_lr = nullptr, int H_kv = 0, int w_dtype = WKV7_F32);
 cudaError_t launch_expire_wait(int spins, int* status, cudaStream_t stream);
+// backward of the recurrence (wkv7_backward.cu)
+long backward_ckpt_chunks(int B, int T, int packed);
+size_t backward_workspace_floats(int B, int T, int H, int packed);
+cudaError_t launch_backward(const BackwardArgs& p, int io_dtype, int w_dtype, cudaStream_t stream);
 
 // Records the first device-side error of a call sequence (first writer wins).
 __device__ __forceinline__ void report_status(int* status, int code) {

@@ -22,7 +22,7 @@ def wk():
 
 def test_header_symbols_exported(wk):
     hdr = open(os.path.join(ROOT, "include", "wkv7.h")).read()
-    declared = set(re.findall(r"^(?:int|const char\*)\s+(wkv7_\w+)\s*\(", hdr, flags=re.M))
+    declared = set(re.findall(r"^(?:int|size_t|const char\*)\s+(wkv7_\w+)\s*\(", hdr, flags=re.M))
     assert declared == set(wk.EXPORTS)
     lib = ctypes.CDLL(wk.LIB_PATH)
     for name in declared:
@@ -158,3 +158,37 @@ def test_decode_fused_rejects_bad_arguments(wk):
     assert call(*args(g=0x901008, rk=0x801000)) == -3  # misaligned gate
     assert call(*args(out=0x201000)) == -1  # out aliases k
     assert call(*args(s_out=0x401000)) == -1  # s_out overlaps a_lr
+
+
+
+# argument tuple for wkv7_backward: 17 pointers, workspace bytes, B, T, H, D, offsets, io, w, stream
+def _bwd(wk, B=1, T=8, H=1, D=64, offs=None, io=1, wd=0, wsb=None, **over):
+    names = ("r", "w", "k", "v", "a", "b", "s0", "dy", "dsT", "dr", "dwl", "dk", "dv", "da", "db", "ds0", "ws")
+    p = {n: 0x1000 + i * 0x100000 for i, n in enumerate(names)}
+    p["s0"] = p["dsT"] = None
+    p.update(over)
+    if wsb is None:
+        wsb = wk.wkv7_backward_workspace_bytes(B, T, H, 64, offs is not None)
+    return tuple(p[n] for n in names) + (wsb, B, T, H, D, offs, io, wd, None)
+
+
+def test_backward_workspace_size(wk):
+    # checkpoints: ceil(T / 64) per sequence (dense) or ceil(T / 64) + B (packed) per head,
+    # plus 64 states per unit; a state is 64 x 64 fp32
+    assert wk.wkv7_backward_workspace_bytes(2, 130, 3, 64, False) == (2 * 3 * 3 + 2 * 3 * 64) * 16384
+    assert wk.wkv7_backward_workspace_bytes(2, 130, 3, 64, True) == ((3 + 2) * 3 + 2 * 3 * 64) * 16384
+    assert wk.wkv7_backward_workspace_bytes(2, 130, 3, 32, False) == 0
+
+
+def test_backward_rejects_bad_arguments(wk):
+    call = wk._binding.raw_call_backward
+    assert call(*_bwd(wk, D=32)) == -2
+    assert call(*_bwd(wk, B=0)) == -1
+    assert call(*_bwd(wk, ds0=None)) == -1
+    assert call(*_bwd(wk, ws=None)) == -1
+    assert call(*_bwd(wk, dy=None)) == -1
+    assert call(*_bwd(wk, wsb=1024)) == -1  # workspace too small
+    assert call(*_bwd(wk, dk=0x1008 + 0xB00000)) == -3  # misaligned
+    assert call(*_bwd(wk, dr=0x1000)) == -1  # dr aliases r
+    assert call(*_bwd(wk, dk=0x1000 + 0x900000)) == -1  # dk aliases dr
+    assert call(*_bwd(wk, ws=0x1000 + 0x700000)) == -1  # workspace overlaps dy

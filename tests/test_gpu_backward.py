@@ -1,0 +1,78 @@
+"""GPU parity of wkv7_backward (gradient of <dy, y> + <dsT, sT> with respect to
+r, w_log, k, v, a, b and s0) against the fp64 oracle's backward, through the C
+ABI.  Same metric and bounds as the forward: max|out - ref| / max|ref| <= 2e-3
+for fp32 inputs and <= 2e-2 for bf16 inputs, for every gradient."""
+import numpy as np
+import pytest
+import torch
+
+import wkv7_inputs as W
+
+pytestmark = pytest.mark.gpu
+
+TOL = {"f32": 2e-3, "bf16": 2e-2}
+NAMES = ("dr", "dw_log", "dk", "dv", "da", "db", "ds0")
+
+
+@pytest.fixture(scope="module")
+def wk():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from linear_recurrent_lm_wkv7_b200 import build
+
+    build.build()
+    import linear_recurrent_lm_wkv7_b200 as wk
+
+    return wk
+
+
+def relerr(out, ref):
+    out = np.asarray(out, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    assert np.all(np.isfinite(out)), "non-finite output"
+    return float(np.max(np.abs(out - ref)) / max(np.max(np.abs(ref)), 1e-30))
+
+
+def check(wk, oracle_mod, inp, seed=0, with_dsT=True):
+    dy, dsT = W.make_upstream(inp.r.shape, inp.B, inp.H, io=inp.io, seed=seed, with_dsT=with_dsT)
+    t = inp.tensors()
+    d = {n: x.cuda() for n, x in t.items()}
+    s0 = inp.s0.cuda() if inp.s0 is not None else None
+    offs = inp.seq_offsets.cuda() if inp.seq_offsets is not None else None
+    got = wk.backward(d["r"], d["w_log"], d["k"], d["v"], d["a"], d["b"], dy.cuda(), s0,
+                      dsT.cuda() if dsT is not None else None, offs)
+    assert wk.wkv7_get_device_status() == 0
+    f64 = lambda x: x.double().numpy() if x is not None else None
+    ref = oracle_mod.backward(*(f64(t[n]) for n in ("r", "w_log", "k", "v", "a", "b")), f64(dy), f64(inp.s0),
+                              f64(dsT), inp.seq_offsets.numpy() if inp.seq_offsets is not None else None)
+    tol = TOL[inp.io]
+    errs = {n: relerr(g.float().cpu().numpy(), rf) for n, g, rf in zip(NAMES, got, ref)}
+    assert all(e <= tol for e in errs.values()), errs
+
+
+def test_backward_tiny_f32(wk, oracle_mod):
+    check(wk, oracle_mod, W.make_prefill(1, 64, 2, io="f32", wdt="f32", s0_std=0.1, seed=1), seed=1)
+
+
+@pytest.mark.parametrize("T", [1, 63, 64, 130])
+@pytest.mark.parametrize("wdt", ["f32", "bf16"])
+def test_backward_dense_bf16(wk, oracle_mod, T, wdt):
+    """bf16 inputs, ragged tails, a partial and several chunks."""
+    check(wk, oracle_mod, W.make_prefill(2, T, 3, io="bf16", wdt=wdt, s0_std=0.1, seed=500 + T), seed=T)
+
+
+def test_backward_dense_f32_no_state(wk, oracle_mod):
+    """fp32 inputs, no initial state and no gradient on the final state."""
+    check(wk, oracle_mod, W.make_prefill(2, 130, 2, io="f32", wdt="f32", s0_std=None, seed=9), seed=9,
+          with_dsT=False)
+
+
+def test_backward_packed_with_pads(wk, oracle_mod):
+    lengths = [0, 5, 64, 100, 1, 130]
+    pads = [3, 0, 7, 1, 0, 63]
+    check(wk, oracle_mod, W.make_packed(lengths, pads, 2, io="bf16", wdt="f32", s0_std=0.1, seed=56), seed=6)
+
+
+def test_backward_prefill_1p5b_full(wk, oracle_mod):
+    """The 1.5B-class prefill (B4 T1024 H32), in the launch configuration of the benchmark."""
+    check(wk, oracle_mod, W.make_workload("prefill_1p5b"), seed=21)

@@ -21,6 +21,8 @@ order r, k, v, kappa, a_lr logit, decay logit, s0):
   kv heads [.., H_kv, D]; a_lr = sigmoid(N(0, 1)) [.., H, D]; log_neglog_w as
   above.  The prologue (normalised kk, a, b and the scaled key) happens inside
   the path under test.
+* backward upstream gradients (make_upstream, its own generator): dy ~ N(0, 1)
+  in the io dtype with the shape of r, dsT ~ N(0, 0.1^2) fp32 [B, H, D, D]
 * packed batches: lengths ~ U{len_lo..len_hi} and pad counts ~ U{0..pad_hi};
   pad tokens carry log_neglog_w = -inf (w = 1) and k = v = a = b = 0, so they
   leave the state unchanged; r stays drawn at pads.
@@ -184,6 +186,15 @@ def make_fused(B, T, H, H_kv, D=64, io="bf16", wdt="f32", s0_std=None, mu_z=0.0,
     cast = lambda t, d: t.to(_DT[d]).contiguous()
     return FusedInputs(cast(r, io), cast(w_log, wdt), cast(k, io), cast(v, io), cast(a_lr, io), s0, seq_offsets,
                        B, T, H, H_kv, D, io, wdt, n_real)
+
+
+def make_upstream(shape, B, H, D=64, io="bf16", seed=0, with_dsT=True, dsT_std=0.1):
+    """Upstream gradients for the backward: dy of the activation shape (io dtype)
+    and dsT [B, H, D, D] fp32 (None when with_dsT is false)."""
+    g = torch.Generator().manual_seed(seed)
+    dy = torch.randn(tuple(shape), generator=g).to(_DT[io]).contiguous()
+    dsT = (torch.randn((B, H, D, D), generator=g) * dsT_std).contiguous() if with_dsT else None
+    return dy, dsT
 
 
 def draw_lengths(n_seq, len_lo, len_hi, pad_hi, seed):
