@@ -63,7 +63,8 @@ typedef enum {
     WKV7_ERR_MISALIGNED = -3,     /* a pointer not 16-byte aligned */
     WKV7_ERR_CUDA = -4,           /* a CUDA runtime call or a launch failed */
     WKV7_ERR_DEVICE_TIMEOUT = -5, /* a bounded device-side wait expired */
-    WKV7_ERR_DEVICE_BOUNDS = -6   /* packed offsets not monotone or beyond T */
+    WKV7_ERR_DEVICE_BOUNDS = -6,  /* packed offsets not monotone or beyond T */
+    WKV7_ERR_SCRATCH_LIMIT = -7   /* wkv7_backward_noalloc: problem needs more than its fixed scratch */
 } wkv7_status;
 
 /*
@@ -198,6 +199,35 @@ int wkv7_backward(const void* r, const void* w_log, const void* k, const void* v
                   void* da, void* db, float* ds0, void* workspace, size_t workspace_bytes,
                   int B, int T, int H, int D, const int32_t* seq_offsets,
                   int io_dtype, int w_dtype, void* stream);
+
+/*
+ * wkv7_backward_noalloc — wkv7_backward with the library's own fixed scratch in
+ * place of a caller workspace, for callers that cannot allocate device memory
+ * at the point of the call (a device-memory budget that forbids new
+ * allocations, runtimes that pass kernels only preallocated buffers, paths that
+ * must not call cudaMalloc because it can synchronise the device).  Nothing is
+ * allocated by the call.  The pages have no counterpart: this is an interface
+ * convenience around the same kernel.
+ *   Arguments, layouts and results as in wkv7_backward, without the workspace.
+ *   Limit: wkv7_backward_workspace_bytes(B, T, H, D, packed) must not exceed
+ *   WKV7_NOALLOC_SCRATCH_BYTES (16 MiB); otherwise WKV7_ERR_SCRATCH_LIMIT is
+ *   returned and nothing is launched.  (For example B = 2, H = 3 and T up to
+ *   a few hundred tokens fit; use wkv7_backward for larger problems.)
+ *   Nothing in the scratch has to start at zero (every element is written
+ *   before it is read), so the call clears nothing.
+ *   There is one scratch per device: calls whose kernels may overlap on the
+ *   same device (unordered streams, several host threads) race on it; the
+ *   caller must order them.
+ *   The first call on each device looks up the scratch's address
+ *   (cudaGetSymbolAddress, which may load the library's module); make that
+ *   first call before any stream capture.
+ */
+#define WKV7_NOALLOC_SCRATCH_BYTES ((size_t)16 << 20)
+int wkv7_backward_noalloc(const void* r, const void* w_log, const void* k, const void* v,
+                          const void* a, const void* b, const float* s0, const void* dy,
+                          const float* dsT, void* dr, void* dw_log, void* dk, void* dv,
+                          void* da, void* db, float* ds0, int B, int T, int H, int D,
+                          const int32_t* seq_offsets, int io_dtype, int w_dtype, void* stream);
 
 /* Human-readable text for a status code (static storage, never NULL). */
 const char* wkv7_status_string(int status);

@@ -18,6 +18,7 @@ from ._binding import (  # noqa: F401
     Wkv7Error,
     _lib,
     wkv7_backward,
+    wkv7_backward_noalloc,
     wkv7_backward_workspace_bytes,
     wkv7_debug_expire_wait,
     wkv7_decode_step,

@@ -23,6 +23,7 @@ STATUS = {
     -4: "WKV7_ERR_CUDA",
     -5: "WKV7_ERR_DEVICE_TIMEOUT",
     -6: "WKV7_ERR_DEVICE_BOUNDS",
+    -7: "WKV7_ERR_SCRATCH_LIMIT",
 }
 # every symbol include/wkv7.h declares
 EXPORTS = (
@@ -33,6 +34,7 @@ EXPORTS = (
     "wkv7_decode_step_fused",
     "wkv7_backward",
     "wkv7_backward_workspace_bytes",
+    "wkv7_backward_noalloc",
     "wkv7_status_string",
     "wkv7_get_device_status",
     "wkv7_debug_expire_wait",
@@ -69,6 +71,8 @@ def _lib():
         lib.wkv7_backward.restype = i
         lib.wkv7_backward_workspace_bytes.argtypes = [i] * 5
         lib.wkv7_backward_workspace_bytes.restype = ctypes.c_size_t
+        lib.wkv7_backward_noalloc.argtypes = [vp] * 16 + [i] * 4 + [vp, i, i, vp]
+        lib.wkv7_backward_noalloc.restype = i
         lib.wkv7_decode_step.argtypes = [vp] * 9 + [i] * 3 + [i, i, vp]
         lib.wkv7_decode_step.restype = i
         lib.wkv7_status_string.argtypes = [i]
@@ -166,6 +170,19 @@ def wkv7_backward(r, w_log, k, v, a, b, s0, dy, dsT, dr, dw_log, dk, dv, da, db,
         raise Wkv7Error(st, "wkv7_backward")
 
 
+def wkv7_backward_noalloc(r, w_log, k, v, a, b, s0, dy, dsT, dr, dw_log, dk, dv, da, db, ds0, B, T, H, D,
+                          seq_offsets=None, stream=None):
+    """Enqueue the backward with the library's fixed scratch: for callers that
+    cannot allocate device memory at the call (see include/wkv7.h for the 16 MiB
+    limit and the rule that overlapping calls must be ordered)."""
+    st = _lib().wkv7_backward_noalloc(_ptr(r), _ptr(w_log), _ptr(k), _ptr(v), _ptr(a), _ptr(b), _ptr(s0), _ptr(dy),
+                                      _ptr(dsT), _ptr(dr), _ptr(dw_log), _ptr(dk), _ptr(dv), _ptr(da), _ptr(db),
+                                      _ptr(ds0), int(B), int(T), int(H), int(D), _ptr(seq_offsets), _dtype_code(r),
+                                      _dtype_code(w_log), _stream(stream))
+    if st != 0:
+        raise Wkv7Error(st, "wkv7_backward_noalloc")
+
+
 def wkv7_decode_step(r, w_log, k, v, a, b, s_in, y, s_out, B, H, D, stream=None):
     """Enqueue one decoding step (see include/wkv7.h)."""
     st = _lib().wkv7_decode_step(_ptr(r), _ptr(w_log), _ptr(k), _ptr(v), _ptr(a), _ptr(b), _ptr(s_in), _ptr(y),
@@ -212,6 +229,10 @@ def raw_call_decode_fused(*args):
 
 def raw_call_backward(*args):
     return int(_lib().wkv7_backward(*args))
+
+
+def raw_call_backward_noalloc(*args):
+    return int(_lib().wkv7_backward_noalloc(*args))
 
 
 def raw_call_decode(*args):

@@ -79,6 +79,7 @@ const char* wkv7_status_string(int status) {
         case WKV7_ERR_CUDA: return "CUDA runtime error";
         case WKV7_ERR_DEVICE_TIMEOUT: return "device-side bounded wait expired";
         case WKV7_ERR_DEVICE_BOUNDS: return "packed sequence offsets out of range";
+        case WKV7_ERR_SCRATCH_LIMIT: return "problem needs more than the fixed scratch of wkv7_backward_noalloc";
         default: return "unknown status";
     }
 }

@@ -192,3 +192,13 @@ def test_backward_rejects_bad_arguments(wk):
     assert call(*_bwd(wk, dr=0x1000)) == -1  # dr aliases r
     assert call(*_bwd(wk, dk=0x1000 + 0x900000)) == -1  # dk aliases dr
     assert call(*_bwd(wk, ws=0x1000 + 0x700000)) == -1  # workspace overlaps dy
+
+
+def test_backward_noalloc_rejects_before_any_cuda_call(wk):
+    call = wk._binding.raw_call_backward_noalloc
+    ptrs = tuple(0x1000 + i * 0x100000 for i in range(16))
+    # B2 T8192 H32 needs (2 x 128 x 32 checkpoints + 2 x 32 x 64 chunk states) x 16 KB = 192 MiB
+    assert call(*ptrs, 2, 8192, 32, 64, None, 1, 0, None) == -7
+    assert wk.wkv7_status_string(-7)
+    assert call(*ptrs, 0, 8, 1, 64, None, 1, 0, None) == -1
+    assert call(*ptrs, 1, 8, 1, 32, None, 1, 0, None) == -2
