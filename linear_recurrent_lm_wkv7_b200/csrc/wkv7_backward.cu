@@ -195,11 +195,18 @@ __global__ void __launch_bounds__(NTHR, 1)
             st_state(cs + static_cast<long>(tt) * SQ, S, rg, cg);
             fwd_step(S, smf, tt, rg, cg);
         }
-        // S is now the state after the chunk's last token
+        // S is now the state after the chunk's last token; the state before each token is
+        // loaded one token ahead (its own elements: no barrier needed)
+        float Sn[4][4];
+        if (nv > 0) ld_state(cs + static_cast<long>(nv - 1) * SQ, Sn, rg, cg);
         for (int tt = nv - 1; tt >= 0; --tt, ++tok) {
             const float* base = smf + tt * kHead;
             float Sp[4][4];
-            ld_state(cs + static_cast<long>(tt) * SQ, Sp, rg, cg);
+#pragma unroll
+            for (int m = 0; m < 4; ++m)
+#pragma unroll
+                for (int c4 = 0; c4 < 4; ++c4) Sp[m][c4] = Sn[m][c4];
+            if (tt > 0) ld_state(cs + static_cast<long>(tt - 1) * SQ, Sn, rg, cg);
             const float4 rj = ld4(base + IN_R * L * kHead + 4 * cg), kj = ld4(base + IN_K * L * kHead + 4 * cg);
             const float4 aj = ld4(base + IN_A * L * kHead + 4 * cg), bj = ld4(base + IN_B * L * kHead + 4 * cg);
             const float4 wj = ld4(base + IN_W * L * kHead + 4 * cg);
