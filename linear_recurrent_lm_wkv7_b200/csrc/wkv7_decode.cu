@@ -93,13 +93,20 @@ __global__ void __launch_bounds__(256, BLOCKS_PER_SM)
     const long first = blockIdx.x, stride = gridDim.x;
     const long nmine = first < units ? (units - first + stride - 1) / stride : 0;
     long n_issued = 0;  // thread 0: units whose copies were issued
+    // sequence and head of the next unit to issue: units are issued in order, so they
+    // advance by the grid stride with one carry (no division per unit)
+    long in_n = first / H;
+    int in_h = static_cast<int>(first % H);
+    const long step_n = stride / H;
+    const int step_h = static_cast<int>(stride % H);
+    const int rep = PRO ? H / H_kv : 1;  // heads per kv head
     auto issue = [&](long j) {
         const long u = first + j * stride;
         uint8_t* base = smem + (j % NST) * ST_BYTES;
         uint64_t* bar = &full[j % NST];
         mbar_arrive_expect_tx(bar, tx);
         // row of k and v: the unit's own, or its kv head's
-        const long ukv = PRO ? (u / H) * H_kv + (u % H) / (H / H_kv) : u;
+        const long ukv = PRO ? in_n * H_kv + in_h / rep : u;
         if (s_in) bulk_load(base, s_in + u * (kHead * kHead), ST_STATE, bar);
         bulk_load(base + O_R, r + u * kHead, IOB, bar);
         bulk_load(base + O_K, k + ukv * kHead, IOB, bar);
@@ -108,8 +115,14 @@ __global__ void __launch_bounds__(256, BLOCKS_PER_SM)
         if constexpr (!PRO) bulk_load(base + O_B, b + u * kHead, IOB, bar);
         bulk_load(base + O_W, wl + u * kHead, WB, bar);
         if constexpr (GATED) {
-            bulk_load(base + O_RK, rk + (u % H) * kHead, kHead * 4, bar);
+            bulk_load(base + O_RK, rk + static_cast<long>(in_h) * kHead, kHead * 4, bar);
             bulk_load(base + O_G, gte + u * kHead, IOB, bar);
+        }
+        in_n += step_n;
+        in_h += step_h;
+        if (in_h >= H) {
+            in_h -= H;
+            ++in_n;
         }
         ++n_issued;
     };
