@@ -188,6 +188,8 @@ int wkv7_decode_step_fused(const void* r, const void* w_log, const void* k, cons
  *   workspace : DEVICE scratch of at least
  *          wkv7_backward_workspace_bytes(B, T, H, D, seq_offsets != NULL) bytes,
  *          owned by the caller and not read before it is written.
+ *          wkv7_backward_workspace_bytes returns 0 for invalid sizes (B <= 0,
+ *          T < 0, H <= 0, D != 64).
  * Every output and the workspace must be disjoint from every input and from
  * each other.  Recurrent form: one block per (sequence, head) recomputes the
  * states of each 64-token chunk from checkpoints and sweeps the tokens backward.
