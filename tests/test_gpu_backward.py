@@ -76,3 +76,16 @@ def test_backward_packed_with_pads(wk, oracle_mod):
 def test_backward_prefill_1p5b_full(wk, oracle_mod):
     """The 1.5B-class prefill (B4 T1024 H32), in the launch configuration of the benchmark."""
     check(wk, oracle_mod, W.make_workload("prefill_1p5b"), seed=21)
+
+
+def test_backward_zero_tokens(wk):
+    """T = 0: no token to differentiate; ds0 is dsT itself, or zero without dsT."""
+    B, H = 2, 3
+    r = torch.empty((B, 0, H, 64), dtype=torch.bfloat16, device="cuda")
+    wl = torch.empty((B, 0, H, 64), dtype=torch.float32, device="cuda")
+    _, dsT = W.make_upstream((B, 0, H, 64), B, H, io="bf16", seed=3)
+    got = wk.backward(r, wl, r, r, r, r, r, None, dsT.cuda())
+    assert wk.wkv7_get_device_status() == 0
+    assert torch.equal(got[6].cpu(), dsT)
+    got = wk.backward(r, wl, r, r, r, r, r)
+    assert torch.count_nonzero(got[6]).item() == 0
