@@ -793,17 +793,15 @@ __global__ void __launch_bounds__(NTHR, 1)
             const long row0 = tb + static_cast<long>(c) * L;
             const int nv = static_cast<int>(len - static_cast<long>(c) * L < L ? len - static_cast<long>(c) * L : L);
             const uint32_t tm_out = tmem + 256u * g + TM_OUT;
-            // gated read-out: this token row's v and g, fetched before waiting for the chunk
-            uint4 vpre[8], gpre[8];
+            // gated read-out: this token row's v and g (128 B each) are brought into L2 before
+            // waiting for the chunk, and read where they are used
+            long goff = 0, gvoff = 0;
             if constexpr (GATED) {
+                goff = (row0 + ts) * tstride + hoff;
+                gvoff = PRO ? (row0 + ts) * tstride_kv + hoff_kv : goff;
                 if (ts < nv) {
-                    const long off = (row0 + ts) * tstride + hoff;
-                    const long voff = PRO ? (row0 + ts) * tstride_kv + hoff_kv : off;
-#pragma unroll
-                    for (int i = 0; i < 8; ++i) {
-                        vpre[i] = *reinterpret_cast<const uint4*>(v + voff + 8 * i);
-                        gpre[i] = *reinterpret_cast<const uint4*>(gte + off + 8 * i);
-                    }
+                    prefetch_line_l2(v + gvoff);
+                    prefetch_line_l2(gte + goff);
                 }
             }
             ok = group_sync_and(bar_id, GROUP,
@@ -836,7 +834,8 @@ __global__ void __launch_bounds__(NTHR, 1)
                             // z = (y / sqrt(D) + u v) (.) g, with v and g of this token row
 #pragma unroll
                             for (int i = 0; i < 32; i += 8) {
-                                const uint4 vq = vpre[4 * q + i / 8], gq4 = gpre[4 * q + i / 8];
+                                const uint4 vq = *reinterpret_cast<const uint4*>(v + gvoff + 32 * q + i);
+                                const uint4 gq4 = *reinterpret_cast<const uint4*>(gte + goff + 32 * q + i);
                                 const uint32_t vw[4] = {vq.x, vq.y, vq.z, vq.w}, gw[4] = {gq4.x, gq4.y, gq4.z, gq4.w};
 #pragma unroll
                                 for (int m = 0; m < 4; ++m) {
