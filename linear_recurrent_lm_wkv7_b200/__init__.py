@@ -5,7 +5,9 @@ The Python layer only marshals arguments to the CUDA library; importing the
 package loads ``libwkv7.so`` and fails loudly if it has not been built.
 Convenience wrappers ``forward``, ``forward_gated``, ``forward_fused``,
 ``decode_step``, ``decode_step_fused`` and ``backward`` allocate outputs with
-torch and call the C entry points.
+torch and call the C entry points; ``forward_host`` runs the prefill on inputs
+and outputs that live in pinned host memory, overlapping the copies with the
+kernels.
 """
 from __future__ import annotations
 
@@ -49,6 +51,61 @@ def forward(r, w_log, k, v, a, b, s0=None, seq_offsets=None, want_state=True, st
     sT = torch.empty((B, H, D, D), dtype=torch.float32, device=r.device) if want_state else None
     wkv7_forward(r, w_log, k, v, a, b, s0, y, sT, B, T, H, D, seq_offsets, stream)
     return y, sT
+
+
+_HOST_STREAMS = {}
+_INPUTS = ("r", "w_log", "k", "v", "a", "b")
+
+
+def forward_host(host, dev, y_host, sT_host, s0=None, parts=4, stream=None):
+    """Prefill of a dense batch whose inputs and outputs live in pinned host memory.
+
+    ``host``: pinned CPU tensors r, w_log, k, v, a, b of shape [B, T, H, D];
+    ``dev``: device staging tensors of the same names and shapes plus ``y`` and
+    ``sT`` ([B, H, D, D] fp32), allocated once by the caller; ``y_host``,
+    ``sT_host``: pinned CPU outputs; ``s0``: optional device initial states.
+    The batch is split by sequence into ``parts`` groups: the upload of group
+    i + 1, the prefill of group i and the download of group i - 1 run on three
+    CUDA streams at once (sequences are independent, so the results equal one
+    call over the whole batch).  Everything is ordered after ``stream`` (default:
+    the current stream), which then waits for all of it: the call is
+    asynchronous like a kernel launch on ``stream``."""
+    import torch
+
+    device = dev["r"].device
+    st = stream if stream is not None else torch.cuda.current_stream(device)
+    idx = device.index if device.index is not None else torch.cuda.current_device()
+    if idx not in _HOST_STREAMS:
+        _HOST_STREAMS[idx] = tuple(torch.cuda.Stream(device) for _ in range(3))
+    s_up, s_run, s_down = _HOST_STREAMS[idx]
+    B, T, H, D = host["r"].shape
+    parts = max(1, min(int(parts), B))
+    bounds = [B * p // parts for p in range(parts + 1)]
+    start = torch.cuda.Event()
+    start.record(st)
+    for s_ in (s_up, s_run, s_down):
+        s_.wait_event(start)
+    for p in range(parts):
+        b0, b1 = bounds[p], bounds[p + 1]
+        if b1 == b0:
+            continue
+        with torch.cuda.stream(s_up):
+            for n in _INPUTS:
+                dev[n][b0:b1].copy_(host[n][b0:b1], non_blocking=True)
+        up = torch.cuda.Event()
+        up.record(s_up)
+        s_run.wait_event(up)
+        wkv7_forward(*(dev[n][b0:b1] for n in _INPUTS), s0[b0:b1] if s0 is not None else None, dev["y"][b0:b1],
+                     dev["sT"][b0:b1], b1 - b0, T, H, D, None, s_run)
+        ran = torch.cuda.Event()
+        ran.record(s_run)
+        s_down.wait_event(ran)
+        with torch.cuda.stream(s_down):
+            y_host[b0:b1].copy_(dev["y"][b0:b1], non_blocking=True)
+            sT_host[b0:b1].copy_(dev["sT"][b0:b1], non_blocking=True)
+    done = torch.cuda.Event()
+    done.record(s_down)
+    st.wait_event(done)
 
 
 def forward_gated(r, w_log, k, v, a, b, r_k, g, s0=None, seq_offsets=None, want_state=True, stream=None):

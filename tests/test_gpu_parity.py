@@ -261,3 +261,28 @@ def test_bad_offsets_reported_not_read(wk):
     wk.wkv7_forward(d["r"], d["w_log"], d["k"], d["v"], d["a"], d["b"], None, y, sT, 2, 20, 1, 64, offs)
     assert wk.wkv7_get_device_status() == -6
     assert wk.wkv7_get_device_status() == 0
+
+
+def test_forward_host_pipeline(wk, oracle_mod):
+    """forward_host (pinned host inputs and outputs, per-sequence groups whose
+    copies overlap the prefill on three streams) equals one device-side call
+    bit for bit and the oracle within the bf16 bound; 3 sequences in 2 groups."""
+    inp = W.make_prefill(3, 130, 3, io="bf16", wdt="f32", s0_std=0.1, seed=91)
+    t = inp.tensors()
+    host = {n: x.pin_memory() for n, x in t.items()}
+    dev = {n: torch.empty_like(x, device="cuda") for n, x in t.items()}
+    dev["y"] = torch.empty(tuple(inp.r.shape), dtype=torch.bfloat16, device="cuda")
+    dev["sT"] = torch.empty((3, 3, 64, 64), dtype=torch.float32, device="cuda")
+    y_h = torch.empty(tuple(inp.r.shape), dtype=torch.bfloat16).pin_memory()
+    sT_h = torch.empty((3, 3, 64, 64), dtype=torch.float32).pin_memory()
+    s0 = inp.s0.cuda()
+    for _ in range(2):  # the second call reuses the staging buffers and streams
+        wk.forward_host(host, dev, y_h, sT_h, s0=s0, parts=2)
+        torch.cuda.synchronize()
+        assert wk.wkv7_get_device_status() == 0
+        d = {n: x.cuda() for n, x in t.items()}
+        y_ref, s_ref = wk.forward(d["r"], d["w_log"], d["k"], d["v"], d["a"], d["b"], s0)
+        assert torch.equal(y_h, y_ref.cpu()) and torch.equal(sT_h, s_ref.cpu())
+    f64 = lambda x: x.double().numpy()
+    yr, sr = oracle_mod.forward(*(f64(t[n]) for n in ("r", "w_log", "k", "v", "a", "b")), f64(inp.s0))
+    assert relerr(y_h.float().numpy(), yr) <= TOL["bf16"] and relerr(sT_h.numpy(), sr) <= TOL["bf16"]
