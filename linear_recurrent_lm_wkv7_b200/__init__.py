@@ -57,19 +57,24 @@ _HOST_STREAMS = {}
 _INPUTS = ("r", "w_log", "k", "v", "a", "b")
 
 
-def forward_host(host, dev, y_host, sT_host, s0=None, parts=4, stream=None):
+def forward_host(host, dev, y_host, sT_host, s0=None, parts=4, t_parts=1, stream=None):
     """Prefill of a dense batch whose inputs and outputs live in pinned host memory.
 
     ``host``: pinned CPU tensors r, w_log, k, v, a, b of shape [B, T, H, D];
     ``dev``: device staging tensors of the same names and shapes plus ``y`` and
     ``sT`` ([B, H, D, D] fp32), allocated once by the caller; ``y_host``,
     ``sT_host``: pinned CPU outputs; ``s0``: optional device initial states.
-    The batch is split by sequence into ``parts`` groups: the upload of group
-    i + 1, the prefill of group i and the download of group i - 1 run on three
-    CUDA streams at once (sequences are independent, so the results equal one
-    call over the whole batch).  Everything is ordered after ``stream`` (default:
-    the current stream), which then waits for all of it: the call is
-    asynchronous like a kernel launch on ``stream``."""
+    The batch is cut into pieces, each contiguous in memory: ``parts`` groups of
+    whole sequences, or, with ``t_parts`` > 1 (for batches of few long
+    sequences), every sequence cut into that many token ranges whose bounds are
+    multiples of 64, a range continuing from the state the previous one left in
+    ``dev["sT"]`` (updated in place).  Every piece costs a few host-side calls, so
+    a handful of large pieces is best.
+    The upload of one piece, the prefill of the previous and the download of the
+    one before run on three CUDA streams at once, and the results equal one call
+    over the whole batch.  Everything is ordered after ``stream`` (default: the
+    current stream), which then waits for all of it: the call is asynchronous
+    like a kernel launch on ``stream``."""
     import torch
 
     device = dev["r"].device
@@ -79,30 +84,40 @@ def forward_host(host, dev, y_host, sT_host, s0=None, parts=4, stream=None):
         _HOST_STREAMS[idx] = tuple(torch.cuda.Stream(device) for _ in range(3))
     s_up, s_run, s_down = _HOST_STREAMS[idx]
     B, T, H, D = host["r"].shape
-    parts = max(1, min(int(parts), B))
-    bounds = [B * p // parts for p in range(parts + 1)]
+    nck = (T + 63) // 64
+    tb = sorted({min(T, 64 * (nck * j // max(1, int(t_parts)))) for j in range(max(1, int(t_parts)))} | {T})
+    if T == 0:
+        tb = [0, 0]  # one empty piece: sT receives s0 (or zeros)
+    if len(tb) > 2:
+        groups = [(b, b + 1) for b in range(B)]
+    else:
+        n = max(1, min(int(parts), B))
+        groups = [(B * p // n, B * (p + 1) // n) for p in range(n)]
     start = torch.cuda.Event()
     start.record(st)
     for s_ in (s_up, s_run, s_down):
         s_.wait_event(start)
-    for p in range(parts):
-        b0, b1 = bounds[p], bounds[p + 1]
+    for b0, b1 in groups:
         if b1 == b0:
             continue
-        with torch.cuda.stream(s_up):
-            for n in _INPUTS:
-                dev[n][b0:b1].copy_(host[n][b0:b1], non_blocking=True)
-        up = torch.cuda.Event()
-        up.record(s_up)
-        s_run.wait_event(up)
-        wkv7_forward(*(dev[n][b0:b1] for n in _INPUTS), s0[b0:b1] if s0 is not None else None, dev["y"][b0:b1],
-                     dev["sT"][b0:b1], b1 - b0, T, H, D, None, s_run)
-        ran = torch.cuda.Event()
-        ran.record(s_run)
-        s_down.wait_event(ran)
-        with torch.cuda.stream(s_down):
-            y_host[b0:b1].copy_(dev["y"][b0:b1], non_blocking=True)
-            sT_host[b0:b1].copy_(dev["sT"][b0:b1], non_blocking=True)
+        for j in range(len(tb) - 1):
+            t0, t1 = tb[j], tb[j + 1]
+            with torch.cuda.stream(s_up):
+                for n in _INPUTS:
+                    dev[n][b0:b1, t0:t1].copy_(host[n][b0:b1, t0:t1], non_blocking=True)
+            up = torch.cuda.Event()
+            up.record(s_up)
+            s_run.wait_event(up)
+            init = (s0[b0:b1] if s0 is not None else None) if j == 0 else dev["sT"][b0:b1]
+            wkv7_forward(*(dev[n][b0:b1, t0:t1] for n in _INPUTS), init, dev["y"][b0:b1, t0:t1],
+                         dev["sT"][b0:b1], b1 - b0, t1 - t0, H, D, None, s_run)
+            ran = torch.cuda.Event()
+            ran.record(s_run)
+            s_down.wait_event(ran)
+            with torch.cuda.stream(s_down):
+                y_host[b0:b1, t0:t1].copy_(dev["y"][b0:b1, t0:t1], non_blocking=True)
+                if j == len(tb) - 2:
+                    sT_host[b0:b1].copy_(dev["sT"][b0:b1], non_blocking=True)
     done = torch.cuda.Event()
     done.record(s_down)
     st.wait_event(done)

@@ -264,9 +264,10 @@ def test_bad_offsets_reported_not_read(wk):
 
 
 def test_forward_host_pipeline(wk, oracle_mod):
-    """forward_host (pinned host inputs and outputs, per-sequence groups whose
-    copies overlap the prefill on three streams) equals one device-side call
-    bit for bit and the oracle within the bf16 bound; 3 sequences in 2 groups."""
+    """forward_host (pinned host inputs and outputs, pieces whose copies overlap
+    the prefill on three streams) equals one device-side call bit for bit and the
+    oracle within the bf16 bound: 3 sequences in 2 groups, and every sequence in
+    3 token ranges chained through the state."""
     inp = W.make_prefill(3, 130, 3, io="bf16", wdt="f32", s0_std=0.1, seed=91)
     t = inp.tensors()
     host = {n: x.pin_memory() for n, x in t.items()}
@@ -276,8 +277,12 @@ def test_forward_host_pipeline(wk, oracle_mod):
     y_h = torch.empty(tuple(inp.r.shape), dtype=torch.bfloat16).pin_memory()
     sT_h = torch.empty((3, 3, 64, 64), dtype=torch.float32).pin_memory()
     s0 = inp.s0.cuda()
-    for _ in range(2):  # the second call reuses the staging buffers and streams
-        wk.forward_host(host, dev, y_h, sT_h, s0=s0, parts=2)
+    # whole sequences in 2 groups, then token ranges [0, 64), [64, 128), [128, 130) of every
+    # sequence with the state carried between ranges; the calls reuse buffers and streams
+    for kw in (dict(parts=2), dict(t_parts=3), dict(parts=2)):
+        y_h.fill_(float("nan"))
+        sT_h.fill_(float("nan"))
+        wk.forward_host(host, dev, y_h, sT_h, s0=s0, **kw)
         torch.cuda.synchronize()
         assert wk.wkv7_get_device_status() == 0
         d = {n: x.cuda() for n, x in t.items()}
