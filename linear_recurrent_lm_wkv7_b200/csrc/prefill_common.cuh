@@ -92,25 +92,6 @@ __device__ __forceinline__ void ld_op_row32(const uint8_t* tile, uint32_t R, uin
     }
 }
 
-// 16 consecutive bf16 elements [c0, c0+16) of one row (two 16-byte accesses)
-__device__ __forceinline__ void st_bf16_row16(uint8_t* tile, uint32_t R, uint32_t row, uint32_t c0, const float* x) {
-#pragma unroll
-    for (int q = 0; q < 2; ++q)
-        *reinterpret_cast<uint4*>(tile + swz(row, (c0 + 8 * q) * 2, R)) =
-            make_uint4(pack_bf16x2(x[8 * q], x[8 * q + 1]), pack_bf16x2(x[8 * q + 2], x[8 * q + 3]),
-                       pack_bf16x2(x[8 * q + 4], x[8 * q + 5]), pack_bf16x2(x[8 * q + 6], x[8 * q + 7]));
-}
-__device__ __forceinline__ void ld_bf16_row16(const uint8_t* tile, uint32_t R, uint32_t row, uint32_t c0, float* x) {
-#pragma unroll
-    for (int q = 0; q < 2; ++q) {
-        const uint4 v = *reinterpret_cast<const uint4*>(tile + swz(row, (c0 + 8 * q) * 2, R));
-        x[8 * q + 0] = bf16lo_to_f32(v.x); x[8 * q + 1] = bf16hi_to_f32(v.x);
-        x[8 * q + 2] = bf16lo_to_f32(v.y); x[8 * q + 3] = bf16hi_to_f32(v.y);
-        x[8 * q + 4] = bf16lo_to_f32(v.z); x[8 * q + 5] = bf16hi_to_f32(v.z);
-        x[8 * q + 6] = bf16lo_to_f32(v.w); x[8 * q + 7] = bf16hi_to_f32(v.w);
-    }
-}
-
 // Descriptor of K-step s of a K-major operand tile with R rows (K = 64 elements).
 template <bool TF32>
 __device__ __forceinline__ uint64_t kmajor_desc(const uint8_t* tile, uint32_t R, uint32_t s) {
@@ -125,27 +106,6 @@ __device__ __forceinline__ uint64_t mnmajor_desc(const uint8_t* tile, uint32_t R
     return sdesc_sw128(addr, R * 128u, 1024);
 }
 
-
-// 32 consecutive fp32 columns written to this thread's TMEM lane (32x32b shape).
-// tcgen05.st reads its source registers asynchronously, so the store is waited
-// for before returning: the caller may reuse the array immediately.
-__device__ __forceinline__ void tmem_st32(uint32_t taddr, const float (&f)[32]) {
-    __syncwarp();  // .sync.aligned: the whole warp must execute it converged
-    asm volatile(
-        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
-        "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
-        "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};\n\t"
-        "tcgen05.wait::st.sync.aligned;" ::"r"(taddr),
-        "f"(f[0]), "f"(f[1]), "f"(f[2]), "f"(f[3]), "f"(f[4]), "f"(f[5]), "f"(f[6]), "f"(f[7]), "f"(f[8]),
-        "f"(f[9]), "f"(f[10]), "f"(f[11]), "f"(f[12]), "f"(f[13]), "f"(f[14]), "f"(f[15]), "f"(f[16]),
-        "f"(f[17]), "f"(f[18]), "f"(f[19]), "f"(f[20]), "f"(f[21]), "f"(f[22]), "f"(f[23]), "f"(f[24]),
-        "f"(f[25]), "f"(f[26]), "f"(f[27]), "f"(f[28]), "f"(f[29]), "f"(f[30]), "f"(f[31])
-        : "memory");
-}
-__device__ __forceinline__ void tmem_st_wait() {
-    __syncwarp();
-    asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
-}
 
 // Barrier over the `nthreads` threads of one warp group (named barrier `id`),
 // returning the AND of `pred` over them.
