@@ -57,6 +57,26 @@ _HOST_STREAMS = {}
 _INPUTS = ("r", "w_log", "k", "v", "a", "b")
 
 
+def host_pieces(B, T, parts=4, t_parts=1):
+    """How ``forward_host`` cuts a dense [B, T, ...] batch: returns ``(groups, bounds)``,
+    sequence groups [b0, b1) and token bounds, so that each piece (group, [t0, t1))
+    is contiguous in memory.  With ``t_parts`` > 1 every sequence is its own group
+    and the token bounds are multiples of 64 (the chunk length), so a range
+    continues exactly where the previous one stopped; otherwise there are ``parts``
+    groups of whole sequences.  T = 0 gives one empty range."""
+    t_parts = max(1, int(t_parts))
+    nck = (T + 63) // 64
+    bounds = sorted({min(T, 64 * (nck * j // t_parts)) for j in range(t_parts)} | {T})
+    if T == 0:
+        bounds = [0, 0]  # one empty piece: sT receives s0 (or zeros)
+    if len(bounds) > 2:
+        groups = [(b, b + 1) for b in range(B)]
+    else:
+        n = max(1, min(int(parts), B))
+        groups = [(B * p // n, B * (p + 1) // n) for p in range(n)]
+    return groups, bounds
+
+
 def forward_host(host, dev, y_host, sT_host, s0=None, parts=4, t_parts=1, stream=None):
     """Prefill of a dense batch whose inputs and outputs live in pinned host memory.
 
@@ -84,15 +104,7 @@ def forward_host(host, dev, y_host, sT_host, s0=None, parts=4, t_parts=1, stream
         _HOST_STREAMS[idx] = tuple(torch.cuda.Stream(device) for _ in range(3))
     s_up, s_run, s_down = _HOST_STREAMS[idx]
     B, T, H, D = host["r"].shape
-    nck = (T + 63) // 64
-    tb = sorted({min(T, 64 * (nck * j // max(1, int(t_parts)))) for j in range(max(1, int(t_parts)))} | {T})
-    if T == 0:
-        tb = [0, 0]  # one empty piece: sT receives s0 (or zeros)
-    if len(tb) > 2:
-        groups = [(b, b + 1) for b in range(B)]
-    else:
-        n = max(1, min(int(parts), B))
-        groups = [(B * p // n, B * (p + 1) // n) for p in range(n)]
+    groups, tb = host_pieces(B, T, parts, t_parts)
     start = torch.cuda.Event()
     start.record(st)
     for s_ in (s_up, s_run, s_down):
