@@ -202,3 +202,24 @@ def test_backward_noalloc_rejects_before_any_cuda_call(wk):
     assert wk.wkv7_status_string(-7)
     assert call(*ptrs, 0, 8, 1, 64, None, 1, 0, None) == -1
     assert call(*ptrs, 1, 8, 1, 32, None, 1, 0, None) == -2
+
+
+def test_c_program_compiles_and_links(wk, tmp_path):
+    """The C ABI is usable from plain C: a C99 program that includes the header and
+    references every entry point compiles and links against the library (nothing
+    is run, so no GPU is needed)."""
+    import shutil
+    import subprocess
+
+    if shutil.which("gcc") is None:
+        pytest.skip("no C compiler")
+    src = tmp_path / "use_wkv7.c"
+    calls = "\n".join(f"    (void)&{name};" for name in sorted(wk.EXPORTS))
+    src.write_text('#include "wkv7.h"\n#include <stdio.h>\nint main(void) {\n' + calls +
+                   '\n    printf("%s\\n", wkv7_status_string(WKV7_OK));\n    return 0;\n}\n')
+    libdir = os.path.dirname(wk.LIB_PATH)
+    cuda_lib = "/usr/local/cuda/lib64"
+    cmd = ["gcc", "-std=c99", "-Wall", "-Werror", "-I", os.path.join(ROOT, "include"), str(src), "-o",
+           str(tmp_path / "use_wkv7"), wk.LIB_PATH, f"-Wl,-rpath-link,{cuda_lib}", f"-Wl,-rpath,{libdir}"]
+    res = subprocess.run(cmd, capture_output=True, text=True)
+    assert res.returncode == 0, res.stderr
