@@ -5,7 +5,11 @@
 One JSON line on rank 0.  `value` is prefill tokens/s of the whole job for the
 B4 T1024 H32 D64 prefill (bf16 inputs, fp32 decay logits, zero initial state),
 timed with CUDA events per launch on the launching stream, L2 flushed (a
-256 MB write) between timed launches.  `e2e` is the same metric through the
+256 MB write) between timed launches.  `long` and `packed` time the same entry
+point on the long-context prefill (B1 T16384 H40, N(0, 0.1^2) initial state;
+the literal decay formula and the long-memory variant) and on the packed
+variable-length prefill (16 sequences, lengths U{512..8192}, pad tokens),
+each with its own roofline.  `e2e` is the same metric through the
 public API from pinned host buffers (host->device copies of the inputs and
 device->host copies of y and sT inside the timed region).  `gated` times the
 same prefill with the gated read-out (wkv7_forward_gated, z instead of y; the
@@ -43,7 +47,7 @@ L2_FLUSH_BYTES = 256 << 20
 # DRAM traffic of one prefill launch (dram__bytes_read.sum + dram__bytes_write.sum)
 # from an ncu capture of this workload, valid only for the kernel sources it was
 # taken on (SHA-256 over the files below); any change makes it null until the
-# capture is repeated.  Summary: profiles/wkv7_prefill_pipe_kernel_prefill_1p5b.md
+# capture is repeated.
 NCU_TRAFFIC = {"sha256": "8bebd1a9fdcffb412393fa4f71b647588418bb938f88825c8a37cdb86ffca3de",
                "bytes": 123540992, "workload": "prefill_1p5b"}
 KERNEL_SOURCES = ("linear_recurrent_lm_wkv7_b200/csrc/wkv7_prefill_pipe.cu",
@@ -75,6 +79,13 @@ def prefill_bytes(n_tokens_heads, io_b, w_b, n_states, with_s0):
     w_log read once (w_b), sT written once (and s0 read once when given)."""
     per = D * (6 * io_b + w_b)
     return n_tokens_heads * per + n_states * D * D * 4 * (2 if with_s0 else 1)
+
+
+def prefill_config(B, T, H, world):
+    """`config` of the headline line, shared by both arms of the benchmark."""
+    return {"workload": PREFILL_WORKLOAD, "B": B, "T": T, "H": H, "D": D, "io": "bf16", "w_log": "f32",
+            "s0": "zero", "chunk": 64, "l2": "flushed (256 MB write) between launches",
+            "parallelism": f"replicas{world}" if world > 1 else "single"}
 
 
 def prefill_flops(n_tokens_heads, L=64):
@@ -187,7 +198,7 @@ def run_reference(args):
             "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": 1000.0 * 4 * 1024 / cb["value"], "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": PREFILL_WORKLOAD, "B": 4, "T": 1024, "H": 32, "D": D},
+            "config": prefill_config(4, 1024, 32, 1),
             "cpu_baseline": cb,
             "e2e": {"value": cb["value"], "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
@@ -252,6 +263,61 @@ def run_ours(args):
     bytes_alg = prefill_bytes(B * T * H, 2, 4, B * H, with_s0=False)
     achieved = bytes_alg / (ms * 1e-3) / 1e9
     flops = prefill_flops(B * T * H)
+
+    def max_over_ranks(x):
+        if world > 1:
+            t_ = torch.tensor([x], device="cuda")
+            dist.all_reduce(t_, op=dist.ReduceOp.MAX)
+            x = float(t_.item())
+        return x
+
+    def prefill_section(name, inp_, label, s0_kind):
+        """Times wkv7_forward on one more prefill workload: per-launch CUDA events,
+        L2 flushed between launches; tokens/s counts real tokens (pads excluded);
+        the roofline bytes are the workload's own (s0 read and sT written)."""
+        d_ = {k_: v_.cuda() for k_, v_ in inp_.tensors().items()}
+        s0_ = inp_.s0.cuda() if inp_.s0 is not None else None
+        offs_ = inp_.seq_offsets.cuda() if inp_.seq_offsets is not None else None
+        y_ = torch.empty_like(d_["r"])
+        sT_ = torch.empty((inp_.B, inp_.H, D, D), dtype=torch.float32, device="cuda")
+
+        def st_():
+            wk.wkv7_forward(d_["r"], d_["w_log"], d_["k"], d_["v"], d_["a"], d_["b"], s0_, y_, sT_, inp_.B, inp_.T,
+                            inp_.H, D, offs_, stream)
+
+        for _ in range(max(3, args.warmup)):
+            st_()
+        torch.cuda.synchronize()
+        tt = time_launches(st_, args.steps, stream, flush)
+        if wk.wkv7_get_device_status() != 0:
+            raise RuntimeError(f"device status set during the {name} run")
+        ms_ = max_over_ranks(sum(tt) / len(tt))
+        slots = inp_.T if inp_.seq_offsets is not None else inp_.B * inp_.T  # tokens in the tensors, pads included
+        bytes_ = prefill_bytes(slots * inp_.H, 2, 4, inp_.B * inp_.H, with_s0=inp_.s0 is not None)
+        ach = bytes_ / (ms_ * 1e-3) / 1e9
+        out = {"workload": name, "variant": label, "B": inp_.B, "H": inp_.H, "tokens": inp_.n_real_tokens,
+               "token_slots": slots, "s0": s0_kind, "tokens_per_s": world * inp_.n_real_tokens / (ms_ * 1e-3),
+               "ms_per_step": ms_,
+               "roofline": {"bound": "hbm", "achieved": ach, "peak": hbm_peak, "unit": "GB/s", "frac": ach / hbm_peak,
+                            "algorithmic_bytes_per_launch": bytes_,
+                            "hbm_time_floor_us": bytes_ / (hbm_peak * 1e9) * 1e6}}
+        if inp_.seq_offsets is not None:
+            out["lengths"] = inp_.lengths
+        del d_, y_, sT_
+        return out
+
+    # ---------------- long-context prefill B1 T16384 H40 (the workload's literal decay formula,
+    # and the labelled long-memory variant), N(0, 0.1^2) initial state
+    long_sections = []
+    for mu_z, label in ((1.0, "decay z ~ N(1,1) (literal formula)"), (-3.0, "decay z ~ N(-3,1) (long memory)")):
+        linp = W.make_workload("prefill_2p9b_long", mu_z=mu_z, seed=2 + 1000 * rank)
+        long_sections.append(prefill_section("prefill_2p9b_long", linp, label, "N(0, 0.1^2)"))
+        del linp
+    # ---------------- packed variable-length prefill: 16 sequences, lengths U{512..8192}, pads U{0..63}
+    pinp = W.make_workload("packed_1p5b", seed=4 + 1000 * rank)
+    packed_section = prefill_section("packed_1p5b", pinp, "16 sequences, pads U{0..63} (w = 1, k = v = a = b = 0)",
+                                     "N(0, 0.1^2)")
+    del pinp
 
     # ---------------- the same prefill with the gated read-out (wkv7_forward_gated)
     rk_h, gate_h = W.make_gate(tuple(dev["r"].shape), H, D, io="bf16", seed=2 + 1000 * rank)
@@ -438,9 +504,7 @@ def run_ours(args):
             "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": {"workload": PREFILL_WORKLOAD, "B": B, "T": T, "H": H, "D": D, "io": "bf16",
-                       "w_log": "f32", "s0": "zero", "chunk": 64, "l2": "flushed (256 MB write) between launches",
-                       "parallelism": f"replicas{world}" if world > 1 else "single"},
+            "config": prefill_config(B, T, H, world),
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
                          "frac": achieved / hbm_peak, "traffic": measured_traffic(), "peak_source": peak_src,
                          "algorithmic_bytes_per_launch": bytes_alg,
@@ -452,6 +516,8 @@ def run_ours(args):
                     "ms_per_step": e2e_ms, "api": "forward_host (per-sequence upload / prefill / download overlapped)"},
             "gpu_launches": args.steps,
             "clocks": clocks,
+            "long": long_sections,
+            "packed": packed_section,
             "gated": {"workload": PREFILL_WORKLOAD, "tokens_per_s": world * tokens / (gms * 1e-3),
                       "ms_per_step": gms,
                       "roofline": {"bound": "hbm", "achieved": gach, "peak": hbm_peak, "unit": "GB/s",

@@ -31,10 +31,18 @@
  *  - D must be 64 (the head size of the RWKV-7 layers the pages describe);
  *    other head sizes return WKV7_ERR_UNSUPPORTED.
  *  - Every pointer must be 16-byte aligned (WKV7_ERR_MISALIGNED otherwise).
- *  - Documented, unchecked precondition: w_log <= -0.5 or w_log = -inf, i.e.
- *    w in [exp(-exp(-0.5)), 1] ~= [0.545, 1], the range produced by the
- *    hxa07D decay parametrisation -softplus(-x) - 0.5.  w_log = -inf gives
- *    w = 1 exactly (used for padding).
+ *  - Decay range.  The hxa07D decay parametrisation -softplus(-x) - 0.5 gives
+ *    w_log <= -0.5, i.e. w in [exp(-exp(-0.5)), 1] ~= [0.545, 1]; w_log = -inf
+ *    gives w = 1 exactly (used for padding).  The prefill works on 64-token
+ *    chunks and scales the operands by the decay accumulated inside a chunk,
+ *    Gamma_t = prod_{s<=t} w_s per key channel, and by 1 / Gamma_t.  It is exact
+ *    (to the stated tolerances) whenever every chunk keeps Gamma_64 >= 1e-30 in
+ *    every channel, i.e. sum of exp(w_log) over the chunk <= 69: always true in
+ *    the parametrised range (Gamma_64 >= e^-38.8) and for any w_log <= 0.
+ *    A chunk that decays further (e.g. w_log > 0.08 on all 64 tokens) is
+ *    detected on the device and reported as WKV7_ERR_DECAY_RANGE through
+ *    wkv7_get_device_status; y and sT of that call are then unspecified.  The
+ *    decode step works token by token and has no such limit.
  *  - Errors in the arguments are detected on the host before anything is
  *    launched and returned as a negative status; nothing is written then.
  *    Errors that only the device can see (a bounded wait that expired, packed
@@ -64,7 +72,8 @@ typedef enum {
     WKV7_ERR_CUDA = -4,           /* a CUDA runtime call or a launch failed */
     WKV7_ERR_DEVICE_TIMEOUT = -5, /* a bounded device-side wait expired */
     WKV7_ERR_DEVICE_BOUNDS = -6,  /* packed offsets not monotone or beyond T */
-    WKV7_ERR_SCRATCH_LIMIT = -7   /* wkv7_backward_noalloc: problem needs more than its fixed scratch */
+    WKV7_ERR_SCRATCH_LIMIT = -7,  /* wkv7_backward_noalloc: problem needs more than its fixed scratch */
+    WKV7_ERR_DECAY_RANGE = -8     /* device: a 64-token chunk decays below the exact range (see above) */
 } wkv7_status;
 
 /*
@@ -220,9 +229,10 @@ int wkv7_backward(const void* r, const void* w_log, const void* k, const void* v
  *   There is one scratch per device: calls whose kernels may overlap on the
  *   same device (unordered streams, several host threads) race on it; the
  *   caller must order them.
- *   The first call on each device looks up the scratch's address
- *   (cudaGetSymbolAddress, which may load the library's module); make that
- *   first call before any stream capture.
+ *   Every call looks up the scratch's address on the current device with
+ *   cudaGetSymbolAddress (no allocation); the first call on a device may load
+ *   the library's module there, so make that first call before any stream
+ *   capture.
  */
 #define WKV7_NOALLOC_SCRATCH_BYTES ((size_t)16 << 20)
 int wkv7_backward_noalloc(const void* r, const void* w_log, const void* k, const void* v,
@@ -236,8 +246,8 @@ const char* wkv7_status_string(int status);
 
 /*
  * Synchronizes `stream`, then reads and clears the status word of the current
- * device.  Returns WKV7_OK, WKV7_ERR_DEVICE_TIMEOUT, WKV7_ERR_DEVICE_BOUNDS, or
- * WKV7_ERR_CUDA if the synchronization itself failed.
+ * device.  Returns WKV7_OK, WKV7_ERR_DEVICE_TIMEOUT, WKV7_ERR_DEVICE_BOUNDS,
+ * WKV7_ERR_DECAY_RANGE, or WKV7_ERR_CUDA if the synchronization itself failed.
  */
 int wkv7_get_device_status(void* stream);
 

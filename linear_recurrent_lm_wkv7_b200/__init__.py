@@ -94,7 +94,12 @@ def forward_host(host, dev, y_host, sT_host, s0=None, parts=4, t_parts=1, stream
     one before run on three CUDA streams at once, and the results equal one call
     over the whole batch.  Everything is ordered after ``stream`` (default: the
     current stream), which then waits for all of it: the call is asynchronous
-    like a kernel launch on ``stream``."""
+    like a kernel launch on ``stream``.
+    The three side streams are created once per device and shared by every call
+    on that device.  Calls from several host threads at once are correct but
+    their copies and kernels serialise on those streams; such calls must not
+    share ``dev`` buffers (nothing orders one call's use of them against
+    another's)."""
     import torch
 
     device = dev["r"].device

@@ -24,6 +24,7 @@ STATUS = {
     -5: "WKV7_ERR_DEVICE_TIMEOUT",
     -6: "WKV7_ERR_DEVICE_BOUNDS",
     -7: "WKV7_ERR_SCRATCH_LIMIT",
+    -8: "WKV7_ERR_DECAY_RANGE",
 }
 # every symbol include/wkv7.h declares
 EXPORTS = (

@@ -1,5 +1,6 @@
 // wkv7_api.cu — the C ABI declared in include/wkv7.h: argument validation on
 // the host, dispatch to the kernels, and the per-device status word.
+#include <atomic>
 #include <cstdint>
 #include <cstring>
 
@@ -13,17 +14,14 @@ namespace {
 __device__ int g_status = 0;
 
 constexpr int kMaxDevices = 64;
-int* g_status_ptr[kMaxDevices] = {};
 
+// Address of the current device's status word.  Looked up on every call
+// (cudaGetSymbolAddress allocates nothing), so that no cached address can
+// outlive a device reset and nothing is shared between host threads.
 int status_ptr(int** out) {
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return WKV7_ERR_CUDA;
-    if (!g_status_ptr[dev]) {
-        void* p = nullptr;
-        if (cudaGetSymbolAddress(&p, g_status) != cudaSuccess) return WKV7_ERR_CUDA;
-        g_status_ptr[dev] = static_cast<int*>(p);
-    }
-    *out = g_status_ptr[dev];
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_status) != cudaSuccess || !p) return WKV7_ERR_CUDA;
+    *out = static_cast<int*>(p);
     return WKV7_OK;
 }
 
@@ -46,15 +44,20 @@ int check_device() {
     return WKV7_OK;
 }
 
+// The device check, remembered per device ordinal (0 unknown, 1 ok, else the
+// status); entries are atomics because host threads may call concurrently.
 int cached_device_check() {
-    static int cache[kMaxDevices] = {};  // 0 unknown, 1 ok, else status
+    static std::atomic<int> cache[kMaxDevices];
     int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return WKV7_ERR_CUDA;
-    if (cache[dev] == 0) {
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) return WKV7_ERR_CUDA;
+    if (dev >= kMaxDevices) return check_device();
+    int c = cache[dev].load(std::memory_order_acquire);
+    if (c == 0) {
         const int s = check_device();
-        cache[dev] = (s == WKV7_OK) ? 1 : s;
+        c = (s == WKV7_OK) ? 1 : s;
+        cache[dev].store(c, std::memory_order_release);
     }
-    return cache[dev] == 1 ? WKV7_OK : cache[dev];
+    return c == 1 ? WKV7_OK : c;
 }
 
 // Zero-token call: sT <- s0 (or zeros).
@@ -80,6 +83,7 @@ const char* wkv7_status_string(int status) {
         case WKV7_ERR_DEVICE_TIMEOUT: return "device-side bounded wait expired";
         case WKV7_ERR_DEVICE_BOUNDS: return "packed sequence offsets out of range";
         case WKV7_ERR_SCRATCH_LIMIT: return "problem needs more than the fixed scratch of wkv7_backward_noalloc";
+        case WKV7_ERR_DECAY_RANGE: return "a 64-token chunk decays below the prefill's exact range (Gamma < 1e-30)";
         default: return "unknown status";
     }
 }

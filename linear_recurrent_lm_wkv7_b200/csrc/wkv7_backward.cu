@@ -279,16 +279,9 @@ __global__ void __launch_bounds__(NTHR, 1)
 template <typename IO, typename WT>
 cudaError_t launch_bwd_typed(const BackwardArgs& p, cudaStream_t stream) {
     auto kern = wkv7_backward_kernel<IO, WT>;
-    static unsigned long long configured = 0;
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
+    static std::atomic<unsigned long long> configured{0};
+    const cudaError_t e = configure_smem_once(kern, static_cast<int>(SMEM_BYTES), configured);
     if (e != cudaSuccess) return e;
-    const unsigned long long bit = 1ull << (dev & 63);
-    if (!(configured & bit)) {
-        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(SMEM_BYTES));
-        if (e != cudaSuccess) return e;
-        configured |= bit;
-    }
     const long units = static_cast<long>(p.B) * p.H;
     kern<<<static_cast<unsigned>(units), NTHR, SMEM_BYTES, stream>>>(
         static_cast<const IO*>(p.r), static_cast<const WT*>(p.w_log), static_cast<const IO*>(p.k),

@@ -207,21 +207,16 @@ __global__ void __launch_bounds__(256, BLOCKS_PER_SM)
 template <typename IO, typename WT, bool PRO, bool GATED>
 cudaError_t launch_typed(const DecodeArgs& p, int* status, cudaStream_t stream) {
     auto kern = wkv7_decode_kernel<IO, WT, PRO, GATED>;
-    static unsigned long long configured = 0;
-    static int sm_count[64] = {};
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
+    static std::atomic<unsigned long long> configured{0};
+    cudaError_t e = configure_smem_once(kern, static_cast<int>(SMEM_BYTES), configured);
     if (e != cudaSuccess) return e;
-    const unsigned long long bit = 1ull << (dev & 63);
-    if (!(configured & bit)) {
-        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
-        if (e != cudaSuccess) return e;
-        e = cudaDeviceGetAttribute(&sm_count[dev & 63], cudaDevAttrMultiProcessorCount, dev);
-        if (e != cudaSuccess) return e;
-        configured |= bit;
-    }
+    int dev = 0, sms = 0;
+    e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return e;
     const long units = static_cast<long>(p.B) * p.H;
-    const long slots = static_cast<long>(BLOCKS_PER_SM) * sm_count[dev & 63];
+    const long slots = static_cast<long>(BLOCKS_PER_SM) * sms;
     const long grid = units < slots ? units : slots;
     kern<<<static_cast<unsigned>(grid), 256, SMEM_BYTES, stream>>>(
         static_cast<const IO*>(p.r), static_cast<const WT*>(p.w_log), static_cast<const IO*>(p.k),

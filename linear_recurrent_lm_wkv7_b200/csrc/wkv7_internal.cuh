@@ -4,6 +4,7 @@
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <cstdint>
 
 #include "wkv7.h"
@@ -11,6 +12,11 @@
 namespace wkv7 {
 
 constexpr int kHead = 64;  // D: head size supported by every kernel
+// Smallest decay a 64-token chunk of the prefill may accumulate in one key
+// channel (Gamma_64 = prod of w over the chunk): the chunked algebra scales
+// operands by 1 / Gamma_t, which must stay far from the fp32 / bf16 overflow
+// at 3.4e38.  Smaller values are reported as WKV7_ERR_DECAY_RANGE.
+constexpr float kMinGammaL = 1e-30f;
 
 struct PrefillArgs {
     const void* r;
@@ -92,6 +98,24 @@ cudaError_t launch_expire_wait(int spins, int* status, cudaStream_t stream);
 long backward_ckpt_chunks(int B, int T, int packed);
 size_t backward_workspace_floats(int B, int T, int H, int packed);
 cudaError_t launch_backward(const BackwardArgs& p, int io_dtype, int w_dtype, cudaStream_t stream);
+
+// Raises `kern`'s dynamic shared-memory limit to `bytes` the first time it is
+// launched on the current device.  `configured` holds one bit per device
+// ordinal below 64 (ordinals from 64 up set the attribute on every call).  Two
+// threads that launch first at the same time may both set it, which is
+// harmless: the call is idempotent.
+template <typename K>
+cudaError_t configure_smem_once(K kern, int bytes, std::atomic<unsigned long long>& configured) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    const unsigned long long bit = dev < 64 ? 1ull << dev : 0ull;
+    if (bit && (configured.load(std::memory_order_acquire) & bit)) return cudaSuccess;
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e != cudaSuccess) return e;
+    configured.fetch_or(bit, std::memory_order_release);
+    return cudaSuccess;
+}
 
 // Records the first device-side error of a call sequence (first writer wins).
 __device__ __forceinline__ void report_status(int* status, int code) {

@@ -27,20 +27,15 @@ namespace {
 constexpr size_t kScratchBytes = WKV7_NOALLOC_SCRATCH_BYTES;
 static __device__ __align__(256) float g_bwd_scratch[kScratchBytes / sizeof(float)];
 
-constexpr int kMaxDevices = 64;
-void* g_scratch_ptr[kMaxDevices] = {};
-
-// Address of this device's scratch, looked up once per device with that device
-// current (the first call on a device does this; it may load the module).
+// Address of the scratch on the current device.  cudaGetSymbolAddress
+// allocates nothing and is cheap, so it runs on every call: no cached address
+// can outlive a device reset, and host threads share no mutable state here.
+// The first call on a device may load the library's module there (which is
+// why that first call should come before any stream capture).
 int scratch_for_current_device(void** out) {
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return WKV7_ERR_CUDA;
-    if (!g_scratch_ptr[dev]) {
-        void* p = nullptr;
-        if (cudaGetSymbolAddress(&p, g_bwd_scratch) != cudaSuccess || !p) return WKV7_ERR_CUDA;
-        g_scratch_ptr[dev] = p;
-    }
-    *out = g_scratch_ptr[dev];
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_bwd_scratch) != cudaSuccess || !p) return WKV7_ERR_CUDA;
+    *out = p;
     return WKV7_OK;
 }
 
@@ -51,9 +46,14 @@ extern "C" int wkv7_backward_noalloc(const void* r, const void* w_log, const voi
                                      void* dw_log, void* dk, void* dv, void* da, void* db, float* ds0, int B, int T,
                                      int H, int D, const int32_t* seq_offsets, int io_dtype, int w_dtype,
                                      void* stream) {
-    // decided before any CUDA call; the remaining checks are wkv7_backward's own
+    // The argument checks that come before the scratch limit, in wkv7_backward's
+    // order, so that both entry points return the same code for the same bad
+    // arguments; the remaining checks are wkv7_backward's own.
     if (B <= 0 || T < 0 || H <= 0 || D <= 0) return WKV7_ERR_INVALID_ARG;
+    const bool dt_ok = (io_dtype == WKV7_F32 || io_dtype == WKV7_BF16) && (w_dtype == WKV7_F32 || w_dtype == WKV7_BF16);
+    if (!dt_ok) return WKV7_ERR_INVALID_ARG;
     if (D != 64) return WKV7_ERR_UNSUPPORTED;
+    if (!ds0) return WKV7_ERR_INVALID_ARG;
     if (wkv7_backward_workspace_bytes(B, T, H, D, seq_offsets ? 1 : 0) > kScratchBytes) return WKV7_ERR_SCRATCH_LIMIT;
     void* ws = nullptr;
     const int st = scratch_for_current_device(&ws);

@@ -457,6 +457,8 @@ __global__ void __launch_bounds__(NT, 1)
                 }
             } else {
                 const float GL = sm.gammaL[jj];
+                // 1 / Gamma_t must stay far inside the fp32 range (false for NaN too)
+                if (!(GL >= kMinGammaL)) report_status(status, WKV7_ERR_DECAY_RANGE);
 #pragma unroll
                 for (int q = 0; q < 2; ++q) {
                     tmem_load32(tmem + lane_base + COL_O + 32 * q, o);
@@ -491,16 +493,9 @@ template <typename IO, typename WT, bool TF32, bool PRO>
 cudaError_t launch_typed(const PrefillArgs& p, cudaStream_t stream) {
     constexpr uint32_t smem = smem_bytes_needed<TF32>();
     auto kern = wkv7_prefill_kernel<IO, WT, TF32, PRO>;
-    static unsigned long long configured = 0;  // one bit per device ordinal
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
+    static std::atomic<unsigned long long> configured{0};
+    const cudaError_t e = configure_smem_once(kern, static_cast<int>(smem), configured);
     if (e != cudaSuccess) return e;
-    const unsigned long long bit = 1ull << (dev & 63);
-    if (!(configured & bit)) {
-        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-        if (e != cudaSuccess) return e;
-        configured |= bit;
-    }
     const long units = static_cast<long>(p.B) * p.H;
     kern<<<static_cast<unsigned>(units), NT, smem, stream>>>(
         static_cast<const IO*>(p.r), static_cast<const WT*>(p.w_log), static_cast<const IO*>(p.k),

@@ -855,6 +855,8 @@ __global__ void __launch_bounds__(NTHR, 1)
                 }
             } else {
                 const float GL = gam_all[g * 128 + (kk_ & 1) * 64 + x];
+                // 1 / Gamma_t must stay far inside the fp32 / bf16 range (false for NaN too)
+                if (!(GL >= kMinGammaL)) report_status(status, WKV7_ERR_DECAY_RANGE);
 #pragma unroll
                 for (int q = 0; q < 2; ++q) {
                     tmem_load32(tm_out + lane_base + 32 * q, o);
@@ -889,16 +891,9 @@ __global__ void __launch_bounds__(NTHR, 1)
 template <typename WT, bool GATED, bool PRO>
 cudaError_t launch_pipe_typed(const PrefillArgs& p, cudaStream_t stream) {
     auto kern = wkv7_prefill_pipe_kernel<WT, GATED, PRO>;
-    static unsigned long long configured = 0;
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
+    static std::atomic<unsigned long long> configured{0};
+    const cudaError_t e = configure_smem_once(kern, static_cast<int>(SMEM_BYTES), configured);
     if (e != cudaSuccess) return e;
-    const unsigned long long bit = 1ull << (dev & 63);
-    if (!(configured & bit)) {
-        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
-        if (e != cudaSuccess) return e;
-        configured |= bit;
-    }
     TmaMaps maps;
     const uint64_t ntok = p.seq_offsets ? static_cast<uint64_t>(p.T) : static_cast<uint64_t>(p.B) * p.T;
     const int H_kv = PRO ? p.H_kv : p.H;

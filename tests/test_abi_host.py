@@ -202,6 +202,12 @@ def test_backward_noalloc_rejects_before_any_cuda_call(wk):
     assert wk.wkv7_status_string(-7)
     assert call(*ptrs, 0, 8, 1, 64, None, 1, 0, None) == -1
     assert call(*ptrs, 1, 8, 1, 32, None, 1, 0, None) == -2
+    # a bad dtype code is an invalid argument even when the problem is also too large,
+    # as wkv7_backward would report it (its checks come before the scratch limit)
+    assert call(*ptrs, 2, 8192, 32, 64, None, 7, 0, None) == -1
+    assert call(*ptrs, 2, 8192, 32, 64, None, 1, 5, None) == -1
+    bwd_same = wk._binding.raw_call_backward
+    assert bwd_same(*ptrs[:16], ptrs[0] + 0x8000000, 1 << 40, 2, 8192, 32, 64, None, 7, 0, None) == -1
 
 
 def test_c_program_compiles_and_links(wk, tmp_path):

@@ -99,6 +99,57 @@ def test_long_memory_decay(wk, oracle_mod):
     check_prefill(wk, oracle_mod, inp)
 
 
+def _constant_decay(inp, value):
+    """The same inputs with every decay logit set to `value` (pad tokens of a
+    packed batch keep their -inf)."""
+    w = inp.w_log
+    pad = torch.isneginf(w.float())
+    inp.w_log = torch.where(pad, w, torch.full_like(w, value)).contiguous()
+    return inp
+
+
+@pytest.mark.parametrize("io,wdt", [("bf16", "f32"), ("bf16", "bf16"), ("f32", "f32")])
+def test_decay_at_the_parametrised_bound(wk, oracle_mod, io, wdt):
+    """w_log = -0.5 on every token (w = 0.545, the fastest decay the hxa07D
+    parametrisation produces): a 64-token chunk decays by e^-38.8 in every
+    channel, the extreme the chunked algebra's 1 / Gamma scaling must carry.
+    Four chunks, the last one ragged, non-zero initial state."""
+    inp = _constant_decay(W.make_prefill(2, 200, 3, io=io, wdt=wdt, s0_std=0.1, seed=120), -0.5)
+    check_prefill(wk, oracle_mod, inp)
+
+
+def test_decay_bound_packed_with_pads(wk, oracle_mod):
+    """w_log = -0.5 on every real token of a packed batch whose pad tokens carry
+    -inf (w = 1): chunks mix the fastest decay with identity steps, and the
+    sequence starts are not chunk aligned."""
+    inp = _constant_decay(W.make_packed([150, 64, 7, 130], [13, 63, 0, 40], 3, io="bf16", wdt="f32",
+                                        s0_std=0.1, seed=121), -0.5)
+    check_prefill(wk, oracle_mod, inp)
+
+
+@pytest.mark.parametrize("io", ["bf16", "f32"])
+def test_decay_inside_exact_range_beyond_bound(wk, oracle_mod, io):
+    """w_log = 0 on every token (w = 0.368, faster than the parametrisation
+    allows): each chunk decays by e^-64, still inside the exact range
+    (Gamma_64 >= 1e-30), so results stay within the parity bounds."""
+    inp = _constant_decay(W.make_prefill(1, 200, 2, io=io, wdt="f32", s0_std=0.1, seed=122), 0.0)
+    check_prefill(wk, oracle_mod, inp)
+    assert wk.wkv7_get_device_status() == 0
+
+
+@pytest.mark.parametrize("io", ["bf16", "f32"])
+def test_decay_beyond_exact_range_is_reported(wk, io):
+    """w_log = 1 on every token (w = 0.066): a 64-token chunk would decay by
+    e^-174, below the exact range; the call reports WKV7_ERR_DECAY_RANGE in the
+    device status instead of returning silently."""
+    inp = _constant_decay(W.make_prefill(1, 130, 2, io=io, wdt="f32", s0_std=0.1, seed=123), 1.0)
+    d, s0, _ = to_dev(inp)
+    assert wk.wkv7_get_device_status() == 0
+    wk.forward(d["r"], d["w_log"], d["k"], d["v"], d["a"], d["b"], s0)
+    assert wk.wkv7_get_device_status() == -8
+    assert wk.wkv7_get_device_status() == 0  # cleared by the read
+
+
 def test_packed_with_pads_and_empty(wk, oracle_mod):
     """Packed batch: empty sequence, sub-chunk sequences, chunk-straddling
     starts, pad tokens (w_log = -inf, k = v = a = b = 0)."""
