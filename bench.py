@@ -4,8 +4,10 @@
 
 One JSON line on rank 0.  `value` is prefill tokens/s of the whole job for the
 B4 T1024 H32 D64 prefill (bf16 inputs, fp32 decay logits, zero initial state),
-timed with CUDA events per launch on the launching stream, L2 flushed (a
-256 MB write) between timed launches.  `long` and `packed` time the same entry
+timed with CUDA events per launch on the launching stream.  Consecutive
+launches alternate between two resident copies of the inputs (2 x 136 MB,
+more than the 126 MB L2), so no launch finds its inputs in L2 and no flush
+kernel has to run between them.  `long` and `packed` time the same entry
 point on the long-context prefill (B1 T16384 H40, N(0, 0.1^2) initial state;
 the literal decay formula and the long-memory variant) and on the packed
 variable-length prefill (16 sequences, lengths U{512..8192}, pad tokens),
@@ -84,7 +86,8 @@ def prefill_bytes(n_tokens_heads, io_b, w_b, n_states, with_s0):
 def prefill_config(B, T, H, world):
     """`config` of the headline line, shared by both arms of the benchmark."""
     return {"workload": PREFILL_WORKLOAD, "B": B, "T": T, "H": H, "D": D, "io": "bf16", "w_log": "f32",
-            "s0": "zero", "chunk": 64, "l2": "flushed (256 MB write) between launches",
+            "s0": "zero", "chunk": 64,
+            "l2": "inputs larger than L2: two input copies (2 x 136 MB) alternated between launches",
             "parallelism": f"replicas{world}" if world > 1 else "single"}
 
 
@@ -231,12 +234,22 @@ def run_ours(args):
     B, T, H = inp.B, inp.T, inp.H
     host = {k: v.pin_memory() for k, v in inp.tensors().items()}
     dev = {k: v.cuda() for k, v in host.items()}
+    # a second resident copy of the inputs: launches alternate between the two, so the
+    # working set (2 x 136 MB) exceeds L2 and every launch reads its inputs from HBM
+    dev2 = {k: v.clone() for k, v in dev.items()}
+    copies = (dev, dev2)
+    alt = {"i": 0}
+
+    def cur():
+        alt["i"] += 1
+        return copies[alt["i"] & 1]
+
     y = torch.empty_like(dev["r"])
     sT = torch.empty((B, H, D, D), dtype=torch.float32, device="cuda")
 
     def step():
-        wk.wkv7_forward(dev["r"], dev["w_log"], dev["k"], dev["v"], dev["a"], dev["b"], None, y, sT, B, T, H, D,
-                        None, stream)
+        x = cur()
+        wk.wkv7_forward(x["r"], x["w_log"], x["k"], x["v"], x["a"], x["b"], None, y, sT, B, T, H, D, None, stream)
 
     for _ in range(args.warmup):
         step()
@@ -248,7 +261,7 @@ def run_ours(args):
     torch.cuda.synchronize()
     clk = ClockSampler(local)
     clk.start()
-    times = time_launches(step, args.steps, stream, flush)
+    times = time_launches(step, args.steps, stream)
     clocks = clk.stop()
     torch.cuda.synchronize()
     if world > 1:
@@ -273,7 +286,7 @@ def run_ours(args):
 
     def prefill_section(name, inp_, label, s0_kind):
         """Times wkv7_forward on one more prefill workload: per-launch CUDA events,
-        L2 flushed between launches; tokens/s counts real tokens (pads excluded);
+        inputs far larger than L2 (no flush needed); tokens/s counts real tokens (pads excluded);
         the roofline bytes are the workload's own (s0 read and sT written)."""
         d_ = {k_: v_.cuda() for k_, v_ in inp_.tensors().items()}
         s0_ = inp_.s0.cuda() if inp_.s0 is not None else None
@@ -288,7 +301,7 @@ def run_ours(args):
         for _ in range(max(3, args.warmup)):
             st_()
         torch.cuda.synchronize()
-        tt = time_launches(st_, args.steps, stream, flush)
+        tt = time_launches(st_, args.steps, stream)
         if wk.wkv7_get_device_status() != 0:
             raise RuntimeError(f"device status set during the {name} run")
         ms_ = max_over_ranks(sum(tt) / len(tt))
@@ -325,13 +338,14 @@ def run_ours(args):
     z = torch.empty_like(dev["r"])
 
     def gstep():
-        wk.wkv7_forward_gated(dev["r"], dev["w_log"], dev["k"], dev["v"], dev["a"], dev["b"], None, rk_d, gate_d, z,
+        x = cur()
+        wk.wkv7_forward_gated(x["r"], x["w_log"], x["k"], x["v"], x["a"], x["b"], None, rk_d, gate_d, z,
                               sT, B, T, H, D, None, stream)
 
     for _ in range(max(3, args.warmup)):
         gstep()
     torch.cuda.synchronize()
-    gtimes = time_launches(gstep, args.steps, stream, flush)
+    gtimes = time_launches(gstep, args.steps, stream, flush)  # gate, r_k and the fused inputs have one copy
     if wk.wkv7_get_device_status() != 0:
         raise RuntimeError("device status set during the gated run")
     gms = sum(gtimes) / len(gtimes)
@@ -379,7 +393,8 @@ def run_ours(args):
     bws = torch.empty(wk.wkv7_backward_workspace_bytes(B, T, H, D, False) // 4, dtype=torch.float32, device="cuda")
 
     def bstep():
-        wk.wkv7_backward(dev["r"], dev["w_log"], dev["k"], dev["v"], dev["a"], dev["b"], None, dyd, None,
+        x = cur()
+        wk.wkv7_backward(x["r"], x["w_log"], x["k"], x["v"], x["a"], x["b"], None, dyd, None,
                          *bgrads, bds0, bws, B, T, H, D, None, stream)
 
     for _ in range(3):
@@ -421,7 +436,7 @@ def run_ours(args):
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         e2e_ms = float(t.item())
     e2e_value = world * tokens / (e2e_ms * 1e-3)
-    del dev, host
+    del dev, dev2, copies, host
 
     # ---------------- decode step (B256 H40, state carried through 128 steps)
     cfg = W.WORKLOADS[DECODE_WORKLOAD]

@@ -154,6 +154,44 @@ int wkv7_forward_fused(const void* r, const void* w_log, const void* k, const vo
                        const int32_t* seq_offsets, int io_dtype, int w_dtype, void* stream);
 
 /*
+ * wkv7_state_map — the affine map that a token range applies to the state, for
+ * splitting long sequences into ranges (across devices or launches).  Each step
+ * S <- S (diag(w_t) + a_t b_t^T) + v_t k_t^T of the generalized delta rule ("RWKV-7
+ * Goose: Expressive Dynamic State Evolution", section "Generalized Delta rule")
+ * is affine in S, so over a range
+ *
+ *     S_end = S_start M + Q      for every start state S_start,
+ *
+ * with M = prod_t (diag(w_t) + a_t b_t^T) (key x key, the tokens in order) and Q
+ * the end state from a zero start.  A range's start state then follows from the
+ * maps of the ranges before it (wkv7_state_apply), and each range runs
+ * wkv7_forward from it; this is what lets the recurrence serve the very long
+ * contexts of the inference-cost table of "RWKV-7 Goose architecture analysis"
+ * (youngju.dev) on several devices, each holding one range.
+ *   r, w_log, k, v, a, b, B, T, H, D, seq_offsets, dtype codes : as in
+ *       wkv7_forward (dense or packed; one map per sequence and head; r is not
+ *       read for the result, but must be a valid tensor of its shape).
+ *   M, Q : [B][H][D][D] fp32 outputs (M[j'][j] key x key; Q[i][j] value x key as
+ *       the state); either may be NULL (not computed), not both.  They must not
+ *       overlap any input or each other.  T == 0 gives M = I, Q = 0.
+ * Cost: two passes of the prefill kernel over the range (Q from a zero state;
+ * M from the identity state with v taken as zero), neither writing y.
+ */
+int wkv7_state_map(const void* r, const void* w_log, const void* k, const void* v,
+                   const void* a, const void* b, float* M, float* Q,
+                   int B, int T, int H, int D, const int32_t* seq_offsets,
+                   int io_dtype, int w_dtype, void* stream);
+
+/*
+ * wkv7_state_apply — S_out = S_in M + Q for n_units (sequence, head) states of
+ * D x D fp32 (layouts as wkv7_state_map's outputs; S_in == NULL means a zero
+ * state, so S_out = Q).  S_out == S_in (in place) is allowed; any other overlap
+ * of S_out with an input is not.  Computed in fp32.
+ */
+int wkv7_state_apply(const float* S_in, const float* M, const float* Q, float* S_out,
+                     int n_units, int D, void* stream);
+
+/*
  * wkv7_decode_step — one token per sequence (RNN mode).
  *   r, w_log, k, v, a, b, y : [B][H][D]
  *   s_in, s_out            : [B][H][D][D] fp32; s_in == s_out (in place) is

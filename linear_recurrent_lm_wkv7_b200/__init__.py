@@ -29,6 +29,8 @@ from ._binding import (  # noqa: F401
     wkv7_forward_fused,
     wkv7_forward_gated,
     wkv7_get_device_status,
+    wkv7_state_apply,
+    wkv7_state_map,
     wkv7_status_string,
     wkv7_version,
 )

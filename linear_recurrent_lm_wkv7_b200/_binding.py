@@ -36,6 +36,8 @@ EXPORTS = (
     "wkv7_backward",
     "wkv7_backward_workspace_bytes",
     "wkv7_backward_noalloc",
+    "wkv7_state_map",
+    "wkv7_state_apply",
     "wkv7_status_string",
     "wkv7_get_device_status",
     "wkv7_debug_expire_wait",
@@ -57,7 +59,7 @@ def _lib():
     if _LIB is None:
         if not os.path.exists(LIB_PATH):
             raise ImportError(
-                f"{LIB_PATH} is missing: build it with `python -m linear_recurrent_lm_wkv7_b200.build`")
+                f"{LIB_PATH} is missing: build it with `python linear_recurrent_lm_wkv7_b200/build.py`")
         lib = ctypes.CDLL(LIB_PATH)
         vp, i = ctypes.c_void_p, ctypes.c_int
         lib.wkv7_forward.argtypes = [vp] * 9 + [i] * 4 + [vp, i, i, vp]
@@ -74,6 +76,10 @@ def _lib():
         lib.wkv7_backward_workspace_bytes.restype = ctypes.c_size_t
         lib.wkv7_backward_noalloc.argtypes = [vp] * 16 + [i] * 4 + [vp, i, i, vp]
         lib.wkv7_backward_noalloc.restype = i
+        lib.wkv7_state_map.argtypes = [vp] * 8 + [i] * 4 + [vp, i, i, vp]
+        lib.wkv7_state_map.restype = i
+        lib.wkv7_state_apply.argtypes = [vp] * 4 + [i, i, vp]
+        lib.wkv7_state_apply.restype = i
         lib.wkv7_decode_step.argtypes = [vp] * 9 + [i] * 3 + [i, i, vp]
         lib.wkv7_decode_step.restype = i
         lib.wkv7_status_string.argtypes = [i]
@@ -184,6 +190,23 @@ def wkv7_backward_noalloc(r, w_log, k, v, a, b, s0, dy, dsT, dr, dw_log, dk, dv,
         raise Wkv7Error(st, "wkv7_backward_noalloc")
 
 
+def wkv7_state_map(r, w_log, k, v, a, b, M, Q, B, T, H, D, seq_offsets=None, stream=None):
+    """Enqueue the affine map of a token range (see include/wkv7.h): S_end = S_start M + Q.
+    M or Q may be None (not computed)."""
+    st = _lib().wkv7_state_map(_ptr(r), _ptr(w_log), _ptr(k), _ptr(v), _ptr(a), _ptr(b), _ptr(M), _ptr(Q), int(B),
+                               int(T), int(H), int(D), _ptr(seq_offsets), _dtype_code(r), _dtype_code(w_log),
+                               _stream(stream))
+    if st != 0:
+        raise Wkv7Error(st, "wkv7_state_map")
+
+
+def wkv7_state_apply(S_in, M, Q, S_out, n_units, D, stream=None):
+    """Enqueue S_out = S_in M + Q over n_units states (S_in None: a zero state)."""
+    st = _lib().wkv7_state_apply(_ptr(S_in), _ptr(M), _ptr(Q), _ptr(S_out), int(n_units), int(D), _stream(stream))
+    if st != 0:
+        raise Wkv7Error(st, "wkv7_state_apply")
+
+
 def wkv7_decode_step(r, w_log, k, v, a, b, s_in, y, s_out, B, H, D, stream=None):
     """Enqueue one decoding step (see include/wkv7.h)."""
     st = _lib().wkv7_decode_step(_ptr(r), _ptr(w_log), _ptr(k), _ptr(v), _ptr(a), _ptr(b), _ptr(s_in), _ptr(y),
@@ -234,6 +257,14 @@ def raw_call_backward(*args):
 
 def raw_call_backward_noalloc(*args):
     return int(_lib().wkv7_backward_noalloc(*args))
+
+
+def raw_call_state_map(*args):
+    return int(_lib().wkv7_state_map(*args))
+
+
+def raw_call_state_apply(*args):
+    return int(_lib().wkv7_state_apply(*args))
 
 
 def raw_call_decode(*args):

@@ -1,6 +1,7 @@
 """Build libwkv7.so in-tree with nvcc for sm_100a.
 
-Usage: ``python -m linear_recurrent_lm_wkv7_b200.build [--force] [--verbose]``.
+Usage: ``python linear_recurrent_lm_wkv7_b200/build.py [--force] [--verbose]`` (run as a
+script: importing the package loads the library, which this builds).
 ``--verbose`` adds ``-Xptxas -v`` (registers, spills, shared memory per kernel).
 """
 from __future__ import annotations
@@ -17,7 +18,7 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libwkv7.so")
 SOURCES = ["wkv7_api.cu", "wkv7_decode.cu", "wkv7_prefill.cu", "wkv7_prefill_pipe.cu", "wkv7_gate.cu",
-           "wkv7_backward.cu", "wkv7_noalloc.cu"]
+           "wkv7_backward.cu", "wkv7_noalloc.cu", "wkv7_state.cu"]
 HEADERS = ["sm100_ptx.cuh", "wkv7_internal.cuh", "prefill_common.cuh", "tma_host.cuh"]
 
 

@@ -246,6 +246,66 @@ int wkv7_decode_step_fused(const void* r, const void* w_log, const void* k, cons
                        stream, true);
 }
 
+int wkv7_state_map(const void* r, const void* w_log, const void* k, const void* v, const void* a, const void* b,
+                   float* M, float* Q, int B, int T, int H, int D, const int32_t* seq_offsets, int io_dtype,
+                   int w_dtype, void* stream) {
+    // ---- host-side validation; nothing is launched on failure
+    if (B <= 0 || T < 0 || H <= 0 || D <= 0) return WKV7_ERR_INVALID_ARG;
+    if (!dtype_ok(io_dtype) || !dtype_ok(w_dtype)) return WKV7_ERR_INVALID_ARG;
+    if (D != wkv7::kHead) return WKV7_ERR_UNSUPPORTED;
+    if (!M && !Q) return WKV7_ERR_INVALID_ARG;
+    if (T > 0 && (!r || !w_log || !k || !v || !a || !b)) return WKV7_ERR_INVALID_ARG;
+    const void* ptrs[] = {r, w_log, k, v, a, b, M, Q, seq_offsets};
+    for (const void* p : ptrs)
+        if (p && !aligned16(p)) return WKV7_ERR_MISALIGNED;
+    const long tokens = seq_offsets ? static_cast<long>(T) : static_cast<long>(B) * T;
+    const size_t n_act = static_cast<size_t>(tokens) * H * D;
+    const size_t n_state = static_cast<size_t>(B) * H * D * D;
+    const size_t io_b = dtype_bytes(io_dtype), w_b = dtype_bytes(w_dtype);
+    if (overlaps(M, n_state * 4, Q, n_state * 4)) return WKV7_ERR_INVALID_ARG;
+    const void* ins[] = {r, k, v, a, b, w_log};
+    for (int i = 0; i < 6; ++i) {
+        const size_t nb = n_act * (i == 5 ? w_b : io_b);
+        if (overlaps(M, n_state * 4, ins[i], nb) || overlaps(Q, n_state * 4, ins[i], nb)) return WKV7_ERR_INVALID_ARG;
+    }
+
+    int dev_ok = cached_device_check();
+    if (dev_ok != WKV7_OK) return dev_ok;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const long units = static_cast<long>(B) * H;
+    if (T == 0) return wkv7::launch_state_identity(M, Q, units, st) == cudaSuccess ? WKV7_OK : WKV7_ERR_CUDA;
+    int* status = nullptr;
+    if (status_ptr(&status) != WKV7_OK) return WKV7_ERR_CUDA;
+    // Q: the end state from a zero start; M: the end state from the identity with v = 0
+    // (the product of the transitions); neither writes y
+    wkv7::PrefillArgs p{r, w_log, k, v, a, b, nullptr, nullptr, Q, B, T, H, seq_offsets, status};
+    if (Q && wkv7::launch_prefill(p, io_dtype, w_dtype, st) != cudaSuccess) return WKV7_ERR_CUDA;
+    p.sT = M;
+    p.zero_v = true;
+    p.s0_identity = true;
+    if (M && wkv7::launch_prefill(p, io_dtype, w_dtype, st) != cudaSuccess) return WKV7_ERR_CUDA;
+    return WKV7_OK;
+}
+
+int wkv7_state_apply(const float* S_in, const float* M, const float* Q, float* S_out, int n_units, int D,
+                     void* stream) {
+    if (n_units <= 0 || D <= 0) return WKV7_ERR_INVALID_ARG;
+    if (D != wkv7::kHead) return WKV7_ERR_UNSUPPORTED;
+    if (!M || !Q || !S_out) return WKV7_ERR_INVALID_ARG;
+    const void* ptrs[] = {S_in, M, Q, S_out};
+    for (const void* p : ptrs)
+        if (p && !aligned16(p)) return WKV7_ERR_MISALIGNED;
+    const size_t nb = static_cast<size_t>(n_units) * D * D * 4;
+    // S_out may be S_in (in place); any other overlap of the output is rejected
+    if (overlaps(S_out, nb, M, nb) || overlaps(S_out, nb, Q, nb)) return WKV7_ERR_INVALID_ARG;
+    if (S_in && S_in != S_out && overlaps(S_out, nb, S_in, nb)) return WKV7_ERR_INVALID_ARG;
+    int dev_ok = cached_device_check();
+    if (dev_ok != WKV7_OK) return dev_ok;
+    return wkv7::launch_state_apply(S_in, M, Q, S_out, n_units, static_cast<cudaStream_t>(stream)) == cudaSuccess
+               ? WKV7_OK
+               : WKV7_ERR_CUDA;
+}
+
 size_t wkv7_backward_workspace_bytes(int B, int T, int H, int D, int packed) {
     if (B <= 0 || T < 0 || H <= 0 || D != wkv7::kHead) return 0;
     return wkv7::backward_workspace_floats(B, T, H, packed ? 1 : 0) * sizeof(float);

@@ -38,6 +38,10 @@ struct PrefillArgs {
     // have H_kv heads; the kernels form kk, a, b and the scaled key themselves
     bool prologue = false;
     int H_kv = 0;
+    // state map (wkv7_state_map): v is treated as zero (v may be any valid pointer),
+    // the initial state is the identity (s0 ignored); y == nullptr writes no y rows
+    bool zero_v = false;
+    bool s0_identity = false;
 };
 
 struct DecodeArgs {
@@ -94,6 +98,11 @@ cudaError_t launch_gate(void* z, const void* r, const void* k, const void* v, co
                         long ntok, int H, int io_dtype, cudaStream_t stream, const void* w_log = nullptr,
                         const void* a_lr = nullptr, int H_kv = 0, int w_dtype = WKV7_F32);
 cudaError_t launch_expire_wait(int spins, int* status, cudaStream_t stream);
+// S_out = S_in M + Q for n (sequence, head) units (S_in null: zero), fp32 (wkv7_state.cu)
+cudaError_t launch_state_apply(const float* S_in, const float* M, const float* Q, float* S_out, long n,
+                               cudaStream_t stream);
+// M <- identity, Q <- 0 for n units (the map of an empty token range); either may be null
+cudaError_t launch_state_identity(float* M, float* Q, long n, cudaStream_t stream);
 // backward of the recurrence (wkv7_backward.cu)
 long backward_ckpt_chunks(int B, int T, int packed);
 size_t backward_workspace_floats(int B, int T, int H, int packed);

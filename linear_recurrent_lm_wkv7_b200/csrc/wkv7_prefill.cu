@@ -133,7 +133,7 @@ __global__ void __launch_bounds__(NT, 1)
     wkv7_prefill_kernel(const IO* __restrict__ r, const WT* __restrict__ wl, const IO* __restrict__ k,
                         const IO* __restrict__ v, const IO* __restrict__ a, const IO* __restrict__ b,
                         const float* s0, IO* __restrict__ y, float* sT, int T, int H,
-                        const int32_t* __restrict__ seq_offsets, int* status, int H_kv) {
+                        const int32_t* __restrict__ seq_offsets, int* status, int H_kv, int map_flags) {
     static_assert(TF32, "this kernel serves fp32 inputs (tf32 operands) only");
     using O = OpType<TF32>;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -189,7 +189,8 @@ __global__ void __launch_bounds__(NT, 1)
     const int jj = tid - 64;
     if (tid >= 64) {
 #pragma unroll
-        for (int i = 0; i < 64; ++i) S[i] = s0 ? s0[sbase + i * kHead + jj] : 0.f;
+        for (int i = 0; i < 64; ++i)
+            S[i] = (map_flags & 2) ? (i == jj ? 1.f : 0.f) : (s0 ? s0[sbase + i * kHead + jj] : 0.f);
         store_state_operand(sm.S, jj, S);
     }
 
@@ -278,7 +279,7 @@ __global__ void __launch_bounds__(NT, 1)
                     gprev = G;
                 }
             }
-            load_v_tile(v, row0, tstride_kv, hoff_kv, nv, sm.V, tid);
+            load_v_tile(v, row0, tstride_kv, hoff_kv, (map_flags & 1) ? 0 : nv, sm.V, tid);  // v = 0: no rows
         }
         fence_proxy_async_smem();
         tc_fence_before();
@@ -448,7 +449,7 @@ __global__ void __launch_bounds__(NT, 1)
 #pragma unroll
                 for (int q = 0; q < 2; ++q) {
                     tmem_load32(tmem + lane_base + COL_O + 32 * q, o);
-                    if (t < nv) {
+                    if (t < nv && y != nullptr) {
                         IO* dst = y + (row0 + t) * tstride + hoff + 32 * q;
 #pragma unroll
                         for (int i = 0; i < 32; i += 4)
@@ -500,7 +501,8 @@ cudaError_t launch_typed(const PrefillArgs& p, cudaStream_t stream) {
     kern<<<static_cast<unsigned>(units), NT, smem, stream>>>(
         static_cast<const IO*>(p.r), static_cast<const WT*>(p.w_log), static_cast<const IO*>(p.k),
         static_cast<const IO*>(p.v), static_cast<const IO*>(p.a), static_cast<const IO*>(p.b), p.s0,
-        static_cast<IO*>(p.y), p.sT, p.T, p.H, p.seq_offsets, p.status, PRO ? p.H_kv : p.H);
+        static_cast<IO*>(p.y), p.sT, p.T, p.H, p.seq_offsets, p.status, PRO ? p.H_kv : p.H,
+        (p.zero_v ? 1 : 0) | (p.s0_identity ? 2 : 0));
     return cudaGetLastError();
 }
 

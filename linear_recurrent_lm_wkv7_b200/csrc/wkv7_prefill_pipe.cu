@@ -154,9 +154,10 @@ __device__ __forceinline__ float2 ld_wlog2(const __nv_bfloat16* p, int i) {
     const uint32_t u = *reinterpret_cast<const uint32_t*>(p + i);
     return make_float2(bf16lo_to_f32(u), bf16hi_to_f32(u));
 }
-// w = exp(-exp(w_log)) for two key channels
+// w = exp(-exp(w_log)) = 2^(-log2(e) 2^(log2(e) w_log)) for two key channels
 __device__ __forceinline__ float2 decay2(float2 lv) {
-    return make_float2(__expf(-__expf(lv.x)), __expf(-__expf(lv.y)));
+    constexpr float kLog2e = 1.4426950408889634f;
+    return make_float2(ex2_ftz(-kLog2e * ex2_ftz(kLog2e * lv.x)), ex2_ftz(-kLog2e * ex2_ftz(kLog2e * lv.y)));
 }
 __device__ __forceinline__ uint32_t pack2(float2 v) { return pack_bf16x2(v.x, v.y); }
 
@@ -205,6 +206,11 @@ __device__ __forceinline__ float sum8_scatter(const float (&pd)[8], int jp) {
 // h / (H / H_kv), the `a` tile carries a_lr, and per token
 //   kk = k / max(||k||, 1e-12),  a = -kk,  b = kk a_lr,  k <- k (1 - w + a_lr);
 // `b` is not read.
+// map_flags (wkv7_state_map; 0 otherwise): kMapZeroV treats v as zero (no V tile is
+// loaded), kMapIdentity starts from the identity state (s0 ignored).  y == nullptr
+// writes no y rows.
+constexpr int kMapZeroV = 1, kMapIdentity = 2;
+
 template <typename WT, bool GATED, bool PRO>
 __global__ void __launch_bounds__(NTHR, 1)
     wkv7_prefill_pipe_kernel(const __nv_bfloat16* __restrict__ r, const WT* __restrict__ wl,
@@ -213,7 +219,7 @@ __global__ void __launch_bounds__(NTHR, 1)
                              const float* s0, __nv_bfloat16* __restrict__ y, float* sT, int T, int H,
                              const int32_t* __restrict__ seq_offsets, int* status,
                              const float* __restrict__ rk, const __nv_bfloat16* __restrict__ gte, int H_kv,
-                             const __grid_constant__ TmaMaps maps) {
+                             int map_flags, const __grid_constant__ TmaMaps maps) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     // 1024-byte aligned base, derived from the shared array so that every tile pointer
     // stays in the shared address space (32-bit addressing)
@@ -330,14 +336,22 @@ __global__ void __launch_bounds__(NTHR, 1)
             mbar_arrive_expect_tx(&bars.vld[g], 8192u);
             tma_load_3d(Vt, &maps.v, &bars.vld[g], 0, hk, static_cast<int>(tb + static_cast<long>(cc) * L));
         };
+        const bool zero_v = (map_flags & kMapZeroV) != 0;
+        if (zero_v) {
+            // v = 0: the V tile is cleared once and never loaded
+            for (int i = tg; i < 512; i += static_cast<int>(GROUP))
+                reinterpret_cast<uint4*>(Vt)[i] = make_uint4(0u, 0u, 0u, 0u);
+            fence_proxy_async_smem();
+        }
         if (g < nchunks) {
             if (tg == 0) {
                 issue_raw(g, 0);
                 issue_raw(g, 1);
                 issue_raw(g, 2);
-                issue_v(g);
+                if (!zero_v) issue_v(g);
             }
-            raw_issued = v_issued = 1;
+            raw_issued = 1;
+            v_issued = zero_v ? 0 : 1;
         }
 
         // matrix descriptors of K-step 0; K-step s adds 2 s (K-major) or 128 s (MN-major)
@@ -392,12 +406,12 @@ __global__ void __launch_bounds__(NTHR, 1)
                 if (tg == 0) {
                     if (kk_ >= 1) {
                         w_ok = mbar_wait(&bars.ready[g], static_cast<uint32_t>(kk_ - 1) & 1u, WAIT_NS);
-                        if (w_ok) issue_v(c);
+                        if (w_ok && !zero_v) issue_v(c);
                     }
                     w_ok = w_ok && mbar_wait(&bars.rrk[g], static_cast<uint32_t>(kk_) & 1u, WAIT_NS) &&
                            mbar_wait(&bars.rab[g], static_cast<uint32_t>(kk_) & 1u, WAIT_NS);
                 }
-                if (kk_ >= 1) ++v_issued;
+                if (kk_ >= 1 && !zero_v) ++v_issued;
                 ok = group_sync_and(bar_id, GROUP, w_ok);
                 if (!ok) break;
                 ++raw_done;
@@ -473,7 +487,7 @@ __global__ void __launch_bounds__(NTHR, 1)
                             wv = decay2(ld_wlog2(rawl, t * 64 + j0));
                             G = __fmul2_rn(gp, wv);
                         }
-                        const float2 iv = make_float2(__fdividef(1.f, G.x), __fdividef(1.f, G.y));
+                        const float2 iv = make_float2(rcp_ftz(G.x), rcp_ftz(G.y));
                         const float2 l = __fmul2_rn(iv, GL);
                         const float2 rf = unpack_bf16x2(rr[e]);
                         float2 kf = unpack_bf16x2(kv[e]), af, bf;
@@ -738,10 +752,11 @@ __global__ void __launch_bounds__(NTHR, 1)
             if (c + 2 < nchunks && tg == 0) issue_raw(c + 2, 2);
             // ---- OUT = [Mrb Z; Bh^T Z] V + [Mrk; Kh^T] V   (the serial group adds [R'; Bh^T W] S0^T)
             {
-                const bool vok = (tg == 0) ? mbar_wait(&bars.vld[g], static_cast<uint32_t>(kk_) & 1u, WAIT_NS) : true;
+                const bool vok =
+                    (tg == 0 && !zero_v) ? mbar_wait(&bars.vld[g], static_cast<uint32_t>(kk_) & 1u, WAIT_NS) : true;
                 ok = group_sync_and(bar_id, GROUP, vok);
                 if (!ok) break;
-                ++v_done;
+                if (!zero_v) ++v_done;
             }
             if (tg == 0) {
                 tc_fence_after();
@@ -780,7 +795,8 @@ __global__ void __launch_bounds__(NTHR, 1)
         const int x = ts - 64;  // key channel owned by lanes 64..127
         if (ts >= 64) {
 #pragma unroll
-            for (int i = 0; i < 64; ++i) S[i] = s0 ? s0[sbase + i * kHead + x] : 0.f;
+            for (int i = 0; i < 64; ++i)
+                S[i] = (map_flags & kMapIdentity) ? (i == x ? 1.f : 0.f) : (s0 ? s0[sbase + i * kHead + x] : 0.f);
             st_op_row32<false>(St, 64, x, 0, S);
             st_op_row32<false>(St, 64, x, 32, S + 32);
         }
@@ -828,7 +844,7 @@ __global__ void __launch_bounds__(NTHR, 1)
 #pragma unroll(GATED ? 2 : 1)
                 for (int q = 0; q < 2; ++q) {
                     tmem_load32(tm_out + lane_base + 32 * q, o);
-                    if (t < nv) {
+                    if (t < nv && y != nullptr) {
                         const long off = (row0 + t) * tstride + hoff + 32 * q;
                         if constexpr (GATED) {
                             // z = (y / sqrt(D) + u v) (.) g, with v and g of this token row
@@ -905,7 +921,8 @@ cudaError_t launch_pipe_typed(const PrefillArgs& p, cudaStream_t stream) {
         static_cast<const __nv_bfloat16*>(p.k), static_cast<const __nv_bfloat16*>(p.v),
         static_cast<const __nv_bfloat16*>(p.a), static_cast<const __nv_bfloat16*>(p.b), p.s0,
         static_cast<__nv_bfloat16*>(p.y), p.sT, p.T, p.H, p.seq_offsets, p.status, p.rk,
-        static_cast<const __nv_bfloat16*>(p.g), H_kv, maps);
+        static_cast<const __nv_bfloat16*>(p.g), H_kv, (p.zero_v ? kMapZeroV : 0) | (p.s0_identity ? kMapIdentity : 0),
+        maps);
     return cudaGetLastError();
 }
 

@@ -1,4 +1,4 @@
-"""Splitting a batch of independent sequences across ranks.
+"""Splitting work across ranks: whole sequences, or one sequence's tokens.
 
 Every (sequence, head) unit of the WKV-7 recurrence is independent of every
 other one (the state is per sequence and head), so a batch shards across GPUs
@@ -8,8 +8,15 @@ decision is which sequences go where; for packed variable-length batches the
 assignment balances token counts (longest sequences first, each to the least
 loaded rank).
 
-Nothing here computes the operator; the collective helpers below exist only to
-gather shards for checking and are not on the compute path.
+A long sequence can also be cut along its tokens (``token_ranges``): the
+recurrence is affine in its start state over any token range, S_end =
+S_start M + Q (``wkv7_state_map``), so each range's start state follows from
+the maps of the ranges before it by an exclusive scan (``start_states``), after
+which every range runs ``wkv7_forward`` on its own.  ``forward_sequence_parallel``
+does this across ranks (the maps, B x H x 64 x 64 fp32 each, are all-gathered
+over the process group; nothing else crosses ranks); ``forward_split`` does the
+same on one device.  The arithmetic of every step runs in the CUDA library; the
+functions here only order the calls.
 """
 from __future__ import annotations
 
@@ -54,3 +61,125 @@ def dense_shard(batch: int, world_size: int, rank: int) -> range:
     base, extra = divmod(batch, world_size)
     start = rank * base + min(rank, extra)
     return range(start, start + base + (1 if rank < extra else 0))
+
+
+def token_ranges(T: int, n_parts: int, chunk: int = 64) -> List[tuple]:
+    """Cut T tokens into ``n_parts`` contiguous ranges ``(t0, t1)`` whose inner
+    bounds are multiples of ``chunk`` (so every range but the last starts a
+    fresh chunk) and whose chunk counts differ by at most one; ranges past the
+    end are empty."""
+    if n_parts <= 0:
+        raise ValueError("n_parts must be positive")
+    nck = (T + chunk - 1) // chunk
+    bounds = [min(T, chunk * (nck * j // n_parts)) for j in range(n_parts)] + [T]
+    return [(bounds[j], bounds[j + 1]) for j in range(n_parts)]
+
+
+def start_states(maps, s0, apply):
+    """Start state of every range from the maps of the ranges before it:
+    S_0 = s0 and S_{j+1} = apply(S_j, M_j, Q_j), the end state of range j.
+    ``maps`` lists (M_j, Q_j) in token order; the last one is not needed.
+    ``apply(S, M, Q)`` returns S M + Q (S may be None for a zero state)."""
+    starts = [s0]
+    S = s0
+    for M, Q in list(maps)[:-1]:
+        S = apply(S, M, Q)
+        starts.append(S)
+    return starts
+
+
+def _device_apply(wk, stream):
+    import torch
+
+    def apply(S, M, Q):
+        out = torch.empty_like(Q)
+        n = Q.numel() // (64 * 64)
+        wk.wkv7_state_apply(S, M, Q, out, n, 64, stream)
+        return out
+
+    return apply
+
+
+def _range_map(wk, x, B, T, H, stream, out=None):
+    """(M, Q) of a dense range [B, T, H, 64] by wkv7_state_map, written into
+    ``out`` ([2, B, H, 64, 64] fp32) when given."""
+    import torch
+
+    if out is None:
+        out = torch.empty((2, B, H, 64, 64), dtype=torch.float32, device=x["r"].device)
+    wk.wkv7_state_map(x["r"], x["w_log"], x["k"], x["v"], x["a"], x["b"], out[0], out[1], B, T, H, 64, None,
+                      stream)
+    return out[0], out[1]
+
+
+def gather_maps(mine, group=None):
+    """Every rank's map, in rank order: ``mine`` is this rank's [2, ...] stack of
+    (M, Q); returns the list of all ranks' stacks (one all-gather over the
+    group, on any backend)."""
+    import torch
+    import torch.distributed as dist
+
+    world = dist.get_world_size(group)
+    out = [torch.empty_like(mine) for _ in range(world)]
+    dist.all_gather(out, mine.contiguous(), group=group)
+    return out
+
+
+def forward_split(r, w_log, k, v, a, b, s0=None, n_parts=2, stream=None):
+    """One device, a dense batch [B, T, H, D] cut along its tokens into
+    ``n_parts`` ranges: the map of every range but the last, the scan for the
+    start states, then one wkv7_forward per range.  Returns ``(y, sT)`` as one
+    call over the whole batch would (within the kernels' tolerance)."""
+    import torch
+
+    import linear_recurrent_lm_wkv7_b200 as wk
+
+    B, T, H, D = r.shape
+    ranges = [rg for rg in token_ranges(T, n_parts) if rg[1] > rg[0]]
+    if not ranges:
+        ranges = [(0, 0)]
+    parts = []
+    for t0, t1 in ranges:
+        parts.append({n: x[:, t0:t1].contiguous() for n, x in
+                      dict(r=r, w_log=w_log, k=k, v=v, a=a, b=b).items()})
+    maps = [_range_map(wk, p, B, t1 - t0, H, stream) for p, (t0, t1) in zip(parts[:-1], ranges[:-1])]
+    maps.append(None)
+    starts = start_states(maps, s0, _device_apply(wk, stream))
+    ys = []
+    sT = torch.empty((B, H, D, D), dtype=torch.float32, device=r.device)
+    for p, (t0, t1), S in zip(parts, ranges, starts):
+        y = torch.empty_like(p["r"])
+        wk.wkv7_forward(p["r"], p["w_log"], p["k"], p["v"], p["a"], p["b"], S, y, sT, B, t1 - t0, H, D, None,
+                        stream)
+        ys.append(y)
+    return torch.cat(ys, dim=1), sT
+
+
+def forward_sequence_parallel(r, w_log, k, v, a, b, s0=None, group=None, stream=None):
+    """Sequence parallelism across the ranks of ``group``: rank j holds token
+    range j (in rank order) of the same dense batch, [B, T_j, H, D] on its own
+    device, and ``s0`` (the batch's initial states, or None) is given on every
+    rank.  Every rank but the last computes its range's map; the maps are
+    all-gathered (one collective of 2 x B x H x 64 x 64 fp32 per rank); rank j
+    folds the maps of ranks < j into its start state and runs wkv7_forward from
+    it.  Returns ``(y_j, sT_j)``: this rank's outputs and the state at the end of
+    its range (the last rank's is the batch's final state)."""
+    import torch
+    import torch.distributed as dist
+
+    import linear_recurrent_lm_wkv7_b200 as wk
+
+    world = dist.get_world_size(group)
+    rank = dist.get_rank(group)
+    B, T, H, D = r.shape
+    x = dict(r=r, w_log=w_log, k=k, v=v, a=a, b=b)
+    mine = torch.zeros((2, B, H, D, D), dtype=torch.float32, device=r.device)
+    if rank < world - 1:  # nobody starts after the last range
+        _range_map(wk, x, B, T, H, stream, out=mine)
+    stacks = gather_maps(mine, group)
+    maps = [(m[0], m[1]) for m in stacks[:rank]] + [None]
+    S = start_states(maps, s0, _device_apply(wk, stream))[-1]
+    y = torch.empty_like(r)
+    sT = torch.empty((B, H, D, D), dtype=torch.float32, device=r.device)
+    wk.wkv7_forward(r, w_log, k, v, a, b, S, y, sT, B, T, H, D, None, stream)
+    return y, sT

@@ -105,6 +105,27 @@ def forward(r, w_log, k, v, a, b, s0=None, seq_offsets=None, n_threads=None, wan
     return y, sT
 
 
+def state_map(w_log, k, v, a, b, seq_offsets=None, n_threads=None):
+    """The affine map of each sequence's token range, S_end = S_start M + Q.
+
+    Each step S <- S (diag(w_t) + a_t b_t^T) + v_t k_t^T of the generalized delta
+    rule is affine in S, so the whole range is too: M = prod_t (diag(w_t) + a_t
+    b_t^T) in token order, which is the end state of the recurrence started from
+    the identity with v = 0, and Q is the end state started from zero.  Both are
+    computed by :func:`forward` exactly so.  Returns ``(M, Q)``, [B, H, D, D]."""
+    v = _f64(v)
+    zeros = np.zeros_like(v)
+    if seq_offsets is not None:
+        B = len(seq_offsets) - 1
+        H, D = v.shape[1], v.shape[2]
+    else:
+        B, _, H, D = v.shape
+    eye = np.broadcast_to(np.eye(D), (B, H, D, D)).copy()
+    _, M = forward(zeros, w_log, k, zeros, a, b, eye, seq_offsets=seq_offsets, n_threads=n_threads, want_y=False)
+    _, Q = forward(zeros, w_log, k, v, a, b, None, seq_offsets=seq_offsets, n_threads=n_threads, want_y=False)
+    return M, Q
+
+
 def decode_step(r, w_log, k, v, a, b, s_in, n_threads=None):
     """One token per sequence: inputs [B, H, D], state [B, H, D, D].
     Returns ``(y, s_out)`` as float64 arrays."""

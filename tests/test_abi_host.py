@@ -229,3 +229,30 @@ def test_c_program_compiles_and_links(wk, tmp_path):
            str(tmp_path / "use_wkv7"), wk.LIB_PATH, f"-Wl,-rpath-link,{cuda_lib}", f"-Wl,-rpath,{libdir}"]
     res = subprocess.run(cmd, capture_output=True, text=True)
     assert res.returncode == 0, res.stderr
+
+
+def test_state_map_and_apply_reject_bad_arguments(wk):
+    call = wk._binding.raw_call_state_map
+    base = 0x10000000
+    ins = [base + i * 0x1000000 for i in range(6)]  # r, w_log, k, v, a, b
+    M, Q = base + 0x8000000, base + 0x9000000
+    ok = lambda **o: [o.get("r", ins[0]), ins[1], ins[2], ins[3], ins[4], ins[5], o.get("M", M), o.get("Q", Q),
+                      o.get("B", 2), o.get("T", 100), o.get("H", 3), o.get("D", 64), None, o.get("io", 1), 0, None]
+    assert call(*ok(B=0)) == -1
+    assert call(*ok(T=-1)) == -1
+    assert call(*ok(D=32)) == -2
+    assert call(*ok(io=9)) == -1
+    assert call(*ok(M=None, Q=None)) == -1  # nothing to compute
+    assert call(*ok(r=None)) == -1
+    assert call(*ok(M=M + 8)) == -3
+    assert call(*ok(Q=M + 4096)) == -1  # M and Q overlap
+    assert call(*ok(M=ins[3] + 64)) == -1  # M overlaps v
+    app = wk._binding.raw_call_state_apply
+    S = base + 0xA000000
+    assert app(S, M, Q, S, 0, 64, None) == -1
+    assert app(S, M, Q, S, 4, 16, None) == -2
+    assert app(S, None, Q, S, 4, 64, None) == -1
+    assert app(S, M, Q, None, 4, 64, None) == -1
+    assert app(S + 4, M, Q, S + 4, 4, 64, None) == -3
+    assert app(S, M, Q, M + 64, 4, 64, None) == -1  # output overlaps M
+    assert app(S, M, Q, S + 4096, 4, 64, None) == -1  # output overlaps S_in without being it

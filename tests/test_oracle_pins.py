@@ -467,3 +467,60 @@ def test_backward_linear_attention_closed_form(oracle_mod):
     np.testing.assert_allclose(dr[0, :, 0], exp_dr, rtol=1e-10, atol=1e-10)
     np.testing.assert_allclose(ds0[0, 0], exp_ds0, rtol=1e-10, atol=1e-10)
     assert np.all(dwl == 0.0)  # w = 1 exactly: dw/dl = -exp(l) w = 0
+
+
+# ------------------------------------------------------------------ state maps (sequence split)
+@pytest.mark.parametrize("T", [1, 3, 8])
+def test_state_map_is_the_transition_product(oracle_mod, T):
+    """M = G_1 G_2 ... G_T with G_t = diag(w_t) + a_t b_t^T materialised as
+    matrices, and Q = the brute-force end state from a zero start (catches a
+    reversed product order, a dropped rank-one term, or v leaking into M)."""
+    rng = np.random.default_rng(40 + T)
+    B, H, D = 1, 2, 64
+    r, w_log, k, v, a, b, _ = _rand_inputs(rng, B, T, H, D, s0=False)
+    M, Q = oracle_mod.state_map(w_log, k, v, a, b)
+    w = np.exp(-np.exp(w_log))
+    for h in range(H):
+        P = np.eye(D)
+        for t in range(T):
+            P = P @ (np.diag(w[0, t, h]) + np.outer(a[0, t, h], b[0, t, h]))
+        np.testing.assert_allclose(M[0, h], P, rtol=0, atol=1e-12)
+        _, S = _brute(r[0, :, h], w_log[0, :, h], k[0, :, h], v[0, :, h], a[0, :, h], b[0, :, h], np.zeros((D, D)))
+        np.testing.assert_allclose(Q[0, h], S, rtol=0, atol=1e-12)
+
+
+def test_state_map_gives_every_end_state(oracle_mod):
+    """For any start state S0 the recurrence ends at S0 M + Q (dense batch and
+    a packed batch with pads and an empty sequence)."""
+    rng = np.random.default_rng(50)
+    B, T, H, D = 2, 150, 2, 64
+    r, w_log, k, v, a, b, S0 = _rand_inputs(rng, B, T, H, D)
+    M, Q = oracle_mod.state_map(w_log, k, v, a, b)
+    _, sT = oracle_mod.forward(r, w_log, k, v, a, b, S0)
+    np.testing.assert_allclose(sT, S0 @ M + Q, rtol=0, atol=1e-10)
+    offs = np.array([0, 70, 70, 200], dtype=np.int32)
+    r, w_log, k, v, a, b, _ = _rand_inputs(rng, 1, 200, H, D, s0=False)
+    pk = [x[0] for x in (r, w_log, k, v, a, b)]
+    pk[1][60:70] = -np.inf  # pad tokens: w = 1, k = v = a = b = 0
+    for i in (2, 3, 4, 5):
+        pk[i][60:70] = 0.0
+    S0 = rng.standard_normal((3, H, D, D))
+    M, Q = oracle_mod.state_map(*pk[1:], seq_offsets=offs)
+    _, sT = oracle_mod.forward(*pk, S0, seq_offsets=offs)
+    np.testing.assert_allclose(sT, S0 @ M + Q, rtol=0, atol=1e-10)
+    np.testing.assert_array_equal(M[1], np.broadcast_to(np.eye(D), (H, D, D)))  # empty sequence: identity
+    np.testing.assert_array_equal(Q[1], 0.0)
+
+
+def test_state_maps_compose_over_ranges(oracle_mod):
+    """The map of [0, T) is the composition of the maps of [0, T1) and [T1, T):
+    M = M1 M2 and Q = Q1 M2 + Q2 (the exclusive scan of a sequence split)."""
+    rng = np.random.default_rng(51)
+    B, T, H, D = 1, 130, 2, 64
+    r, w_log, k, v, a, b, _ = _rand_inputs(rng, B, T, H, D, s0=False)
+    T1 = 64
+    M, Q = oracle_mod.state_map(w_log, k, v, a, b)
+    M1, Q1 = oracle_mod.state_map(*(x[:, :T1] for x in (w_log, k, v, a, b)))
+    M2, Q2 = oracle_mod.state_map(*(x[:, T1:] for x in (w_log, k, v, a, b)))
+    np.testing.assert_allclose(M, M1 @ M2, rtol=0, atol=1e-11)
+    np.testing.assert_allclose(Q, Q1 @ M2 + Q2, rtol=0, atol=1e-11)

@@ -94,3 +94,71 @@ def test_two_gloo_ranks_reproduce_full_run(tmp_path, oracle_mod):
             pos += n
             seen.add(i)
     assert seen == set(range(len(offs) - 1))
+
+
+# ------------------------------------------------------------------ one sequence cut across ranks
+def test_token_ranges_cover_in_chunk_steps():
+    for T in (0, 1, 63, 64, 100, 16384, 16385):
+        for n in (1, 2, 3, 4, 8):
+            rg = sharding.token_ranges(T, n)
+            assert len(rg) == n and rg[0][0] == 0 and rg[-1][1] == T
+            assert all(rg[j][1] == rg[j + 1][0] for j in range(n - 1))
+            assert all(t0 % 64 == 0 for t0, _ in rg[1:] if t0 < T)
+            sizes = [(t1 - t0 + 63) // 64 for t0, t1 in rg]
+            assert max(sizes) - min(sizes) <= 1
+
+
+def test_start_states_fold_the_maps_in_order():
+    rng = np.random.default_rng(3)
+    maps = [(rng.standard_normal((4, 4)), rng.standard_normal((4, 4))) for _ in range(4)]
+    s0 = rng.standard_normal((4, 4))
+    apply = lambda S, M, Q: (S @ M if S is not None else 0.0) + Q
+    st = sharding.start_states(maps + [None], s0, apply)
+    assert len(st) == 5 and st[0] is s0
+    S = s0
+    for j, (M, Q) in enumerate(maps):
+        S = S @ M + Q
+        np.testing.assert_allclose(st[j + 1], S)
+    assert sharding.start_states([None], None, apply) == [None]
+
+
+def _seq_worker(rank, world, port, out_dir):
+    """Rank j holds token range j of one batch; its map (the oracle stands in for
+    wkv7_state_map), the all-gather of the maps over gloo, the scan, and the
+    range's forward from its start state."""
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    import oracle
+    import wkv7_inputs as W
+
+    inp = W.make_prefill(2, 300, 2, io="bf16", wdt="f32", s0_std=0.1, seed=33)
+    t = {k: v.double().numpy() for k, v in inp.tensors().items()}
+    t0, t1 = sharding.token_ranges(inp.T, world)[rank]
+    part = {n: x[:, t0:t1] for n, x in t.items()}
+    if rank < world - 1:
+        M, Q = oracle.state_map(*(part[n] for n in ("w_log", "k", "v", "a", "b")))
+    else:
+        M = Q = np.zeros((inp.B, inp.H, 64, 64))
+    stacks = sharding.gather_maps(torch.from_numpy(np.stack([M, Q])), None)
+    maps = [(m[0].numpy(), m[1].numpy()) for m in stacks[:rank]] + [None]
+    apply = lambda S, M_, Q_: (S @ M_ if S is not None else 0.0) + Q_
+    S = sharding.start_states(maps, inp.s0.double().numpy(), apply)[-1]
+    y, sT = oracle.forward(*(part[n] for n in ("r", "w_log", "k", "v", "a", "b")), S)
+    np.save(os.path.join(out_dir, f"seq_y{rank}.npy"), y)
+    np.save(os.path.join(out_dir, f"seq_s{rank}.npy"), sT)
+    dist.barrier()
+    dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world", [2, 3])
+def test_gloo_ranks_split_one_sequence(tmp_path, oracle_mod, world):
+    mp.start_processes(_seq_worker, args=(world, _free_port(), str(tmp_path)), nprocs=world, start_method="spawn")
+    import wkv7_inputs as W
+
+    inp = W.make_prefill(2, 300, 2, io="bf16", wdt="f32", s0_std=0.1, seed=33)
+    t = {k: v.double().numpy() for k, v in inp.tensors().items()}
+    y_full, s_full = oracle_mod.forward(*(t[n] for n in ("r", "w_log", "k", "v", "a", "b")), inp.s0.double().numpy())
+    ys = [np.load(tmp_path / f"seq_y{j}.npy") for j in range(world)]
+    np.testing.assert_allclose(np.concatenate(ys, axis=1), y_full, rtol=0, atol=1e-10)
+    np.testing.assert_allclose(np.load(tmp_path / f"seq_s{world - 1}.npy"), s_full, rtol=0, atol=1e-10)
