@@ -50,8 +50,8 @@ L2_FLUSH_BYTES = 256 << 20
 # from an ncu capture of this workload, valid only for the kernel sources it was
 # taken on (SHA-256 over the files below); any change makes it null until the
 # capture is repeated.
-NCU_TRAFFIC = {"sha256": "8bebd1a9fdcffb412393fa4f71b647588418bb938f88825c8a37cdb86ffca3de",
-               "bytes": 123540992, "workload": "prefill_1p5b"}
+NCU_TRAFFIC = {"sha256": "562574fe34746ba9ddad5b430b02e29e0ec96ab2207b675fb2fea8a2ac46d9c5",
+               "bytes": 130046208, "workload": "prefill_1p5b"}
 KERNEL_SOURCES = ("linear_recurrent_lm_wkv7_b200/csrc/wkv7_prefill_pipe.cu",
                   "linear_recurrent_lm_wkv7_b200/csrc/prefill_common.cuh",
                   "linear_recurrent_lm_wkv7_b200/csrc/sm100_ptx.cuh")
@@ -326,6 +326,33 @@ def run_ours(args):
         linp = W.make_workload("prefill_2p9b_long", mu_z=mu_z, seed=2 + 1000 * rank)
         long_sections.append(prefill_section("prefill_2p9b_long", linp, label, "N(0, 0.1^2)"))
         del linp
+    # ---------------- the same long sequence cut into 3 token ranges that run side by side
+    # (sharding.forward_long: range 0 with the map of range 1, then ranges 1 and 2)
+    from linear_recurrent_lm_wkv7_b200 import sharding
+
+    linp = W.make_workload("prefill_2p9b_long", seed=2 + 1000 * rank)
+    ld_ = {k_: v_.cuda() for k_, v_ in linp.tensors().items()}
+    ls0 = linp.s0.cuda()
+
+    def lsplit():
+        sharding.forward_long(ld_["r"], ld_["w_log"], ld_["k"], ld_["v"], ld_["a"], ld_["b"], ls0, 3, stream)
+
+    for _ in range(max(3, args.warmup)):
+        lsplit()
+    torch.cuda.synchronize()
+    lt = time_launches(lsplit, args.steps, stream)
+    if wk.wkv7_get_device_status() != 0:
+        raise RuntimeError("device status set during the long split run")
+    lms = max_over_ranks(sum(lt) / len(lt))
+    lbytes = prefill_bytes(linp.T * linp.H, 2, 4, linp.H, with_s0=True)
+    lach = lbytes / (lms * 1e-3) / 1e9
+    long_split = {"workload": "prefill_2p9b_long", "variant": "decay z ~ N(1,1); 3 token ranges side by side",
+                  "tokens_per_s": world * linp.T / (lms * 1e-3), "ms_per_step": lms,
+                  "launches_per_step": 6,
+                  "roofline": {"bound": "hbm", "achieved": lach, "peak": hbm_peak, "unit": "GB/s",
+                               "frac": lach / hbm_peak, "algorithmic_bytes_per_launch": lbytes,
+                               "hbm_time_floor_us": lbytes / (hbm_peak * 1e9) * 1e6}}
+    del ld_, linp, ls0
     # ---------------- packed variable-length prefill: 16 sequences, lengths U{512..8192}, pads U{0..63}
     pinp = W.make_workload("packed_1p5b", seed=4 + 1000 * rank)
     packed_section = prefill_section("packed_1p5b", pinp, "16 sequences, pads U{0..63} (w = 1, k = v = a = b = 0)",
@@ -532,6 +559,7 @@ def run_ours(args):
             "gpu_launches": args.steps,
             "clocks": clocks,
             "long": long_sections,
+            "long_split": long_split,
             "packed": packed_section,
             "gated": {"workload": PREFILL_WORKLOAD, "tokens_per_s": world * tokens / (gms * 1e-3),
                       "ms_per_step": gms,

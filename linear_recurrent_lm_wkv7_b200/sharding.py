@@ -183,3 +183,84 @@ def forward_sequence_parallel(r, w_log, k, v, a, b, s0=None, group=None, stream=
     sT = torch.empty((B, H, D, D), dtype=torch.float32, device=r.device)
     wk.wkv7_forward(r, w_log, k, v, a, b, S, y, sT, B, T, H, D, None, stream)
     return y, sT
+
+
+_SIDE_STREAMS = {}
+
+
+def _side_streams(device, n):
+    import torch
+
+    idx = device.index if device.index is not None else torch.cuda.current_device()
+    have = _SIDE_STREAMS.setdefault(idx, [])
+    while len(have) < n:
+        have.append(torch.cuda.Stream(device))
+    return have[:n]
+
+
+def forward_long(r, w_log, k, v, a, b, s0=None, n_parts=3, stream=None):
+    """One long sequence (a dense batch with B = 1) on one device, cut into
+    ``n_parts`` token ranges that run side by side.  A single sequence has only
+    H (sequence, head) units, fewer than the SMs; cutting it multiplies the
+    units that run at once.  Phase 1, concurrently: range 0 from s0 (which
+    gives y of range 0 and the start state of range 1) and the map of every
+    middle range (its Q and its M as two separate launches); then the start
+    states by the scan; phase 2, concurrently: ranges 1 .. n_parts-1 from their
+    start states.  Work on the side streams is ordered after ``stream``
+    (default: the current stream), which then waits for all of it.  Returns
+    ``(y, sT)`` as one wkv7_forward call would (within the kernels' tolerance);
+    with H = 40 heads and 148 SMs, n_parts = 3 keeps each phase within one wave
+    of blocks (3 x 40 in phase 1, 2 x 40 in phase 2)."""
+    import torch
+
+    import linear_recurrent_lm_wkv7_b200 as wk
+
+    B, T, H, D = r.shape
+    if B != 1:
+        raise ValueError("forward_long takes one sequence (B = 1)")
+    ranges = [rg for rg in token_ranges(T, n_parts) if rg[1] > rg[0]]
+    y = torch.empty_like(r)
+    sT = torch.empty((1, H, D, D), dtype=torch.float32, device=r.device)
+    st = stream if stream is not None else torch.cuda.current_stream(r.device)
+    if len(ranges) <= 1:
+        wk.wkv7_forward(r, w_log, k, v, a, b, s0, y, sT, B, T, H, D, None, st)
+        return y, sT
+    P = len(ranges)
+    view = lambda x, rg: x[:, rg[0]:rg[1]]  # contiguous for B = 1
+    part = lambda rg: [view(x, rg) for x in (r, w_log, k, v, a, b)]
+    state = lambda: torch.empty((1, H, D, D), dtype=torch.float32, device=r.device)
+    # every buffer is allocated on the caller's stream before the side streams start
+    starts = [None] + [state() for _ in range(1, P)]
+    maps = [(state(), state()) for _ in range(1, P - 1)]
+    ends = [state() for _ in range(1, P - 1)] + [sT]
+    side = _side_streams(r.device, max(1 + 2 * (P - 2), P - 1))
+    start = torch.cuda.Event()
+    start.record(st)
+    for s_ in side:
+        s_.wait_event(start)
+    # ---- phase 1: range 0 from s0; the maps (Q and M as two launches) of the middle ranges
+    t_of = lambda j: ranges[j][1] - ranges[j][0]
+    wk.wkv7_forward(*part(ranges[0]), s0, view(y, ranges[0]), starts[1], B, t_of(0), H, D, None, side[0])
+    for j in range(1, P - 1):
+        Mj, Qj = maps[j - 1]
+        wk.wkv7_state_map(*part(ranges[j]), None, Qj, B, t_of(j), H, D, None, side[2 * j - 1])
+        wk.wkv7_state_map(*part(ranges[j]), Mj, None, B, t_of(j), H, D, None, side[2 * j])
+    for s_ in side[:1 + 2 * (P - 2)]:
+        e = torch.cuda.Event()
+        e.record(s_)
+        st.wait_event(e)
+    # ---- the scan, on the caller's stream: S_{j+1} = S_j M_j + Q_j
+    for j in range(2, P):
+        Mj, Qj = maps[j - 2]
+        wk.wkv7_state_apply(starts[j - 1], Mj, Qj, starts[j], H, D, st)
+    scan = torch.cuda.Event()
+    scan.record(st)
+    # ---- phase 2: ranges 1 .. P-1 from their start states
+    for j in range(1, P):
+        s_ = side[j - 1]
+        s_.wait_event(scan)
+        wk.wkv7_forward(*part(ranges[j]), starts[j], view(y, ranges[j]), ends[j - 1], B, t_of(j), H, D, None, s_)
+        e = torch.cuda.Event()
+        e.record(s_)
+        st.wait_event(e)
+    return y, sT

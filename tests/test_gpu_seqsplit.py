@@ -131,3 +131,25 @@ def test_sequence_parallel_single_rank_group(wk):
         dist.destroy_process_group()
     y_ref, s_ref = wk.forward(d["r"], d["w_log"], d["k"], d["v"], d["a"], d["b"], s0)
     assert torch.equal(y, y_ref) and torch.equal(sT, s_ref)
+
+
+@pytest.mark.parametrize("n_parts", [2, 3, 5])
+def test_long_prefill_overlapped_ranges(wk, oracle_mod, n_parts):
+    """forward_long: one sequence (B1 T16384 H40, N(0, 0.1^2) initial state) whose
+    ranges run side by side on several streams (range 0 with the maps of the
+    middle ranges, then the other ranges from their scanned start states); y and
+    the final state against the oracle on three sampled heads."""
+    from linear_recurrent_lm_wkv7_b200 import sharding
+
+    inp = W.make_workload("prefill_2p9b_long")
+    t = inp.tensors()
+    d = {n: x.cuda() for n, x in t.items()}
+    y, sT = sharding.forward_long(d["r"], d["w_log"], d["k"], d["v"], d["a"], d["b"], inp.s0.cuda(), n_parts)
+    torch.cuda.synchronize()
+    assert wk.wkv7_get_device_status() == 0
+    heads = [0, 19, 39]
+    hs = lambda x: f64(x[..., heads, :].contiguous())
+    yr, sr = oracle_mod.forward(*(hs(t[n]) for n in ("r", "w_log", "k", "v", "a", "b")),
+                                f64(inp.s0[:, heads].contiguous()))
+    assert relerr(y.float().cpu()[..., heads, :], yr) <= TOL["bf16"]
+    assert relerr(sT.cpu()[:, heads], sr) <= TOL["bf16"]
