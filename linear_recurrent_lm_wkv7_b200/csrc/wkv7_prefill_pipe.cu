@@ -27,10 +27,13 @@
 // serial group; each owns its shared-memory tiles and TMEM columns, except the
 // [R'; Bh^T W] tile that the serial group reads, which is shared.
 // Synchronisation: a prep group hands a chunk to the serial group through
-// `ready[g]` (MMA commit + release arrive); the serial group releases the
-// shared tile (and the group's OUT columns) through `freeg[g]`, one barrier per
-// prep group so that no waiter can be two phases behind (a parity wait would
-// then return on the wrong phase).
+// `ready[g]` (MMA commit + release arrive).  The serial group releases the
+// shared tile through `asfree[g]` as soon as its product has read it, and the
+// group's OUT columns through `freeg[g]` once it has read them; both have one
+// barrier per prep group, whose phases are that group's chunks.  A waiter has
+// always waited for the phase before the one it waits for (during the group's
+// previous chunk), so no parity wait can be two phases behind (it would then
+// return on the wrong phase).
 // Inputs arrive by TMA into tiles of the group that are dead at that point of
 // the previous chunk: w_log of chunk c + 2 into BK once T is built, r and k into
 // NQ once P has consumed Q, a and b into RAM once the conversion has read Rt; V
@@ -66,7 +69,7 @@ constexpr uint32_t OFF_GAMMA = OFF_S + 8192;          // Gamma_L [2 groups][2 sl
 constexpr uint32_t OFF_RED = OFF_GAMMA + 2 * 2 * 64 * 4;  // block products [2 groups][4][64] fp32
 constexpr uint32_t OFF_U = OFF_RED + 2 * 4 * 64 * 4;    // gated read-out: u [2 groups][2 slots][64] fp32
 constexpr uint32_t OFF_BAR = OFF_U + 2 * 2 * 64 * 4;
-constexpr uint32_t SMEM_USED = OFF_BAR + 16 * 8 + 16;
+constexpr uint32_t SMEM_USED = OFF_BAR + 18 * 8 + 16;
 // raw TMA staging inside a group's tiles (dead at the time of the load)
 constexpr uint32_t RAW_R = OFF_NQ, RAW_K = OFF_NQ + 8192, RAW_A = OFF_RAM, RAW_B = OFF_RAM + 8192, RAW_L = OFF_BK;
 constexpr uint32_t SMEM_BYTES = SMEM_USED + 1024;      // alignment slack
@@ -173,6 +176,7 @@ struct Bars {
     uint64_t* ready;  // [2] OUT-pre complete and chunk tiles published (count 2)
     uint64_t* freeg;  // [2] serial group done with a chunk of prep group g (shared tile, OUT columns)
     uint64_t* ser;    // serial MMA completion
+    uint64_t* asfree; // [2] the serial product of a chunk of prep group g has read the shared tile
     uint64_t* rl;     // [2] TMA of a group's raw w_log tile
     uint64_t* rrk;    // [2] TMA of a group's raw r, k tiles
     uint64_t* rab;    // [2] TMA of a group's raw a, b tiles
@@ -232,12 +236,13 @@ __global__ void __launch_bounds__(NTHR, 1)
         bars.mma = p;
         bars.ready = p + 2;
         bars.ser = p + 4;
+        bars.asfree = p + 16;
         bars.rl = p + 6;
         bars.rrk = p + 8;
         bars.rab = p + 10;
         bars.vld = p + 12;
         bars.freeg = p + 14;
-        bars.tmem_slot = reinterpret_cast<uint32_t*>(p + 16);
+        bars.tmem_slot = reinterpret_cast<uint32_t*>(p + 18);
     }
 
     // ---- the unit and its tokens
@@ -275,6 +280,8 @@ __global__ void __launch_bounds__(NTHR, 1)
             mbar_init(&bars.freeg[g], 1);
         }
         mbar_init(bars.ser, 1);
+        mbar_init(&bars.asfree[0], 1);
+        mbar_init(&bars.asfree[1], 1);
         fence_mbar_init();
     }
     if (warp == 0) {
@@ -707,8 +714,7 @@ __global__ void __launch_bounds__(NTHR, 1)
                     mma_ss<false>(tm_gp, dQt + 2 * s, dAZ + 128 * s, ID_KM128, s > 0);
                 mma_commit(&bars.mma[g]);
             }
-            // the shared [R'; Bh^T W] tile and this group's OUT columns are free once
-            // the serial group is done with chunk c-1
+            // the shared [R'; Bh^T W] tile is free once the serial product of chunk c-1 has read it
             mma_pending = true;
             {
                 bool w1 = true;
@@ -716,7 +722,7 @@ __global__ void __launch_bounds__(NTHR, 1)
                     w1 = mbar_wait(&bars.mma[g], mma_phase, WAIT_NS);
                     // chunk c - 1 belongs to the other group; it is that group's ((c - 1) >> 1)-th
                     if (c >= 1)
-                        w1 = w1 && mbar_wait(&bars.freeg[(c - 1) & 1], static_cast<uint32_t>((c - 1) >> 1) & 1u, WAIT_NS);
+                        w1 = w1 && mbar_wait(&bars.asfree[(c - 1) & 1], static_cast<uint32_t>((c - 1) >> 1) & 1u, WAIT_NS);
                 }
                 ok = group_sync_and(bar_id, GROUP, w1);
             }
@@ -752,8 +758,10 @@ __global__ void __launch_bounds__(NTHR, 1)
             if (c + 2 < nchunks && tg == 0) issue_raw(c + 2, 2);
             // ---- OUT = [Mrb Z; Bh^T Z] V + [Mrk; Kh^T] V   (the serial group adds [R'; Bh^T W] S0^T)
             {
-                const bool vok =
-                    (tg == 0 && !zero_v) ? mbar_wait(&bars.vld[g], static_cast<uint32_t>(kk_) & 1u, WAIT_NS) : true;
+                // ... and the serial group must have read this group's OUT columns of its previous chunk
+                bool vok = (tg == 0 && !zero_v) ? mbar_wait(&bars.vld[g], static_cast<uint32_t>(kk_) & 1u, WAIT_NS) : true;
+                if (tg == 0 && kk_ >= 1)
+                    vok = vok && mbar_wait(&bars.freeg[g], static_cast<uint32_t>(kk_ - 1) & 1u, WAIT_NS);
                 ok = group_sync_and(bar_id, GROUP, vok);
                 if (!ok) break;
                 if (!zero_v) ++v_done;
@@ -833,6 +841,7 @@ __global__ void __launch_bounds__(NTHR, 1)
             ser_pending = true;
             ok = group_sync_and(bar_id, GROUP, ts == 0 ? mbar_wait(bars.ser, ser_phase, WAIT_NS) : true);
             if (!ok) break;
+            if (ts == 0) mbar_arrive(&bars.asfree[g]);  // the shared tile is free for the next chunk's conversion
             ser_pending = false;
             ser_phase ^= 1u;
             tc_fence_after();
