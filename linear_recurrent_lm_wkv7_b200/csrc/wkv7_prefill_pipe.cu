@@ -247,7 +247,29 @@ __global__ void __launch_bounds__(NTHR, 1)
 
     // ---- the unit and its tokens
     const int unit = blockIdx.x;
-    const int n = unit / H, h = unit % H;
+    const int h = unit % H;
+    int n = unit / H;
+    // A packed batch of at most NTHR sequences is taken longest first: blocks are
+    // started roughly in index order, so the long sequences (the longest chains)
+    // start early and the short ones fill in behind them.  Block n' runs the
+    // sequence of length rank n' (ties by index); the ranks are a permutation even
+    // for offsets that the bounds check below rejects.
+    if (seq_offsets && static_cast<int>(gridDim.x) / H <= NTHR) {
+        const int nseq = static_cast<int>(gridDim.x) / H;
+        long* lens = reinterpret_cast<long*>(sm + OFF_AS);  // scratch, before the tile is used
+        int* pick = reinterpret_cast<int*>(sm + OFF_AS + 8 * NTHR);
+        if (tid < nseq) lens[tid] = static_cast<long>(seq_offsets[tid + 1]) - seq_offsets[tid];
+        __syncthreads();
+        if (tid < nseq) {
+            const long li = lens[tid];
+            int rank = 0;
+            for (int j = 0; j < nseq; ++j) rank += (lens[j] > li || (lens[j] == li && j < tid)) ? 1 : 0;
+            if (rank == n) *pick = tid;
+        }
+        __syncthreads();
+        n = *pick;
+        __syncthreads();  // every thread has its sequence before the scratch is reused
+    }
     const int hk = PRO ? h / (H / H_kv) : h;  // kv head of k and v
     long tb = 0, len = 0;
     if (seq_offsets) {
