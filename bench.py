@@ -570,7 +570,7 @@ def run_ours(args):
                       "roofline": {"bound": "hbm", "achieved": fach, "peak": hbm_peak, "unit": "GB/s",
                                    "frac": fach / hbm_peak, "algorithmic_bytes_per_launch": fbytes}},
             "backward": {"workload": PREFILL_WORKLOAD, "tokens_per_s": world * tokens / (bms * 1e-3),
-                         "ms_per_step": bms, "form": "recurrent (chunk checkpoints, per-token sweep)",
+                         "ms_per_step": bms, "form": "chunked (WY): chunk maps, boundary scans, per-chunk gradients on tf32 tensor cores",
                          "roofline": {"bound": "hbm", "achieved": bach, "peak": hbm_peak, "unit": "GB/s",
                                       "frac": bach / hbm_peak, "algorithmic_bytes_per_launch": bbytes}},
             "decode": {"workload": DECODE_WORKLOAD, "B": dB, "H": dH, "steps_per_s": 1000.0 / dms,

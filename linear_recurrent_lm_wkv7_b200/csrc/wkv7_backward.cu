@@ -299,15 +299,18 @@ long backward_ckpt_chunks(int B, int T, int packed) {
     return packed ? per + B : static_cast<long>(B) * per;
 }
 
+// The larger of the two forms' needs, so that one size serves both input types.
 size_t backward_workspace_floats(int B, int T, int H, int packed) {
-    return static_cast<size_t>(backward_ckpt_chunks(B, T, packed)) * H * SQ +
-           static_cast<size_t>(B) * H * L * SQ;
+    const size_t recurrent = static_cast<size_t>(backward_ckpt_chunks(B, T, packed)) * H * SQ +
+                             static_cast<size_t>(B) * H * L * SQ;
+    const size_t chunked = backward_chunked_workspace_floats(B, T, H, packed);
+    return recurrent > chunked ? recurrent : chunked;
 }
 
+// bf16 inputs take the chunked form (wkv7_backward_chunk.cu); fp32 inputs keep
+// this recurrent kernel, whose fp32 arithmetic holds their tighter bound.
 cudaError_t launch_backward(const BackwardArgs& p, int io_dtype, int w_dtype, cudaStream_t stream) {
-    if (io_dtype == WKV7_BF16)
-        return w_dtype == WKV7_BF16 ? launch_bwd_typed<__nv_bfloat16, __nv_bfloat16>(p, stream)
-                                    : launch_bwd_typed<__nv_bfloat16, float>(p, stream);
+    if (io_dtype == WKV7_BF16) return launch_backward_chunked(p, w_dtype, stream);
     return w_dtype == WKV7_BF16 ? launch_bwd_typed<float, __nv_bfloat16>(p, stream)
                                 : launch_bwd_typed<float, float>(p, stream);
 }

@@ -1,0 +1,933 @@
+// wkv7_backward_chunk.cu — gradient of the WKV-7 recurrence in chunked (WY)
+// form, for bf16 inputs.
+//
+// Per 64-token chunk, tokens as rows (row t of X is token t of the chunk), with
+// Gamma_t = prod_{s<=t} w_s (per key column), Gamma_{-1} = 1, Gamma_L its last row:
+//   At = a (.) Gamma_{t-1},  Rt = r (.) Gamma_t,  Bt = b / Gamma_t,  Kt = k / Gamma_t
+//   Nab = tril(At Bt^T, -1), Nak = tril(At Kt^T, -1), Mrb = tril(Rt Bt^T), Mrk = tril(Rt Kt^T)
+//   T = (I - Nab)^{-1},  U = T (At S0^T + Nak V)     (row t of U: S_{t-1} a_t)
+//   Y = Rt S0^T + Mrb U + Mrk V,   S_L = S0 diag(Gamma_L) + U^T Bt diag(Gamma_L) + V^T Kt diag(Gamma_L)
+// (the chunk-parallel form of the generalized delta rule of "RWKV-7 Goose:
+// Expressive Dynamic State Evolution", section "Generalized Delta rule"; the
+// pages call the model trainable in parallel but print no backward).
+//
+// Reverse-mode through these products, with dSLg = dS_L diag(Gamma_L):
+//   dX = T^T (Mrb^T dY + Bt dSLg^T)                      dV = Mrk^T dY + Kt dSLg^T + Nak^T dX
+//   dNab = tril(dX U^T, -1), dNak = tril(dX V^T, -1), dMrb = tril(dY U^T), dMrk = tril(dY V^T)
+//   dAt = dX S0 + dNab Bt + dNak Kt                       dRt = dY S0 + dMrb Bt + dMrk Kt
+//   dBt' = U dSLg + dNab^T At + dMrb^T Rt                 dKt' = V dSLg + dNak^T At + dMrk^T Rt
+//   da = dAt (.) Gamma_{t-1},  dr = dRt (.) Gamma_t,  db = dBt' / Gamma_t,  dk = dKt' / Gamma_t
+//   d log w_s = sum_{t>=s} (dr_t r_t - db_t b_t - dk_t k_t) + sum_{t>s} da_t a_t
+//               + colsum(dS_L (.) S_L)                 d w_log = d log w (.) (-exp(w_log))
+// and the chunk's maps between its end and start: S_L = S0 M^T + Qf and
+// dS0 = Q + dS_L M with
+//   M = diag(Gamma_L) (I + Bt^T T At),  Q = dY^T (Rt + Mrb T At),
+//   Qf = V^T (Kt + Nak^T T^T Bt) diag(Gamma_L).
+//
+// Three launches:
+//   1. bwd_map_kernel, one block per (chunk, head): M, Q, Qf of the chunk;
+//   2. bwd_scan_kernel, one block per (sequence, head) and direction: the forward
+//      scan S <- S M^T + Qf writes the state at every chunk boundary, the backward
+//      scan dS <- Q + dS M writes dS_L of every chunk and ds0 (fp32 CUDA cores);
+//   3. bwd_grad_kernel, one block per (chunk, head): every gradient of the chunk.
+// Products are warp-level tf32 tensor-core products (m16n8k8, fp32 accumulate)
+// on fp32 tiles in shared memory: 64 x 64 products chained through elementwise
+// steps and masks, each small enough that a register accumulator beats a round
+// trip through tensor memory.
+#include <cstdint>
+
+#include "prefill_common.cuh"
+#include "wkv7_internal.cuh"
+
+namespace wkv7 {
+namespace {
+
+constexpr int L = 64;
+constexpr int D = kHead;
+constexpr int SQ = D * D;
+constexpr int NTHR = 512;  // 16 warps; warp w owns the 16 x 16 block (16 (w / 4), 16 (w % 4)) of a 64 x 64 result
+constexpr int TILE = 64 * 64;
+
+// 64 x 64 fp32 tile, row-major, with the 8-column groups of row r XOR-permuted by
+// h(r) = (r mod 4) ^ bit 2 of r, which depends on r mod 8 only.  The permutation
+// leaves the offset within a group alone, so a step of 8 columns is one XOR away
+// and a step of 8 rows is additive; every fragment pattern below hits 32
+// distinct banks per 16 lanes.
+__device__ __forceinline__ int hsw(int row) { return (row & 3) ^ ((row >> 2) & 1); }
+__device__ __forceinline__ int sx(int row, int col) { return (row << 6) + (col ^ (hsw(row) << 3)); }
+
+__device__ __forceinline__ void mma_tf32(float* d, const uint32_t (&a)[4], const uint32_t (&b)[2]) {
+    asm("mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+        "{%0, %1, %2, %3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
+}
+
+// Fragment offsets of one operand, per lane, for the k-steps of one product.
+// An m16n8k8 product sums over its 8 k in any order both operands agree on:
+// lane t4 supplies k = t4 from position 2 t4 of the 8-step and k = t4 + 4 from
+// 2 t4 + 1, so a row-contiguous operand reads both with one 64-bit load.
+//   along rows (the 16 or 8 rows r0 + l of the operand run along its M or N; the
+//   k-steps run along its columns from c0): offsets of (r0 + l, c0 + 8 s + 2 t4)
+//   across rows (the k-steps run down its rows from k0; the M or N positions
+//   are columns c0 + l): offsets of (k0 + 8 s + 2 t4 + e, c0 + l)
+// r0, c0, k0 are multiples of 8 (all callers use multiples of 16 or 8).
+struct AlongRows {
+    int base, q0, h;  // row offset, first 8-column group, row's permutation
+    __device__ __forceinline__ AlongRows(int row, int c0, int t4) : base((row << 6) + 2 * t4), q0(c0 >> 3), h(hsw(row)) {}
+    __device__ __forceinline__ int at(int s) const { return base + (((q0 + s) ^ h) << 3); }
+};
+struct AcrossRows {
+    int base0, base1;  // offsets of (k0 + 2 t4 + e, col)
+    __device__ __forceinline__ AcrossRows(int k0, int col, int t4) {
+        const int r0 = k0 + 2 * t4;
+        base0 = (r0 << 6) + (col ^ (hsw(r0) << 3));
+        base1 = ((r0 + 1) << 6) + (col ^ (hsw(r0 + 1) << 3));
+    }
+};
+
+// acc (16 x 16) += sum_{kk < 8 nk} op(A)(ar + m, ac + kk) op(B)(bk + kk, bn + n)   (one warp)
+// with op(X) = X, or X^T when the flag is set.  acc[4 h + 2 q + e] is row
+// gq + 8 q, column 8 h + 2 t4 + e of the block (lane = 4 gq + t4).
+template <bool TA, bool TB>
+__device__ __forceinline__ void gemm16(float (&acc)[8], const float* A, int ar, int ac, const float* B, int bk, int bn,
+                                       int nk, int gq, int t4) {
+    if (!TA && !TB) {
+        const AlongRows a0(ar + gq, ac, t4), a1(ar + gq + 8, ac, t4);
+        const AcrossRows b0(bk, bn + gq, t4), b1(bk, bn + 8 + gq, t4);
+#pragma unroll 4
+        for (int s = 0; s < nk; ++s) {
+            const float2 x0 = *reinterpret_cast<const float2*>(A + a0.at(s));
+            const float2 x1 = *reinterpret_cast<const float2*>(A + a1.at(s));
+            const uint32_t a[4] = {__float_as_uint(x0.x), __float_as_uint(x1.x), __float_as_uint(x0.y),
+                                   __float_as_uint(x1.y)};
+            const uint32_t p[2] = {__float_as_uint(B[b0.base0 + 512 * s]), __float_as_uint(B[b0.base1 + 512 * s])};
+            const uint32_t q[2] = {__float_as_uint(B[b1.base0 + 512 * s]), __float_as_uint(B[b1.base1 + 512 * s])};
+            mma_tf32(acc, a, p);
+            mma_tf32(acc + 4, a, q);
+        }
+    } else if (!TA && TB) {
+        const AlongRows a0(ar + gq, ac, t4), a1(ar + gq + 8, ac, t4);
+        const AlongRows b0(bn + gq, bk, t4), b1(bn + 8 + gq, bk, t4);
+#pragma unroll 4
+        for (int s = 0; s < nk; ++s) {
+            const float2 x0 = *reinterpret_cast<const float2*>(A + a0.at(s));
+            const float2 x1 = *reinterpret_cast<const float2*>(A + a1.at(s));
+            const float2 y0 = *reinterpret_cast<const float2*>(B + b0.at(s));
+            const float2 y1 = *reinterpret_cast<const float2*>(B + b1.at(s));
+            const uint32_t a[4] = {__float_as_uint(x0.x), __float_as_uint(x1.x), __float_as_uint(x0.y),
+                                   __float_as_uint(x1.y)};
+            const uint32_t p[2] = {__float_as_uint(y0.x), __float_as_uint(y0.y)};
+            const uint32_t q[2] = {__float_as_uint(y1.x), __float_as_uint(y1.y)};
+            mma_tf32(acc, a, p);
+            mma_tf32(acc + 4, a, q);
+        }
+    } else if (TA && !TB) {
+        const AcrossRows a0(ac, ar + gq, t4), a1(ac, ar + gq + 8, t4);
+        const AcrossRows b0(bk, bn + gq, t4), b1(bk, bn + 8 + gq, t4);
+#pragma unroll 4
+        for (int s = 0; s < nk; ++s) {
+            const int o = 512 * s;
+            const uint32_t a[4] = {__float_as_uint(A[a0.base0 + o]), __float_as_uint(A[a1.base0 + o]),
+                                   __float_as_uint(A[a0.base1 + o]), __float_as_uint(A[a1.base1 + o])};
+            const uint32_t p[2] = {__float_as_uint(B[b0.base0 + o]), __float_as_uint(B[b0.base1 + o])};
+            const uint32_t q[2] = {__float_as_uint(B[b1.base0 + o]), __float_as_uint(B[b1.base1 + o])};
+            mma_tf32(acc, a, p);
+            mma_tf32(acc + 4, a, q);
+        }
+    } else {
+        const AcrossRows a0(ac, ar + gq, t4), a1(ac, ar + gq + 8, t4);
+        const AlongRows b0(bn + gq, bk, t4), b1(bn + 8 + gq, bk, t4);
+#pragma unroll 4
+        for (int s = 0; s < nk; ++s) {
+            const int o = 512 * s;
+            const float2 y0 = *reinterpret_cast<const float2*>(B + b0.at(s));
+            const float2 y1 = *reinterpret_cast<const float2*>(B + b1.at(s));
+            const uint32_t a[4] = {__float_as_uint(A[a0.base0 + o]), __float_as_uint(A[a1.base0 + o]),
+                                   __float_as_uint(A[a0.base1 + o]), __float_as_uint(A[a1.base1 + o])};
+            const uint32_t p[2] = {__float_as_uint(y0.x), __float_as_uint(y0.y)};
+            const uint32_t q[2] = {__float_as_uint(y1.x), __float_as_uint(y1.y)};
+            mma_tf32(acc, a, p);
+            mma_tf32(acc + 4, a, q);
+        }
+    }
+}
+
+__device__ __forceinline__ void zero8(float (&acc)[8]) {
+#pragma unroll
+    for (int e = 0; e < 8; ++e) acc[e] = 0.f;
+}
+
+// row / column of acc[e] within the warp's 16 x 16 block
+__device__ __forceinline__ int frag_row(int e, int gq) { return gq + 8 * ((e >> 1) & 1); }
+__device__ __forceinline__ int frag_col(int e, int t4) { return 8 * (e >> 2) + 2 * t4 + (e & 1); }
+
+// Stores acc as the block (r0, c0) of C (tf32-rounded).  MASK 1 keeps col < row,
+// MASK 2 keeps col <= row (row, col in C's coordinates).
+template <int MASK>
+__device__ __forceinline__ void st16(float* C, const float (&acc)[8], int r0, int c0, int gq, int t4) {
+#pragma unroll
+    for (int e = 0; e < 8; e += 2) {
+        const int row = r0 + frag_row(e, gq), col = c0 + frag_col(e, t4);
+        float x0 = acc[e], x1 = acc[e + 1];
+        if (MASK == 1) {
+            x0 = col < row ? x0 : 0.f;
+            x1 = col + 1 < row ? x1 : 0.f;
+        } else if (MASK == 2) {
+            x0 = col <= row ? x0 : 0.f;
+            x1 = col + 1 <= row ? x1 : 0.f;
+        }
+        *reinterpret_cast<float2*>(C + sx(row, col)) = make_float2(round_tf32(x0), round_tf32(x1));
+    }
+}
+
+__device__ __forceinline__ float2 bf2_to_f2(uint32_t u) { return make_float2(bf16lo_to_f32(u), bf16hi_to_f32(u)); }
+__device__ __forceinline__ void unpack8(uint4 u, float (&x)[8]) {
+    float2 p = bf2_to_f2(u.x);
+    x[0] = p.x; x[1] = p.y;
+    p = bf2_to_f2(u.y);
+    x[2] = p.x; x[3] = p.y;
+    p = bf2_to_f2(u.z);
+    x[4] = p.x; x[5] = p.y;
+    p = bf2_to_f2(u.w);
+    x[6] = p.x; x[7] = p.y;
+}
+__device__ __forceinline__ void ld_wlog8(const float* p, float (&x)[8]) {
+    const float4 a = *reinterpret_cast<const float4*>(p), b = *reinterpret_cast<const float4*>(p + 4);
+    x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w; x[4] = b.x; x[5] = b.y; x[6] = b.z; x[7] = b.w;
+}
+__device__ __forceinline__ void ld_wlog8(const __nv_bfloat16* p, float (&x)[8]) {
+    unpack8(*reinterpret_cast<const uint4*>(p), x);
+}
+__device__ __forceinline__ void st8(float* tile, int row, int c0, const float (&x)[8], bool rnd) {
+    float y[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) y[e] = rnd ? round_tf32(x[e]) : x[e];
+    *reinterpret_cast<float4*>(tile + sx(row, c0)) = make_float4(y[0], y[1], y[2], y[3]);
+    *reinterpret_cast<float4*>(tile + sx(row, c0 + 4)) = make_float4(y[4], y[5], y[6], y[7]);
+}
+__device__ __forceinline__ void ld8(const float* tile, int row, int c0, float (&x)[8]) {
+    const float4 a = *reinterpret_cast<const float4*>(tile + sx(row, c0));
+    const float4 b = *reinterpret_cast<const float4*>(tile + sx(row, c0 + 4));
+    x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w; x[4] = b.x; x[5] = b.y; x[6] = b.z; x[7] = b.w;
+}
+
+// Where one chunk sits: its first token row, its length, and the workspace
+// region of its (sequence, head) unit.  A unit of nch chunks owns 4 (nch + 1)
+// states of D x D floats: M[0..nch], Q[0..nch] (dS_L after the backward scan),
+// Qf[0..nch], and the state at every chunk boundary S[0..nch]; the units of
+// sequence n start at state 4 H (cbase_n + n), head h at 4 h (nch_n + 1) within.
+struct ChunkLoc {
+    long row0;    // token row of the chunk's first token
+    long region;  // float offset of the unit's region in the workspace
+    int c;        // chunk index within the sequence
+    int nch;      // chunks of the sequence
+    int nv;       // tokens of the chunk (1 .. 64)
+};
+
+__device__ __forceinline__ long unit_region(long cbase, int n, int h, int H, int nch) {
+    return (4L * H * (cbase + n) + 4L * h * (nch + 1)) * SQ;
+}
+
+// Chunk g (counted over all sequences) of head h.  Returns false past the last
+// chunk, or after reporting WKV7_ERR_DEVICE_BOUNDS for offsets that are not
+// monotone, leave [0, T], or need more chunks than the workspace holds.
+__device__ bool locate_chunk(long g, int h, int B, int T, int H, const int32_t* offs, long ckpt_chunks, int* status,
+                             ChunkLoc& o) {
+    if (!offs) {
+        const long cps = (static_cast<long>(T) + L - 1) / L;
+        if (cps == 0 || g >= static_cast<long>(B) * cps) return false;
+        const int n = static_cast<int>(g / cps);
+        o.c = static_cast<int>(g % cps);
+        o.nch = static_cast<int>(cps);
+        o.row0 = static_cast<long>(n) * T + static_cast<long>(o.c) * L;
+        const long rest = static_cast<long>(T) - static_cast<long>(o.c) * L;
+        o.nv = static_cast<int>(rest < L ? rest : L);
+        o.region = unit_region(static_cast<long>(n) * cps, n, h, H, o.nch);
+        return true;
+    }
+    long cbase = 0;
+    for (int n = 0; n < B; ++n) {
+        const long o0 = offs[n], o1 = offs[n + 1];
+        if (o0 < 0 || o1 < o0 || o1 > T) {
+            report_status(status, WKV7_ERR_DEVICE_BOUNDS);
+            return false;
+        }
+        const long nc = (o1 - o0 + L - 1) / L;
+        if (g < cbase + nc) {
+            if (cbase + nc > ckpt_chunks) {
+                report_status(status, WKV7_ERR_DEVICE_BOUNDS);
+                return false;
+            }
+            o.c = static_cast<int>(g - cbase);
+            o.nch = static_cast<int>(nc);
+            o.row0 = o0 + static_cast<long>(o.c) * L;
+            const long rest = o1 - o.row0;
+            o.nv = static_cast<int>(rest < L ? rest : L);
+            o.region = unit_region(cbase, n, h, H, o.nch);
+            return true;
+        }
+        cbase += nc;
+    }
+    return false;
+}
+
+// Thread 0 locates the block's chunk; the others read it from shared memory.
+__device__ bool locate_block_chunk(int B, int T, int H, const int32_t* offs, long ckpt_chunks, int* status,
+                                   ChunkLoc& o, ChunkLoc* sh, int* sh_ok) {
+    if (threadIdx.x == 0) {
+        ChunkLoc x{};
+        const bool ok = locate_chunk(blockIdx.x, blockIdx.y, B, T, H, offs, ckpt_chunks, status, x);
+        *sh = x;
+        *sh_ok = ok ? 1 : 0;
+    }
+    __syncthreads();
+    o = *sh;
+    return *sh_ok != 0;
+}
+
+// Stages the chunk's inputs of one head as fp32 tiles: GAM = Gamma (running
+// products of w = exp(-exp(w_log)) down the tokens), AT, RT, BT, KT (the scaled
+// operands, tf32-rounded), VV and DY (bf16 values, exact in tf32); GL = Gamma_L.
+// Rows t >= nv are identity steps (w = 1, every other input 0).  seg: 8 x 64
+// floats of scratch.  Ends with a block barrier.
+template <typename WT>
+__device__ void stage_chunk(float* GAM, float* AT, float* RT, float* BT, float* KT, float* VV, float* DY, float* GL,
+                            float* seg, const __nv_bfloat16* r, const WT* wl, const __nv_bfloat16* k,
+                            const __nv_bfloat16* v, const __nv_bfloat16* a, const __nv_bfloat16* b,
+                            const __nv_bfloat16* dy, long row0, int nv, long tstride, long hoff) {
+    const int tid = threadIdx.x;
+    const int t = tid >> 3, c0 = 8 * (tid & 7);
+    float rr[8], kk[8], aa[8], bb[8], x[8];
+    if (t < nv) {
+        const long off = (row0 + t) * tstride + hoff + c0;
+        unpack8(__ldg(reinterpret_cast<const uint4*>(r + off)), rr);
+        unpack8(__ldg(reinterpret_cast<const uint4*>(k + off)), kk);
+        unpack8(__ldg(reinterpret_cast<const uint4*>(a + off)), aa);
+        unpack8(__ldg(reinterpret_cast<const uint4*>(b + off)), bb);
+        unpack8(__ldg(reinterpret_cast<const uint4*>(v + off)), x);
+        st8(VV, t, c0, x, false);
+        unpack8(__ldg(reinterpret_cast<const uint4*>(dy + off)), x);
+        st8(DY, t, c0, x, false);
+        ld_wlog8(wl + off, x);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) x[e] = expf(-expf(x[e]));
+    } else {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            rr[e] = kk[e] = aa[e] = bb[e] = 0.f;
+            x[e] = 0.f;
+        }
+        st8(VV, t, c0, x, false);
+        st8(DY, t, c0, x, false);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) x[e] = 1.f;
+    }
+    st8(GAM, t, c0, x, false);
+    __syncthreads();
+    {
+        // running products: thread (column j, segment s of 8 tokens)
+        const int j = tid & 63, s = tid >> 6;
+        float p[8], run = 1.f;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            run *= GAM[sx(8 * s + i, j)];
+            p[i] = run;
+        }
+        seg[s * 64 + j] = run;
+        __syncthreads();
+        float pre = 1.f;
+        for (int q = 0; q < s; ++q) pre *= seg[q * 64 + j];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) GAM[sx(8 * s + i, j)] = pre * p[i];
+        if (s == 7) GL[j] = pre * p[7];
+    }
+    __syncthreads();
+    {
+        float g[8], gp[8];
+        ld8(GAM, t, c0, g);
+        if (t > 0) {
+            ld8(GAM, t - 1, c0, gp);
+        } else {
+#pragma unroll
+            for (int e = 0; e < 8; ++e) gp[e] = 1.f;
+        }
+        float o1[8], o2[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            o1[e] = aa[e] * gp[e];
+            o2[e] = rr[e] * g[e];
+        }
+        st8(AT, t, c0, o1, true);
+        st8(RT, t, c0, o2, true);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            const float inv = __frcp_rn(g[e]);
+            o1[e] = bb[e] * inv;
+            o2[e] = kk[e] * inv;
+        }
+        st8(BT, t, c0, o1, true);
+        st8(KT, t, c0, o2, true);
+    }
+    __syncthreads();
+}
+
+// Tm = (I - N)^{-1} for strictly lower-triangular N (both 64 x 64 tiles):
+//  (1) the 16 x 16 diagonal blocks D_b = (I - N_bb)^{-1}: thread 16 b + c computes
+//      column c by forward substitution;
+//  (2) T_{b+1,b} = D_{b+1} (N_{b+1,b} D_b) for b = 0, 2;
+//  (3) T_hl = T_hi (N_hl T_lo) for the 32 x 32 halves.
+// Intermediate products live in the upper-right 32 x 32 quadrant of Tm (zero in
+// T), which is cleared at the end.  Every thread of the block calls this; it
+// starts and ends with the caller's data in place (barriers inside).
+__device__ void invert_unit_lower(const float* N, float* Tm) {
+    const int tid = threadIdx.x, w = tid >> 5, lane = tid & 31, gq = lane >> 2, t4 = lane & 3;
+    if (tid < 64) {
+        const int r0 = 16 * (tid >> 4), c = tid & 15;
+        float x[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            float p = (i == c) ? 1.f : 0.f;
+#pragma unroll
+            for (int j = 0; j < i; ++j) p = fmaf(N[sx(r0 + i, r0 + j)], x[j], p);
+            x[i] = p;
+        }
+#pragma unroll
+        for (int i = 0; i < 16; ++i) Tm[sx(r0 + i, r0 + c)] = round_tf32(x[i]);
+    } else {
+        // blocks (0, 1) and (2, 3) are zero in T and not used as scratch
+        for (int e = tid - 64; e < 512; e += NTHR - 64) {
+            const int row = e >> 4, col = e & 15;  // 32 rows x 16 columns
+            if (row < 16) Tm[sx(row, 16 + col)] = 0.f;   // rows 0 .. 15, columns 16 .. 31
+            else Tm[sx(16 + row, 48 + col)] = 0.f;       // rows 32 .. 47, columns 48 .. 63
+        }
+    }
+    __syncthreads();
+    if (w < 2) {
+        // Y_b = N_{b+1,b} D_b -> quadrant block (w, 2 + w)
+        float acc[8];
+        zero8(acc);
+        const int b0 = 32 * w;
+        gemm16<false, false>(acc, N, b0 + 16, b0, Tm, b0, b0, 2, gq, t4);
+        st16<0>(Tm, acc, 16 * w, 32 + 16 * w, gq, t4);
+    }
+    __syncthreads();
+    if (w < 2) {
+        // T_{b+1,b} = D_{b+1} Y_b
+        float acc[8];
+        zero8(acc);
+        const int b0 = 32 * w;
+        gemm16<false, false>(acc, Tm, b0 + 16, b0 + 16, Tm, 16 * w, 32 + 16 * w, 2, gq, t4);
+        st16<0>(Tm, acc, b0 + 16, b0, gq, t4);
+    }
+    __syncthreads();
+    if (w < 4) {
+        // X = N_hl T_lo -> quadrant (T_lo is zero above its diagonal: k from 16 ni)
+        const int mi = w >> 1, ni = w & 1;
+        float acc[8];
+        zero8(acc);
+        gemm16<false, false>(acc, N, 32 + 16 * mi, 16 * ni, Tm, 16 * ni, 16 * ni, 4 - 2 * ni, gq, t4);
+        st16<0>(Tm, acc, 16 * mi, 32 + 16 * ni, gq, t4);
+    }
+    __syncthreads();
+    if (w < 4) {
+        // T_hl = T_hi X (T_hi is zero right of its diagonal: k up to 16 mi + 16)
+        const int mi = w >> 1, ni = w & 1;
+        float acc[8];
+        zero8(acc);
+        gemm16<false, false>(acc, Tm, 32 + 16 * mi, 32, Tm, 0, 32 + 16 * ni, 2 + 2 * mi, gq, t4);
+        st16<0>(Tm, acc, 32 + 16 * mi, 16 * ni, gq, t4);
+    }
+    __syncthreads();
+    for (int e = tid; e < 1024; e += NTHR) Tm[sx(e >> 5, 32 + (e & 31))] = 0.f;
+    __syncthreads();
+}
+
+// shared memory of the map and gradient kernels: 13 tiles, Gamma_L, 8 x 64 scratch,
+// 64 column sums, the chunk's location
+constexpr int N_TILES = 13;
+constexpr size_t SMEM_BYTES =
+    sizeof(float) * (N_TILES * TILE + 64 + 8 * 64 + 64) + sizeof(ChunkLoc) + 16;
+
+struct Smem {
+    float* tile[N_TILES];
+    float* GL;
+    float* seg;
+    float* csum;
+    ChunkLoc* loc;
+    int* ok;
+};
+__device__ __forceinline__ Smem carve(float* smf) {
+    Smem s;
+#pragma unroll
+    for (int i = 0; i < N_TILES; ++i) s.tile[i] = smf + i * TILE;
+    s.GL = smf + N_TILES * TILE;
+    s.seg = s.GL + 64;
+    s.csum = s.seg + 8 * 64;
+    s.loc = reinterpret_cast<ChunkLoc*>(s.csum + 64);
+    s.ok = reinterpret_cast<int*>(s.loc + 1);
+    return s;
+}
+
+// acc -> block (r0, c0) of a row-major 64 x 64 fp32 matrix in global memory
+__device__ __forceinline__ void st16_global(float* G, const float (&acc)[8], int r0, int c0, int gq, int t4) {
+#pragma unroll
+    for (int e = 0; e < 8; e += 2) {
+        const int row = r0 + frag_row(e, gq), col = c0 + frag_col(e, t4);
+        *reinterpret_cast<float2*>(G + row * 64 + col) = make_float2(acc[e], acc[e + 1]);
+    }
+}
+
+// Nab = tril(At Bt^T, -1), Nak = tril(At Kt^T, -1), Mrb = tril(Rt Bt^T) (each warp its
+// block of all three; blocks above the diagonal are zero)
+__device__ __forceinline__ void masks_abk(const float* AT, const float* RT, const float* BT, const float* KT,
+                                          float* NAB, float* NAK, float* MRB, int m0, int n0, int gq, int t4) {
+    float acc[8];
+    zero8(acc);
+    if (n0 > m0) {
+        st16<0>(NAB, acc, m0, n0, gq, t4);
+        st16<0>(NAK, acc, m0, n0, gq, t4);
+        st16<0>(MRB, acc, m0, n0, gq, t4);
+        return;
+    }
+    gemm16<false, true>(acc, AT, m0, 0, BT, 0, n0, 8, gq, t4);
+    st16<1>(NAB, acc, m0, n0, gq, t4);
+    zero8(acc);
+    gemm16<false, true>(acc, AT, m0, 0, KT, 0, n0, 8, gq, t4);
+    st16<1>(NAK, acc, m0, n0, gq, t4);
+    zero8(acc);
+    gemm16<false, true>(acc, RT, m0, 0, BT, 0, n0, 8, gq, t4);
+    st16<2>(MRB, acc, m0, n0, gq, t4);
+}
+
+enum { T_GAM = 0, T_AT, T_RT, T_BT, T_KT, T_VV, T_DY, T_X0, T_X1, T_X2, T_X3, T_X4, T_X5 };
+
+// ---- 1. the chunk's maps M, Q, Qf
+template <typename WT>
+__global__ void __launch_bounds__(NTHR, 1)
+    bwd_map_kernel(const __nv_bfloat16* __restrict__ r, const WT* __restrict__ wl, const __nv_bfloat16* __restrict__ k,
+                   const __nv_bfloat16* __restrict__ v, const __nv_bfloat16* __restrict__ a,
+                   const __nv_bfloat16* __restrict__ b, const __nv_bfloat16* __restrict__ dy, float* __restrict__ ws,
+                   int B, int T, int H, const int32_t* __restrict__ offs, long ckpt_chunks, int* status) {
+    extern __shared__ __align__(16) float smf[];
+    const Smem sm = carve(smf);
+    ChunkLoc lc;
+    if (!locate_block_chunk(B, T, H, offs, ckpt_chunks, status, lc, sm.loc, sm.ok)) return;
+    float *GAM = sm.tile[T_GAM], *AT = sm.tile[T_AT], *RT = sm.tile[T_RT], *BT = sm.tile[T_BT], *KT = sm.tile[T_KT];
+    float *VV = sm.tile[T_VV], *DY = sm.tile[T_DY];
+    float *NAB = sm.tile[T_X0], *NAK = sm.tile[T_X1], *MRB = sm.tile[T_X2], *TT = sm.tile[T_X3];
+    float *TA = sm.tile[T_X4], *TB = sm.tile[T_X5];
+    const int tid = threadIdx.x, w = tid >> 5, gq = (tid & 31) >> 2, t4 = tid & 3;
+    const int m0 = 16 * (w >> 2), n0 = 16 * (w & 3);
+    const long tstride = static_cast<long>(H) * D, hoff = static_cast<long>(blockIdx.y) * D;
+
+    stage_chunk<WT>(GAM, AT, RT, BT, KT, VV, DY, sm.GL, sm.seg, r, wl, k, v, a, b, dy, lc.row0, lc.nv, tstride, hoff);
+    if (tid < 64 && !(sm.GL[tid] >= kMinGammaL)) report_status(status, WKV7_ERR_DECAY_RANGE);
+    masks_abk(AT, RT, BT, KT, NAB, NAK, MRB, m0, n0, gq, t4);
+    __syncthreads();
+    invert_unit_lower(NAB, TT);
+    {
+        float acc[8];
+        zero8(acc);  // TA = T At (T is zero right of its diagonal)
+        gemm16<false, false>(acc, TT, m0, 0, AT, 0, n0, (m0 + 16) / 8, gq, t4);
+        st16<0>(TA, acc, m0, n0, gq, t4);
+        zero8(acc);  // TB = T^T Bt (T^T is zero left of its diagonal)
+        gemm16<true, false>(acc, TT, m0, m0, BT, m0, n0, (64 - m0) / 8, gq, t4);
+        st16<0>(TB, acc, m0, n0, gq, t4);
+    }
+    __syncthreads();
+    float* Mg = ws + lc.region + static_cast<long>(lc.c) * SQ;
+    float* Qg = ws + lc.region + static_cast<long>(lc.nch + 1 + lc.c) * SQ;
+    float* Qfg = ws + lc.region + static_cast<long>(2 * (lc.nch + 1) + lc.c) * SQ;
+    {
+        float acc[8];
+        zero8(acc);  // M = diag(Gamma_L) (I + Bt^T TA)
+        gemm16<true, false>(acc, BT, m0, 0, TA, 0, n0, 8, gq, t4);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            const int row = m0 + frag_row(e, gq), col = n0 + frag_col(e, t4);
+            acc[e] = sm.GL[row] * (acc[e] + (row == col ? 1.f : 0.f));
+        }
+        st16_global(Mg, acc, m0, n0, gq, t4);
+        zero8(acc);  // W = Rt + Mrb TA -> NAB
+        gemm16<false, false>(acc, MRB, m0, 0, TA, 0, n0, (m0 + 16) / 8, gq, t4);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) acc[e] += RT[sx(m0 + frag_row(e, gq), n0 + frag_col(e, t4))];
+        st16<0>(NAB, acc, m0, n0, gq, t4);
+        zero8(acc);  // Z = Kt + Nak^T TB -> TT
+        gemm16<true, false>(acc, NAK, m0, m0, TB, m0, n0, (64 - m0) / 8, gq, t4);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) acc[e] += KT[sx(m0 + frag_row(e, gq), n0 + frag_col(e, t4))];
+        st16<0>(TT, acc, m0, n0, gq, t4);
+    }
+    __syncthreads();
+    {
+        float acc[8];
+        zero8(acc);  // Q = dY^T W
+        gemm16<true, false>(acc, DY, m0, 0, NAB, 0, n0, 8, gq, t4);
+        st16_global(Qg, acc, m0, n0, gq, t4);
+        zero8(acc);  // Qf = V^T Z diag(Gamma_L)
+        gemm16<true, false>(acc, VV, m0, 0, TT, 0, n0, 8, gq, t4);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) acc[e] *= sm.GL[n0 + frag_col(e, t4)];
+        st16_global(Qfg, acc, m0, n0, gq, t4);
+    }
+}
+
+// ---- 2. the scans over a unit's chunks (fp32): direction 0 runs S <- S M^T + Qf
+// forward from s0 and writes S[c] before every chunk c and S[nch] at the end;
+// direction 1 runs dS <- Q + dS M backward from dsT, writes dS_L[c] over the
+// Q slot c after reading it, and ds0 at the end.  Thread (i0, j0) keeps the
+// 4 x 4 block rows i0.., columns j0.. of the state; the next chunk's M and
+// addend are loaded into registers while the current product runs.
+constexpr int SCAN_THR = 256;
+constexpr int SP = 68;  // padded row stride of the scan's shared matrices
+
+__global__ void __launch_bounds__(SCAN_THR)
+    bwd_scan_kernel(const float* __restrict__ s0, const float* __restrict__ dsT, float* __restrict__ ds0,
+                    float* __restrict__ ws, int B, int T, int H, const int32_t* __restrict__ offs, long ckpt_chunks,
+                    int* status) {
+    __shared__ __align__(16) float Sx[64 * SP];
+    __shared__ __align__(16) float Xm[64 * SP];
+    __shared__ long sh_cbase;
+    __shared__ int sh_nch, sh_ok;
+    const int tid = threadIdx.x, unit = blockIdx.x, dir = blockIdx.y;
+    const int n = unit / H, h = unit % H;
+    if (tid == 0) {
+        long cbase = 0;
+        int nch = 0, ok = 1;
+        if (!offs) {
+            const long cps = (static_cast<long>(T) + L - 1) / L;
+            cbase = static_cast<long>(n) * cps;
+            nch = static_cast<int>(cps);
+        } else {
+            for (int m = 0; m <= n && ok; ++m) {
+                const long o0 = offs[m], o1 = offs[m + 1];
+                if (o0 < 0 || o1 < o0 || o1 > T) {
+                    ok = 0;
+                } else if (m < n) {
+                    cbase += (o1 - o0 + L - 1) / L;
+                } else {
+                    nch = static_cast<int>((o1 - o0 + L - 1) / L);
+                }
+            }
+            if (ok && cbase + nch > ckpt_chunks) ok = 0;
+            if (!ok) report_status(status, WKV7_ERR_DEVICE_BOUNDS);
+        }
+        sh_cbase = cbase;
+        sh_nch = nch;
+        sh_ok = ok;
+    }
+    __syncthreads();
+    if (!sh_ok) return;
+    const int nch = sh_nch;
+    float* Mb = ws + unit_region(sh_cbase, n, h, H, nch);
+    float* Qb = Mb + static_cast<long>(nch + 1) * SQ;
+    float* Qfb = Qb + static_cast<long>(nch + 1) * SQ;
+    float* Sb = Qfb + static_cast<long>(nch + 1) * SQ;
+    float* addb = dir == 0 ? Qfb : Qb;
+    const int i0 = 4 * (tid >> 4), j0 = 4 * (tid & 15);
+    const long sbase = static_cast<long>(unit) * SQ;
+
+    float st[4][4];
+    {
+        const float* init = dir == 0 ? s0 : dsT;
+#pragma unroll
+        for (int p = 0; p < 4; ++p) {
+            const float4 x = init ? *reinterpret_cast<const float4*>(init + sbase + (i0 + p) * 64 + j0)
+                                  : make_float4(0.f, 0.f, 0.f, 0.f);
+            st[p][0] = x.x; st[p][1] = x.y; st[p][2] = x.z; st[p][3] = x.w;
+        }
+    }
+    float4 mreg[4], areg[4];
+    auto prefetch = [&](int c) {
+#pragma unroll
+        for (int p = 0; p < 4; ++p) {
+            mreg[p] = *reinterpret_cast<const float4*>(Mb + static_cast<long>(c) * SQ + (i0 + p) * 64 + j0);
+            areg[p] = *reinterpret_cast<const float4*>(addb + static_cast<long>(c) * SQ + (i0 + p) * 64 + j0);
+        }
+    };
+    if (nch > 0) prefetch(dir == 0 ? 0 : nch - 1);
+    for (int s = 0; s < nch; ++s) {
+        const int c = dir == 0 ? s : nch - 1 - s;
+        float* out = (dir == 0 ? Sb : Qb) + static_cast<long>(c) * SQ;
+        float acc[4][4];
+#pragma unroll
+        for (int p = 0; p < 4; ++p) {
+            const float4 x = make_float4(st[p][0], st[p][1], st[p][2], st[p][3]);
+            *reinterpret_cast<float4*>(out + (i0 + p) * 64 + j0) = x;
+            *reinterpret_cast<float4*>(Sx + (i0 + p) * SP + j0) = x;
+            acc[p][0] = areg[p].x; acc[p][1] = areg[p].y; acc[p][2] = areg[p].z; acc[p][3] = areg[p].w;
+            if (dir == 1) {
+                *reinterpret_cast<float4*>(Xm + (i0 + p) * SP + j0) = mreg[p];
+            } else {
+                Xm[(j0 + 0) * SP + i0 + p] = mreg[p].x;
+                Xm[(j0 + 1) * SP + i0 + p] = mreg[p].y;
+                Xm[(j0 + 2) * SP + i0 + p] = mreg[p].z;
+                Xm[(j0 + 3) * SP + i0 + p] = mreg[p].w;
+            }
+        }
+        __syncthreads();
+        if (s + 1 < nch) prefetch(dir == 0 ? c + 1 : c - 1);
+#pragma unroll 2
+        for (int kk = 0; kk < 64; kk += 4) {
+            float4 sv[4], xv[4];
+#pragma unroll
+            for (int p = 0; p < 4; ++p) {
+                sv[p] = *reinterpret_cast<const float4*>(Sx + (i0 + p) * SP + kk);
+                xv[p] = *reinterpret_cast<const float4*>(Xm + (kk + p) * SP + j0);
+            }
+#pragma unroll
+            for (int p = 0; p < 4; ++p) {
+                const float sk[4] = {sv[p].x, sv[p].y, sv[p].z, sv[p].w};
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    acc[p][0] = fmaf(sk[q], xv[q].x, acc[p][0]);
+                    acc[p][1] = fmaf(sk[q], xv[q].y, acc[p][1]);
+                    acc[p][2] = fmaf(sk[q], xv[q].z, acc[p][2]);
+                    acc[p][3] = fmaf(sk[q], xv[q].w, acc[p][3]);
+                }
+            }
+        }
+        __syncthreads();
+#pragma unroll
+        for (int p = 0; p < 4; ++p)
+#pragma unroll
+            for (int q = 0; q < 4; ++q) st[p][q] = acc[p][q];
+    }
+    float* fin = dir == 0 ? Sb + static_cast<long>(nch) * SQ : ds0 + sbase;
+#pragma unroll
+    for (int p = 0; p < 4; ++p)
+        *reinterpret_cast<float4*>(fin + (i0 + p) * 64 + j0) = make_float4(st[p][0], st[p][1], st[p][2], st[p][3]);
+}
+
+// bf16 pair -> (row0 + row, col .. col + 1) of a [tokens][H][D] tensor
+__device__ __forceinline__ void st_pair(__nv_bfloat16* p, long off, float x0, float x1) {
+    *reinterpret_cast<uint32_t*>(p + off) = pack_bf16x2(x0, x1);
+}
+
+// ---- 3. every gradient of one chunk, from S0 = S[c], S_L = S[c + 1] and dS_L
+template <typename WT>
+__global__ void __launch_bounds__(NTHR, 1)
+    bwd_grad_kernel(const __nv_bfloat16* __restrict__ r, const WT* __restrict__ wl, const __nv_bfloat16* __restrict__ k,
+                    const __nv_bfloat16* __restrict__ v, const __nv_bfloat16* __restrict__ a,
+                    const __nv_bfloat16* __restrict__ b, const __nv_bfloat16* __restrict__ dy,
+                    __nv_bfloat16* __restrict__ dr, WT* __restrict__ dwl, __nv_bfloat16* __restrict__ dk,
+                    __nv_bfloat16* __restrict__ dv, __nv_bfloat16* __restrict__ da, __nv_bfloat16* __restrict__ db,
+                    const float* __restrict__ ws, int B, int T, int H, const int32_t* __restrict__ offs,
+                    long ckpt_chunks, int* status) {
+    extern __shared__ __align__(16) float smf[];
+    const Smem sm = carve(smf);
+    ChunkLoc lc;
+    if (!locate_block_chunk(B, T, H, offs, ckpt_chunks, status, lc, sm.loc, sm.ok)) return;
+    float *GAM = sm.tile[T_GAM], *AT = sm.tile[T_AT], *RT = sm.tile[T_RT], *BT = sm.tile[T_BT], *KT = sm.tile[T_KT];
+    float *VV = sm.tile[T_VV], *DY = sm.tile[T_DY];
+    float *W0 = sm.tile[T_X0], *W1 = sm.tile[T_X1], *W2 = sm.tile[T_X2], *W3 = sm.tile[T_X3];
+    float *S0 = sm.tile[T_X4], *DS = sm.tile[T_X5];
+    const int tid = threadIdx.x, w = tid >> 5, gq = (tid & 31) >> 2, t4 = tid & 3;
+    const int m0 = 16 * (w >> 2), n0 = 16 * (w & 3);
+    const long tstride = static_cast<long>(H) * D, hoff = static_cast<long>(blockIdx.y) * D;
+    const int nv = lc.nv;
+
+    stage_chunk<WT>(GAM, AT, RT, BT, KT, VV, DY, sm.GL, sm.seg, r, wl, k, v, a, b, dy, lc.row0, nv, tstride, hoff);
+    {
+        // S0 and dSLg = dS_L diag(Gamma_L) as tiles; column sums of dS_L (.) S_L
+        const float* S0g = ws + lc.region + static_cast<long>(3 * (lc.nch + 1) + lc.c) * SQ;
+        const float* SLg = S0g + SQ;
+        const float* dSg = ws + lc.region + static_cast<long>(lc.nch + 1 + lc.c) * SQ;
+        const int j = tid & 63, s = tid >> 6;
+        const float gl = sm.GL[j];
+        float cs = 0.f;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const int row = 8 * s + i;
+            const float d = dSg[row * 64 + j];
+            cs = fmaf(d, SLg[row * 64 + j], cs);
+            S0[sx(row, j)] = round_tf32(S0g[row * 64 + j]);
+            DS[sx(row, j)] = round_tf32(d * gl);
+        }
+        sm.seg[s * 64 + j] = cs;
+    }
+    masks_abk(AT, RT, BT, KT, W0, W1, W2, m0, n0, gq, t4);  // W0 = Nab, W1 = Nak, W2 = Mrb
+    __syncthreads();
+    if (tid < 64) {
+        float cs = 0.f;
+#pragma unroll
+        for (int s = 0; s < 8; ++s) cs += sm.seg[s * 64 + tid];
+        sm.csum[tid] = cs;
+    }
+    invert_unit_lower(W0, W3);  // W3 = T
+    float acc[8];
+    // X = At S0^T + Nak V -> W0
+    zero8(acc);
+    gemm16<false, true>(acc, AT, m0, 0, S0, 0, n0, 8, gq, t4);
+    gemm16<false, false>(acc, W1, m0, 0, VV, 0, n0, (m0 + 16) / 8, gq, t4);
+    st16<0>(W0, acc, m0, n0, gq, t4);
+    __syncthreads();
+    // U = T X -> W0
+    zero8(acc);
+    gemm16<false, false>(acc, W3, m0, 0, W0, 0, n0, (m0 + 16) / 8, gq, t4);
+    __syncthreads();
+    st16<0>(W0, acc, m0, n0, gq, t4);
+    // dU = Mrb^T dY + Bt dSLg^T -> W2
+    zero8(acc);
+    gemm16<true, false>(acc, W2, m0, m0, DY, m0, n0, (64 - m0) / 8, gq, t4);
+    gemm16<false, true>(acc, BT, m0, 0, DS, 0, n0, 8, gq, t4);
+    __syncthreads();
+    st16<0>(W2, acc, m0, n0, gq, t4);
+    __syncthreads();
+    // dX = T^T dU -> W3
+    zero8(acc);
+    gemm16<true, false>(acc, W3, m0, m0, W2, m0, n0, (64 - m0) / 8, gq, t4);
+    __syncthreads();
+    st16<0>(W3, acc, m0, n0, gq, t4);
+    // Mrk = tril(Rt Kt^T) -> W2
+    zero8(acc);
+    if (n0 <= m0) gemm16<false, true>(acc, RT, m0, 0, KT, 0, n0, 8, gq, t4);
+    st16<2>(W2, acc, m0, n0, gq, t4);
+    __syncthreads();
+    // dV = Mrk^T dY + Kt dSLg^T + Nak^T dX
+    zero8(acc);
+    gemm16<true, false>(acc, W2, m0, m0, DY, m0, n0, (64 - m0) / 8, gq, t4);
+    gemm16<false, true>(acc, KT, m0, 0, DS, 0, n0, 8, gq, t4);
+    gemm16<true, false>(acc, W1, m0, m0, W3, m0, n0, (64 - m0) / 8, gq, t4);
+#pragma unroll
+    for (int e = 0; e < 8; e += 2) {
+        const int row = m0 + frag_row(e, gq), col = n0 + frag_col(e, t4);
+        if (row < nv) st_pair(dv, (lc.row0 + row) * tstride + hoff + col, acc[e], acc[e + 1]);
+    }
+    // the four accumulated gradients: dAt, dRt, dBt', dKt'
+    float gA[8], gR[8], gB[8], gK[8];
+    zero8(gA);
+    zero8(gR);
+    zero8(gB);
+    zero8(gK);
+    gemm16<false, false>(gA, W3, m0, 0, S0, 0, n0, 8, gq, t4);  // dX S0
+    gemm16<false, false>(gR, DY, m0, 0, S0, 0, n0, 8, gq, t4);  // dY S0
+    gemm16<false, false>(gB, W0, m0, 0, DS, 0, n0, 8, gq, t4);  // U dSLg
+    gemm16<false, false>(gK, VV, m0, 0, DS, 0, n0, 8, gq, t4);  // V dSLg
+    __syncthreads();
+    // dNab = tril(dX U^T, -1) -> W1, dNak = tril(dX V^T, -1) -> W2
+    zero8(acc);
+    if (n0 <= m0) gemm16<false, true>(acc, W3, m0, 0, W0, 0, n0, 8, gq, t4);
+    st16<1>(W1, acc, m0, n0, gq, t4);
+    zero8(acc);
+    if (n0 <= m0) gemm16<false, true>(acc, W3, m0, 0, VV, 0, n0, 8, gq, t4);
+    st16<1>(W2, acc, m0, n0, gq, t4);
+    __syncthreads();
+    gemm16<false, false>(gA, W1, m0, 0, BT, 0, n0, (m0 + 16) / 8, gq, t4);   // dNab Bt
+    gemm16<false, false>(gA, W2, m0, 0, KT, 0, n0, (m0 + 16) / 8, gq, t4);   // dNak Kt
+    gemm16<true, false>(gB, W1, m0, m0, AT, m0, n0, (64 - m0) / 8, gq, t4);  // dNab^T At
+    gemm16<true, false>(gK, W2, m0, m0, AT, m0, n0, (64 - m0) / 8, gq, t4);  // dNak^T At
+    __syncthreads();
+    // dMrb = tril(dY U^T) -> W1, dMrk = tril(dY V^T) -> W2
+    zero8(acc);
+    if (n0 <= m0) gemm16<false, true>(acc, DY, m0, 0, W0, 0, n0, 8, gq, t4);
+    st16<2>(W1, acc, m0, n0, gq, t4);
+    zero8(acc);
+    if (n0 <= m0) gemm16<false, true>(acc, DY, m0, 0, VV, 0, n0, 8, gq, t4);
+    st16<2>(W2, acc, m0, n0, gq, t4);
+    __syncthreads();
+    gemm16<false, false>(gR, W1, m0, 0, BT, 0, n0, (m0 + 16) / 8, gq, t4);   // dMrb Bt
+    gemm16<false, false>(gR, W2, m0, 0, KT, 0, n0, (m0 + 16) / 8, gq, t4);   // dMrk Kt
+    gemm16<true, false>(gB, W1, m0, m0, RT, m0, n0, (64 - m0) / 8, gq, t4);  // dMrb^T Rt
+    gemm16<true, false>(gK, W2, m0, m0, RT, m0, n0, (64 - m0) / 8, gq, t4);  // dMrk^T Rt
+    __syncthreads();
+    // da, dr, db, dk; the terms of d log w: W1 = da (.) a, W2 = dr (.) r - db (.) b - dk (.) k
+#pragma unroll
+    for (int e = 0; e < 8; e += 2) {
+        const int row = m0 + frag_row(e, gq), col = n0 + frag_col(e, t4);
+        float o[4][2];
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+            const int cc = col + u, ix = sx(row, cc);
+            const float g = GAM[ix], gp = row > 0 ? GAM[sx(row - 1, cc)] : 1.f, ig = __frcp_rn(g);
+            const float xa = gA[e + u], xr = gR[e + u], xb = gB[e + u], xk = gK[e + u];
+            o[0][u] = xa * gp;
+            o[1][u] = xr * g;
+            o[2][u] = xb * ig;
+            o[3][u] = xk * ig;
+            W1[ix] = xa * AT[ix];
+            W2[ix] = xr * RT[ix] - xb * BT[ix] - xk * KT[ix];
+        }
+        if (row < nv) {
+            const long off = (lc.row0 + row) * tstride + hoff + col;
+            st_pair(da, off, o[0][0], o[0][1]);
+            st_pair(dr, off, o[1][0], o[1][1]);
+            st_pair(db, off, o[2][0], o[2][1]);
+            st_pair(dk, off, o[3][0], o[3][1]);
+        }
+    }
+    __syncthreads();
+    {
+        // d log w_s = sum_{t >= s} g_t with g_t = W2[t] + W1[t + 1] (t < 63) and
+        // g_63 = W2[63] + colsum(dS_L (.) S_L): thread (column j, tokens 8 s .. 8 s + 7)
+        const int j = tid & 63, s = tid >> 6;
+        float x[8], run = 0.f;
+#pragma unroll
+        for (int i = 7; i >= 0; --i) {
+            const int t = 8 * s + i;
+            run += W2[sx(t, j)] + (t < 63 ? W1[sx(t + 1, j)] : sm.csum[j]);
+            x[i] = run;
+        }
+        sm.seg[s * 64 + j] = run;
+        __syncthreads();
+        float later = 0.f;
+        for (int q = s + 1; q < 8; ++q) later += sm.seg[q * 64 + j];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const int t = 8 * s + i;
+            if (t < nv) {
+                const long off = (lc.row0 + t) * tstride + hoff + j;
+                const float el = expf(to_f32(wl[off]));
+                dwl[off] = from_f32<WT>(-(x[i] + later) * el);
+            }
+        }
+    }
+}
+
+template <typename WT>
+cudaError_t launch_chunked_typed(const BackwardArgs& p, cudaStream_t stream) {
+    static std::atomic<unsigned long long> cfg_map{0}, cfg_grad{0};
+    auto map = bwd_map_kernel<WT>;
+    auto grad = bwd_grad_kernel<WT>;
+    cudaError_t e = configure_smem_once(map, static_cast<int>(SMEM_BYTES), cfg_map);
+    if (e != cudaSuccess) return e;
+    e = configure_smem_once(grad, static_cast<int>(SMEM_BYTES), cfg_grad);
+    if (e != cudaSuccess) return e;
+    using bf = __nv_bfloat16;
+    const bf *r = static_cast<const bf*>(p.r), *k = static_cast<const bf*>(p.k), *v = static_cast<const bf*>(p.v);
+    const bf *a = static_cast<const bf*>(p.a), *b = static_cast<const bf*>(p.b), *dy = static_cast<const bf*>(p.dy);
+    const WT* wl = static_cast<const WT*>(p.w_log);
+    const dim3 cgrid(static_cast<unsigned>(p.ckpt_chunks), static_cast<unsigned>(p.H));
+    if (p.ckpt_chunks > 0) {
+        map<<<cgrid, NTHR, SMEM_BYTES, stream>>>(r, wl, k, v, a, b, dy, p.ws, p.B, p.T, p.H, p.seq_offsets,
+                                                 p.ckpt_chunks, p.status);
+        e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+    }
+    bwd_scan_kernel<<<dim3(static_cast<unsigned>(p.B) * p.H, 2), SCAN_THR, 0, stream>>>(
+        p.s0, p.dsT, p.ds0, p.ws, p.B, p.T, p.H, p.seq_offsets, p.ckpt_chunks, p.status);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    if (p.ckpt_chunks > 0) {
+        grad<<<cgrid, NTHR, SMEM_BYTES, stream>>>(r, wl, k, v, a, b, dy, static_cast<bf*>(p.dr),
+                                                  static_cast<WT*>(p.dw_log), static_cast<bf*>(p.dk),
+                                                  static_cast<bf*>(p.dv), static_cast<bf*>(p.da), static_cast<bf*>(p.db),
+                                                  p.ws, p.B, p.T, p.H, p.seq_offsets, p.ckpt_chunks, p.status);
+        e = cudaGetLastError();
+    }
+    return e;
+}
+
+}  // namespace
+
+size_t backward_chunked_workspace_floats(int B, int T, int H, int packed) {
+    return static_cast<size_t>(4) * H * (backward_ckpt_chunks(B, T, packed) + B) * SQ;
+}
+
+cudaError_t launch_backward_chunked(const BackwardArgs& p, int w_dtype, cudaStream_t stream) {
+    return w_dtype == WKV7_BF16 ? launch_chunked_typed<__nv_bfloat16>(p, stream) : launch_chunked_typed<float>(p, stream);
+}
+
+}  // namespace wkv7

@@ -80,7 +80,7 @@ struct BackwardArgs {
     void* da;
     void* db;
     float* ds0;
-    float* ws;  // workspace: chunk checkpoints, then one chunk of states per unit
+    float* ws;  // workspace (layout owned by the kernel that uses it)
     int B, T, H;
     const int32_t* seq_offsets;
     long ckpt_chunks;  // checkpoint slots per head in the workspace
@@ -107,6 +107,9 @@ cudaError_t launch_state_identity(float* M, float* Q, long n, cudaStream_t strea
 long backward_ckpt_chunks(int B, int T, int packed);
 size_t backward_workspace_floats(int B, int T, int H, int packed);
 cudaError_t launch_backward(const BackwardArgs& p, int io_dtype, int w_dtype, cudaStream_t stream);
+// chunked (WY) form for bf16 inputs (wkv7_backward_chunk.cu)
+size_t backward_chunked_workspace_floats(int B, int T, int H, int packed);
+cudaError_t launch_backward_chunked(const BackwardArgs& p, int w_dtype, cudaStream_t stream);
 
 // Raises `kern`'s dynamic shared-memory limit to `bytes` the first time it is
 // launched on the current device.  `configured` holds one bit per device

@@ -65,10 +65,10 @@ def test_backward_noalloc_packed(wk):
 
 
 def test_backward_noalloc_at_the_limit(wk):
-    """B1 H2 T28672: 2 x 448 chunk checkpoints plus 2 x 64 recomputed states of
-    16 KiB each fill the 16 MiB scratch exactly; T + 1 needs one checkpoint more
-    per head and is refused before anything is launched."""
-    B, T, H = 1, 28672, 2
+    """B1 H1 T16320 (255 chunks): the chunked form's 4 x (255 + 1) states of
+    16 KiB fill the 16 MiB scratch exactly; T + 1 needs a chunk more and is
+    refused before anything is launched."""
+    B, T, H = 1, 16320, 1
     assert wk.wkv7_backward_workspace_bytes(B, T, H, 64, False) == LIMIT
     inp = W.make_prefill(B, T, H, io="bf16", wdt="f32", s0_std=0.1, seed=81)
     _run_both(wk, inp, seed=82)
