@@ -546,7 +546,7 @@ __global__ void __launch_bounds__(NTHR, 1)
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
             const int row = m0 + frag_row(e, gq), col = n0 + frag_col(e, t4);
-            acc[e] = sm.GL[row] * (acc[e] + (row == col ? 1.f : 0.f));
+            acc[e] = round_tf32(sm.GL[row] * (acc[e] + (row == col ? 1.f : 0.f)));  // a tf32 operand of the scan
         }
         st16_global(Mg, acc, m0, n0, gq, t4);
         zero8(acc);  // W = Rt + Mrb TA -> NAB
@@ -574,21 +574,43 @@ __global__ void __launch_bounds__(NTHR, 1)
     }
 }
 
-// ---- 2. the scans over a unit's chunks (fp32): direction 0 runs S <- S M^T + Qf
+// ---- 2. the scans over a unit's chunks: direction 0 runs S <- S M^T + Qf
 // forward from s0 and writes S[c] before every chunk c and S[nch] at the end;
-// direction 1 runs dS <- Q + dS M backward from dsT, writes dS_L[c] over the
-// Q slot c after reading it, and ds0 at the end.  Thread (i0, j0) keeps the
-// 4 x 4 block rows i0.., columns j0.. of the state; the next chunk's M and
-// addend are loaded into registers while the current product runs.
-constexpr int SCAN_THR = 256;
-constexpr int SP = 68;  // padded row stride of the scan's shared matrices
+// direction 1 runs dS <- Q + dS M backward from dsT, writes dS_L[c] over the Q
+// slot c after reading it, and ds0 at the end.  Warp w keeps rows 16 w ..
+// 16 w + 15 of the state in registers, laid out as the accumulator of m16n8k8
+// products; with the k order of gemm16 those registers are also the A
+// fragments of the next product, so the state never leaves the registers.  M
+// (tf32 from the map kernel) and the addend stream through a three-stage
+// cp.async ring; the state enters the product as tf32 high and low parts
+// (S = S_hi + S_lo, two products), which keeps the scan at fp32 accuracy over
+// many chunks.
+constexpr int SCAN_THR = 128;
+
+__device__ __forceinline__ void cp_async16(float* dst, const float* src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
+// row-major 64 x 64 fp32 matrix (global) -> tile in the sx layout, 8 16-byte pieces per thread
+__device__ __forceinline__ void tile_async(float* tile, const float* g) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        const int q = threadIdx.x + SCAN_THR * i, row = q >> 4, col = (q & 15) << 2;
+        cp_async16(tile + sx(row, col), g + row * 64 + col);
+    }
+}
+
+constexpr int SCAN_STAGES = 3;
+constexpr size_t SCAN_SMEM = sizeof(float) * 2 * SCAN_STAGES * TILE;
 
 __global__ void __launch_bounds__(SCAN_THR)
     bwd_scan_kernel(const float* __restrict__ s0, const float* __restrict__ dsT, float* __restrict__ ds0,
                     float* __restrict__ ws, int B, int T, int H, const int32_t* __restrict__ offs, long ckpt_chunks,
                     int* status) {
-    __shared__ __align__(16) float Sx[64 * SP];
-    __shared__ __align__(16) float Xm[64 * SP];
+    extern __shared__ __align__(128) float scan_smem[];  // M[stage] then addend[stage], sx layout
     __shared__ long sh_cbase;
     __shared__ int sh_nch, sh_ok;
     const int tid = threadIdx.x, unit = blockIdx.x, dir = blockIdx.y;
@@ -625,80 +647,99 @@ __global__ void __launch_bounds__(SCAN_THR)
     float* Qb = Mb + static_cast<long>(nch + 1) * SQ;
     float* Qfb = Qb + static_cast<long>(nch + 1) * SQ;
     float* Sb = Qfb + static_cast<long>(nch + 1) * SQ;
-    float* addb = dir == 0 ? Qfb : Qb;
-    const int i0 = 4 * (tid >> 4), j0 = 4 * (tid & 15);
+    const float* addb = dir == 0 ? Qfb : Qb;
+    const int w = tid >> 5, gq = (tid & 31) >> 2, t4 = tid & 3, r0 = 16 * w;
     const long sbase = static_cast<long>(unit) * SQ;
+    // element e of n-tile j: row r0 + gq + 8 (e >> 1), column 8 j + 2 t4 + (e & 1)
+    auto frow = [&](int e) { return r0 + gq + 8 * (e >> 1); };
+    auto fcol = [&](int j) { return 8 * j + 2 * t4; };
 
-    float st[4][4];
+    float st[8][4];
     {
         const float* init = dir == 0 ? s0 : dsT;
 #pragma unroll
-        for (int p = 0; p < 4; ++p) {
-            const float4 x = init ? *reinterpret_cast<const float4*>(init + sbase + (i0 + p) * 64 + j0)
-                                  : make_float4(0.f, 0.f, 0.f, 0.f);
-            st[p][0] = x.x; st[p][1] = x.y; st[p][2] = x.z; st[p][3] = x.w;
-        }
+        for (int j = 0; j < 8; ++j)
+#pragma unroll
+            for (int e = 0; e < 4; e += 2) {
+                const float2 x = init ? *reinterpret_cast<const float2*>(init + sbase + frow(e) * 64 + fcol(j))
+                                      : make_float2(0.f, 0.f);
+                st[j][e] = x.x;
+                st[j][e + 1] = x.y;
+            }
     }
-    float4 mreg[4], areg[4];
-    auto prefetch = [&](int c) {
-#pragma unroll
-        for (int p = 0; p < 4; ++p) {
-            mreg[p] = *reinterpret_cast<const float4*>(Mb + static_cast<long>(c) * SQ + (i0 + p) * 64 + j0);
-            areg[p] = *reinterpret_cast<const float4*>(addb + static_cast<long>(c) * SQ + (i0 + p) * 64 + j0);
+    auto chunk_of = [&](int s) { return dir == 0 ? s : nch - 1 - s; };
+    auto fetch = [&](int s) {  // M and addend of step s -> stage s % 3 (one commit group per step)
+        if (s < nch) {
+            const long c = chunk_of(s);
+            float* stage = scan_smem + 2 * (s % SCAN_STAGES) * TILE;
+            tile_async(stage, Mb + c * SQ);
+            tile_async(stage + TILE, addb + c * SQ);
         }
+        cp_async_commit();
     };
-    if (nch > 0) prefetch(dir == 0 ? 0 : nch - 1);
+    fetch(0);
+    fetch(1);
     for (int s = 0; s < nch; ++s) {
-        const int c = dir == 0 ? s : nch - 1 - s;
+        const int c = chunk_of(s);
+        fetch(s + 2);
+        cp_async_wait<2>();
+        __syncthreads();  // step s's tiles have landed for every thread
+        const float* M = scan_smem + 2 * (s % SCAN_STAGES) * TILE;
+        const float* A = M + TILE;
+        // the state before chunk c: forward S[c]; backward dS_L[c] over the Q slot, whose copy has completed
         float* out = (dir == 0 ? Sb : Qb) + static_cast<long>(c) * SQ;
-        float acc[4][4];
+        float acc[8][4];
 #pragma unroll
-        for (int p = 0; p < 4; ++p) {
-            const float4 x = make_float4(st[p][0], st[p][1], st[p][2], st[p][3]);
-            *reinterpret_cast<float4*>(out + (i0 + p) * 64 + j0) = x;
-            *reinterpret_cast<float4*>(Sx + (i0 + p) * SP + j0) = x;
-            acc[p][0] = areg[p].x; acc[p][1] = areg[p].y; acc[p][2] = areg[p].z; acc[p][3] = areg[p].w;
-            if (dir == 1) {
-                *reinterpret_cast<float4*>(Xm + (i0 + p) * SP + j0) = mreg[p];
-            } else {
-                Xm[(j0 + 0) * SP + i0 + p] = mreg[p].x;
-                Xm[(j0 + 1) * SP + i0 + p] = mreg[p].y;
-                Xm[(j0 + 2) * SP + i0 + p] = mreg[p].z;
-                Xm[(j0 + 3) * SP + i0 + p] = mreg[p].w;
-            }
-        }
-        __syncthreads();
-        if (s + 1 < nch) prefetch(dir == 0 ? c + 1 : c - 1);
-#pragma unroll 2
-        for (int kk = 0; kk < 64; kk += 4) {
-            float4 sv[4], xv[4];
+        for (int j = 0; j < 8; ++j)
 #pragma unroll
-            for (int p = 0; p < 4; ++p) {
-                sv[p] = *reinterpret_cast<const float4*>(Sx + (i0 + p) * SP + kk);
-                xv[p] = *reinterpret_cast<const float4*>(Xm + (kk + p) * SP + j0);
+            for (int e = 0; e < 4; e += 2) {
+                *reinterpret_cast<float2*>(out + frow(e) * 64 + fcol(j)) = make_float2(st[j][e], st[j][e + 1]);
+                const float2 x = *reinterpret_cast<const float2*>(A + sx(frow(e), fcol(j)));
+                acc[j][e] = x.x;
+                acc[j][e + 1] = x.y;
             }
 #pragma unroll
-            for (int p = 0; p < 4; ++p) {
-                const float sk[4] = {sv[p].x, sv[p].y, sv[p].z, sv[p].w};
+        for (int kb = 0; kb < 8; ++kb) {
+            uint32_t ahi[4], alo[4];
+            const float av[4] = {st[kb][0], st[kb][2], st[kb][1], st[kb][3]};
 #pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    acc[p][0] = fmaf(sk[q], xv[q].x, acc[p][0]);
-                    acc[p][1] = fmaf(sk[q], xv[q].y, acc[p][1]);
-                    acc[p][2] = fmaf(sk[q], xv[q].z, acc[p][2]);
-                    acc[p][3] = fmaf(sk[q], xv[q].w, acc[p][3]);
+            for (int i = 0; i < 4; ++i) {
+                const float hi = round_tf32(av[i]);
+                ahi[i] = __float_as_uint(hi);
+                alo[i] = __float_as_uint(round_tf32(av[i] - hi));
+            }
+            uint32_t bf[8][2];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                if (dir == 0) {  // B(k, n) = M[n][k]
+                    const float2 y = *reinterpret_cast<const float2*>(M + sx(8 * j + gq, 8 * kb + 2 * t4));
+                    bf[j][0] = __float_as_uint(y.x);
+                    bf[j][1] = __float_as_uint(y.y);
+                } else {         // B(k, n) = M[k][n]
+                    bf[j][0] = __float_as_uint(M[sx(8 * kb + 2 * t4, 8 * j + gq)]);
+                    bf[j][1] = __float_as_uint(M[sx(8 * kb + 2 * t4 + 1, 8 * j + gq)]);
                 }
             }
+            // the high parts into all eight accumulators, then the low parts: eight
+            // independent products between two that share an accumulator
+#pragma unroll
+            for (int j = 0; j < 8; ++j) mma_tf32(acc[j], ahi, bf[j]);
+#pragma unroll
+            for (int j = 0; j < 8; ++j) mma_tf32(acc[j], alo, bf[j]);
         }
-        __syncthreads();
+        __syncthreads();  // every warp is done with this stage before step s + 3 refills it
 #pragma unroll
-        for (int p = 0; p < 4; ++p)
+        for (int j = 0; j < 8; ++j)
 #pragma unroll
-            for (int q = 0; q < 4; ++q) st[p][q] = acc[p][q];
+            for (int e = 0; e < 4; ++e) st[j][e] = acc[j][e];
     }
+    cp_async_wait<0>();
     float* fin = dir == 0 ? Sb + static_cast<long>(nch) * SQ : ds0 + sbase;
 #pragma unroll
-    for (int p = 0; p < 4; ++p)
-        *reinterpret_cast<float4*>(fin + (i0 + p) * 64 + j0) = make_float4(st[p][0], st[p][1], st[p][2], st[p][3]);
+    for (int j = 0; j < 8; ++j)
+#pragma unroll
+        for (int e = 0; e < 4; e += 2)
+            *reinterpret_cast<float2*>(fin + frow(e) * 64 + fcol(j)) = make_float2(st[j][e], st[j][e + 1]);
 }
 
 // bf16 pair -> (row0 + row, col .. col + 1) of a [tokens][H][D] tensor
@@ -906,7 +947,10 @@ cudaError_t launch_chunked_typed(const BackwardArgs& p, cudaStream_t stream) {
         e = cudaGetLastError();
         if (e != cudaSuccess) return e;
     }
-    bwd_scan_kernel<<<dim3(static_cast<unsigned>(p.B) * p.H, 2), SCAN_THR, 0, stream>>>(
+    static std::atomic<unsigned long long> cfg_scan{0};
+    e = configure_smem_once(bwd_scan_kernel, static_cast<int>(SCAN_SMEM), cfg_scan);
+    if (e != cudaSuccess) return e;
+    bwd_scan_kernel<<<dim3(static_cast<unsigned>(p.B) * p.H, 2), SCAN_THR, SCAN_SMEM, stream>>>(
         p.s0, p.dsT, p.ds0, p.ws, p.B, p.T, p.H, p.seq_offsets, p.ckpt_chunks, p.status);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
