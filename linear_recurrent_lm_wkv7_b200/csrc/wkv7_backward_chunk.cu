@@ -153,6 +153,12 @@ __device__ __forceinline__ void gemm16(float (&acc)[8], const float* A, int ar, 
     }
 }
 
+constexpr float kLog2e = 1.4426950408889634f;
+// w = exp(-exp(l)) and exp(l) by the hardware 2^x (subnormals flushed: a w that
+// small fails the decay-range check anyway)
+__device__ __forceinline__ float decay(float l) { return ex2_ftz(-kLog2e * ex2_ftz(kLog2e * l)); }
+__device__ __forceinline__ float exp_l(float l) { return ex2_ftz(kLog2e * l); }
+
 __device__ __forceinline__ void zero8(float (&acc)[8]) {
 #pragma unroll
     for (int e = 0; e < 8; ++e) acc[e] = 0.f;
@@ -286,6 +292,30 @@ __device__ bool locate_block_chunk(int B, int T, int H, const int32_t* offs, lon
     return *sh_ok != 0;
 }
 
+// L2 prefetch of the inputs of the block `ahead` places later in launch order
+// (dense batches; with one block per SM that is about the next block this SM
+// runs, so its staging finds its rows in L2).  One thread per 128-byte row piece.
+template <typename WT>
+__device__ __forceinline__ void prefetch_ahead(const __nv_bfloat16* r, const WT* wl, const __nv_bfloat16* k,
+                                               const __nv_bfloat16* v, const __nv_bfloat16* a,
+                                               const __nv_bfloat16* b, const __nv_bfloat16* dy, int B, int T, int H,
+                                               const int32_t* offs, unsigned ahead) {
+    if (offs || threadIdx.x >= 64) return;
+    const unsigned id = blockIdx.y * gridDim.x + blockIdx.x + ahead;
+    if (id >= gridDim.x * gridDim.y) return;
+    const long cps = (static_cast<long>(T) + L - 1) / L;
+    const int h = static_cast<int>(id / gridDim.x);
+    const long g = id % gridDim.x;
+    const long n = g / cps, c = g % cps;
+    const int t = threadIdx.x;
+    if (n >= B || c * L + t >= T) return;
+    const long off = (n * T + c * L + t) * static_cast<long>(H) * D + static_cast<long>(h) * D;
+    const void* rows[7] = {r + off, k + off, v + off, a + off, b + off, dy + off, wl + off};
+#pragma unroll
+    for (int q = 0; q < 7; ++q) asm volatile("prefetch.global.L2 [%0];" ::"l"(rows[q]));
+    if constexpr (sizeof(WT) == 4) asm volatile("prefetch.global.L2 [%0];" ::"l"(wl + off + 32));
+}
+
 // Stages the chunk's inputs of one head as fp32 tiles: GAM = Gamma (running
 // products of w = exp(-exp(w_log)) down the tokens), AT, RT, BT, KT (the scaled
 // operands, tf32-rounded), VV and DY (bf16 values, exact in tf32); GL = Gamma_L.
@@ -311,7 +341,7 @@ __device__ void stage_chunk(float* GAM, float* AT, float* RT, float* BT, float* 
         st8(DY, t, c0, x, false);
         ld_wlog8(wl + off, x);
 #pragma unroll
-        for (int e = 0; e < 8; ++e) x[e] = expf(-expf(x[e]));
+        for (int e = 0; e < 8; ++e) x[e] = decay(x[e]);
     } else {
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
@@ -521,6 +551,7 @@ __global__ void __launch_bounds__(NTHR, 1)
     const int m0 = 16 * (w >> 2), n0 = 16 * (w & 3);
     const long tstride = static_cast<long>(H) * D, hoff = static_cast<long>(blockIdx.y) * D;
 
+    prefetch_ahead<WT>(r, wl, k, v, a, b, dy, B, T, H, offs, 148);
     stage_chunk<WT>(GAM, AT, RT, BT, KT, VV, DY, sm.GL, sm.seg, r, wl, k, v, a, b, dy, lc.row0, lc.nv, tstride, hoff);
     if (tid < 64 && !(sm.GL[tid] >= kMinGammaL)) report_status(status, WKV7_ERR_DECAY_RANGE);
     masks_abk(AT, RT, BT, KT, NAB, NAK, MRB, m0, n0, gq, t4);
@@ -594,11 +625,12 @@ __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commi
 template <int N>
 __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
 
-// row-major 64 x 64 fp32 matrix (global) -> tile in the sx layout, 8 16-byte pieces per thread
+// row-major 64 x 64 fp32 matrix (global) -> tile in the sx layout, by a block of NT threads
+template <int NT>
 __device__ __forceinline__ void tile_async(float* tile, const float* g) {
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-        const int q = threadIdx.x + SCAN_THR * i, row = q >> 4, col = (q & 15) << 2;
+    for (int i = 0; i < 1024 / NT; ++i) {
+        const int q = threadIdx.x + NT * i, row = q >> 4, col = (q & 15) << 2;
         cp_async16(tile + sx(row, col), g + row * 64 + col);
     }
 }
@@ -672,8 +704,8 @@ __global__ void __launch_bounds__(SCAN_THR)
         if (s < nch) {
             const long c = chunk_of(s);
             float* stage = scan_smem + 2 * (s % SCAN_STAGES) * TILE;
-            tile_async(stage, Mb + c * SQ);
-            tile_async(stage + TILE, addb + c * SQ);
+            tile_async<SCAN_THR>(stage, Mb + c * SQ);
+            tile_async<SCAN_THR>(stage + TILE, addb + c * SQ);
         }
         cp_async_commit();
     };
@@ -769,23 +801,31 @@ __global__ void __launch_bounds__(NTHR, 1)
     const int m0 = 16 * (w >> 2), n0 = 16 * (w & 3);
     const long tstride = static_cast<long>(H) * D, hoff = static_cast<long>(blockIdx.y) * D;
     const int nv = lc.nv;
-
-    stage_chunk<WT>(GAM, AT, RT, BT, KT, VV, DY, sm.GL, sm.seg, r, wl, k, v, a, b, dy, lc.row0, nv, tstride, hoff);
     {
-        // S0 and dSLg = dS_L diag(Gamma_L) as tiles; column sums of dS_L (.) S_L
+        // S0 -> S0, dS_L -> DS, S_L -> W3 (free until the inverse), in flight during the staging
         const float* S0g = ws + lc.region + static_cast<long>(3 * (lc.nch + 1) + lc.c) * SQ;
-        const float* SLg = S0g + SQ;
         const float* dSg = ws + lc.region + static_cast<long>(lc.nch + 1 + lc.c) * SQ;
+        tile_async<NTHR>(S0, S0g);
+        tile_async<NTHR>(DS, dSg);
+        tile_async<NTHR>(W3, S0g + SQ);
+        cp_async_commit();
+    }
+    prefetch_ahead<WT>(r, wl, k, v, a, b, dy, B, T, H, offs, 148);
+    stage_chunk<WT>(GAM, AT, RT, BT, KT, VV, DY, sm.GL, sm.seg, r, wl, k, v, a, b, dy, lc.row0, nv, tstride, hoff);
+    cp_async_wait<0>();
+    __syncthreads();
+    {
+        // S0 tf32-rounded and dSLg = dS_L diag(Gamma_L) in place; column sums of dS_L (.) S_L
         const int j = tid & 63, s = tid >> 6;
         const float gl = sm.GL[j];
         float cs = 0.f;
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
-            const int row = 8 * s + i;
-            const float d = dSg[row * 64 + j];
-            cs = fmaf(d, SLg[row * 64 + j], cs);
-            S0[sx(row, j)] = round_tf32(S0g[row * 64 + j]);
-            DS[sx(row, j)] = round_tf32(d * gl);
+            const int ix = sx(8 * s + i, j);
+            const float d = DS[ix];
+            cs = fmaf(d, W3[ix], cs);
+            S0[ix] = round_tf32(S0[ix]);
+            DS[ix] = round_tf32(d * gl);
         }
         sm.seg[s * 64 + j] = cs;
     }
@@ -874,7 +914,19 @@ __global__ void __launch_bounds__(NTHR, 1)
     gemm16<true, false>(gB, W1, m0, m0, RT, m0, n0, (64 - m0) / 8, gq, t4);  // dMrb^T Rt
     gemm16<true, false>(gK, W2, m0, m0, RT, m0, n0, (64 - m0) / 8, gq, t4);  // dMrk^T Rt
     __syncthreads();
-    // da, dr, db, dk; the terms of d log w: W1 = da (.) a, W2 = dr (.) r - db (.) b - dk (.) k
+    // d log w needs exp(w_log) of this thread's column j and tokens 8 s .. 8 s + 7 at the end:
+    // load them now, behind the element-wise work
+    const int jc = tid & 63, sc = tid >> 6;
+    float el[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        const int t = 8 * sc + i;
+        el[i] = t < nv ? to_f32(wl[(lc.row0 + t) * tstride + hoff + jc]) : 0.f;
+    }
+    // da, dr, db, dk -> bf16 rows in OB (the dead S0 and DS tiles: 4 x 64 rows of 128 bytes, 32-bit
+    // words XOR-permuted by 4 (row mod 8)); the terms of d log w: W1 = da (.) a,
+    // W2 = dr (.) r - db (.) b - dk (.) k
+    uint32_t* OB = reinterpret_cast<uint32_t*>(S0);
 #pragma unroll
     for (int e = 0; e < 8; e += 2) {
         const int row = m0 + frag_row(e, gq), col = n0 + frag_col(e, t4);
@@ -891,19 +943,27 @@ __global__ void __launch_bounds__(NTHR, 1)
             W1[ix] = xa * AT[ix];
             W2[ix] = xr * RT[ix] - xb * BT[ix] - xk * KT[ix];
         }
-        if (row < nv) {
-            const long off = (lc.row0 + row) * tstride + hoff + col;
-            st_pair(da, off, o[0][0], o[0][1]);
-            st_pair(dr, off, o[1][0], o[1][1]);
-            st_pair(db, off, o[2][0], o[2][1]);
-            st_pair(dk, off, o[3][0], o[3][1]);
-        }
+        const int word = (row << 5) + ((col >> 1) ^ ((row & 7) << 2));
+#pragma unroll
+        for (int q = 0; q < 4; ++q) OB[q * 2048 + word] = pack_bf16x2(o[q][0], o[q][1]);
     }
     __syncthreads();
     {
+        // coalesced copy-out: 4 tensors x 64 rows x 8 pieces of 16 bytes
+        __nv_bfloat16* const dst[4] = {da, dr, db, dk};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const int q = tid + NTHR * i, tsr = q >> 9, row = (q >> 3) & 63, pc = q & 7;
+            if (row < nv) {
+                const uint4 x = *reinterpret_cast<const uint4*>(OB + tsr * 2048 + (row << 5) + ((4 * pc) ^ ((row & 7) << 2)));
+                *reinterpret_cast<uint4*>(dst[tsr] + (lc.row0 + row) * tstride + hoff + 8 * pc) = x;
+            }
+        }
+    }
+    {
         // d log w_s = sum_{t >= s} g_t with g_t = W2[t] + W1[t + 1] (t < 63) and
         // g_63 = W2[63] + colsum(dS_L (.) S_L): thread (column j, tokens 8 s .. 8 s + 7)
-        const int j = tid & 63, s = tid >> 6;
+        const int j = jc, s = sc;
         float x[8], run = 0.f;
 #pragma unroll
         for (int i = 7; i >= 0; --i) {
@@ -920,8 +980,7 @@ __global__ void __launch_bounds__(NTHR, 1)
             const int t = 8 * s + i;
             if (t < nv) {
                 const long off = (lc.row0 + t) * tstride + hoff + j;
-                const float el = expf(to_f32(wl[off]));
-                dwl[off] = from_f32<WT>(-(x[i] + later) * el);
+                dwl[off] = from_f32<WT>(-(x[i] + later) * exp_l(el[i]));
             }
         }
     }
