@@ -89,3 +89,48 @@ def test_backward_zero_tokens(wk):
     assert torch.equal(got[6].cpu(), dsT)
     got = wk.backward(r, wl, r, r, r, r, r)
     assert torch.count_nonzero(got[6]).item() == 0
+
+
+def _constant_decay(inp, value):
+    """The same inputs with every decay logit set to `value` (pad tokens of a
+    packed batch keep their -inf)."""
+    w = inp.w_log
+    pad = torch.isneginf(w.float())
+    inp.w_log = torch.where(pad, w, torch.full_like(w, value)).contiguous()
+    return inp
+
+
+@pytest.mark.parametrize("wdt", ["f32", "bf16"])
+def test_backward_decay_at_the_bound(wk, oracle_mod, wdt):
+    """w_log = -0.5 on every token (w = 0.545): a 64-token chunk decays by e^-38.8,
+    the extreme the chunked form's 1 / Gamma scaling carries through every product
+    of the adjoint.  Four chunks, the last ragged, non-zero initial state and dsT."""
+    inp = _constant_decay(W.make_prefill(2, 200, 3, io="bf16", wdt=wdt, s0_std=0.1, seed=130), -0.5)
+    check(wk, oracle_mod, inp, seed=131)
+
+
+def test_backward_decay_bound_packed_with_pads(wk, oracle_mod):
+    """The bound on every real token of a packed batch whose pads carry -inf (w = 1)."""
+    inp = _constant_decay(W.make_packed([150, 64, 7, 130], [13, 63, 0, 40], 3, io="bf16", wdt="f32",
+                                        s0_std=0.1, seed=132), -0.5)
+    check(wk, oracle_mod, inp, seed=133)
+
+
+def test_backward_decay_beyond_exact_range_is_reported(wk):
+    """w_log = 1 (w = e^-e): Gamma of a 64-token chunk falls below 1e-30, outside the
+    chunked form's exact range; the backward of bf16 inputs reports
+    WKV7_ERR_DECAY_RANGE (-8) like the prefill, instead of returning inf or NaN
+    with status OK."""
+    inp = _constant_decay(W.make_prefill(1, 130, 2, io="bf16", wdt="f32", s0_std=0.1, seed=134), 1.0)
+    dy, dsT = W.make_upstream(inp.r.shape, inp.B, inp.H, io=inp.io, seed=135)
+    d = {n: x.cuda() for n, x in inp.tensors().items()}
+    wk.backward(d["r"], d["w_log"], d["k"], d["v"], d["a"], d["b"], dy.cuda(), inp.s0.cuda(), dsT.cuda())
+    assert wk.wkv7_get_device_status() == -8
+    assert wk.wkv7_get_device_status() == 0  # read and cleared
+
+
+def test_backward_long_sequence(wk, oracle_mod):
+    """B1 T4096 H2: 64 chunks, so both boundary scans run 64 steps; their fp32
+    accuracy (tf32 high and low parts of the carried state) keeps the first
+    chunk's gradients and ds0 within the bound."""
+    check(wk, oracle_mod, W.make_prefill(1, 4096, 2, io="bf16", wdt="f32", s0_std=0.1, seed=136), seed=137)
