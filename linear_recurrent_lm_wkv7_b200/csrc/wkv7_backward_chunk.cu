@@ -319,25 +319,28 @@ __device__ __forceinline__ void prefetch_ahead(const __nv_bfloat16* r, const WT*
 // Stages the chunk's inputs of one head as fp32 tiles: GAM = Gamma (running
 // products of w = exp(-exp(w_log)) down the tokens), AT, RT, BT, KT (the scaled
 // operands, tf32-rounded), VV and DY (bf16 values, exact in tf32); GL = Gamma_L.
-// Rows t >= nv are identity steps (w = 1, every other input 0).  seg: 8 x 64
-// floats of scratch.  Ends with a block barrier.
+// Rows t >= nv are identity steps (w = 1, every other input 0).  The inputs are
+// read from rows 0 .. nv - 1 of r .. dy (each pointing at the chunk's first token
+// row of this head) with a row stride of rs elements: the tensors in global
+// memory, or copies of the rows in shared memory.  seg: 8 x 64 floats of
+// scratch.  Ends with a block barrier.
 template <typename WT>
 __device__ void stage_chunk(float* GAM, float* AT, float* RT, float* BT, float* KT, float* VV, float* DY, float* GL,
                             float* seg, const __nv_bfloat16* r, const WT* wl, const __nv_bfloat16* k,
                             const __nv_bfloat16* v, const __nv_bfloat16* a, const __nv_bfloat16* b,
-                            const __nv_bfloat16* dy, long row0, int nv, long tstride, long hoff) {
+                            const __nv_bfloat16* dy, long rs, int nv) {
     const int tid = threadIdx.x;
     const int t = tid >> 3, c0 = 8 * (tid & 7);
     float rr[8], kk[8], aa[8], bb[8], x[8];
     if (t < nv) {
-        const long off = (row0 + t) * tstride + hoff + c0;
-        unpack8(__ldg(reinterpret_cast<const uint4*>(r + off)), rr);
-        unpack8(__ldg(reinterpret_cast<const uint4*>(k + off)), kk);
-        unpack8(__ldg(reinterpret_cast<const uint4*>(a + off)), aa);
-        unpack8(__ldg(reinterpret_cast<const uint4*>(b + off)), bb);
-        unpack8(__ldg(reinterpret_cast<const uint4*>(v + off)), x);
+        const long off = t * rs + c0;
+        unpack8(*reinterpret_cast<const uint4*>(r + off), rr);
+        unpack8(*reinterpret_cast<const uint4*>(k + off), kk);
+        unpack8(*reinterpret_cast<const uint4*>(a + off), aa);
+        unpack8(*reinterpret_cast<const uint4*>(b + off), bb);
+        unpack8(*reinterpret_cast<const uint4*>(v + off), x);
         st8(VV, t, c0, x, false);
-        unpack8(__ldg(reinterpret_cast<const uint4*>(dy + off)), x);
+        unpack8(*reinterpret_cast<const uint4*>(dy + off), x);
         st8(DY, t, c0, x, false);
         ld_wlog8(wl + off, x);
 #pragma unroll
@@ -477,7 +480,7 @@ __device__ void invert_unit_lower(const float* N, float* Tm) {
 // 64 column sums, the chunk's location
 constexpr int N_TILES = 13;
 constexpr size_t SMEM_BYTES =
-    sizeof(float) * (N_TILES * TILE + 64 + 8 * 64 + 64) + sizeof(ChunkLoc) + 16;
+    sizeof(float) * (N_TILES * TILE + 64 + 8 * 64 + 64) + 2 * sizeof(ChunkLoc) + 16;
 
 struct Smem {
     float* tile[N_TILES];
@@ -494,8 +497,8 @@ __device__ __forceinline__ Smem carve(float* smf) {
     s.GL = smf + N_TILES * TILE;
     s.seg = s.GL + 64;
     s.csum = s.seg + 8 * 64;
-    s.loc = reinterpret_cast<ChunkLoc*>(s.csum + 64);
-    s.ok = reinterpret_cast<int*>(s.loc + 1);
+    s.loc = reinterpret_cast<ChunkLoc*>(s.csum + 64);  // two slots (the map kernel's current and next chunk)
+    s.ok = reinterpret_cast<int*>(s.loc + 2);
     return s;
 }
 
@@ -507,6 +510,13 @@ __device__ __forceinline__ void st16_global(float* G, const float (&acc)[8], int
         *reinterpret_cast<float2*>(G + row * 64 + col) = make_float2(acc[e], acc[e + 1]);
     }
 }
+
+__device__ __forceinline__ void cp_async16(void* dst, const void* src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
 
 // Nab = tril(At Bt^T, -1), Nak = tril(At Kt^T, -1), Mrb = tril(Rt Bt^T) (each warp its
 // block of all three; blocks above the diagonal are zero)
@@ -532,7 +542,41 @@ __device__ __forceinline__ void masks_abk(const float* AT, const float* RT, cons
 
 enum { T_GAM = 0, T_AT, T_RT, T_BT, T_KT, T_VV, T_DY, T_X0, T_X1, T_X2, T_X3, T_X4, T_X5 };
 
-// ---- 1. the chunk's maps M, Q, Qf
+// Raw input rows of one chunk and head into shared memory (per-thread 16-byte
+// cp.async): rows 0 .. nv - 1 of r, k, a, b, v, dy (bf16, 128 bytes each) into
+// two 16 KB tiles' worth of row-major buffers R2 = [r | k], A2 = [a | b],
+// V2 = [v | dy], and the w_log rows (64 or 128 bytes) into W1.  One commit group.
+template <typename WT>
+__device__ __forceinline__ void issue_raw(float* R2, float* A2, float* V2, float* W1, const __nv_bfloat16* r,
+                                          const WT* wl, const __nv_bfloat16* k, const __nv_bfloat16* v,
+                                          const __nv_bfloat16* a, const __nv_bfloat16* b, const __nv_bfloat16* dy,
+                                          long o, long tstride, int nv) {
+    const int tid = threadIdx.x, t = tid >> 3, pc = tid & 7;  // 64 rows x 8 pieces of 16 bytes
+    if (t < nv) {
+        const long go = o + t * tstride + 8 * pc;
+        __nv_bfloat16* rr = reinterpret_cast<__nv_bfloat16*>(R2);
+        __nv_bfloat16* aa = reinterpret_cast<__nv_bfloat16*>(A2);
+        __nv_bfloat16* vv = reinterpret_cast<__nv_bfloat16*>(V2);
+        const int so = t * 64 + 8 * pc;
+        cp_async16(rr + so, r + go);
+        cp_async16(rr + 4096 + so, k + go);
+        cp_async16(aa + so, a + go);
+        cp_async16(aa + 4096 + so, b + go);
+        cp_async16(vv + so, v + go);
+        cp_async16(vv + 4096 + so, dy + go);
+        WT* ww = reinterpret_cast<WT*>(W1);
+        constexpr int PER_ROW = 64 * sizeof(WT) / 16;  // 16-byte pieces per w_log row
+#pragma unroll
+        for (int q = pc; q < PER_ROW; q += 8) cp_async16(ww + t * 64 + q * (16 / sizeof(WT)), wl + o + t * tstride + q * (16 / sizeof(WT)));
+    }
+    cp_async_commit();
+}
+
+// ---- 1. the chunk's maps M, Q, Qf.  A persistent grid walks over the
+// (chunk, head) items; while an item's last products run, the raw rows of the
+// block's next item are copied into four tiles that are dead by then (NAK,
+// MRB, TA, TB), so the next staging reads shared memory instead of waiting for
+// global loads.
 template <typename WT>
 __global__ void __launch_bounds__(NTHR, 1)
     bwd_map_kernel(const __nv_bfloat16* __restrict__ r, const WT* __restrict__ wl, const __nv_bfloat16* __restrict__ k,
@@ -541,68 +585,110 @@ __global__ void __launch_bounds__(NTHR, 1)
                    int B, int T, int H, const int32_t* __restrict__ offs, long ckpt_chunks, int* status) {
     extern __shared__ __align__(16) float smf[];
     const Smem sm = carve(smf);
-    ChunkLoc lc;
-    if (!locate_block_chunk(B, T, H, offs, ckpt_chunks, status, lc, sm.loc, sm.ok)) return;
     float *GAM = sm.tile[T_GAM], *AT = sm.tile[T_AT], *RT = sm.tile[T_RT], *BT = sm.tile[T_BT], *KT = sm.tile[T_KT];
     float *VV = sm.tile[T_VV], *DY = sm.tile[T_DY];
     float *NAB = sm.tile[T_X0], *NAK = sm.tile[T_X1], *MRB = sm.tile[T_X2], *TT = sm.tile[T_X3];
     float *TA = sm.tile[T_X4], *TB = sm.tile[T_X5];
     const int tid = threadIdx.x, w = tid >> 5, gq = (tid & 31) >> 2, t4 = tid & 3;
     const int m0 = 16 * (w >> 2), n0 = 16 * (w & 3);
-    const long tstride = static_cast<long>(H) * D, hoff = static_cast<long>(blockIdx.y) * D;
+    const long tstride = static_cast<long>(H) * D;
+    const long n_items = ckpt_chunks * H;  // item = h * ckpt_chunks + chunk
+    const __nv_bfloat16* raw = reinterpret_cast<const __nv_bfloat16*>(NAK);  // [r | k], then [a | b] in MRB ...
+    const __nv_bfloat16* rawa = reinterpret_cast<const __nv_bfloat16*>(MRB);
+    const __nv_bfloat16* rawv = reinterpret_cast<const __nv_bfloat16*>(TA);
+    const WT* raww = reinterpret_cast<const WT*>(TB);
+    auto locate_item = [&](long item, int slot) {  // thread 0
+        ChunkLoc x{};
+        const bool ok = item < n_items &&
+                        locate_chunk(item % ckpt_chunks, static_cast<int>(item / ckpt_chunks), B, T, H, offs,
+                                     ckpt_chunks, status, x);
+        sm.loc[slot] = x;
+        sm.ok[slot] = ok ? 1 : 0;
+    };
+    auto head_of = [&](long item) { return static_cast<long>(item / ckpt_chunks) * D; };
 
-    prefetch_ahead<WT>(r, wl, k, v, a, b, dy, B, T, H, offs, 148);
-    stage_chunk<WT>(GAM, AT, RT, BT, KT, VV, DY, sm.GL, sm.seg, r, wl, k, v, a, b, dy, lc.row0, lc.nv, tstride, hoff);
-    if (tid < 64 && !(sm.GL[tid] >= kMinGammaL)) report_status(status, WKV7_ERR_DECAY_RANGE);
-    masks_abk(AT, RT, BT, KT, NAB, NAK, MRB, m0, n0, gq, t4);
+    long item = blockIdx.x;
+    int cur = 0;
+    if (tid == 0) locate_item(item, 0);
     __syncthreads();
-    invert_unit_lower(NAB, TT);
-    {
-        float acc[8];
-        zero8(acc);  // TA = T At (T is zero right of its diagonal)
-        gemm16<false, false>(acc, TT, m0, 0, AT, 0, n0, (m0 + 16) / 8, gq, t4);
-        st16<0>(TA, acc, m0, n0, gq, t4);
-        zero8(acc);  // TB = T^T Bt (T^T is zero left of its diagonal)
-        gemm16<true, false>(acc, TT, m0, m0, BT, m0, n0, (64 - m0) / 8, gq, t4);
-        st16<0>(TB, acc, m0, n0, gq, t4);
-    }
-    __syncthreads();
-    float* Mg = ws + lc.region + static_cast<long>(lc.c) * SQ;
-    float* Qg = ws + lc.region + static_cast<long>(lc.nch + 1 + lc.c) * SQ;
-    float* Qfg = ws + lc.region + static_cast<long>(2 * (lc.nch + 1) + lc.c) * SQ;
-    {
-        float acc[8];
-        zero8(acc);  // M = diag(Gamma_L) (I + Bt^T TA)
-        gemm16<true, false>(acc, BT, m0, 0, TA, 0, n0, 8, gq, t4);
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-            const int row = m0 + frag_row(e, gq), col = n0 + frag_col(e, t4);
-            acc[e] = round_tf32(sm.GL[row] * (acc[e] + (row == col ? 1.f : 0.f)));  // a tf32 operand of the scan
+    if (sm.ok[0])
+        issue_raw<WT>(NAK, MRB, TA, TB, r, wl, k, v, a, b, dy, sm.loc[0].row0 * tstride + head_of(item), tstride,
+                      sm.loc[0].nv);
+    else
+        cp_async_commit();
+    for (; item < n_items; item += gridDim.x, cur ^= 1) {
+        const long next = item + gridDim.x;
+        if (tid == 0) locate_item(next, cur ^ 1);  // read by every thread after the barriers below
+        cp_async_wait<0>();
+        __syncthreads();  // this item's raw rows have landed; the previous item's products are done
+        const ChunkLoc lc = sm.loc[cur];
+        const bool ok = sm.ok[cur] != 0;
+        auto prefetch_next = [&]() {
+            if (sm.ok[cur ^ 1])
+                issue_raw<WT>(NAK, MRB, TA, TB, r, wl, k, v, a, b, dy,
+                              sm.loc[cur ^ 1].row0 * tstride + head_of(next), tstride, sm.loc[cur ^ 1].nv);
+            else
+                cp_async_commit();
+        };
+        if (!ok) {
+            prefetch_next();
+            continue;
         }
-        st16_global(Mg, acc, m0, n0, gq, t4);
-        zero8(acc);  // W = Rt + Mrb TA -> NAB
-        gemm16<false, false>(acc, MRB, m0, 0, TA, 0, n0, (m0 + 16) / 8, gq, t4);
+        stage_chunk<WT>(GAM, AT, RT, BT, KT, VV, DY, sm.GL, sm.seg, raw, raww, raw + 4096, rawv, rawa, rawa + 4096,
+                        rawv + 4096, 64, lc.nv);
+        if (tid < 64 && !(sm.GL[tid] >= kMinGammaL)) report_status(status, WKV7_ERR_DECAY_RANGE);
+        masks_abk(AT, RT, BT, KT, NAB, NAK, MRB, m0, n0, gq, t4);
+        __syncthreads();
+        invert_unit_lower(NAB, TT);
+        {
+            float acc[8];
+            zero8(acc);  // TA = T At (T is zero right of its diagonal)
+            gemm16<false, false>(acc, TT, m0, 0, AT, 0, n0, (m0 + 16) / 8, gq, t4);
+            st16<0>(TA, acc, m0, n0, gq, t4);
+            zero8(acc);  // TB = T^T Bt (T^T is zero left of its diagonal)
+            gemm16<true, false>(acc, TT, m0, m0, BT, m0, n0, (64 - m0) / 8, gq, t4);
+            st16<0>(TB, acc, m0, n0, gq, t4);
+        }
+        __syncthreads();
+        float* Mg = ws + lc.region + static_cast<long>(lc.c) * SQ;
+        float* Qg = ws + lc.region + static_cast<long>(lc.nch + 1 + lc.c) * SQ;
+        float* Qfg = ws + lc.region + static_cast<long>(2 * (lc.nch + 1) + lc.c) * SQ;
+        {
+            float acc[8];
+            zero8(acc);  // M = diag(Gamma_L) (I + Bt^T TA)
+            gemm16<true, false>(acc, BT, m0, 0, TA, 0, n0, 8, gq, t4);
 #pragma unroll
-        for (int e = 0; e < 8; ++e) acc[e] += RT[sx(m0 + frag_row(e, gq), n0 + frag_col(e, t4))];
-        st16<0>(NAB, acc, m0, n0, gq, t4);
-        zero8(acc);  // Z = Kt + Nak^T TB -> TT
-        gemm16<true, false>(acc, NAK, m0, m0, TB, m0, n0, (64 - m0) / 8, gq, t4);
+            for (int e = 0; e < 8; ++e) {
+                const int row = m0 + frag_row(e, gq), col = n0 + frag_col(e, t4);
+                acc[e] = round_tf32(sm.GL[row] * (acc[e] + (row == col ? 1.f : 0.f)));  // a tf32 operand of the scan
+            }
+            st16_global(Mg, acc, m0, n0, gq, t4);
+            zero8(acc);  // W = Rt + Mrb TA -> NAB
+            gemm16<false, false>(acc, MRB, m0, 0, TA, 0, n0, (m0 + 16) / 8, gq, t4);
 #pragma unroll
-        for (int e = 0; e < 8; ++e) acc[e] += KT[sx(m0 + frag_row(e, gq), n0 + frag_col(e, t4))];
-        st16<0>(TT, acc, m0, n0, gq, t4);
+            for (int e = 0; e < 8; ++e) acc[e] += RT[sx(m0 + frag_row(e, gq), n0 + frag_col(e, t4))];
+            st16<0>(NAB, acc, m0, n0, gq, t4);
+            zero8(acc);  // Z = Kt + Nak^T TB -> TT
+            gemm16<true, false>(acc, NAK, m0, m0, TB, m0, n0, (64 - m0) / 8, gq, t4);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) acc[e] += KT[sx(m0 + frag_row(e, gq), n0 + frag_col(e, t4))];
+            st16<0>(TT, acc, m0, n0, gq, t4);
+        }
+        __syncthreads();
+        prefetch_next();  // NAK, MRB, TA and TB are dead: the next item's raw rows go there
+        {
+            float acc[8];
+            zero8(acc);  // Q = dY^T W
+            gemm16<true, false>(acc, DY, m0, 0, NAB, 0, n0, 8, gq, t4);
+            st16_global(Qg, acc, m0, n0, gq, t4);
+            zero8(acc);  // Qf = V^T Z diag(Gamma_L)
+            gemm16<true, false>(acc, VV, m0, 0, TT, 0, n0, 8, gq, t4);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) acc[e] *= sm.GL[n0 + frag_col(e, t4)];
+            st16_global(Qfg, acc, m0, n0, gq, t4);
+        }
     }
-    __syncthreads();
-    {
-        float acc[8];
-        zero8(acc);  // Q = dY^T W
-        gemm16<true, false>(acc, DY, m0, 0, NAB, 0, n0, 8, gq, t4);
-        st16_global(Qg, acc, m0, n0, gq, t4);
-        zero8(acc);  // Qf = V^T Z diag(Gamma_L)
-        gemm16<true, false>(acc, VV, m0, 0, TT, 0, n0, 8, gq, t4);
-#pragma unroll
-        for (int e = 0; e < 8; ++e) acc[e] *= sm.GL[n0 + frag_col(e, t4)];
-        st16_global(Qfg, acc, m0, n0, gq, t4);
-    }
+    cp_async_wait<0>();  // nothing may still be landing when the block exits
 }
 
 // ---- 2. the scans over a unit's chunks: direction 0 runs S <- S M^T + Qf
@@ -618,12 +704,6 @@ __global__ void __launch_bounds__(NTHR, 1)
 // many chunks.
 constexpr int SCAN_THR = 128;
 
-__device__ __forceinline__ void cp_async16(float* dst, const float* src) {
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-template <int N>
-__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
 
 // row-major 64 x 64 fp32 matrix (global) -> tile in the sx layout, by a block of NT threads
 template <int NT>
@@ -811,7 +891,11 @@ __global__ void __launch_bounds__(NTHR, 1)
         cp_async_commit();
     }
     prefetch_ahead<WT>(r, wl, k, v, a, b, dy, B, T, H, offs, 148);
-    stage_chunk<WT>(GAM, AT, RT, BT, KT, VV, DY, sm.GL, sm.seg, r, wl, k, v, a, b, dy, lc.row0, nv, tstride, hoff);
+    {
+        const long o = lc.row0 * tstride + hoff;
+        stage_chunk<WT>(GAM, AT, RT, BT, KT, VV, DY, sm.GL, sm.seg, r + o, wl + o, k + o, v + o, a + o, b + o, dy + o,
+                        tstride, nv);
+    }
     cp_async_wait<0>();
     __syncthreads();
     {
@@ -1001,7 +1085,14 @@ cudaError_t launch_chunked_typed(const BackwardArgs& p, cudaStream_t stream) {
     const WT* wl = static_cast<const WT*>(p.w_log);
     const dim3 cgrid(static_cast<unsigned>(p.ckpt_chunks), static_cast<unsigned>(p.H));
     if (p.ckpt_chunks > 0) {
-        map<<<cgrid, NTHR, SMEM_BYTES, stream>>>(r, wl, k, v, a, b, dy, p.ws, p.B, p.T, p.H, p.seq_offsets,
+        int dev = 0, sms = 0;
+        e = cudaGetDevice(&dev);
+        if (e != cudaSuccess) return e;
+        e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+        if (e != cudaSuccess) return e;
+        const long items = p.ckpt_chunks * p.H;
+        const unsigned mgrid = static_cast<unsigned>(items < sms ? items : sms);
+        map<<<mgrid, NTHR, SMEM_BYTES, stream>>>(r, wl, k, v, a, b, dy, p.ws, p.B, p.T, p.H, p.seq_offsets,
                                                  p.ckpt_chunks, p.status);
         e = cudaGetLastError();
         if (e != cudaSuccess) return e;
