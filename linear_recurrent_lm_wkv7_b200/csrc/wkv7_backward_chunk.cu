@@ -25,7 +25,7 @@
 //   Qf = V^T (Kt + Nak^T T^T Bt) diag(Gamma_L).
 //
 // Three launches:
-//   1. bwd_map_kernel, one block per (chunk, head): M, Q, Qf of the chunk;
+//   1. bwd_map_kernel, a persistent grid over the (chunk, head) items: M, Q, Qf of each chunk;
 //   2. bwd_scan_kernel, one block per (sequence, head) and direction: the forward
 //      scan S <- S M^T + Qf writes the state at every chunk boundary, the backward
 //      scan dS <- Q + dS M writes dS_L of every chunk and ds0 (fp32 CUDA cores);
