@@ -28,7 +28,8 @@
 //   1. bwd_map_kernel, a persistent grid over the (chunk, head) items: M, Q, Qf of each chunk;
 //   2. bwd_scan_kernel, one block per (sequence, head) and direction: the forward
 //      scan S <- S M^T + Qf writes the state at every chunk boundary, the backward
-//      scan dS <- Q + dS M writes dS_L of every chunk and ds0 (fp32 CUDA cores);
+//      scan dS <- Q + dS M writes dS_L of every chunk and ds0 (the carried state
+//      enters each product as tf32 high and low parts, which keeps fp32 accuracy);
 //   3. bwd_grad_kernel, one block per (chunk, head): every gradient of the chunk.
 // Products are warp-level tf32 tensor-core products (m16n8k8, fp32 accumulate)
 // on fp32 tiles in shared memory: 64 x 64 products chained through elementwise
