@@ -354,7 +354,9 @@ def run_ours(args):
                                "hbm_time_floor_us": lbytes / (hbm_peak * 1e9) * 1e6}}
     del ld_, linp, ls0
     # ---------------- packed variable-length prefill: 16 sequences, lengths U{512..8192}, pads U{0..63}
-    pinp = W.make_workload("packed_1p5b", seed=4 + 1000 * rank)
+    # the same packed draw on every rank: the lengths (and so the real-token count and the bytes)
+    # are equal across ranks, so world x tokens is the job's count
+    pinp = W.make_workload("packed_1p5b", seed=4)
     packed_section = prefill_section("packed_1p5b", pinp, "16 sequences, pads U{0..63} (w = 1, k = v = a = b = 0)",
                                      "N(0, 0.1^2)")
     del pinp
