@@ -134,3 +134,26 @@ def test_backward_long_sequence(wk, oracle_mod):
     accuracy (tf32 high and low parts of the carried state) keeps the first
     chunk's gradients and ds0 within the bound."""
     check(wk, oracle_mod, W.make_prefill(1, 4096, 2, io="bf16", wdt="f32", s0_std=0.1, seed=136), seed=137)
+
+
+def test_backward_many_short_packed(wk, oracle_mod):
+    """40 packed sequences of 1 .. 70 tokens with pads: the persistent map kernel's
+    items include chunk slots past the last real chunk (the packed workspace bound
+    is ceil(T / 64) + B chunks per head), and most sequences are one ragged chunk."""
+    g = torch.Generator().manual_seed(140)
+    lengths = torch.randint(1, 71, (40,), generator=g).tolist()
+    pads = torch.randint(0, 4, (40,), generator=g).tolist()
+    check(wk, oracle_mod, W.make_packed(lengths, pads, 2, io="bf16", wdt="f32", s0_std=0.1, seed=141), seed=142)
+
+
+def test_backward_is_deterministic(wk):
+    """No atomics anywhere: two calls on the same inputs give the same bits."""
+    inp = W.make_prefill(2, 300, 3, io="bf16", wdt="f32", s0_std=0.1, seed=143)
+    dy, dsT = W.make_upstream(inp.r.shape, inp.B, inp.H, io=inp.io, seed=144)
+    d = {n: x.cuda() for n, x in inp.tensors().items()}
+    args = (d["r"], d["w_log"], d["k"], d["v"], d["a"], d["b"], dy.cuda(), inp.s0.cuda(), dsT.cuda())
+    first = wk.backward(*args)
+    second = wk.backward(*args)
+    assert wk.wkv7_get_device_status() == 0
+    for x, y in zip(first, second):
+        assert torch.equal(x, y)
