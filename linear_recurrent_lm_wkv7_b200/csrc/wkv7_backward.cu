@@ -1,4 +1,7 @@
-// wkv7_backward.cu — gradient of the WKV-7 recurrence (recurrent form).
+// wkv7_backward.cu — gradient of the WKV-7 recurrence in recurrent form, for fp32
+// inputs (fp32 arithmetic throughout, which their tighter bound needs; bf16 inputs
+// take the chunked form of wkv7_backward_chunk.cu).  Also the entry point's
+// workspace size and dispatch.
 //
 // For L = sum_t <dy_t, y_t> + <dsT, S_T> the chain rule through one step
 // S_t = S_{t-1} diag(w_t) + (S_{t-1} a_t) b_t^T + v_t k_t^T, y_t = S_t r_t gives,
@@ -19,7 +22,7 @@
 //      workspace (checkpoints);
 //   2. chunks in reverse: stage the chunk's inputs in shared memory (fp32),
 //      recompute its 64 states from the checkpoint into a per-unit scratch of
-//      the workspace (1 MB, mostly L2-resident), then sweep its tokens downwards.
+//      the workspace (1 MB), then sweep its tokens downwards.
 #include <cstdint>
 
 #include "wkv7_internal.cuh"
