@@ -128,6 +128,26 @@ __device__ __forceinline__ void load_v_tile(const float* __restrict__ v, long ro
     }
 }
 
+constexpr float kLog2e = 1.4426950408889634f;
+
+// L2 prefetch of the rows of one chunk (up to 64 tokens from row0, nrows of them):
+// thread tid takes token tid / 2 and one 128-byte half of each 256-byte fp32 row.
+template <typename IO, typename WT>
+__device__ __forceinline__ void prefetch_chunk_rows(const IO* r, const WT* wl, const IO* k, const IO* v, const IO* a,
+                                                    const IO* b, long row0, long nrows, long tstride, long hoff,
+                                                    long tstride_kv, long hoff_kv, int tid, bool pro) {
+    const int t = tid >> 1, half = tid & 1;
+    if (t >= nrows) return;
+    const long off = (row0 + t) * tstride + hoff + 32 * half;
+    const long offkv = (row0 + t) * tstride_kv + hoff_kv + 32 * half;
+    prefetch_line_l2(r + off);
+    prefetch_line_l2(a + off);
+    prefetch_line_l2(k + offkv);
+    prefetch_line_l2(v + offkv);
+    if (!pro) prefetch_line_l2(b + off);
+    prefetch_line_l2(wl + (row0 + t) * tstride + hoff + (sizeof(WT) == 4 ? 32 * half : 0));
+}
+
 template <typename IO, typename WT, bool TF32, bool PRO>
 __global__ void __launch_bounds__(NT, 1)
     wkv7_prefill_kernel(const IO* __restrict__ r, const WT* __restrict__ wl, const IO* __restrict__ k,
@@ -194,6 +214,7 @@ __global__ void __launch_bounds__(NT, 1)
         store_state_operand(sm.S, jj, S);
     }
 
+    if (nchunks > 0) prefetch_chunk_rows(r, wl, k, v, a, b, tb, len, tstride, hoff, tstride_kv, hoff_kv, tid, PRO);
     bool ok = true;
     uint32_t phase = 0;          // parity of the next MMA completion
     bool mma_pending = false;    // an MMA commit not yet waited for
@@ -201,20 +222,25 @@ __global__ void __launch_bounds__(NT, 1)
         const long row0 = tb + static_cast<long>(c) * L;  // first token of the chunk
         const int nv = static_cast<int>(len - static_cast<long>(c) * L < L ? len - static_cast<long>(c) * L : L);
 
+        // the next chunk's rows into L2 while this one is worked on (its loads then hit L2)
+        if (c + 1 < nchunks) prefetch_chunk_rows(r, wl, k, v, a, b, row0 + L, len - static_cast<long>(c + 1) * L,
+                                                  tstride, hoff, tstride_kv, hoff_kv, tid, PRO);
         // ---- p1: decay products and scaled operand tiles.  Thread (j, half).
         {
             const int j = tid & 63, hf = tid >> 6;
             float cp[32];
             float prod = 1.f;
+            // every decay logit of the thread's 32 tokens is loaded before the first product
+            float lv[32];
 #pragma unroll
             for (int q = 0; q < 32; ++q) {
                 const int t = hf * 32 + q;
-                float w = 1.f;
-                if (t < nv) {
-                    const float l = to_f32(wl[(row0 + t) * tstride + hoff + j]);
-                    w = expf(-expf(l));
-                }
-                prod *= w;
+                lv[q] = t < nv ? to_f32(wl[(row0 + t) * tstride + hoff + j]) : -INFINITY;
+            }
+#pragma unroll
+            for (int q = 0; q < 32; ++q) {
+                // w = exp(-exp(l)) by the hardware 2^x (w_log = -inf gives w = 1 exactly)
+                prod *= ex2_ftz(-kLog2e * ex2_ftz(kLog2e * lv[q]));
                 cp[q] = prod;
             }
             sm.red[hf * 64 + j] = prod;
@@ -346,15 +372,17 @@ __global__ void __launch_bounds__(NT, 1)
             for (int t = 0; t < 64; ++t) {
                 float acc = col < 64 ? ld_op<TF32>(sm.RA, 128, 64 + t, col) : sm.MAK[t * NSTRIDE + (col - 64)];
                 const float* nrow = sm.NAB + t * NSTRIDE;
+                // four partial sums: a quarter of the dependent chain
+                float a1 = 0.f, a2 = 0.f, a3 = 0.f;
 #pragma unroll
                 for (int i = 0; i < t; i += 4) {
                     const float4 nv4 = *reinterpret_cast<const float4*>(nrow + i);
                     acc = fmaf(nv4.x, x[i], acc);
-                    acc = fmaf(nv4.y, x[i + 1], acc);
-                    acc = fmaf(nv4.z, x[i + 2], acc);
-                    acc = fmaf(nv4.w, x[i + 3], acc);
+                    a1 = fmaf(nv4.y, x[i + 1], a1);
+                    a2 = fmaf(nv4.z, x[i + 2], a2);
+                    a3 = fmaf(nv4.w, x[i + 3], a3);
                 }
-                x[t] = acc;
+                x[t] = (acc + a1) + (a2 + a3);
             }
             st_op_row32<TF32>(sm.WZ, 128, col, 0, x);
             st_op_row32<TF32>(sm.WZ, 128, col, 32, x + 32);
