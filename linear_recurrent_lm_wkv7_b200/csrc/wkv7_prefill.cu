@@ -68,6 +68,7 @@ struct Smem {
     uint8_t* AS;   // [R' ; Bh^T W]        128 x 64, K-major over key channels    (aliases NAB, MAK)
     uint8_t* V;    // V: 64 values x 64 tokens (K-major)
     uint8_t* S;    // S^T: 64 values x 64 keys (K-major)
+    float* XS;     // solver columns: XS[t][col], 64 tokens x 128 columns fp32
     float* gammaL; // Gamma_L per key channel
     float* red;    // per-half products of w (2 x 64), then (prologue) 1 / ||k_t|| per token (64)
     uint64_t* bar; // MMA completion barrier
@@ -80,8 +81,8 @@ __host__ __device__ constexpr uint32_t smem_bytes_needed() {
     using O = OpType<TF32>;
     constexpr uint32_t solver = 2u * 64u * NSTRIDE * 4u;
     constexpr uint32_t r4 = ((solver > O::TILE128 ? solver : O::TILE128) + 1023u) & ~1023u;
-    return 1024u /* alignment slack */ + 3u * O::TILE128 + O::TILE64 + r4 + 2u * O::TILE64 + 64u * 4u + 192u * 4u +
-           64u;
+    return 1024u /* alignment slack */ + 3u * O::TILE128 + O::TILE64 + r4 + 2u * O::TILE64 + 64u * NT * 4u +
+           64u * 4u + 192u * 4u + 64u;
 }
 
 template <bool TF32>
@@ -98,6 +99,7 @@ __device__ __forceinline__ Smem carve(uint8_t* raw) {
     s.NAB = reinterpret_cast<float*>(p); s.MAK = s.NAB + 64 * NSTRIDE; s.AS = p; p += r4;
     s.V = p; p += O::TILE64;
     s.S = p; p += O::TILE64;
+    s.XS = reinterpret_cast<float*>(p); p += 64 * NT * 4;
     s.gammaL = reinterpret_cast<float*>(p); p += 64 * 4;
     s.red = reinterpret_cast<float*>(p); p += 192 * 4;
     s.bar = reinterpret_cast<uint64_t*>(p); p += 8;
@@ -362,30 +364,49 @@ __global__ void __launch_bounds__(NT, 1)
         tc_fence_before();
         __syncthreads();
 
-        // ---- [W | Z] = (I - Nab)^{-1} [At | Mak]: forward substitution, column `tid`
+        // ---- [W | Z] = (I - Nab)^{-1} [At | Mak]: forward substitution, column `tid`, in blocks of
+        // four rows: the rows of a block accumulate their products with the solved rows above as
+        // four independent sums, then take the 4 x 4 triangle; the column lives in XS
         {
             const int col = tid;
-            float x[64];
+            float* xs = sm.XS;
+#pragma unroll 1
+            for (int t0 = 0; t0 < 64; t0 += 4) {
+                float acc[4];
 #pragma unroll
-            for (int t = 0; t < 64; ++t) x[t] = 0.f;
+                for (int q = 0; q < 4; ++q)
+                    acc[q] = col < 64 ? ld_op<TF32>(sm.RA, 128, 64 + t0 + q, col) : sm.MAK[(t0 + q) * NSTRIDE + (col - 64)];
+                const float* n0 = sm.NAB + t0 * NSTRIDE;  // rows t0 .. t0 + 3
+#pragma unroll 2
+                for (int i = 0; i < t0; i += 4) {
+                    const float x0 = xs[i * NT + col], x1 = xs[(i + 1) * NT + col];
+                    const float x2 = xs[(i + 2) * NT + col], x3 = xs[(i + 3) * NT + col];
 #pragma unroll
-            for (int t = 0; t < 64; ++t) {
-                float acc = col < 64 ? ld_op<TF32>(sm.RA, 128, 64 + t, col) : sm.MAK[t * NSTRIDE + (col - 64)];
-                const float* nrow = sm.NAB + t * NSTRIDE;
-                // four partial sums: a quarter of the dependent chain
-                float a1 = 0.f, a2 = 0.f, a3 = 0.f;
-#pragma unroll
-                for (int i = 0; i < t; i += 4) {
-                    const float4 nv4 = *reinterpret_cast<const float4*>(nrow + i);
-                    acc = fmaf(nv4.x, x[i], acc);
-                    a1 = fmaf(nv4.y, x[i + 1], a1);
-                    a2 = fmaf(nv4.z, x[i + 2], a2);
-                    a3 = fmaf(nv4.w, x[i + 3], a3);
+                    for (int q = 0; q < 4; ++q) {
+                        const float4 n4 = *reinterpret_cast<const float4*>(n0 + q * NSTRIDE + i);
+                        acc[q] = fmaf(n4.x, x0, acc[q]);
+                        acc[q] = fmaf(n4.y, x1, acc[q]);
+                        acc[q] = fmaf(n4.z, x2, acc[q]);
+                        acc[q] = fmaf(n4.w, x3, acc[q]);
+                    }
                 }
-                x[t] = (acc + a1) + (a2 + a3);
+                const float y0 = acc[0];
+                const float y1 = fmaf(n0[NSTRIDE + t0], y0, acc[1]);
+                const float y2 = fmaf(n0[2 * NSTRIDE + t0 + 1], y1, fmaf(n0[2 * NSTRIDE + t0], y0, acc[2]));
+                const float y3 = fmaf(n0[3 * NSTRIDE + t0 + 2], y2,
+                                      fmaf(n0[3 * NSTRIDE + t0 + 1], y1, fmaf(n0[3 * NSTRIDE + t0], y0, acc[3])));
+                xs[t0 * NT + col] = y0;
+                xs[(t0 + 1) * NT + col] = y1;
+                xs[(t0 + 2) * NT + col] = y2;
+                xs[(t0 + 3) * NT + col] = y3;
             }
-            st_op_row32<TF32>(sm.WZ, 128, col, 0, x);
-            st_op_row32<TF32>(sm.WZ, 128, col, 32, x + 32);
+#pragma unroll
+            for (int hlf = 0; hlf < 2; ++hlf) {
+                float x[32];
+#pragma unroll
+                for (int q = 0; q < 32; ++q) x[q] = xs[(32 * hlf + q) * NT + col];
+                st_op_row32<TF32>(sm.WZ, 128, col, 32 * hlf, x);
+            }
         }
         fence_proxy_async_smem();
         __syncthreads();
