@@ -239,15 +239,13 @@ int wkv7_decode_step_fused(const void* r, const void* w_log, const void* k, cons
  *          T < 0, H <= 0, D != 64).
  * Every output and the workspace must be disjoint from every input and from
  * each other.
- * bf16 inputs (io_dtype WKV7_BF16) take the chunked form: per 64-token chunk the
- * maps between the chunk's end and start state are formed in parallel, two scans
- * over the chunks give the state and its gradient at every chunk boundary, and
- * every chunk's gradients follow in parallel from the WY products of the chunk
- * (tf32 tensor-core products, fp32 accumulation).  Its decay range is the
- * prefill's: a chunk whose Gamma falls below 1e-30 sets WKV7_ERR_DECAY_RANGE.
- * fp32 inputs take the recurrent form: one block per (sequence, head) recomputes
- * the states of each chunk from checkpoints and sweeps the tokens backward in
- * fp32, with no range condition.
+ * Chunked form: per 64-token chunk the maps between the chunk's end and start
+ * state are formed in parallel, two scans over the chunks give the state and
+ * its gradient at every chunk boundary, and every chunk's gradients follow in
+ * parallel from the WY products of the chunk (tf32 tensor-core products, fp32
+ * accumulation; fp32 inputs enter as tf32 high and low parts, three products
+ * each, which keeps fp32 accuracy).  Its decay range is the prefill's: a chunk
+ * whose Gamma falls below 1e-30 sets WKV7_ERR_DECAY_RANGE.
  */
 size_t wkv7_backward_workspace_bytes(int B, int T, int H, int D, int packed);
 int wkv7_backward(const void* r, const void* w_log, const void* k, const void* v,
@@ -269,7 +267,7 @@ int wkv7_backward(const void* r, const void* w_log, const void* k, const void* v
  *   Limit: wkv7_backward_workspace_bytes(B, T, H, D, packed) must not exceed
  *   WKV7_NOALLOC_SCRATCH_BYTES (16 MiB); otherwise WKV7_ERR_SCRATCH_LIMIT is
  *   returned and nothing is launched.  (For example B = 2, H = 3 and T up to
- *   2624 tokens fit; use wkv7_backward for larger problems.)
+ *   3520 tokens fit; use wkv7_backward for larger problems.)
  *   Nothing in the scratch has to start at zero (every element is written
  *   before it is read), so the call clears nothing.
  *   There is one scratch per device: calls whose kernels may overlap on the

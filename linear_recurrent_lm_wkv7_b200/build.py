@@ -18,7 +18,7 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libwkv7.so")
 SOURCES = ["wkv7_api.cu", "wkv7_decode.cu", "wkv7_prefill.cu", "wkv7_prefill_pipe.cu", "wkv7_gate.cu",
-           "wkv7_backward.cu", "wkv7_backward_chunk.cu", "wkv7_noalloc.cu", "wkv7_state.cu"]
+           "wkv7_backward.cu", "wkv7_noalloc.cu", "wkv7_state.cu"]
 HEADERS = ["sm100_ptx.cuh", "wkv7_internal.cuh", "prefill_common.cuh", "tma_host.cuh"]
 
 

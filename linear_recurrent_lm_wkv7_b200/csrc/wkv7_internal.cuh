@@ -103,13 +103,10 @@ cudaError_t launch_state_apply(const float* S_in, const float* M, const float* Q
                                cudaStream_t stream);
 // M <- identity, Q <- 0 for n units (the map of an empty token range); either may be null
 cudaError_t launch_state_identity(float* M, float* Q, long n, cudaStream_t stream);
-// backward of the recurrence (wkv7_backward.cu)
+// backward of the recurrence in chunked form (wkv7_backward.cu)
 long backward_ckpt_chunks(int B, int T, int packed);
 size_t backward_workspace_floats(int B, int T, int H, int packed);
 cudaError_t launch_backward(const BackwardArgs& p, int io_dtype, int w_dtype, cudaStream_t stream);
-// chunked (WY) form for bf16 inputs (wkv7_backward_chunk.cu)
-size_t backward_chunked_workspace_floats(int B, int T, int H, int packed);
-cudaError_t launch_backward_chunked(const BackwardArgs& p, int w_dtype, cudaStream_t stream);
 
 // Raises `kern`'s dynamic shared-memory limit to `bytes` the first time it is
 // launched on the current device.  `configured` holds one bit per device

@@ -173,14 +173,13 @@ def _bwd(wk, B=1, T=8, H=1, D=64, offs=None, io=1, wd=0, wsb=None, **over):
 
 
 def test_backward_workspace_size(wk):
-    # the larger of the two forms' needs; a state is 64 x 64 fp32, C chunk slots per head
-    # (C = ceil(T / 64) per sequence dense, ceil(T / 64) + B packed):
-    #   recurrent: C checkpoints per head plus 64 states per unit
-    #   chunked:   4 (C + B) per head (M, Q, Qf and the boundary states, one spare slot each)
-    assert wk.wkv7_backward_workspace_bytes(2, 130, 3, 64, False) == (2 * 3 * 3 + 2 * 3 * 64) * 16384
-    assert wk.wkv7_backward_workspace_bytes(2, 130, 3, 64, True) == ((3 + 2) * 3 + 2 * 3 * 64) * 16384
-    assert wk.wkv7_backward_workspace_bytes(1, 16320, 1, 64, False) == 4 * (255 + 1) * 16384
-    assert wk.wkv7_backward_workspace_bytes(2, 8192, 3, 64, True) == 4 * 3 * (128 + 2 + 2) * 16384
+    # a state is 64 x 64 fp32; C chunk slots per head (C = ceil(T / 64) per sequence
+    # dense, ceil(T / 64) + B packed); 3 (C + B) states per head: M, Q and Qf, with
+    # the boundary states over Qf, one spare slot of each per sequence
+    assert wk.wkv7_backward_workspace_bytes(2, 130, 3, 64, False) == 3 * 3 * (6 + 2) * 16384
+    assert wk.wkv7_backward_workspace_bytes(2, 130, 3, 64, True) == 3 * 3 * (5 + 2) * 16384
+    assert wk.wkv7_backward_workspace_bytes(1, 21760, 1, 64, False) == 3 * (340 + 1) * 16384
+    assert wk.wkv7_backward_workspace_bytes(2, 8192, 3, 64, True) == 3 * 3 * (128 + 2 + 2) * 16384
     assert wk.wkv7_backward_workspace_bytes(2, 130, 3, 32, False) == 0
 
 

@@ -4,8 +4,8 @@ workspace.  Checked through the C ABI against wkv7_backward with a caller
 workspace: the same kernel on the same inputs, so the gradients must agree bit
 for bit (a race or a stale value in the shared scratch would show up as a
 difference).  Two calls in a row per case; a dense case, a packed case (whose
-checkpoint count is B + ceil(T/64) per head), and the largest problem that fits
-the 16 MiB scratch exactly.  One element more is refused on the host.
+chunk count is B + ceil(T/64) per head), and the longest sequence whose
+workspace fits the 16 MiB scratch.  One token more is refused on the host.
 
 This file sorts last so that a run stopping at its first failure has run every
 other test before it; it also passes on its own in a fresh process."""
@@ -65,11 +65,11 @@ def test_backward_noalloc_packed(wk):
 
 
 def test_backward_noalloc_at_the_limit(wk):
-    """B1 H1 T16320 (255 chunks): the chunked form's 4 x (255 + 1) states of
-    16 KiB fill the 16 MiB scratch exactly; T + 1 needs a chunk more and is
-    refused before anything is launched."""
-    B, T, H = 1, 16320, 1
-    assert wk.wkv7_backward_workspace_bytes(B, T, H, 64, False) == LIMIT
+    """B1 H1 T21760 (340 chunks), the longest sequence that fits: the chunked
+    form's 3 x (340 + 1) states of 16 KiB take 16 MiB less one state; T + 1
+    needs a chunk more (three states) and is refused before anything is launched."""
+    B, T, H = 1, 21760, 1
+    assert wk.wkv7_backward_workspace_bytes(B, T, H, 64, False) == LIMIT - 16384
     inp = W.make_prefill(B, T, H, io="bf16", wdt="f32", s0_std=0.1, seed=81)
     _run_both(wk, inp, seed=82)
 
