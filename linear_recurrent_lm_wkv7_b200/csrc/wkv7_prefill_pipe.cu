@@ -286,8 +286,6 @@ __global__ void __launch_bounds__(NTHR, 1)
     }
     const long tstride = static_cast<long>(H) * kHead;
     const long hoff = static_cast<long>(h) * kHead;
-    const long tstride_kv = static_cast<long>(PRO ? H_kv : H) * kHead;
-    const long hoff_kv = static_cast<long>(hk) * kHead;
     const long sbase = (static_cast<long>(n) * H + h) * kHead * kHead;
     const int nchunks = static_cast<int>((len + L - 1) / L);
 
@@ -587,15 +585,24 @@ __global__ void __launch_bounds__(NTHR, 1)
             {
                 const bool tok = tg < 64;
                 const int t = tok ? tg : tg - 64;
+                // gated read-out: u_t v_t joins y_t through the diagonal of Mrk, as 8 u_t (the
+                // serial group scales the row by 1 / sqrt(D) = 1 / 8)
+                float du = 0.f;
+                if constexpr (GATED)
+                    if (tok) du = 8.f * reinterpret_cast<const float*>(sm + OFF_U)[g * 128 + (kk_ & 1) * 64 + t];
 #pragma unroll 1
                 for (int qq = 0; qq < 4; ++qq) {
                     float x[32];
                     tmem_load32(tm_gp + lane_base + 32 * qq, x);
                     const int c0 = 32 * (qq & 1);
                     const int lim = t - c0 - (tok ? 0 : 1);  // columns c0 + i with i <= lim are kept
+                    const float dd = qq >= 2 ? du : 0.f;
 #pragma unroll
-                    for (int i = 0; i < 32; ++i)
+                    for (int i = 0; i < 32; ++i) {
                         if (i > lim) x[i] = 0.f;
+                        if constexpr (GATED)
+                            if (i == lim) x[i] += dd;
+                    }
                     if (!tok && qq < 2) {
 #pragma unroll
                         for (int i = 0; i < 32; i += 4)
@@ -839,16 +846,12 @@ __global__ void __launch_bounds__(NTHR, 1)
             const long row0 = tb + static_cast<long>(c) * L;
             const int nv = static_cast<int>(len - static_cast<long>(c) * L < L ? len - static_cast<long>(c) * L : L);
             const uint32_t tm_out = tmem + 256u * g + TM_OUT;
-            // gated read-out: this token row's v and g (128 B each) are brought into L2 before
-            // waiting for the chunk, and read where they are used
-            long goff = 0, gvoff = 0;
+            // gated read-out: this token row of g (128 B) is brought into L2 before waiting
+            // for the chunk, and read where it is used
+            long goff = 0;
             if constexpr (GATED) {
                 goff = (row0 + ts) * tstride + hoff;
-                gvoff = PRO ? (row0 + ts) * tstride_kv + hoff_kv : goff;
-                if (ts < nv) {
-                    prefetch_line_l2(v + gvoff);
-                    prefetch_line_l2(gte + goff);
-                }
+                if (ts < nv) prefetch_line_l2(gte + goff);
             }
             ok = group_sync_and(bar_id, GROUP,
                                 ts == 0 ? mbar_wait(&bars.ready[g], static_cast<uint32_t>(kk_) & 1u, WAIT_NS) : true);
@@ -870,25 +873,23 @@ __global__ void __launch_bounds__(NTHR, 1)
             float o[32];
             if (ts < 64) {
                 const int t = ts;
-                float uu = 0.f;
-                if constexpr (GATED) uu = reinterpret_cast<const float*>(sm + OFF_U)[g * 128 + (kk_ & 1) * 64 + t];
 #pragma unroll(GATED ? 2 : 1)
                 for (int q = 0; q < 2; ++q) {
                     tmem_load32(tm_out + lane_base + 32 * q, o);
                     if (t < nv && y != nullptr) {
                         const long off = (row0 + t) * tstride + hoff + 32 * q;
                         if constexpr (GATED) {
-                            // z = (y / sqrt(D) + u v) (.) g, with v and g of this token row
+                            // z = (y + 8 u v) / 8 (.) g: the row already holds y + 8 u v (the
+                            // diagonal of Mrk), so only g of this token row is read
 #pragma unroll
                             for (int i = 0; i < 32; i += 8) {
-                                const uint4 vq = *reinterpret_cast<const uint4*>(v + gvoff + 32 * q + i);
                                 const uint4 gq4 = *reinterpret_cast<const uint4*>(gte + goff + 32 * q + i);
-                                const uint32_t vw[4] = {vq.x, vq.y, vq.z, vq.w}, gw[4] = {gq4.x, gq4.y, gq4.z, gq4.w};
+                                const uint32_t gw[4] = {gq4.x, gq4.y, gq4.z, gq4.w};
 #pragma unroll
                                 for (int m = 0; m < 4; ++m) {
-                                    const float2 vf = unpack_bf16x2(vw[m]), gf = unpack_bf16x2(gw[m]);
-                                    o[i + 2 * m] = (o[i + 2 * m] * 0.125f + uu * vf.x) * gf.x;
-                                    o[i + 2 * m + 1] = (o[i + 2 * m + 1] * 0.125f + uu * vf.y) * gf.y;
+                                    const float2 gf = unpack_bf16x2(gw[m]);
+                                    o[i + 2 * m] = o[i + 2 * m] * 0.125f * gf.x;
+                                    o[i + 2 * m + 1] = o[i + 2 * m + 1] * 0.125f * gf.y;
                                 }
                             }
                         }
