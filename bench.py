@@ -352,7 +352,31 @@ def run_ours(args):
                   "roofline": {"bound": "hbm", "achieved": lach, "peak": hbm_peak, "unit": "GB/s",
                                "frac": lach / hbm_peak, "algorithmic_bytes_per_launch": lbytes,
                                "hbm_time_floor_us": lbytes / (hbm_peak * 1e9) * 1e6}}
-    del ld_, linp, ls0
+    # ---------------- the same long sequence through the two-phase prefill (wkv7_forward_long):
+    # every chunk's state-independent part in parallel, then one state pass per head
+    lws = torch.empty(wk.wkv7_forward_long_workspace_bytes(1, linp.T, linp.H, 64), dtype=torch.uint8, device="cuda")
+    ly = torch.empty_like(ld_["r"])
+    lsT = torch.empty_like(ls0)
+
+    def ltwo():
+        wk.wkv7_forward_long(ld_["r"], ld_["w_log"], ld_["k"], ld_["v"], ld_["a"], ld_["b"], ls0, ly, lsT, lws, 1,
+                             linp.T, linp.H, 64, stream)
+
+    for _ in range(max(3, args.warmup)):
+        ltwo()
+    torch.cuda.synchronize()
+    l2t = time_launches(ltwo, args.steps, stream)
+    if wk.wkv7_get_device_status() != 0:
+        raise RuntimeError("device status set during the two-phase long run")
+    l2ms = max_over_ranks(sum(l2t) / len(l2t))
+    l2ach = lbytes / (l2ms * 1e-3) / 1e9
+    long_two_phase = {"workload": "prefill_2p9b_long", "variant": "decay z ~ N(1,1); two-phase (wkv7_forward_long)",
+                      "tokens_per_s": world * linp.T / (l2ms * 1e-3), "ms_per_step": l2ms,
+                      "launches_per_step": 2, "workspace_bytes": lws.numel(),
+                      "roofline": {"bound": "hbm", "achieved": l2ach, "peak": hbm_peak, "unit": "GB/s",
+                                   "frac": l2ach / hbm_peak, "algorithmic_bytes_per_launch": lbytes,
+                                   "hbm_time_floor_us": lbytes / (hbm_peak * 1e9) * 1e6}}
+    del ld_, linp, ls0, lws, ly, lsT
     # ---------------- packed variable-length prefill: 16 sequences, lengths U{512..8192}, pads U{0..63}
     # the same packed draw on every rank: the lengths (and so the real-token count and the bytes)
     # are equal across ranks, so world x tokens is the job's count
@@ -562,6 +586,7 @@ def run_ours(args):
             "clocks": clocks,
             "long": long_sections,
             "long_split": long_split,
+            "long_two_phase": long_two_phase,
             "packed": packed_section,
             "gated": {"workload": PREFILL_WORKLOAD, "tokens_per_s": world * tokens / (gms * 1e-3),
                       "ms_per_step": gms,

@@ -154,6 +154,39 @@ int wkv7_forward_fused(const void* r, const void* w_log, const void* k, const vo
                        const int32_t* seq_offsets, int io_dtype, int w_dtype, void* stream);
 
 /*
+ * wkv7_forward_long — wkv7_forward for dense batches with few (sequence, head)
+ * units and long sequences, in two phases through a caller workspace.  Same
+ * result as wkv7_forward (the same chunk algebra; "RWKV-7 Goose architecture
+ * analysis", its Q5 on chunk-wise parallel WKV and its inference-cost table by
+ * sequence length, up to 1M tokens).  Every 64-token chunk's output splits into a
+ * part that does not depend on the chunk's start state and one product with
+ * that state, so
+ *   phase 1 forms the state-independent part of every chunk of every sequence
+ *           (one block per SM, each taking every SM-th chunk and head, so all
+ *           SMs stay busy even when B x H is small) and writes it to the
+ *           workspace;
+ *   phase 2 carries the state through the chunks of each (sequence, head), with
+ *           one tensor-core product per chunk (a (sequence, head) split over up
+ *           to four blocks by columns of the state).
+ *   r, w_log, k, v, a, b, s0, y, sT, B, T, H, D : as in wkv7_forward for a
+ *          dense batch (no seq_offsets); bf16 inputs only (io_dtype WKV7_BF16;
+ *          WKV7_F32 returns WKV7_ERR_UNSUPPORTED: use wkv7_forward), w_log fp32
+ *          or bf16.
+ *   workspace : DEVICE scratch of at least wkv7_forward_long_workspace_bytes(B,
+ *          T, H, D) bytes (49,408 per 64-token chunk and head), owned by the
+ *          caller, 16-byte aligned, not read before it is written; it must not
+ *          overlap any input or output.  wkv7_forward_long_workspace_bytes
+ *          returns 0 for invalid sizes (B <= 0, T < 0, H <= 0, D != 64).
+ * Decay range and status codes as in wkv7_forward.  T == 0: sT receives s0 (or
+ * zeros) and the workspace is not touched.
+ */
+size_t wkv7_forward_long_workspace_bytes(int B, int T, int H, int D);
+int wkv7_forward_long(const void* r, const void* w_log, const void* k, const void* v,
+                      const void* a, const void* b, const float* s0, void* y, float* sT,
+                      void* workspace, size_t workspace_bytes, int B, int T, int H, int D,
+                      int io_dtype, int w_dtype, void* stream);
+
+/*
  * wkv7_state_map — the affine map that a token range applies to the state, for
  * splitting long sequences into ranges (across devices or launches).  Each step
  * S <- S (diag(w_t) + a_t b_t^T) + v_t k_t^T of the generalized delta rule ("RWKV-7

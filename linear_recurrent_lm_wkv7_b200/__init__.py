@@ -3,7 +3,7 @@ decode step behind a C ABI (``include/wkv7.h``, ``libwkv7.so``).
 
 The Python layer only marshals arguments to the CUDA library; importing the
 package loads ``libwkv7.so`` and fails loudly if it has not been built.
-Convenience wrappers ``forward``, ``forward_gated``, ``forward_fused``,
+Convenience wrappers ``forward``, ``forward_long``, ``forward_gated``, ``forward_fused``,
 ``decode_step``, ``decode_step_fused`` and ``backward`` allocate outputs with
 torch and call the C entry points; ``forward_host`` runs the prefill on inputs
 and outputs that live in pinned host memory, overlapping the copies with the
@@ -28,6 +28,8 @@ from ._binding import (  # noqa: F401
     wkv7_forward,
     wkv7_forward_fused,
     wkv7_forward_gated,
+    wkv7_forward_long,
+    wkv7_forward_long_workspace_bytes,
     wkv7_get_device_status,
     wkv7_state_apply,
     wkv7_state_map,
@@ -52,6 +54,24 @@ def forward(r, w_log, k, v, a, b, s0=None, seq_offsets=None, want_state=True, st
     y = torch.empty_like(r)
     sT = torch.empty((B, H, D, D), dtype=torch.float32, device=r.device) if want_state else None
     wkv7_forward(r, w_log, k, v, a, b, s0, y, sT, B, T, H, D, seq_offsets, stream)
+    return y, sT
+
+
+def forward_long(r, w_log, k, v, a, b, s0=None, want_state=True, workspace=None, stream=None):
+    """Two-phase prefill of a dense batch [B, T, H, D] (bf16 inputs) for few,
+    long sequences: every chunk's state-independent work in parallel, then one
+    state pass per (sequence, head).  ``workspace`` (a device tensor of at least
+    ``wkv7_forward_long_workspace_bytes`` bytes) is allocated when not given.
+    Returns ``(y, sT)`` like ``forward``."""
+    import torch
+
+    B, T, H, D = r.shape
+    if workspace is None:
+        nbytes = wkv7_forward_long_workspace_bytes(B, T, H, D)
+        workspace = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=r.device)
+    y = torch.empty_like(r)
+    sT = torch.empty((B, H, D, D), dtype=torch.float32, device=r.device) if want_state else None
+    wkv7_forward_long(r, w_log, k, v, a, b, s0, y, sT, workspace, B, T, H, D, stream)
     return y, sT
 
 

@@ -31,6 +31,8 @@ EXPORTS = (
     "wkv7_forward",
     "wkv7_forward_gated",
     "wkv7_forward_fused",
+    "wkv7_forward_long",
+    "wkv7_forward_long_workspace_bytes",
     "wkv7_decode_step",
     "wkv7_decode_step_fused",
     "wkv7_backward",
@@ -76,6 +78,10 @@ def _lib():
         lib.wkv7_backward_workspace_bytes.restype = ctypes.c_size_t
         lib.wkv7_backward_noalloc.argtypes = [vp] * 16 + [i] * 4 + [vp, i, i, vp]
         lib.wkv7_backward_noalloc.restype = i
+        lib.wkv7_forward_long.argtypes = [vp] * 10 + [ctypes.c_size_t] + [i] * 4 + [i, i, vp]
+        lib.wkv7_forward_long.restype = i
+        lib.wkv7_forward_long_workspace_bytes.argtypes = [i] * 4
+        lib.wkv7_forward_long_workspace_bytes.restype = ctypes.c_size_t
         lib.wkv7_state_map.argtypes = [vp] * 8 + [i] * 4 + [vp, i, i, vp]
         lib.wkv7_state_map.restype = i
         lib.wkv7_state_apply.argtypes = [vp] * 4 + [i, i, vp]
@@ -161,6 +167,20 @@ def wkv7_decode_step_fused(r, w_log, k, v, a_lr, s_in, r_k, g, out, s_out, B, H,
         raise Wkv7Error(st, "wkv7_decode_step_fused")
 
 
+def wkv7_forward_long_workspace_bytes(B, T, H, D) -> int:
+    return int(_lib().wkv7_forward_long_workspace_bytes(int(B), int(T), int(H), int(D)))
+
+
+def wkv7_forward_long(r, w_log, k, v, a, b, s0, y, sT, workspace, B, T, H, D, stream=None):
+    """Enqueue the two-phase prefill for long sequences (see include/wkv7.h)."""
+    nbytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    st = _lib().wkv7_forward_long(_ptr(r), _ptr(w_log), _ptr(k), _ptr(v), _ptr(a), _ptr(b), _ptr(s0), _ptr(y),
+                                  _ptr(sT), _ptr(workspace), int(nbytes), int(B), int(T), int(H), int(D),
+                                  _dtype_code(r), _dtype_code(w_log), _stream(stream))
+    if st != 0:
+        raise Wkv7Error(st, "wkv7_forward_long")
+
+
 def wkv7_backward_workspace_bytes(B, T, H, D, packed) -> int:
     return int(_lib().wkv7_backward_workspace_bytes(int(B), int(T), int(H), int(D), 1 if packed else 0))
 
@@ -237,6 +257,10 @@ def wkv7_version() -> int:
 def raw_call_forward(*args):
     """Direct C call with raw integer pointers (used by host-validation tests)."""
     return int(_lib().wkv7_forward(*args))
+
+
+def raw_call_forward_long(*args):
+    return int(_lib().wkv7_forward_long(*args))
 
 
 def raw_call_forward_gated(*args):

@@ -17,7 +17,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libwkv7.so")
-SOURCES = ["wkv7_api.cu", "wkv7_decode.cu", "wkv7_prefill.cu", "wkv7_prefill_pipe.cu", "wkv7_gate.cu",
+SOURCES = ["wkv7_api.cu", "wkv7_decode.cu", "wkv7_prefill.cu", "wkv7_prefill_pipe.cu", "wkv7_prefill_long.cu", "wkv7_gate.cu",
            "wkv7_backward.cu", "wkv7_noalloc.cu", "wkv7_state.cu"]
 HEADERS = ["sm100_ptx.cuh", "wkv7_internal.cuh", "prefill_common.cuh", "tma_host.cuh"]
 

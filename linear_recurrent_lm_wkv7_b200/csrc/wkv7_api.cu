@@ -246,6 +246,58 @@ int wkv7_decode_step_fused(const void* r, const void* w_log, const void* k, cons
                        stream, true);
 }
 
+size_t wkv7_forward_long_workspace_bytes(int B, int T, int H, int D) {
+    if (B <= 0 || T < 0 || H <= 0 || D != wkv7::kHead) return 0;
+    return wkv7::prefill_long_workspace_bytes(B, T, H);
+}
+
+int wkv7_forward_long(const void* r, const void* w_log, const void* k, const void* v, const void* a, const void* b,
+                      const float* s0, void* y, float* sT, void* workspace, size_t workspace_bytes, int B, int T,
+                      int H, int D, int io_dtype, int w_dtype, void* stream) {
+    // ---- host-side validation; nothing is launched on failure
+    if (B <= 0 || T < 0 || H <= 0 || D <= 0) return WKV7_ERR_INVALID_ARG;
+    if (!dtype_ok(io_dtype) || !dtype_ok(w_dtype)) return WKV7_ERR_INVALID_ARG;
+    if (D != wkv7::kHead || io_dtype != WKV7_BF16) return WKV7_ERR_UNSUPPORTED;
+    if (T > 0 && (!r || !w_log || !k || !v || !a || !b || !y || !workspace)) return WKV7_ERR_INVALID_ARG;
+    const void* ptrs[] = {r, w_log, k, v, a, b, s0, y, sT, workspace};
+    for (const void* p : ptrs)
+        if (p && !aligned16(p)) return WKV7_ERR_MISALIGNED;
+    const size_t need = wkv7::prefill_long_workspace_bytes(B, T, H);
+    if (T > 0 && workspace_bytes < need) return WKV7_ERR_INVALID_ARG;
+    const size_t n_act = static_cast<size_t>(B) * T * H * D;
+    const size_t n_state = static_cast<size_t>(B) * H * D * D;
+    const size_t io_b = dtype_bytes(io_dtype), w_b = dtype_bytes(w_dtype);
+    const void* ins[] = {r, k, v, a, b, w_log, s0};
+    const size_t in_b[] = {n_act * io_b, n_act * io_b, n_act * io_b, n_act * io_b, n_act * io_b, n_act * w_b,
+                           n_state * 4};
+    // outputs and workspace: disjoint from every input and from each other (sT may be s0)
+    const void* outs[] = {y, sT, T > 0 ? workspace : nullptr};
+    const size_t out_b[] = {n_act * io_b, n_state * 4, need};
+    for (int o = 0; o < 3; ++o) {
+        for (int i = 0; i < 7; ++i) {
+            if (o == 1 && i == 6 && sT == s0) continue;
+            if (overlaps(outs[o], out_b[o], ins[i], in_b[i])) return WKV7_ERR_INVALID_ARG;
+        }
+        for (int o2 = o + 1; o2 < 3; ++o2)
+            if (overlaps(outs[o], out_b[o], outs[o2], out_b[o2])) return WKV7_ERR_INVALID_ARG;
+    }
+
+    int dev_ok = cached_device_check();
+    if (dev_ok != WKV7_OK) return dev_ok;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (T == 0) {
+        if (!sT) return WKV7_OK;
+        const long n = static_cast<long>(n_state);
+        const int blocks = static_cast<int>((n + 255) / 256 < 1184 ? (n + 255) / 256 : 1184);
+        copy_or_zero_states<<<blocks, 256, 0, st>>>(s0, sT, n);
+        return cudaGetLastError() == cudaSuccess ? WKV7_OK : WKV7_ERR_CUDA;
+    }
+    int* status = nullptr;
+    if (status_ptr(&status) != WKV7_OK) return WKV7_ERR_CUDA;
+    wkv7::PrefillArgs p{r, w_log, k, v, a, b, s0, y, sT, B, T, H, nullptr, status};
+    return wkv7::launch_prefill_long(p, w_dtype, workspace, st) == cudaSuccess ? WKV7_OK : WKV7_ERR_CUDA;
+}
+
 int wkv7_state_map(const void* r, const void* w_log, const void* k, const void* v, const void* a, const void* b,
                    float* M, float* Q, int B, int T, int H, int D, const int32_t* seq_offsets, int io_dtype,
                    int w_dtype, void* stream) {

@@ -42,6 +42,12 @@ struct PrefillArgs {
     // the initial state is the identity (s0 ignored); y == nullptr writes no y rows
     bool zero_v = false;
     bool s0_identity = false;
+    // two-phase prefill (wkv7_forward_long), first phase: each chunk's
+    // state-independent results go to the workspace arrays below (layouts in
+    // wkv7_prefill_pipe.cu)
+    uint8_t* ex_as = nullptr;
+    float* ex_out = nullptr;
+    float* ex_gam = nullptr;
 };
 
 struct DecodeArgs {
@@ -90,6 +96,11 @@ struct BackwardArgs {
 cudaError_t launch_prefill(const PrefillArgs& p, int io_dtype, int w_dtype, cudaStream_t stream);
 // warp-specialised kernel for bf16 inputs (wkv7_prefill_pipe.cu)
 cudaError_t launch_prefill_pipe(const PrefillArgs& p, int w_dtype, cudaStream_t stream);
+// its export mode: the first phase of the two-phase prefill (dense bf16 batches)
+cudaError_t launch_prefill_pipe_export(const PrefillArgs& p, int w_dtype, cudaStream_t stream);
+// two-phase prefill (wkv7_prefill_long.cu): workspace bytes, and both phases
+size_t prefill_long_workspace_bytes(int B, int T, int H);
+cudaError_t launch_prefill_long(const PrefillArgs& p, int w_dtype, void* ws, cudaStream_t stream);
 cudaError_t launch_decode(const DecodeArgs& p, int io_dtype, int w_dtype, int* status, cudaStream_t stream);
 // z <- (z / sqrt(D) + (sum_d r k rk) v) * g in place over ntok x H rows (wkv7_gate.cu).
 // With a_lr non-null (after the fused prologue) the key is k (1 - w + a_lr) with

@@ -214,8 +214,17 @@ __device__ __forceinline__ float sum8_scatter(const float (&pd)[8], int jp) {
 // loaded), kMapIdentity starts from the identity state (s0 ignored).  y == nullptr
 // writes no y rows.
 constexpr int kMapZeroV = 1, kMapIdentity = 2;
+// EXPORT (first phase of wkv7_forward_long, dense batches): no chunk depends on
+// another, so the grid is persistent: block i takes chunks i, i + gridDim.x, ...
+// of the list of every (sequence n, chunk j, head h) in the order
+// slot = (n * chunks per sequence + j) * H + h, through one continuous pipeline,
+// and the serial group, instead of the state pass, writes each chunk's
+// state-independent results to its workspace slot: the [R'; Bh^T W] tile as it
+// is in shared memory (ex_as, 16 KB), the OUT product so far (ex_out, 128 rows x
+// 64 fp32 in 16 column quads, quad-major: element (row, col) at
+// ((col / 4) * 128 + row) * 4 + col % 4) and Gamma_L (ex_gam, 64 fp32).
 
-template <typename WT, bool GATED, bool PRO>
+template <typename WT, bool GATED, bool PRO, bool EXPORT = false>
 __global__ void __launch_bounds__(NTHR, 1)
     wkv7_prefill_pipe_kernel(const __nv_bfloat16* __restrict__ r, const WT* __restrict__ wl,
                              const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restrict__ v,
@@ -223,7 +232,9 @@ __global__ void __launch_bounds__(NTHR, 1)
                              const float* s0, __nv_bfloat16* __restrict__ y, float* sT, int T, int H,
                              const int32_t* __restrict__ seq_offsets, int* status,
                              const float* __restrict__ rk, const __nv_bfloat16* __restrict__ gte, int H_kv,
-                             int map_flags, const __grid_constant__ TmaMaps maps) {
+                             int map_flags, int B, uint8_t* __restrict__ ex_as,
+                             float* __restrict__ ex_out, float* __restrict__ ex_gam,
+                             const __grid_constant__ TmaMaps maps) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     // 1024-byte aligned base, derived from the shared array so that every tile pointer
     // stays in the shared address space (32-bit addressing)
@@ -270,7 +281,6 @@ __global__ void __launch_bounds__(NTHR, 1)
         n = *pick;
         __syncthreads();  // every thread has its sequence before the scratch is reused
     }
-    const int hk = PRO ? h / (H / H_kv) : h;  // kv head of k and v
     long tb = 0, len = 0;
     if (seq_offsets) {
         const long o0 = seq_offsets[n], o1 = seq_offsets[n + 1];
@@ -287,7 +297,33 @@ __global__ void __launch_bounds__(NTHR, 1)
     const long tstride = static_cast<long>(H) * kHead;
     const long hoff = static_cast<long>(h) * kHead;
     const long sbase = (static_cast<long>(n) * H + h) * kHead * kHead;
-    const int nchunks = static_cast<int>((len + L - 1) / L);
+    int nchunks = static_cast<int>((len + L - 1) / L);
+    // EXPORT: this block's c-th chunk is slot blockIdx.x + c * gridDim.x
+    const long nch_seq = (static_cast<long>(T) + L - 1) / L;
+    if constexpr (EXPORT) {
+        const long total = static_cast<long>(B) * nch_seq * H;
+        nchunks = static_cast<int>((total - blockIdx.x + gridDim.x - 1) / gridDim.x);
+    }
+    auto slot_of = [&](int c) { return static_cast<long>(blockIdx.x) + static_cast<long>(c) * gridDim.x; };
+    // first token row, head and valid rows of this block's c-th chunk
+    auto chunk_t0 = [&](int c) -> long {
+        if constexpr (EXPORT) {
+            const long q = slot_of(c) / H;
+            return (q / nch_seq) * T + (q % nch_seq) * L;
+        } else {
+            return tb + static_cast<long>(c) * L;
+        }
+    };
+    auto chunk_h = [&](int c) -> int {
+        if constexpr (EXPORT) return static_cast<int>(slot_of(c) % H);
+        else return h;
+    };
+    auto chunk_nv = [&](int c) -> int {
+        long rem;
+        if constexpr (EXPORT) rem = T - (slot_of(c) / H % nch_seq) * L;
+        else rem = len - static_cast<long>(c) * L;
+        return static_cast<int>(rem < L ? rem : L);
+    };
 
     if (tid == 0) {
         for (int g = 0; g < 2; ++g) {
@@ -342,7 +378,8 @@ __global__ void __launch_bounds__(NTHR, 1)
         constexpr uint32_t WB = sizeof(WT);
         // one thread each; `which`: 0 = w_log, 1 = r and k, 2 = a and b
         auto issue_raw = [&](int cc, int which) {
-            const int t0 = static_cast<int>(tb + static_cast<long>(cc) * L);
+            const int t0 = static_cast<int>(chunk_t0(cc));
+            const int h = chunk_h(cc), hk = PRO ? h / (H / H_kv) : h;
             if (which == 0) {
                 mbar_arrive_expect_tx(&bars.rl[g], 4096u * WB);
                 tma_load_3d(gt + RAW_L, &maps.wl, &bars.rl[g], 0, h, t0);
@@ -361,7 +398,8 @@ __global__ void __launch_bounds__(NTHR, 1)
         };
         auto issue_v = [&](int cc) {  // one thread
             mbar_arrive_expect_tx(&bars.vld[g], 8192u);
-            tma_load_3d(Vt, &maps.v, &bars.vld[g], 0, hk, static_cast<int>(tb + static_cast<long>(cc) * L));
+            const int hv = PRO ? chunk_h(cc) / (H / H_kv) : chunk_h(cc);
+            tma_load_3d(Vt, &maps.v, &bars.vld[g], 0, hv, static_cast<int>(chunk_t0(cc)));
         };
         const bool zero_v = (map_flags & kMapZeroV) != 0;
         if (zero_v) {
@@ -401,7 +439,7 @@ __global__ void __launch_bounds__(NTHR, 1)
 
         for (int c = g; c < nchunks; c += 2) {
             const int kk_ = c >> 1;
-            const int nv = static_cast<int>(len - static_cast<long>(c) * L < L ? len - static_cast<long>(c) * L : L);
+            const int nv = chunk_nv(c);
 
             // ---- p1: decay products and the scaled operand tiles
             {
@@ -821,6 +859,46 @@ __global__ void __launch_bounds__(NTHR, 1)
             }
             for (int i = v_done; i < v_issued; ++i) mbar_wait(&bars.vld[g], static_cast<uint32_t>(i) & 1u, WAIT_NS);
         }
+    } else if constexpr (EXPORT) {
+        // =========================================================== export group
+        const int ts = tid - 256;
+        const uint32_t bar_id = 3;
+        const float* gam_all = reinterpret_cast<const float*>(sm + OFF_GAMMA);
+        for (int c = 0; c < nchunks; ++c) {
+            const int g = c & 1, kk_ = c >> 1;
+            const uint32_t tm_out = tmem + 256u * g + TM_OUT;
+            ok = group_sync_and(bar_id, GROUP,
+                                ts == 0 ? mbar_wait(&bars.ready[g], static_cast<uint32_t>(kk_) & 1u, WAIT_NS) : true);
+            if (!ok) break;
+            tc_fence_after();
+            const long slot = slot_of(c);
+            if (ts == 0) {
+                // the shared tile as it is, by one bulk copy (the prep group fenced it for the
+                // async proxy before publishing the chunk)
+                bulk_store(ex_as + slot * 16384, sm + OFF_AS, 16384u);
+                bulk_commit();
+            }
+            float* orow = ex_out + slot * 8192 + ts * 4;
+#pragma unroll 1
+            for (int q = 0; q < 2; ++q) {
+                float o[32];
+                tmem_load32(tm_out + lane_base + 32 * q, o);
+#pragma unroll
+                for (int i = 0; i < 8; ++i)
+                    *reinterpret_cast<float4*>(orow + (8 * q + i) * 512) =
+                        make_float4(o[4 * i], o[4 * i + 1], o[4 * i + 2], o[4 * i + 3]);
+            }
+            if (ts < 64) ex_gam[slot * 64 + ts] = gam_all[g * 128 + (kk_ & 1) * 64 + ts];
+            if (ts == 0) {
+                bulk_wait_read<0>();                        // the copy has read the shared tile
+                mbar_arrive(&bars.asfree[g]);
+            }
+            tc_fence_before();
+            group_sync(bar_id, GROUP);
+            if (ts == 0) mbar_arrive(&bars.freeg[g]);
+        }
+        if (ts == 0) bulk_wait_all();  // every tile copy has landed before the block exits
+        if (!ok && ts == 0) report_status(status, WKV7_ERR_DEVICE_TIMEOUT);
     } else {
         // =========================================================== serial group
         const int ts = tid - 256;
@@ -844,7 +922,7 @@ __global__ void __launch_bounds__(NTHR, 1)
         for (int c = 0; c < nchunks; ++c) {
             const int g = c & 1, kk_ = c >> 1;
             const long row0 = tb + static_cast<long>(c) * L;
-            const int nv = static_cast<int>(len - static_cast<long>(c) * L < L ? len - static_cast<long>(c) * L : L);
+            const int nv = chunk_nv(c);
             const uint32_t tm_out = tmem + 256u * g + TM_OUT;
             // gated read-out: this token row of g (128 B) is brought into L2 before waiting
             // for the chunk, and read where it is used
@@ -936,9 +1014,9 @@ __global__ void __launch_bounds__(NTHR, 1)
     }
 }
 
-template <typename WT, bool GATED, bool PRO>
+template <typename WT, bool GATED, bool PRO, bool EXPORT = false>
 cudaError_t launch_pipe_typed(const PrefillArgs& p, cudaStream_t stream) {
-    auto kern = wkv7_prefill_pipe_kernel<WT, GATED, PRO>;
+    auto kern = wkv7_prefill_pipe_kernel<WT, GATED, PRO, EXPORT>;
     static std::atomic<unsigned long long> configured{0};
     const cudaError_t e = configure_smem_once(kern, static_cast<int>(SMEM_BYTES), configured);
     if (e != cudaSuccess) return e;
@@ -947,18 +1025,31 @@ cudaError_t launch_pipe_typed(const PrefillArgs& p, cudaStream_t stream) {
     const int H_kv = PRO ? p.H_kv : p.H;
     if (!make_prefill_maps(&maps, p.r, p.w_log, p.k, p.v, p.a, PRO ? nullptr : p.b, p.H, H_kv, ntok, sizeof(WT)))
         return cudaErrorInvalidValue;
-    const long units = static_cast<long>(p.B) * p.H;
+    long units = static_cast<long>(p.B) * p.H;
+    if (EXPORT) {  // persistent: one block per SM, or one per chunk when there are fewer
+        int dev = 0, sms = 0;
+        cudaError_t e2 = cudaGetDevice(&dev);
+        if (e2 == cudaSuccess) e2 = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+        if (e2 != cudaSuccess) return e2;
+        const long total = static_cast<long>(p.B) * ((static_cast<long>(p.T) + L - 1) / L) * p.H;
+        units = total < sms ? total : sms;
+    }
     kern<<<static_cast<unsigned>(units), NTHR, SMEM_BYTES, stream>>>(
         static_cast<const __nv_bfloat16*>(p.r), static_cast<const WT*>(p.w_log),
         static_cast<const __nv_bfloat16*>(p.k), static_cast<const __nv_bfloat16*>(p.v),
         static_cast<const __nv_bfloat16*>(p.a), static_cast<const __nv_bfloat16*>(p.b), p.s0,
         static_cast<__nv_bfloat16*>(p.y), p.sT, p.T, p.H, p.seq_offsets, p.status, p.rk,
         static_cast<const __nv_bfloat16*>(p.g), H_kv, (p.zero_v ? kMapZeroV : 0) | (p.s0_identity ? kMapIdentity : 0),
-        maps);
+        p.B, p.ex_as, p.ex_out, p.ex_gam, maps);
     return cudaGetLastError();
 }
 
 }  // namespace
+
+cudaError_t launch_prefill_pipe_export(const PrefillArgs& p, int w_dtype, cudaStream_t stream) {
+    return w_dtype == WKV7_BF16 ? launch_pipe_typed<__nv_bfloat16, false, false, true>(p, stream)
+                                : launch_pipe_typed<float, false, false, true>(p, stream);
+}
 
 cudaError_t launch_prefill_pipe(const PrefillArgs& p, int w_dtype, cudaStream_t stream) {
     if (p.prologue) {

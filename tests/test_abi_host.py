@@ -213,6 +213,41 @@ def test_backward_noalloc_rejects_before_any_cuda_call(wk):
     assert bwd_same(*ptrs[:16], ptrs[0] + 0x8000000, 1 << 40, 2, 8192, 32, 64, None, 7, 0, None) == -1
 
 
+# argument tuple for wkv7_forward_long: 10 pointers, workspace bytes, B, T, H, D, io, w, stream
+def _fwd_long(wk, B=1, T=130, H=2, D=64, io=1, wd=0, wsb=None, **over):
+    names = ("r", "w", "k", "v", "a", "b", "s0", "y", "sT", "ws")
+    p = {n: 0x1000 + i * 0x1000000 for i, n in enumerate(names)}
+    p["s0"] = p["sT"] = None
+    p.update(over)
+    if wsb is None:
+        wsb = wk.wkv7_forward_long_workspace_bytes(B, T, H, 64)
+    return tuple(p[n] for n in names) + (wsb, B, T, H, D, io, wd, None)
+
+
+def test_forward_long_workspace_size(wk):
+    # 16 KB tile + 32 KB fp32 block + 256 B of decay per 64-token chunk and head
+    assert wk.wkv7_forward_long_workspace_bytes(2, 130, 3, 64) == 2 * 3 * 3 * 49408
+    assert wk.wkv7_forward_long_workspace_bytes(1, 16384, 40, 64) == 256 * 40 * 49408
+    assert wk.wkv7_forward_long_workspace_bytes(1, 0, 1, 64) == 0
+    assert wk.wkv7_forward_long_workspace_bytes(0, 64, 1, 64) == 0
+    assert wk.wkv7_forward_long_workspace_bytes(1, 64, 1, 32) == 0
+
+
+def test_forward_long_rejects_bad_arguments(wk):
+    call = wk._binding.raw_call_forward_long
+    assert call(*_fwd_long(wk, io=0)) == -2  # fp32 inputs: use wkv7_forward
+    assert call(*_fwd_long(wk, D=32)) == -2
+    assert call(*_fwd_long(wk, B=0)) == -1
+    assert call(*_fwd_long(wk, io=3)) == -1
+    assert call(*_fwd_long(wk, ws=None)) == -1
+    assert call(*_fwd_long(wk, y=None)) == -1
+    assert call(*_fwd_long(wk, wsb=1024)) == -1  # workspace too small
+    assert call(*_fwd_long(wk, ws=0x1008 + 0x9000000)) == -3  # misaligned
+    assert call(*_fwd_long(wk, ws=0x1000 + 0x3000000)) == -1  # workspace overlaps v
+    assert call(*_fwd_long(wk, y=0x1000 + 0x9000000)) == -1  # y aliases the workspace
+    assert call(*_fwd_long(wk, sT=0x1000 + 0x4000000)) == -1  # sT overlaps a
+
+
 def test_c_program_compiles_and_links(wk, tmp_path):
     """The C ABI is usable from plain C: a C99 program that includes the header and
     references every entry point compiles and links against the library (nothing
