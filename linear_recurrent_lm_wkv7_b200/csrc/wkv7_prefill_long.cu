@@ -20,8 +20,13 @@
 //            columns of its operand tile (the rest stay zero), reads the whole
 //            [R'; Bh^T W] tile but only its NV columns of OUTpre, and writes its NV
 //            columns of y and sT.
-// Phase 2 streams the workspace through a four-stage ring of bulk copies issued
-// by a producer warp (full / empty mbarriers, bounded waits).
+// Phase 2 streams the workspace through a ring of bulk copies (8, 6 or 4 stages)
+// issued by a producer warp (full / empty mbarriers, bounded waits), which also
+// prefetches the chunk one ring-depth ahead into L2.  The product is issued as
+// tcgen05 (N = 64, the block's NV columns first in the operand tile, zeros after):
+// a warp-level mma.sync form of it, with the state in accumulator registers, was
+// measured slower (about 1.3 K cycles per chunk against 0.7 K: four or eight warps,
+// each with ~180 dependent instructions per chunk on one scheduler).
 #include "prefill_common.cuh"
 #include "sm100_ptx.cuh"
 #include "wkv7_internal.cuh"
@@ -34,22 +39,30 @@ constexpr uint32_t AS_BYTES = 16384;     // [R'; Bh^T W], 128 rows x 64 bf16, 12
 constexpr uint32_t OUT_BYTES = 32768;    // OUTpre, 128 x 64 fp32 (column quads, quad-major)
 constexpr uint32_t GAM_BYTES = 256;      // Gamma_L, 64 fp32
 constexpr uint32_t SLOT_BYTES = AS_BYTES + OUT_BYTES + GAM_BYTES;
-constexpr int NST = 4;                   // ring stages
 constexpr int NCOMP = 128;               // compute threads: TMEM lanes 0..127
 constexpr int NTHR = NCOMP + 32;         // + one producer warp
 constexpr uint64_t WAIT_NS = 1000000000ull;
 constexpr uint32_t ID_KM64 = idesc_f32acc(1, 128, 64, 0, 1);  // bf16, B MN-major, N = 64
 
-// per-block geometry for NV value columns
+// per-block geometry for NV value columns: with 16 columns two blocks share an SM
+// (four chunks in flight each), with 32 or 64 one block holds six or four
 template <int NV>
 struct ScanGeom {
     static constexpr uint32_t OUT_PART = NV * 512u;  // this block's columns of OUTpre (NV / 4 quads)
     static constexpr uint32_t BYTES = AS_BYTES + OUT_PART + GAM_BYTES;  // one chunk's bulk copies
     static constexpr uint32_t STAGE = (BYTES + 1023u) / 1024u * 1024u;  // the AS tile is 1024-aligned
+    static constexpr int NST = NV == 32 ? 6 : 4;                         // ring stages
     static constexpr uint32_t OFF_ST = NST * STAGE;                     // S0^T, bf16 MN-major (64 x 64)
     static constexpr uint32_t OFF_BAR = OFF_ST + 8192;                  // full[NST], empty[NST], mma, tmem slot
     static constexpr uint32_t SMEM = OFF_BAR + (2 * NST + 2) * 8 + 1024;
+    static_assert(SMEM <= 227u * 1024u, "shared memory");
 };
+
+// L2 prefetch of global bytes (a hint: nothing waits for it); 16-byte aligned, size a
+// multiple of 16, all inside one allocation
+__device__ __forceinline__ void prefetch_l2_bulk(const void* src, uint32_t bytes) {
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
+}
 
 // the first NV fp32 columns of this thread's TMEM lane (NV = 16, 32 or 64)
 template <int NV>
@@ -82,7 +95,7 @@ __global__ void __launch_bounds__(NTHR, 1)
                           const float* __restrict__ ex_gam, const float* s0, __nv_bfloat16* __restrict__ y,
                           float* sT, int T, int H, int* status) {
     using G = ScanGeom<NV>;
-    constexpr int NPART = 64 / NV;
+    constexpr int NPART = 64 / NV, NST = G::NST;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     uint64_t* full = reinterpret_cast<uint64_t*>(sm + G::OFF_BAR);
@@ -130,6 +143,11 @@ __global__ void __launch_bounds__(NTHR, 1)
                 }
                 if (*reinterpret_cast<volatile int*>(&abort_flag)) break;
                 const long slot = (cbase + c) * H + h;
+                if (c + NST < nch) {  // the chunk one ring-depth ahead: from DRAM into L2
+                    const long ps = slot + static_cast<long>(NST) * H;
+                    prefetch_l2_bulk(ex_as + ps * AS_BYTES, AS_BYTES);
+                    prefetch_l2_bulk(ex_out + ps * (OUT_BYTES / 4) + v0 * 128, G::OUT_PART);
+                }
                 uint8_t* stage = sm + st * G::STAGE;
                 mbar_arrive_expect_tx(&full[st], G::BYTES);
                 bulk_load(stage, ex_as + slot * AS_BYTES, AS_BYTES, &full[st]);
@@ -170,18 +188,23 @@ __global__ void __launch_bounds__(NTHR, 1)
             const uint8_t* stage = sm + st * G::STAGE;
             const long row0 = static_cast<long>(n) * T + static_cast<long>(c) * L;
             const int nv = T - c * L < L ? T - c * L : L;
-            ok = group_sync_and(bar_id, NCOMP,
-                                ts == 0 ? mbar_wait(&full[st], static_cast<uint32_t>(c / NST) & 1u, WAIT_NS) : true);
-            if (!ok) break;
-            tc_fence_after();
+            // one thread waits for the stage, issues the product and waits for it; the
+            // product's completion means every copy of the stage has landed (one full
+            // barrier), so the other threads only wait for the product
+            bool w_ok = true;
             if (ts == 0) {
-                const uint64_t dAS = kmajor_desc<false>(stage, 128, 0);
+                w_ok = mbar_wait(&full[st], static_cast<uint32_t>(c / NST) & 1u, WAIT_NS);
+                if (w_ok) {
+                    tc_fence_after();
+                    const uint64_t dAS = kmajor_desc<false>(stage, 128, 0);
 #pragma unroll
-                for (uint32_t s = 0; s < 4; ++s) mma_ss<false>(tmem, dAS + 2 * s, dSt + 128 * s, ID_KM64, s > 0);
-                mma_commit(mma_bar);
+                    for (uint32_t s = 0; s < 4; ++s) mma_ss<false>(tmem, dAS + 2 * s, dSt + 128 * s, ID_KM64, s > 0);
+                    mma_commit(mma_bar);
+                    mma_pending = true;
+                    w_ok = mbar_wait(mma_bar, mma_phase, WAIT_NS);
+                }
             }
-            mma_pending = true;
-            ok = group_sync_and(bar_id, NCOMP, ts == 0 ? mbar_wait(mma_bar, mma_phase, WAIT_NS) : true);
+            ok = group_sync_and(bar_id, NCOMP, w_ok);
             if (!ok) break;
             mma_pending = false;
             mma_phase ^= 1u;
@@ -270,10 +293,11 @@ cudaError_t launch_prefill_long(const PrefillArgs& p, int w_dtype, void* ws, cud
     if (e != cudaSuccess) return e;
     e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     if (e != cudaSuccess) return e;
-    // value columns per block: as few as keep the blocks within two per SM
+    // value columns per block: as few as keep every block of the grid resident at once
+    // (up to two per SM with 16 columns, one with 32)
     const long units = static_cast<long>(p.B) * p.H;
     if (units * 4 <= 2L * sms) return launch_scan<16>(p, q, stream);
-    if (units * 2 <= 2L * sms) return launch_scan<32>(p, q, stream);
+    if (units * 2 <= sms) return launch_scan<32>(p, q, stream);
     return launch_scan<64>(p, q, stream);
 }
 
