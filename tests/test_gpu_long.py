@@ -140,3 +140,20 @@ def test_long_is_deterministic(wk):
     b = wk.forward_long(*args)
     for x, z in zip(a, b):
         assert torch.equal(x, z)
+
+
+def test_million_token_context(wk, oracle_mod):
+    """B1 T1048576 H1 with the long-memory decay draw (median w 0.97) and a
+    non-zero initial state: 16,384 chunks of state carried through both prefill
+    forms (the pages' long-context claim reaches 1M tokens).  Every output is
+    compared with the oracle's."""
+    inp = W.make_prefill(1, 1 << 20, 1, io="bf16", wdt="f32", s0_std=0.1, mu_z=-3.0, seed=902)
+    yr, sr = oracle_forward(oracle_mod, inp)
+    y, sT = run_long(wk, inp)
+    ey, es = relerr(y, yr), relerr(sT, sr)
+    assert ey <= TOL and es <= TOL, (ey, es)
+    d = {k: t.cuda() for k, t in inp.tensors().items()}
+    y1, s1 = wk.forward(d["r"], d["w_log"], d["k"], d["v"], d["a"], d["b"], inp.s0.cuda())
+    assert wk.wkv7_get_device_status() == 0
+    e1y, e1s = relerr(y1.float().cpu().numpy(), yr), relerr(s1.cpu().numpy(), sr)
+    assert e1y <= TOL and e1s <= TOL, (e1y, e1s)
