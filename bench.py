@@ -306,7 +306,8 @@ def run_ours(args):
             raise RuntimeError(f"device status set during the {name} run")
         ms_ = max_over_ranks(sum(tt) / len(tt))
         slots = inp_.T if inp_.seq_offsets is not None else inp_.B * inp_.T  # tokens in the tensors, pads included
-        bytes_ = prefill_bytes(slots * inp_.H, 2, 4, inp_.B * inp_.H, with_s0=inp_.s0 is not None)
+        io_b_, w_b_ = (4 if inp_.io == "f32" else 2), (4 if inp_.wdt == "f32" else 2)
+        bytes_ = prefill_bytes(slots * inp_.H, io_b_, w_b_, inp_.B * inp_.H, with_s0=inp_.s0 is not None)
         ach = bytes_ / (ms_ * 1e-3) / 1e9
         out = {"workload": name, "variant": label, "B": inp_.B, "H": inp_.H, "tokens": inp_.n_real_tokens,
                "token_slots": slots, "s0": s0_kind, "tokens_per_s": world * inp_.n_real_tokens / (ms_ * 1e-3),
@@ -384,6 +385,11 @@ def run_ours(args):
     packed_section = prefill_section("packed_1p5b", pinp, "16 sequences, pads U{0..63} (w = 1, k = v = a = b = 0)",
                                      "N(0, 0.1^2)")
     del pinp
+
+    # ---------------- the headline shape with fp32 inputs (the tf32 kernel; fp32 y)
+    finp = W.make_prefill(B, T, H, io="f32", wdt="f32", s0_std=None, seed=1 + 1000 * rank)
+    f32_section = prefill_section("prefill_1p5b_f32", finp, "fp32 inputs and outputs", "zero")
+    del finp
 
     # ---------------- the same prefill with the gated read-out (wkv7_forward_gated)
     rk_h, gate_h = W.make_gate(tuple(dev["r"].shape), H, D, io="bf16", seed=2 + 1000 * rank)
@@ -588,6 +594,7 @@ def run_ours(args):
             "long_split": long_split,
             "long_two_phase": long_two_phase,
             "packed": packed_section,
+            "prefill_f32": f32_section,
             "gated": {"workload": PREFILL_WORKLOAD, "tokens_per_s": world * tokens / (gms * 1e-3),
                       "ms_per_step": gms,
                       "roofline": {"bound": "hbm", "achieved": gach, "peak": hbm_peak, "unit": "GB/s",
