@@ -188,6 +188,91 @@ __device__ __forceinline__ void gemm16(float (&acc)[8], const float* A, int ar, 
     }
 }
 
+// The fragments of one k-step of gemm16's operands, as separate loaders, so that
+// gemm16_2 can run two independent products through the same k-steps.
+template <bool T>
+struct OpA;  // A: 16 rows (M) x 8 k
+template <>
+struct OpA<false> {
+    AlongRows r0, r1;
+    __device__ __forceinline__ OpA(int ar, int ac, int gq, int t4) : r0(ar + gq, ac, t4), r1(ar + gq + 8, ac, t4) {}
+    __device__ __forceinline__ void load(const float* A, int s, uint32_t (&a)[4]) const {
+        const float2 x0 = *reinterpret_cast<const float2*>(A + r0.at(s));
+        const float2 x1 = *reinterpret_cast<const float2*>(A + r1.at(s));
+        a[0] = __float_as_uint(x0.x);
+        a[1] = __float_as_uint(x1.x);
+        a[2] = __float_as_uint(x0.y);
+        a[3] = __float_as_uint(x1.y);
+    }
+};
+template <>
+struct OpA<true> {
+    AcrossRows c0, c1;
+    __device__ __forceinline__ OpA(int ar, int ac, int gq, int t4) : c0(ac, ar + gq, t4), c1(ac, ar + gq + 8, t4) {}
+    __device__ __forceinline__ void load(const float* A, int s, uint32_t (&a)[4]) const {
+        const int o = 512 * s;
+        a[0] = __float_as_uint(A[c0.base0 + o]);
+        a[1] = __float_as_uint(A[c1.base0 + o]);
+        a[2] = __float_as_uint(A[c0.base1 + o]);
+        a[3] = __float_as_uint(A[c1.base1 + o]);
+    }
+};
+template <bool T>
+struct OpB;  // B: 8 k x 16 columns (N), as two n-tiles
+template <>
+struct OpB<false> {
+    AcrossRows b0, b1;
+    __device__ __forceinline__ OpB(int bk, int bn, int gq, int t4) : b0(bk, bn + gq, t4), b1(bk, bn + 8 + gq, t4) {}
+    __device__ __forceinline__ void load(const float* B, int s, uint32_t (&p)[2], uint32_t (&q)[2]) const {
+        const int o = 512 * s;
+        p[0] = __float_as_uint(B[b0.base0 + o]);
+        p[1] = __float_as_uint(B[b0.base1 + o]);
+        q[0] = __float_as_uint(B[b1.base0 + o]);
+        q[1] = __float_as_uint(B[b1.base1 + o]);
+    }
+};
+template <>
+struct OpB<true> {
+    AlongRows b0, b1;
+    __device__ __forceinline__ OpB(int bk, int bn, int gq, int t4) : b0(bn + gq, bk, t4), b1(bn + 8 + gq, bk, t4) {}
+    __device__ __forceinline__ void load(const float* B, int s, uint32_t (&p)[2], uint32_t (&q)[2]) const {
+        const float2 y0 = *reinterpret_cast<const float2*>(B + b0.at(s));
+        const float2 y1 = *reinterpret_cast<const float2*>(B + b1.at(s));
+        p[0] = __float_as_uint(y0.x);
+        p[1] = __float_as_uint(y0.y);
+        q[0] = __float_as_uint(y1.x);
+        q[1] = __float_as_uint(y1.y);
+    }
+};
+
+// Two independent products of gemm16's form (each with its own operand orientations
+// and k-step count), advanced together: each k-step issues both products' fragment
+// loads and then their four products, so the two accumulator chains overlap.
+template <bool TA1, bool TB1, bool TA2, bool TB2, bool SP>
+__device__ __forceinline__ void gemm16_2(float (&acc1)[8], const float* A1, int ar1, int ac1, const float* B1, int bk1,
+                                         int bn1, int nk1, float (&acc2)[8], const float* A2, int ar2, int ac2,
+                                         const float* B2, int bk2, int bn2, int nk2, int gq, int t4) {
+    const OpA<TA1> x1(ar1, ac1, gq, t4);
+    const OpA<TA2> x2(ar2, ac2, gq, t4);
+    const OpB<TB1> y1(bk1, bn1, gq, t4);
+    const OpB<TB2> y2(bk2, bn2, gq, t4);
+    const int nk = nk1 > nk2 ? nk1 : nk2;
+#pragma unroll(SP ? 1 : 2)
+    for (int s = 0; s < nk; ++s) {
+        uint32_t a1[4], a2[4], p1[2], q1[2], p2[2], q2[2];
+        if (s < nk1) {
+            x1.load(A1, s, a1);
+            y1.load(B1, s, p1, q1);
+        }
+        if (s < nk2) {
+            x2.load(A2, s, a2);
+            y2.load(B2, s, p2, q2);
+        }
+        if (s < nk1) mma_pair<SP>(acc1, a1, p1, q1);
+        if (s < nk2) mma_pair<SP>(acc2, a2, p2, q2);
+    }
+}
+
 constexpr float kLog2e = 1.4426950408889634f;
 // w = exp(-exp(l)) and exp(l) by the hardware 2^x (subnormals flushed: a w that
 // small fails the decay-range check anyway)
@@ -711,9 +796,13 @@ __global__ void __launch_bounds__(NTHR, 1)
         float* Qg = ws + lc.region + static_cast<long>(lc.nch + 1 + lc.c) * SQ;
         float* Qfg = ws + lc.region + static_cast<long>(2 * (lc.nch + 1) + lc.c) * SQ;
         {
-            float acc[8];
-            zero8(acc);  // M = diag(Gamma_L) (I + Bt^T TA)
+            float acc[8], accw[8];
+            // M = diag(Gamma_L) (I + Bt^T TA), and W = Rt + Mrb TA -> NAB (one after the other: run
+            // together, as in the gradient kernel, they were slower here)
+            zero8(acc);
+            zero8(accw);
             gemm16<true, false, SP>(acc, BT, m0, 0, TA, 0, n0, 8, gq, t4);
+            gemm16<false, false, SP>(accw, MRB, m0, 0, TA, 0, n0, (m0 + 16) / 8, gq, t4);
 #pragma unroll
             for (int e = 0; e < 8; ++e) {
                 const int row = m0 + frag_row(e, gq), col = n0 + frag_col(e, t4);
@@ -721,11 +810,9 @@ __global__ void __launch_bounds__(NTHR, 1)
                 acc[e] = SP ? mv : round_tf32(mv);  // an operand of the scan (tf32 unless split)
             }
             st16_global(Mg, acc, m0, n0, gq, t4);
-            zero8(acc);  // W = Rt + Mrb TA -> NAB
-            gemm16<false, false, SP>(acc, MRB, m0, 0, TA, 0, n0, (m0 + 16) / 8, gq, t4);
 #pragma unroll
-            for (int e = 0; e < 8; ++e) acc[e] += RT[sx(m0 + frag_row(e, gq), n0 + frag_col(e, t4))];
-            st16<0, !SP>(NAB, acc, m0, n0, gq, t4);
+            for (int e = 0; e < 8; ++e) accw[e] += RT[sx(m0 + frag_row(e, gq), n0 + frag_col(e, t4))];
+            st16<0, !SP>(NAB, accw, m0, n0, gq, t4);
             zero8(acc);  // Z = Kt + Nak^T TB -> TT
             gemm16<true, false, SP>(acc, NAK, m0, m0, TB, m0, n0, (64 - m0) / 8, gq, t4);
 #pragma unroll
@@ -735,15 +822,16 @@ __global__ void __launch_bounds__(NTHR, 1)
         __syncthreads();
         prefetch_next();  // NAK, MRB, TA and TB are dead: the next item's raw rows go there
         {
-            float acc[8];
-            zero8(acc);  // Q = dY^T W
+            float acc[8], accf[8];
+            // Q = dY^T W, and Qf = V^T Z diag(Gamma_L)
+            zero8(acc);
+            zero8(accf);
             gemm16<true, false, SP>(acc, DY, m0, 0, NAB, 0, n0, 8, gq, t4);
+            gemm16<true, false, SP>(accf, VV, m0, 0, TT, 0, n0, 8, gq, t4);
             st16_global(Qg, acc, m0, n0, gq, t4);
-            zero8(acc);  // Qf = V^T Z diag(Gamma_L)
-            gemm16<true, false, SP>(acc, VV, m0, 0, TT, 0, n0, 8, gq, t4);
 #pragma unroll
-            for (int e = 0; e < 8; ++e) acc[e] *= sm.GL[n0 + frag_col(e, t4)];
-            st16_global(Qfg, acc, m0, n0, gq, t4);
+            for (int e = 0; e < 8; ++e) accf[e] *= sm.GL[n0 + frag_col(e, t4)];
+            st16_global(Qfg, accf, m0, n0, gq, t4);
         }
     }
     cp_async_wait<0>();  // nothing may still be landing when the block exits
@@ -997,9 +1085,15 @@ __global__ void __launch_bounds__(NTHR, 1)
     invert_unit_lower<SP>(W0, W3);  // W3 = T
     float acc[8];
     // X = At S0^T + Nak V -> W0
-    zero8(acc);
-    gemm16<false, true, SP>(acc, AT, m0, 0, S0, 0, n0, 8, gq, t4);
-    gemm16<false, false, SP>(acc, W1, m0, 0, VV, 0, n0, (m0 + 16) / 8, gq, t4);
+    {
+        float acc2[8];
+        zero8(acc);
+        zero8(acc2);
+        gemm16_2<false, true, false, false, SP>(acc, AT, m0, 0, S0, 0, n0, 8, acc2, W1, m0, 0, VV, 0, n0,
+                                                (m0 + 16) / 8, gq, t4);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) acc[e] += acc2[e];
+    }
     st16<0, !SP>(W0, acc, m0, n0, gq, t4);
     __syncthreads();
     // U = T X -> W0
@@ -1008,9 +1102,15 @@ __global__ void __launch_bounds__(NTHR, 1)
     __syncthreads();
     st16<0, !SP>(W0, acc, m0, n0, gq, t4);
     // dU = Mrb^T dY + Bt dSLg^T -> W2
-    zero8(acc);
-    gemm16<true, false, SP>(acc, W2, m0, m0, DY, m0, n0, (64 - m0) / 8, gq, t4);
-    gemm16<false, true, SP>(acc, BT, m0, 0, DS, 0, n0, 8, gq, t4);
+    {
+        float acc2[8];
+        zero8(acc);
+        zero8(acc2);
+        gemm16_2<true, false, false, true, SP>(acc, W2, m0, m0, DY, m0, n0, (64 - m0) / 8, acc2, BT, m0, 0, DS, 0, n0,
+                                               8, gq, t4);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) acc[e] += acc2[e];
+    }
     __syncthreads();
     st16<0, !SP>(W2, acc, m0, n0, gq, t4);
     __syncthreads();
@@ -1025,10 +1125,16 @@ __global__ void __launch_bounds__(NTHR, 1)
     st16<2, !SP>(W2, acc, m0, n0, gq, t4);
     __syncthreads();
     // dV = Mrk^T dY + Kt dSLg^T + Nak^T dX
-    zero8(acc);
-    gemm16<true, false, SP>(acc, W2, m0, m0, DY, m0, n0, (64 - m0) / 8, gq, t4);
-    gemm16<false, true, SP>(acc, KT, m0, 0, DS, 0, n0, 8, gq, t4);
-    gemm16<true, false, SP>(acc, W1, m0, m0, W3, m0, n0, (64 - m0) / 8, gq, t4);
+    {
+        float acc2[8];
+        zero8(acc);
+        zero8(acc2);
+        gemm16_2<false, true, true, false, SP>(acc, KT, m0, 0, DS, 0, n0, 8, acc2, W1, m0, m0, W3, m0, n0,
+                                               (64 - m0) / 8, gq, t4);
+        gemm16<true, false, SP>(acc2, W2, m0, m0, DY, m0, n0, (64 - m0) / 8, gq, t4);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) acc[e] += acc2[e];
+    }
 #pragma unroll
     for (int e = 0; e < 8; e += 2) {
         const int row = m0 + frag_row(e, gq), col = n0 + frag_col(e, t4);
@@ -1040,36 +1146,56 @@ __global__ void __launch_bounds__(NTHR, 1)
     zero8(gR);
     zero8(gB);
     zero8(gK);
-    gemm16<false, false, SP>(gA, W3, m0, 0, S0, 0, n0, 8, gq, t4);  // dX S0
-    gemm16<false, false, SP>(gR, DY, m0, 0, S0, 0, n0, 8, gq, t4);  // dY S0
-    gemm16<false, false, SP>(gB, W0, m0, 0, DS, 0, n0, 8, gq, t4);  // U dSLg
-    gemm16<false, false, SP>(gK, VV, m0, 0, DS, 0, n0, 8, gq, t4);  // V dSLg
+    gemm16_2<false, false, false, false, SP>(gA, W3, m0, 0, S0, 0, n0, 8, gR, DY, m0, 0, S0, 0, n0, 8, gq,
+                                             t4);  // dX S0, dY S0
+    gemm16_2<false, false, false, false, SP>(gB, W0, m0, 0, DS, 0, n0, 8, gK, VV, m0, 0, DS, 0, n0, 8, gq,
+                                             t4);  // U dSLg, V dSLg
     __syncthreads();
     // dNab = tril(dX U^T, -1) -> W1, dNak = tril(dX V^T, -1) -> W2
-    zero8(acc);
-    if (n0 <= m0) gemm16<false, true, SP>(acc, W3, m0, 0, W0, 0, n0, 8, gq, t4);
-    st16<1, !SP>(W1, acc, m0, n0, gq, t4);
-    zero8(acc);
-    if (n0 <= m0) gemm16<false, true, SP>(acc, W3, m0, 0, VV, 0, n0, 8, gq, t4);
-    st16<1, !SP>(W2, acc, m0, n0, gq, t4);
+    {
+        float acc2[8];
+        zero8(acc);
+        zero8(acc2);
+        if (n0 <= m0)
+            gemm16_2<false, true, false, true, SP>(acc, W3, m0, 0, W0, 0, n0, 8, acc2, W3, m0, 0, VV, 0, n0, 8, gq, t4);
+        st16<1, !SP>(W1, acc, m0, n0, gq, t4);
+        st16<1, !SP>(W2, acc2, m0, n0, gq, t4);
+    }
     __syncthreads();
-    gemm16<false, false, SP>(gA, W1, m0, 0, BT, 0, n0, (m0 + 16) / 8, gq, t4);   // dNab Bt
-    gemm16<false, false, SP>(gA, W2, m0, 0, KT, 0, n0, (m0 + 16) / 8, gq, t4);   // dNak Kt
-    gemm16<true, false, SP>(gB, W1, m0, m0, AT, m0, n0, (64 - m0) / 8, gq, t4);  // dNab^T At
-    gemm16<true, false, SP>(gK, W2, m0, m0, AT, m0, n0, (64 - m0) / 8, gq, t4);  // dNak^T At
+    {
+        float tmp[8];  // dNak Kt, added to gA after the pair
+        zero8(tmp);
+        gemm16_2<false, false, false, false, SP>(gA, W1, m0, 0, BT, 0, n0, (m0 + 16) / 8, tmp, W2, m0, 0, KT, 0, n0,
+                                                 (m0 + 16) / 8, gq, t4);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) gA[e] += tmp[e];
+    }
+    // dNab^T At, dNak^T At
+    gemm16_2<true, false, true, false, SP>(gB, W1, m0, m0, AT, m0, n0, (64 - m0) / 8, gK, W2, m0, m0, AT, m0, n0,
+                                           (64 - m0) / 8, gq, t4);
     __syncthreads();
     // dMrb = tril(dY U^T) -> W1, dMrk = tril(dY V^T) -> W2
-    zero8(acc);
-    if (n0 <= m0) gemm16<false, true, SP>(acc, DY, m0, 0, W0, 0, n0, 8, gq, t4);
-    st16<2, !SP>(W1, acc, m0, n0, gq, t4);
-    zero8(acc);
-    if (n0 <= m0) gemm16<false, true, SP>(acc, DY, m0, 0, VV, 0, n0, 8, gq, t4);
-    st16<2, !SP>(W2, acc, m0, n0, gq, t4);
+    {
+        float acc2[8];
+        zero8(acc);
+        zero8(acc2);
+        if (n0 <= m0)
+            gemm16_2<false, true, false, true, SP>(acc, DY, m0, 0, W0, 0, n0, 8, acc2, DY, m0, 0, VV, 0, n0, 8, gq, t4);
+        st16<2, !SP>(W1, acc, m0, n0, gq, t4);
+        st16<2, !SP>(W2, acc2, m0, n0, gq, t4);
+    }
     __syncthreads();
-    gemm16<false, false, SP>(gR, W1, m0, 0, BT, 0, n0, (m0 + 16) / 8, gq, t4);   // dMrb Bt
-    gemm16<false, false, SP>(gR, W2, m0, 0, KT, 0, n0, (m0 + 16) / 8, gq, t4);   // dMrk Kt
-    gemm16<true, false, SP>(gB, W1, m0, m0, RT, m0, n0, (64 - m0) / 8, gq, t4);  // dMrb^T Rt
-    gemm16<true, false, SP>(gK, W2, m0, m0, RT, m0, n0, (64 - m0) / 8, gq, t4);  // dMrk^T Rt
+    {
+        float tmp[8];  // dMrk Kt, added to gR after the pair
+        zero8(tmp);
+        gemm16_2<false, false, false, false, SP>(gR, W1, m0, 0, BT, 0, n0, (m0 + 16) / 8, tmp, W2, m0, 0, KT, 0, n0,
+                                                 (m0 + 16) / 8, gq, t4);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) gR[e] += tmp[e];
+    }
+    // dMrb^T Rt, dMrk^T Rt
+    gemm16_2<true, false, true, false, SP>(gB, W1, m0, m0, RT, m0, n0, (64 - m0) / 8, gK, W2, m0, m0, RT, m0, n0,
+                                           (64 - m0) / 8, gq, t4);
     __syncthreads();
     // d log w needs exp(w_log) of this thread's column j and tokens 8 s .. 8 s + 7 at the end:
     // load them now, behind the element-wise work
