@@ -48,7 +48,9 @@ namespace wkv7 {
 namespace {
 
 constexpr int L = 64;          // chunk length (tokens)
-constexpr int NT = 128;        // threads per block: one per TMEM lane
+constexpr int NT = 256;        // threads per block: the first 128 own one TMEM lane each
+constexpr int NL = 128;        // TMEM lanes (and columns of the triangular solve)
+constexpr int XSTRIDE = 132;   // fp32 row stride of the solver's columns (bank spread of 4 per row)
 constexpr int NSTRIDE = 68;    // fp32 row stride of the solver matrices (bank-conflict padding)
 constexpr uint32_t COL_G = 0;    // TMEM columns of G   (128)
 constexpr uint32_t COL_P = 128;  // TMEM columns of P   (128)
@@ -68,9 +70,9 @@ struct Smem {
     uint8_t* AS;   // [R' ; Bh^T W]        128 x 64, K-major over key channels    (aliases NAB, MAK)
     uint8_t* V;    // V: 64 values x 64 tokens (K-major)
     uint8_t* S;    // S^T: 64 values x 64 keys (K-major)
-    float* XS;     // solver columns: XS[t][col], 64 tokens x 128 columns fp32
+    float* XS;     // solver columns: XS[t][col], 64 tokens x 128 columns fp32 (row stride XSTRIDE)
     float* gammaL; // Gamma_L per key channel
-    float* red;    // per-half products of w (2 x 64), then (prologue) 1 / ||k_t|| per token (64)
+    float* red;    // per-quarter products of w (4 x 64), then (prologue) 1 / ||k_t|| per token (64)
     uint64_t* bar; // MMA completion barrier
     uint32_t* tmem_slot;
 };
@@ -81,8 +83,8 @@ __host__ __device__ constexpr uint32_t smem_bytes_needed() {
     using O = OpType<TF32>;
     constexpr uint32_t solver = 2u * 64u * NSTRIDE * 4u;
     constexpr uint32_t r4 = ((solver > O::TILE128 ? solver : O::TILE128) + 1023u) & ~1023u;
-    return 1024u /* alignment slack */ + 3u * O::TILE128 + O::TILE64 + r4 + 2u * O::TILE64 + 64u * NT * 4u +
-           64u * 4u + 192u * 4u + 64u;
+    return 1024u /* alignment slack */ + 3u * O::TILE128 + O::TILE64 + r4 + 2u * O::TILE64 + 64u * XSTRIDE * 4u +
+           64u * 4u + 320u * 4u + 64u;
 }
 
 template <bool TF32>
@@ -99,9 +101,9 @@ __device__ __forceinline__ Smem carve(uint8_t* raw) {
     s.NAB = reinterpret_cast<float*>(p); s.MAK = s.NAB + 64 * NSTRIDE; s.AS = p; p += r4;
     s.V = p; p += O::TILE64;
     s.S = p; p += O::TILE64;
-    s.XS = reinterpret_cast<float*>(p); p += 64 * NT * 4;
+    s.XS = reinterpret_cast<float*>(p); p += 64 * XSTRIDE * 4;
     s.gammaL = reinterpret_cast<float*>(p); p += 64 * 4;
-    s.red = reinterpret_cast<float*>(p); p += 192 * 4;
+    s.red = reinterpret_cast<float*>(p); p += 320 * 4;
     s.bar = reinterpret_cast<uint64_t*>(p); p += 8;
     s.tmem_slot = reinterpret_cast<uint32_t*>(p);
     return s;
@@ -118,7 +120,7 @@ __device__ __forceinline__ void store_state_operand(uint8_t* tile, int jj, const
 __device__ __forceinline__ void load_v_tile(const float* __restrict__ v, long row0, long tstride, long hoff, int nv,
                                             uint8_t* tile, int tid) {
 #pragma unroll
-    for (int it = 0; it < 8; ++it) {
+    for (int it = 0; it < 1024 / NT; ++it) {
         const int q = tid + it * NT;
         const int row = q >> 4, ch = q & 15;
         float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -139,7 +141,7 @@ __device__ __forceinline__ void prefetch_chunk_rows(const IO* r, const WT* wl, c
                                                     const IO* b, long row0, long nrows, long tstride, long hoff,
                                                     long tstride_kv, long hoff_kv, int tid, bool pro) {
     const int t = tid >> 1, half = tid & 1;
-    if (t >= nrows) return;
+    if (tid >= 2 * L || t >= nrows) return;
     const long off = (row0 + t) * tstride + hoff + 32 * half;
     const long offkv = (row0 + t) * tstride_kv + hoff_kv + 32 * half;
     prefetch_line_l2(r + off);
@@ -209,7 +211,7 @@ __global__ void __launch_bounds__(NT, 1)
     // ---- state: threads 64..127 own key channel j = tid - 64 (a row of S^T)
     float S[64];
     const int jj = tid - 64;
-    if (tid >= 64) {
+    if (tid >= 64 && tid < NL) {
 #pragma unroll
         for (int i = 0; i < 64; ++i)
             S[i] = (map_flags & 2) ? (i == jj ? 1.f : 0.f) : (s0 ? s0[sbase + i * kHead + jj] : 0.f);
@@ -229,50 +231,56 @@ __global__ void __launch_bounds__(NT, 1)
                                                   tstride, hoff, tstride_kv, hoff_kv, tid, PRO);
         // ---- p1: decay products and scaled operand tiles.  Thread (j, half).
         {
-            const int j = tid & 63, hf = tid >> 6;
-            float cp[32];
+            const int j = tid & 63, hf = tid >> 6;  // key channel j, tokens 16 hf .. 16 hf + 15
+            float cp[16];
             float prod = 1.f;
-            // every decay logit of the thread's 32 tokens is loaded before the first product
-            float lv[32];
+            // every decay logit of the thread's 16 tokens is loaded before the first product
+            float lv[16];
 #pragma unroll
-            for (int q = 0; q < 32; ++q) {
-                const int t = hf * 32 + q;
+            for (int q = 0; q < 16; ++q) {
+                const int t = hf * 16 + q;
                 lv[q] = t < nv ? to_f32(wl[(row0 + t) * tstride + hoff + j]) : -INFINITY;
             }
 #pragma unroll
-            for (int q = 0; q < 32; ++q) {
+            for (int q = 0; q < 16; ++q) {
                 // w = exp(-exp(l)) by the hardware 2^x (w_log = -inf gives w = 1 exactly)
                 prod *= ex2_ftz(-kLog2e * ex2_ftz(kLog2e * lv[q]));
                 cp[q] = prod;
             }
             sm.red[hf * 64 + j] = prod;
             if constexpr (PRO) {
-                // 1 / max(||k_t||, 1e-12) of token t = tid / 2: each thread of the pair sums 32 channels
-                const int t = tid >> 1, c0 = (tid & 1) * 32;
+                // 1 / max(||k_t||, 1e-12) of token t = tid / 4: each thread of the quad sums 16 channels
+                const int t = tid >> 2, c0 = (tid & 3) * 16;
                 float ss = 0.f;
                 if (t < nv) {
                     const IO* kr = k + (row0 + t) * tstride_kv + hoff_kv + c0;
 #pragma unroll 8
-                    for (int i = 0; i < 32; ++i) {
+                    for (int i = 0; i < 16; ++i) {
                         const float x = to_f32(kr[i]);
                         ss = fmaf(x, x, ss);
                     }
                 }
                 ss += __shfl_xor_sync(0xffffffffu, ss, 1);
-                if ((tid & 1) == 0) sm.red[128 + t] = 1.f / fmaxf(sqrtf(ss), 1e-12f);
+                ss += __shfl_xor_sync(0xffffffffu, ss, 2);
+                if ((tid & 3) == 0) sm.red[256 + t] = 1.f / fmaxf(sqrtf(ss), 1e-12f);
             }
             __syncthreads();
-            const float pre = hf ? sm.red[j] : 1.f;
-            const float GL = sm.red[j] * sm.red[64 + j];
+            float pre = 1.f, GL = 1.f;
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const float x = sm.red[q * 64 + j];
+                if (q < hf) pre *= x;
+                GL *= x;
+            }
             if (hf == 0) sm.gammaL[j] = GL;
             float gprev = pre;
 #pragma unroll
-            for (int g = 0; g < 4; ++g) {
+            for (int g = 0; g < 2; ++g) {
                 // batches of 8 tokens: all loads of a batch are issued before its stores
                 float rr[8], kk[8], aa[8], bb[8];
 #pragma unroll
                 for (int e = 0; e < 8; ++e) {
-                    const int t = hf * 32 + g * 8 + e;
+                    const int t = hf * 16 + g * 8 + e;
                     rr[e] = kk[e] = aa[e] = bb[e] = 0.f;
                     if (t < nv) {
                         const long off = (row0 + t) * tstride + hoff + j;
@@ -288,12 +296,12 @@ __global__ void __launch_bounds__(NT, 1)
                 }
 #pragma unroll
                 for (int e = 0; e < 8; ++e) {
-                    const int t = hf * 32 + g * 8 + e;
+                    const int t = hf * 16 + g * 8 + e;
                     const float G = pre * cp[g * 8 + e];
                     const float inv = 1.f / G;
                     const float invL = inv * GL;
                     if constexpr (PRO) {
-                        const float w = G / gprev, kn = kk[e] * sm.red[128 + t];  // w_t and kk
+                        const float w = G / gprev, kn = kk[e] * sm.red[256 + t];  // w_t and kk
                         bb[e] = kn * aa[e];
                         kk[e] *= 1.f - w + aa[e];
                         aa[e] = -kn;
@@ -343,7 +351,7 @@ __global__ void __launch_bounds__(NT, 1)
                         if (32 * q + i > t) g[i] = 0.f;
                     st_op_row32<TF32>(sm.BH, 128, t, 32 * q, g);
                 }
-            } else {
+            } else if (tid < NL) {
                 const int t = tid - 64;
 #pragma unroll
                 for (int q = 0; q < 4; ++q) {
@@ -364,23 +372,28 @@ __global__ void __launch_bounds__(NT, 1)
         tc_fence_before();
         __syncthreads();
 
-        // ---- [W | Z] = (I - Nab)^{-1} [At | Mak]: forward substitution, column `tid`, in blocks of
-        // four rows: the rows of a block accumulate their products with the solved rows above as
-        // four independent sums, then take the 4 x 4 triangle; the column lives in XS
+        // ---- [W | Z] = (I - Nab)^{-1} [At | Mak]: forward substitution of 128 columns in blocks of
+        // four rows.  Warp w takes columns 16 w .. 16 w + 15; lanes l and l + 16 share a column and
+        // split the products with the solved rows above a block (even and odd blocks of four rows,
+        // which the row stride of XS puts in different banks), add them with one shuffle, and both
+        // take the 4 x 4 triangle; the column lives in XS
         {
-            const int col = tid;
+            const int lane = tid & 31, part = lane >> 4;
+            const int col = 16 * warp + (lane & 15);
             float* xs = sm.XS;
 #pragma unroll 1
             for (int t0 = 0; t0 < 64; t0 += 4) {
                 float acc[4];
 #pragma unroll
                 for (int q = 0; q < 4; ++q)
-                    acc[q] = col < 64 ? ld_op<TF32>(sm.RA, 128, 64 + t0 + q, col) : sm.MAK[(t0 + q) * NSTRIDE + (col - 64)];
+                    acc[q] = part ? 0.f
+                                  : (col < 64 ? ld_op<TF32>(sm.RA, 128, 64 + t0 + q, col)
+                                              : sm.MAK[(t0 + q) * NSTRIDE + (col - 64)]);
                 const float* n0 = sm.NAB + t0 * NSTRIDE;  // rows t0 .. t0 + 3
 #pragma unroll 2
-                for (int i = 0; i < t0; i += 4) {
-                    const float x0 = xs[i * NT + col], x1 = xs[(i + 1) * NT + col];
-                    const float x2 = xs[(i + 2) * NT + col], x3 = xs[(i + 3) * NT + col];
+                for (int i = 4 * part; i < t0; i += 8) {
+                    const float x0 = xs[i * XSTRIDE + col], x1 = xs[(i + 1) * XSTRIDE + col];
+                    const float x2 = xs[(i + 2) * XSTRIDE + col], x3 = xs[(i + 3) * XSTRIDE + col];
 #pragma unroll
                     for (int q = 0; q < 4; ++q) {
                         const float4 n4 = *reinterpret_cast<const float4*>(n0 + q * NSTRIDE + i);
@@ -390,23 +403,26 @@ __global__ void __launch_bounds__(NT, 1)
                         acc[q] = fmaf(n4.w, x3, acc[q]);
                     }
                 }
+#pragma unroll
+                for (int q = 0; q < 4; ++q) acc[q] += __shfl_xor_sync(0xffffffffu, acc[q], 16);
                 const float y0 = acc[0];
                 const float y1 = fmaf(n0[NSTRIDE + t0], y0, acc[1]);
                 const float y2 = fmaf(n0[2 * NSTRIDE + t0 + 1], y1, fmaf(n0[2 * NSTRIDE + t0], y0, acc[2]));
                 const float y3 = fmaf(n0[3 * NSTRIDE + t0 + 2], y2,
                                       fmaf(n0[3 * NSTRIDE + t0 + 1], y1, fmaf(n0[3 * NSTRIDE + t0], y0, acc[3])));
-                xs[t0 * NT + col] = y0;
-                xs[(t0 + 1) * NT + col] = y1;
-                xs[(t0 + 2) * NT + col] = y2;
-                xs[(t0 + 3) * NT + col] = y3;
+                if (part == 0) {
+                    xs[t0 * XSTRIDE + col] = y0;
+                    xs[(t0 + 1) * XSTRIDE + col] = y1;
+                    xs[(t0 + 2) * XSTRIDE + col] = y2;
+                    xs[(t0 + 3) * XSTRIDE + col] = y3;
+                }
+                __syncwarp();  // the block's rows are in XS for both lanes of the column
             }
+            // the column -> the K-major [W | Z]^T tile: one half of it per lane of the pair
+            float x[32];
 #pragma unroll
-            for (int hlf = 0; hlf < 2; ++hlf) {
-                float x[32];
-#pragma unroll
-                for (int q = 0; q < 32; ++q) x[q] = xs[(32 * hlf + q) * NT + col];
-                st_op_row32<TF32>(sm.WZ, 128, col, 32 * hlf, x);
-            }
+            for (int q = 0; q < 32; ++q) x[q] = xs[(32 * part + q) * XSTRIDE + col];
+            st_op_row32<TF32>(sm.WZ, 128, col, 32 * part, x);
         }
         fence_proxy_async_smem();
         __syncthreads();
@@ -449,7 +465,7 @@ __global__ void __launch_bounds__(NT, 1)
                     for (int i = 0; i < 32; ++i) p[i] += (32 * q + i <= t) ? e[i] : 0.f;
                     st_op_row32<TF32>(sm.AQ, 128, t, 32 * q, p);
                 }
-            } else {
+            } else if (tid < NL) {
                 const int j = tid - 64;
 #pragma unroll
                 for (int q = 0; q < 2; ++q) {
@@ -505,7 +521,7 @@ __global__ void __launch_bounds__(NT, 1)
                             *reinterpret_cast<float4*>(dst + i) = make_float4(o[i], o[i + 1], o[i + 2], o[i + 3]);
                     }
                 }
-            } else {
+            } else if (tid < NL) {
                 const float GL = sm.gammaL[jj];
                 // 1 / Gamma_t must stay far inside the fp32 range (false for NaN too)
                 if (!(GL >= kMinGammaL)) report_status(status, WKV7_ERR_DECAY_RANGE);
@@ -527,7 +543,7 @@ __global__ void __launch_bounds__(NT, 1)
         // let an MMA still in flight finish (bounded) before the block releases
         // TMEM and its shared memory
         if (mma_pending) mbar_wait(sm.bar, phase, WAIT_LIMIT_NS);
-    } else if (sT && tid >= 64) {
+    } else if (sT && tid >= 64 && tid < NL) {
 #pragma unroll
         for (int i = 0; i < 64; ++i) sT[sbase + i * kHead + jj] = S[i];
     }
