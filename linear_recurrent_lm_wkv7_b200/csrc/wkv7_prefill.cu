@@ -373,29 +373,29 @@ __global__ void __launch_bounds__(NT, 1)
         __syncthreads();
 
         // ---- [W | Z] = (I - Nab)^{-1} [At | Mak]: forward substitution of 128 columns in blocks of
-        // four rows.  Warp w takes columns 16 w .. 16 w + 15; lanes l and l + 16 share a column and
-        // split the products with the solved rows above a block (even and odd blocks of four rows,
-        // which the row stride of XS puts in different banks), add them with one shuffle, and both
-        // take the 4 x 4 triangle; the column lives in XS
+        // sixteen rows.  Warp w takes columns 16 w .. 16 w + 15; lanes l and l + 16 share a column and
+        // split the products with the solved rows above a block (alternate groups of four rows,
+        // which the row stride of XS puts in different banks), add them with shuffles, and both
+        // take the 16 x 16 triangle; the column lives in XS
         {
             const int lane = tid & 31, part = lane >> 4;
             const int col = 16 * warp + (lane & 15);
             float* xs = sm.XS;
 #pragma unroll 1
-            for (int t0 = 0; t0 < 64; t0 += 4) {
-                float acc[4];
+            for (int t0 = 0; t0 < 64; t0 += 16) {
+                float acc[16];
 #pragma unroll
-                for (int q = 0; q < 4; ++q)
+                for (int q = 0; q < 16; ++q)
                     acc[q] = part ? 0.f
                                   : (col < 64 ? ld_op<TF32>(sm.RA, 128, 64 + t0 + q, col)
                                               : sm.MAK[(t0 + q) * NSTRIDE + (col - 64)]);
-                const float* n0 = sm.NAB + t0 * NSTRIDE;  // rows t0 .. t0 + 3
+                const float* n0 = sm.NAB + t0 * NSTRIDE;  // rows t0 .. t0 + 15
 #pragma unroll 2
                 for (int i = 4 * part; i < t0; i += 8) {
                     const float x0 = xs[i * XSTRIDE + col], x1 = xs[(i + 1) * XSTRIDE + col];
                     const float x2 = xs[(i + 2) * XSTRIDE + col], x3 = xs[(i + 3) * XSTRIDE + col];
 #pragma unroll
-                    for (int q = 0; q < 4; ++q) {
+                    for (int q = 0; q < 16; ++q) {
                         const float4 n4 = *reinterpret_cast<const float4*>(n0 + q * NSTRIDE + i);
                         acc[q] = fmaf(n4.x, x0, acc[q]);
                         acc[q] = fmaf(n4.y, x1, acc[q]);
@@ -404,17 +404,19 @@ __global__ void __launch_bounds__(NT, 1)
                     }
                 }
 #pragma unroll
-                for (int q = 0; q < 4; ++q) acc[q] += __shfl_xor_sync(0xffffffffu, acc[q], 16);
-                const float y0 = acc[0];
-                const float y1 = fmaf(n0[NSTRIDE + t0], y0, acc[1]);
-                const float y2 = fmaf(n0[2 * NSTRIDE + t0 + 1], y1, fmaf(n0[2 * NSTRIDE + t0], y0, acc[2]));
-                const float y3 = fmaf(n0[3 * NSTRIDE + t0 + 2], y2,
-                                      fmaf(n0[3 * NSTRIDE + t0 + 1], y1, fmaf(n0[3 * NSTRIDE + t0], y0, acc[3])));
+                for (int q = 0; q < 16; ++q) acc[q] += __shfl_xor_sync(0xffffffffu, acc[q], 16);
+                // the 16 x 16 unit lower triangle of the block
+                float yv[16];
+#pragma unroll
+                for (int q = 0; q < 16; ++q) {
+                    float yq = acc[q];
+#pragma unroll
+                    for (int r = 0; r < q; ++r) yq = fmaf(n0[q * NSTRIDE + t0 + r], yv[r], yq);
+                    yv[q] = yq;
+                }
                 if (part == 0) {
-                    xs[t0 * XSTRIDE + col] = y0;
-                    xs[(t0 + 1) * XSTRIDE + col] = y1;
-                    xs[(t0 + 2) * XSTRIDE + col] = y2;
-                    xs[(t0 + 3) * XSTRIDE + col] = y3;
+#pragma unroll
+                    for (int q = 0; q < 16; ++q) xs[(t0 + q) * XSTRIDE + col] = yv[q];
                 }
                 __syncwarp();  // the block's rows are in XS for both lanes of the column
             }
