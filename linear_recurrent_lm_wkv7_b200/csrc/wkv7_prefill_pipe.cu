@@ -318,6 +318,13 @@ __global__ void __launch_bounds__(NTHR, 1)
         if constexpr (EXPORT) return static_cast<int>(slot_of(c) % H);
         else return h;
     };
+    // kv head of k and v (the fused prologue shares them over H / H_kv heads); fixed per
+    // block except in EXPORT mode, which has no prologue
+    const int hk_unit = PRO ? h / (H / H_kv) : h;
+    auto chunk_hk = [&](int c) -> int {
+        if constexpr (EXPORT) return chunk_h(c);
+        else return hk_unit;
+    };
     auto chunk_nv = [&](int c) -> int {
         long rem;
         if constexpr (EXPORT) rem = T - (slot_of(c) / H % nch_seq) * L;
@@ -379,7 +386,7 @@ __global__ void __launch_bounds__(NTHR, 1)
         // one thread each; `which`: 0 = w_log, 1 = r and k, 2 = a and b
         auto issue_raw = [&](int cc, int which) {
             const int t0 = static_cast<int>(chunk_t0(cc));
-            const int h = chunk_h(cc), hk = PRO ? h / (H / H_kv) : h;
+            const int h = chunk_h(cc), hk = chunk_hk(cc);
             if (which == 0) {
                 mbar_arrive_expect_tx(&bars.rl[g], 4096u * WB);
                 tma_load_3d(gt + RAW_L, &maps.wl, &bars.rl[g], 0, h, t0);
@@ -398,8 +405,7 @@ __global__ void __launch_bounds__(NTHR, 1)
         };
         auto issue_v = [&](int cc) {  // one thread
             mbar_arrive_expect_tx(&bars.vld[g], 8192u);
-            const int hv = PRO ? chunk_h(cc) / (H / H_kv) : chunk_h(cc);
-            tma_load_3d(Vt, &maps.v, &bars.vld[g], 0, hv, static_cast<int>(chunk_t0(cc)));
+            tma_load_3d(Vt, &maps.v, &bars.vld[g], 0, chunk_hk(cc), static_cast<int>(chunk_t0(cc)));
         };
         const bool zero_v = (map_flags & kMapZeroV) != 0;
         if (zero_v) {
