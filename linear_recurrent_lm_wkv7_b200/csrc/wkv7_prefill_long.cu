@@ -20,13 +20,13 @@
 //            columns of its operand tile (the rest stay zero), reads the whole
 //            [R'; Bh^T W] tile but only its NV columns of OUTpre, and writes its NV
 //            columns of y and sT.
-// Phase 2 streams the workspace through a ring of bulk copies (8, 6 or 4 stages)
+// Phase 2 streams the workspace through a ring of bulk copies (4 or 6 stages)
 // issued by a producer warp (full / empty mbarriers, bounded waits), which also
 // prefetches the chunk one ring-depth ahead into L2.  The product is issued as
 // tcgen05 (N = 64, the block's NV columns first in the operand tile, zeros after):
 // a warp-level mma.sync form of it, with the state in accumulator registers, was
-// measured slower (about 1.3 K cycles per chunk against 0.7 K: four or eight warps,
-// each with ~180 dependent instructions per chunk on one scheduler).
+// measured slower on B1 T16384 H40 (268 us with four warps, 329 us with eight,
+// against 176 us: each warp has ~180 dependent instructions per chunk).
 #include "prefill_common.cuh"
 #include "sm100_ptx.cuh"
 #include "wkv7_internal.cuh"
