@@ -69,7 +69,7 @@ constexpr uint32_t OFF_GAMMA = OFF_S + 8192;          // Gamma_L [2 groups][2 sl
 constexpr uint32_t OFF_RED = OFF_GAMMA + 2 * 2 * 64 * 4;  // block products [2 groups][4][64] fp32
 constexpr uint32_t OFF_U = OFF_RED + 2 * 4 * 64 * 4;    // gated read-out: u [2 groups][2 slots][64] fp32
 constexpr uint32_t OFF_BAR = OFF_U + 2 * 2 * 64 * 4;
-constexpr uint32_t SMEM_USED = OFF_BAR + 18 * 8 + 16;
+constexpr uint32_t SMEM_USED = OFF_BAR + 22 * 8 + 16;
 // raw TMA staging inside a group's tiles (dead at the time of the load)
 constexpr uint32_t RAW_R = OFF_NQ, RAW_K = OFF_NQ + 8192, RAW_A = OFF_RAM, RAW_B = OFF_RAM + 8192, RAW_L = OFF_BK;
 constexpr uint32_t SMEM_BYTES = SMEM_USED + 1024;      // alignment slack
@@ -181,6 +181,8 @@ struct Bars {
     uint64_t* rrk;    // [2] TMA of a group's raw r, k tiles
     uint64_t* rab;    // [2] TMA of a group's raw a, b tiles
     uint64_t* vld;    // [2] TMA of a group's V tile
+    uint64_t* p1done; // [2] SERIAL_P1: the serial group has done pass 1 of a chunk of prep group g (from 2 on)
+    uint64_t* rls;    // [2] SERIAL_P1: TMA of a group's raw w_log tile for its chunks from 2 on
     uint32_t* tmem_slot;
 };
 
@@ -201,6 +203,23 @@ __device__ __forceinline__ float sum8_scatter(const float (&pd)[8], int jp) {
     q1 += __shfl_xor_sync(0xffffffffu, q1, 2);
     q1 += __shfl_xor_sync(0xffffffffu, q1, 1);
     return q1;
+}
+
+// Pass 1 of a chunk: the product of w over each thread's 16 tokens, per key channel
+// (thread (jp, tq) of a 128-thread group: key channels 2 jp, 2 jp + 1, tokens
+// 16 tq .. 16 tq + 15), into red[tq][j]; with fp32 w_log the running products
+// overwrite the thread's own w_log elements.
+template <typename WT>
+__device__ __forceinline__ void decay_pass(WT* rawl, float* red, int tq, int j0) {
+    float2 pw = make_float2(1.f, 1.f);
+#pragma unroll 4
+    for (int e = 0; e < 16; ++e) {
+        const int i = (16 * tq + e) * 64 + j0;
+        pw = __fmul2_rn(pw, decay2(ld_wlog2(rawl, i)));
+        if constexpr (sizeof(WT) == 4) *reinterpret_cast<float2*>(rawl + i) = pw;
+    }
+    red[tq * 64 + j0] = pw.x;
+    red[tq * 64 + j0 + 1] = pw.y;
 }
 
 // GATED: the output rows are z = (y / sqrt(D) + u v) (.) g with u = sum_d r k rk
@@ -235,6 +254,11 @@ __global__ void __launch_bounds__(NTHR, 1)
                              int map_flags, int B, uint8_t* __restrict__ ex_as,
                              float* __restrict__ ex_out, float* __restrict__ ex_gam,
                              const __grid_constant__ TmaMaps maps) {
+    // With the fused prologue (the longest pass 2) the serial group also runs pass 1 of each prep
+    // group's chunks from the second on, off the prep chains (fused + gated 107 -> 100 us on
+    // B4 T1024 H32 with 8 kv heads); for the other variants the extra work on the serial warps
+    // cost more than it saved (plain +0.7 %, gated +3 %, packed +1.5 %), so they keep it.
+    constexpr bool SERIAL_P1 = PRO;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     // 1024-byte aligned base, derived from the shared array so that every tile pointer
     // stays in the shared address space (32-bit addressing)
@@ -253,7 +277,9 @@ __global__ void __launch_bounds__(NTHR, 1)
         bars.rab = p + 10;
         bars.vld = p + 12;
         bars.freeg = p + 14;
-        bars.tmem_slot = reinterpret_cast<uint32_t*>(p + 18);
+        bars.p1done = p + 18;
+        bars.rls = p + 20;
+        bars.tmem_slot = reinterpret_cast<uint32_t*>(p + 22);
     }
 
     // ---- the unit and its tokens
@@ -341,6 +367,8 @@ __global__ void __launch_bounds__(NTHR, 1)
             mbar_init(&bars.rab[g], 1);
             mbar_init(&bars.vld[g], 1);
             mbar_init(&bars.freeg[g], 1);
+            mbar_init(&bars.p1done[g], 1);
+            mbar_init(&bars.rls[g], 1);
         }
         mbar_init(bars.ser, 1);
         mbar_init(&bars.asfree[0], 1);
@@ -357,6 +385,29 @@ __global__ void __launch_bounds__(NTHR, 1)
     const uint32_t tmem = *bars.tmem_slot;
     const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
     bool ok = true;
+    // SERIAL_P1: pass 1 of chunk cn (>= 2) by the serial group (thread ts, named barrier 3)
+    // for prep group cn & 1, run while that group finishes chunk cn - 2 (whose inverse has
+    // released the tile the w_log of chunk cn lands in, on rls: the serial group is its only
+    // waiter, one phase per chunk in order); the group waits on p1done instead of running
+    // the pass on its own chain.
+    auto serial_pass1 = [&](int cn, int ts) -> bool {
+        const int gn = cn & 1;
+        WT* rl_n = reinterpret_cast<WT*>(sm + gn * GROUP_TILES + RAW_L);
+        float* red_n = reinterpret_cast<float*>(sm + OFF_RED) + gn * 256;
+        if (!group_sync_and(3, GROUP,
+                            ts == 0 ? mbar_wait(&bars.rls[gn], static_cast<uint32_t>((cn >> 1) - 1) & 1u, WAIT_NS)
+                                    : true))
+            return false;
+        const int nvn = chunk_nv(cn);
+        if (nvn < L) {  // tokens past the end of the sequence are identity steps (w = 1)
+            for (int i = nvn * 64 + ts; i < L * 64; i += static_cast<int>(GROUP)) rl_n[i] = neg_inf_of<WT>();
+            group_sync(3, GROUP);
+        }
+        decay_pass<WT>(rl_n, red_n, ts >> 5, 2 * (ts & 31));
+        group_sync(3, GROUP);
+        if (ts == 0) mbar_arrive(&bars.p1done[gn]);
+        return true;
+    };
 
     if (warp < 8) {
         // =========================================================== prep groups
@@ -388,8 +439,11 @@ __global__ void __launch_bounds__(NTHR, 1)
             const int t0 = static_cast<int>(chunk_t0(cc));
             const int h = chunk_h(cc), hk = chunk_hk(cc);
             if (which == 0) {
-                mbar_arrive_expect_tx(&bars.rl[g], 4096u * WB);
-                tma_load_3d(gt + RAW_L, &maps.wl, &bars.rl[g], 0, h, t0);
+                // the first chunk's tile completes on rl (the group waits); later ones on rls,
+                // whose only waiter is the serial group, in chunk order
+                uint64_t* bl = (SERIAL_P1 && cc >= 2) ? &bars.rls[g] : &bars.rl[g];
+                mbar_arrive_expect_tx(bl, 4096u * WB);
+                tma_load_3d(gt + RAW_L, &maps.wl, bl, 0, h, t0);
             } else if (which == 1) {
                 mbar_arrive_expect_tx(&bars.rrk[g], 2u * 8192u);
                 tma_load_3d(gt + RAW_R, &maps.r, &bars.rrk[g], 0, h, t0);
@@ -448,28 +502,25 @@ __global__ void __launch_bounds__(NTHR, 1)
             const int nv = chunk_nv(c);
 
             // ---- p1: decay products and the scaled operand tiles
-            {
-                const bool w_ok = (tg == 0) ? mbar_wait(&bars.rl[g], static_cast<uint32_t>(kk_) & 1u, WAIT_NS) : true;
-                ok = group_sync_and(bar_id, GROUP, w_ok);
+            const bool ragged = nv < L;  // group-uniform
+            if (!SERIAL_P1 || kk_ == 0) {
+                // pass 1 here (with SERIAL_P1 only for the group's first chunk)
+                ok = group_sync_and(bar_id, GROUP,
+                                    (tg == 0) ? mbar_wait(&bars.rl[g], static_cast<uint32_t>(kk_) & 1u, WAIT_NS)
+                                              : true);
+                if (!ok) break;
+                if (ragged) {
+                    // tokens past the end of the sequence are identity steps: w_log = -inf (w = 1)
+                    for (int i = nv * 64 + tg; i < L * 64; i += static_cast<int>(GROUP)) rawl_w[i] = neg_inf_of<WT>();
+                    group_sync(bar_id, GROUP);
+                }
+                decay_pass<WT>(rawl_w, red, tq, j0);
+            } else {
+                ok = group_sync_and(bar_id, GROUP,
+                                    (tg == 0) ? mbar_wait(&bars.p1done[g], static_cast<uint32_t>(kk_ - 1) & 1u, WAIT_NS)
+                                              : true);
                 if (!ok) break;
             }
-            const bool ragged = nv < L;  // group-uniform
-            if (ragged) {
-                // tokens past the end of the sequence are identity steps: w_log = -inf (w = 1)
-                for (int i = nv * 64 + tg; i < L * 64; i += static_cast<int>(GROUP)) rawl_w[i] = neg_inf_of<WT>();
-                group_sync(bar_id, GROUP);
-            }
-            // pass 1: product of w over this thread's 16 tokens, per key channel.  With fp32
-            // w_log the running products overwrite the thread's own w_log elements.
-            float2 pw = make_float2(1.f, 1.f);
-#pragma unroll 4
-            for (int e = 0; e < 16; ++e) {
-                const int i = (16 * tq + e) * 64 + j0;
-                pw = __fmul2_rn(pw, decay2(ld_wlog2(rawl, i)));
-                if constexpr (sizeof(WT) == 4) *reinterpret_cast<float2*>(rawl_w + i) = pw;
-            }
-            red[tq * 64 + j0] = pw.x;
-            red[tq * 64 + j0 + 1] = pw.y;
             {
                 // pass 2 rewrites BH and MK and V is reloaded: the previous OUT product of this
                 // group (chunk c-2) must have read them
@@ -859,7 +910,8 @@ __global__ void __launch_bounds__(NTHR, 1)
             if (issued_out > 0) mbar_wait(&bars.ready[g], static_cast<uint32_t>(issued_out - 1) & 1u, WAIT_NS);
             // a chunk's raw loads are issued in three batches; wait for every one that may be in flight
             for (int i = raw_done; i < raw_issued; ++i) {
-                mbar_wait(&bars.rl[g], static_cast<uint32_t>(i) & 1u, WAIT_NS);
+                if (!SERIAL_P1 || i == 0) mbar_wait(&bars.rl[g], static_cast<uint32_t>(i) & 1u, WAIT_NS);
+                else mbar_wait(&bars.rls[g], static_cast<uint32_t>(i - 1) & 1u, WAIT_NS);
                 mbar_wait(&bars.rrk[g], static_cast<uint32_t>(i) & 1u, WAIT_NS);
                 mbar_wait(&bars.rab[g], static_cast<uint32_t>(i) & 1u, WAIT_NS);
             }
@@ -873,6 +925,7 @@ __global__ void __launch_bounds__(NTHR, 1)
         for (int c = 0; c < nchunks; ++c) {
             const int g = c & 1, kk_ = c >> 1;
             const uint32_t tm_out = tmem + 256u * g + TM_OUT;
+            if (SERIAL_P1 && c + 2 < nchunks && !(ok = serial_pass1(c + 2, ts))) break;  // as in the serial group
             ok = group_sync_and(bar_id, GROUP,
                                 ts == 0 ? mbar_wait(&bars.ready[g], static_cast<uint32_t>(kk_) & 1u, WAIT_NS) : true);
             if (!ok) break;
@@ -937,6 +990,9 @@ __global__ void __launch_bounds__(NTHR, 1)
                 goff = (row0 + ts) * tstride + hoff;
                 if (ts < nv) prefetch_line_l2(gte + goff);
             }
+            // while group g finishes chunk c: pass 1 of its chunk c + 2 (its w_log tile lands
+            // once that group's inverse of chunk c is done)
+            if (SERIAL_P1 && c + 2 < nchunks && !(ok = serial_pass1(c + 2, ts))) break;
             ok = group_sync_and(bar_id, GROUP,
                                 ts == 0 ? mbar_wait(&bars.ready[g], static_cast<uint32_t>(kk_) & 1u, WAIT_NS) : true);
             if (!ok) break;
