@@ -94,6 +94,15 @@ def test_fused_packed_with_pads(wk, oracle_mod, gated):
     check_prefill(wk, oracle_mod, inp, gated, seed=9)
 
 
+@pytest.mark.parametrize("wdt", ["f32", "bf16"])
+@pytest.mark.parametrize("gated", [False, True])
+def test_fused_many_chunks_ragged(wk, oracle_mod, wdt, gated):
+    """11 chunks per sequence with a ragged tail: the serial group runs pass 1 (the decay
+    products) of each prep group's chunks after the first, handed over chunk by chunk."""
+    inp = W.make_fused(2, 700, 4, 2, io="bf16", wdt=wdt, s0_std=0.1, seed=900 + gated)
+    check_prefill(wk, oracle_mod, inp, gated, seed=12)
+
+
 def test_fused_gated_full_size(wk, oracle_mod):
     """The 1.5B-class prefill (B4 T1024 H32) with 8 kv heads and the read-out, in
     the launch configuration of the benchmark."""
