@@ -171,7 +171,8 @@ int wkv7_forward_fused(const void* r, const void* w_log, const void* k, const vo
  *   r, w_log, k, v, a, b, s0, y, sT, B, T, H, D : as in wkv7_forward for a
  *          dense batch (no seq_offsets); bf16 inputs only (io_dtype WKV7_BF16;
  *          WKV7_F32 returns WKV7_ERR_UNSUPPORTED: use wkv7_forward), w_log fp32
- *          or bf16.
+ *          or bf16.  B x T and B x ceil(T / 64) x H must be below 2^31
+ *          (WKV7_ERR_UNSUPPORTED otherwise).
  *   workspace : DEVICE scratch of at least wkv7_forward_long_workspace_bytes(B,
  *          T, H, D) bytes (49,408 per 64-token chunk and head), owned by the
  *          caller, 16-byte aligned, not read before it is written; it must not

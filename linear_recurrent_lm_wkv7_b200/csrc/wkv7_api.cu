@@ -258,6 +258,10 @@ int wkv7_forward_long(const void* r, const void* w_log, const void* k, const voi
     if (B <= 0 || T < 0 || H <= 0 || D <= 0) return WKV7_ERR_INVALID_ARG;
     if (!dtype_ok(io_dtype) || !dtype_ok(w_dtype)) return WKV7_ERR_INVALID_ARG;
     if (D != wkv7::kHead || io_dtype != WKV7_BF16) return WKV7_ERR_UNSUPPORTED;
+    // the first phase numbers token rows and (sequence, chunk, head) slots in 32 bits
+    if (static_cast<long long>(B) * T >= (1LL << 31) ||
+        static_cast<long long>(B) * ((T + 63) / 64) * H >= (1LL << 31))
+        return WKV7_ERR_UNSUPPORTED;
     if (T > 0 && (!r || !w_log || !k || !v || !a || !b || !y || !workspace)) return WKV7_ERR_INVALID_ARG;
     const void* ptrs[] = {r, w_log, k, v, a, b, s0, y, sT, workspace};
     for (const void* p : ptrs)

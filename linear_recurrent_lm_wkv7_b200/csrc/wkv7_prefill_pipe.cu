@@ -331,29 +331,64 @@ __global__ void __launch_bounds__(NTHR, 1)
         nchunks = static_cast<int>((total - blockIdx.x + gridDim.x - 1) / gridDim.x);
     }
     auto slot_of = [&](int c) { return static_cast<long>(blockIdx.x) + static_cast<long>(c) * gridDim.x; };
-    // first token row, head and valid rows of this block's c-th chunk
-    auto chunk_t0 = [&](int c) -> long {
-        if constexpr (EXPORT) {
-            const long q = slot_of(c) / H;
-            return (q / nch_seq) * T + (q % nch_seq) * L;
-        } else {
-            return tb + static_cast<long>(c) * L;
-        }
-    };
-    auto chunk_h = [&](int c) -> int {
-        if constexpr (EXPORT) return static_cast<int>(slot_of(c) % H);
-        else return h;
-    };
+    // EXPORT: slot = (n * nch_seq + j) * H + h, in 32-bit arithmetic (the host keeps every slot
+    // below 2^31)
+    const uint32_t H32 = static_cast<uint32_t>(H), nch32 = static_cast<uint32_t>(nch_seq);
+    auto slot_q = [&](int c) -> uint32_t { return static_cast<uint32_t>(slot_of(c)) / H32; };
     // kv head of k and v (the fused prologue shares them over H / H_kv heads); fixed per
     // block except in EXPORT mode, which has no prologue
     const int hk_unit = PRO ? h / (H / H_kv) : h;
-    auto chunk_hk = [&](int c) -> int {
-        if constexpr (EXPORT) return chunk_h(c);
-        else return hk_unit;
-    };
+    // valid rows of this block's c-th chunk
     auto chunk_nv = [&](int c) -> int {
         long rem;
-        if constexpr (EXPORT) rem = T - (slot_of(c) / H % nch_seq) * L;
+        if constexpr (EXPORT) rem = T - static_cast<long>(slot_q(c) % nch32) * L;
+        else rem = len - static_cast<long>(c) * L;
+        return static_cast<int>(rem < L ? rem : L);
+    };
+    // EXPORT: (sequence n, chunk j, head h) of a prep group's chunk.  A group's consecutive
+    // slots are 2 x gridDim.x apart; that step is split into heads, chunks and sequences once,
+    // so each next position follows by additions with carries (no division per chunk)
+    struct Pos {
+        uint32_t n, j, h;
+    };
+    auto pos_of = [&](int c) -> Pos {
+        if constexpr (EXPORT) {
+            const uint32_t sl = static_cast<uint32_t>(slot_of(c)), q = sl / H32;
+            return Pos{q / nch32, q % nch32, sl - q * H32};
+        } else {
+            return Pos{0u, 0u, 0u};
+        }
+    };
+    const uint32_t step_q = EXPORT ? 2u * gridDim.x / H32 : 0u;
+    const uint32_t step_h = EXPORT ? 2u * gridDim.x - step_q * H32 : 0u;
+    const uint32_t step_j = EXPORT ? step_q % nch32 : 0u, step_n = EXPORT ? step_q / nch32 : 0u;
+    auto advance2 = [&](Pos p) -> Pos {
+        if constexpr (EXPORT) {
+            p.h += step_h;
+            uint32_t cy = p.h >= H32 ? 1u : 0u;
+            p.h -= cy * H32;
+            p.j += step_j + cy;  // < 2 nch32
+            cy = p.j >= nch32 ? 1u : 0u;
+            p.j -= cy * nch32;
+            p.n += step_n + cy;
+        }
+        return p;
+    };
+    auto pos_t0 = [&](int c, const Pos& p) -> long {
+        if constexpr (EXPORT) return static_cast<long>(p.n) * T + static_cast<long>(p.j) * L;
+        else return tb + static_cast<long>(c) * L;
+    };
+    auto pos_h = [&](const Pos& p) -> int {
+        if constexpr (EXPORT) return static_cast<int>(p.h);
+        else return h;
+    };
+    auto pos_hk = [&](const Pos& p) -> int {
+        if constexpr (EXPORT) return static_cast<int>(p.h);
+        else return hk_unit;
+    };
+    auto pos_nv = [&](int c, const Pos& p) -> int {
+        long rem;
+        if constexpr (EXPORT) rem = T - static_cast<long>(p.j) * L;
         else rem = len - static_cast<long>(c) * L;
         return static_cast<int>(rem < L ? rem : L);
     };
@@ -435,9 +470,9 @@ __global__ void __launch_bounds__(NTHR, 1)
         int raw_issued = 0, raw_done = 0, v_issued = 0, v_done = 0;  // TMA loads (chunks) of this group
         constexpr uint32_t WB = sizeof(WT);
         // one thread each; `which`: 0 = w_log, 1 = r and k, 2 = a and b
-        auto issue_raw = [&](int cc, int which) {
-            const int t0 = static_cast<int>(chunk_t0(cc));
-            const int h = chunk_h(cc), hk = chunk_hk(cc);
+        auto issue_raw = [&](int cc, const Pos& pc, int which) {
+            const int t0 = static_cast<int>(pos_t0(cc, pc));
+            const int h = pos_h(pc), hk = pos_hk(pc);
             if (which == 0) {
                 // the first chunk's tile completes on rl (the group waits); later ones on rls,
                 // whose only waiter is the serial group, in chunk order
@@ -457,10 +492,12 @@ __global__ void __launch_bounds__(NTHR, 1)
                 tma_load_3d(gt + RAW_B, &maps.b, &bars.rab[g], 0, h, t0);
             }
         };
-        auto issue_v = [&](int cc) {  // one thread
+        auto issue_v = [&](int cc, const Pos& pc) {  // one thread
             mbar_arrive_expect_tx(&bars.vld[g], 8192u);
-            tma_load_3d(Vt, &maps.v, &bars.vld[g], 0, chunk_hk(cc), static_cast<int>(chunk_t0(cc)));
+            tma_load_3d(Vt, &maps.v, &bars.vld[g], 0, pos_hk(pc), static_cast<int>(pos_t0(cc, pc)));
         };
+        Pos pcur = pos_of(g);          // this group's chunk c
+        Pos pnext = advance2(pcur);    // and its chunk c + 2
         const bool zero_v = (map_flags & kMapZeroV) != 0;
         if (zero_v) {
             // v = 0: the V tile is cleared once and never loaded
@@ -470,10 +507,10 @@ __global__ void __launch_bounds__(NTHR, 1)
         }
         if (g < nchunks) {
             if (tg == 0) {
-                issue_raw(g, 0);
-                issue_raw(g, 1);
-                issue_raw(g, 2);
-                if (!zero_v) issue_v(g);
+                issue_raw(g, pcur, 0);
+                issue_raw(g, pcur, 1);
+                issue_raw(g, pcur, 2);
+                if (!zero_v) issue_v(g, pcur);
             }
             raw_issued = 1;
             v_issued = zero_v ? 0 : 1;
@@ -499,7 +536,7 @@ __global__ void __launch_bounds__(NTHR, 1)
 
         for (int c = g; c < nchunks; c += 2) {
             const int kk_ = c >> 1;
-            const int nv = chunk_nv(c);
+            const int nv = pos_nv(c, pcur);
 
             // ---- p1: decay products and the scaled operand tiles
             const bool ragged = nv < L;  // group-uniform
@@ -528,7 +565,7 @@ __global__ void __launch_bounds__(NTHR, 1)
                 if (tg == 0) {
                     if (kk_ >= 1) {
                         w_ok = mbar_wait(&bars.ready[g], static_cast<uint32_t>(kk_ - 1) & 1u, WAIT_NS);
-                        if (w_ok && !zero_v) issue_v(c);
+                        if (w_ok && !zero_v) issue_v(c, pcur);
                     }
                     w_ok = w_ok && mbar_wait(&bars.rrk[g], static_cast<uint32_t>(kk_) & 1u, WAIT_NS) &&
                            mbar_wait(&bars.rab[g], static_cast<uint32_t>(kk_) & 1u, WAIT_NS);
@@ -800,7 +837,7 @@ __global__ void __launch_bounds__(NTHR, 1)
             group_sync(bar_id, GROUP);
             // BK (the fp32 T) is dead: load the w_log tile of this group's next chunk
             if (c + 2 < nchunks) {
-                if (tg == 0) issue_raw(c + 2, 0);
+                if (tg == 0) issue_raw(c + 2, pnext, 0);
                 ++raw_issued;  // counted at the first of the chunk's three raw loads
             }
 
@@ -855,7 +892,7 @@ __global__ void __launch_bounds__(NTHR, 1)
             mma_phase ^= 1u;
             tc_fence_after();
             // NQ (Q) has been consumed by P: load r and k of this group's next chunk
-            if (c + 2 < nchunks && tg == 0) issue_raw(c + 2, 1);
+            if (c + 2 < nchunks && tg == 0) issue_raw(c + 2, pnext, 1);
             {
                 // P columns 0..63 -> AS (token rows get Rt added: R' = Rt + Mrb W; key rows Bh^T W),
                 // columns 64..127 -> BH ([Mrb Z; Bh^T Z])
@@ -879,7 +916,7 @@ __global__ void __launch_bounds__(NTHR, 1)
             group_sync(bar_id, GROUP);
 
             // RAM (Rt, At, Mak) is dead: load a and b of this group's next chunk
-            if (c + 2 < nchunks && tg == 0) issue_raw(c + 2, 2);
+            if (c + 2 < nchunks && tg == 0) issue_raw(c + 2, pnext, 2);
             // ---- OUT = [Mrb Z; Bh^T Z] V + [Mrk; Kh^T] V   (the serial group adds [R'; Bh^T W] S0^T)
             {
                 // ... and the serial group must have read this group's OUT columns of its previous chunk
@@ -902,6 +939,8 @@ __global__ void __launch_bounds__(NTHR, 1)
                 mbar_arrive(&bars.ready[g]);  // this chunk's [R'; Bh^T W] and Gamma_L are published
             }
             ++issued_out;
+            pcur = pnext;
+            pnext = advance2(pnext);
         }
         if (!ok && tg == 0) report_status(status, WKV7_ERR_DEVICE_TIMEOUT);
         // drain: an unwaited G/Q/P product, and the last OUT-pre product
@@ -937,6 +976,13 @@ __global__ void __launch_bounds__(NTHR, 1)
                 bulk_store(ex_as + slot * 16384, sm + OFF_AS, 16384u);
                 bulk_commit();
             }
+            if (ts < 64) ex_gam[slot * 64 + ts] = gam_all[g * 128 + (kk_ & 1) * 64 + ts];
+            if (ts == 0) {
+                // the other group's next conversion waits for the shared tile: release it
+                // before the OUT columns are read
+                bulk_wait_read<0>();                        // the copy has read the shared tile
+                mbar_arrive(&bars.asfree[g]);
+            }
             float* orow = ex_out + slot * 8192 + ts * 4;
 #pragma unroll 1
             for (int q = 0; q < 2; ++q) {
@@ -946,11 +992,6 @@ __global__ void __launch_bounds__(NTHR, 1)
                 for (int i = 0; i < 8; ++i)
                     *reinterpret_cast<float4*>(orow + (8 * q + i) * 512) =
                         make_float4(o[4 * i], o[4 * i + 1], o[4 * i + 2], o[4 * i + 3]);
-            }
-            if (ts < 64) ex_gam[slot * 64 + ts] = gam_all[g * 128 + (kk_ & 1) * 64 + ts];
-            if (ts == 0) {
-                bulk_wait_read<0>();                        // the copy has read the shared tile
-                mbar_arrive(&bars.asfree[g]);
             }
             tc_fence_before();
             group_sync(bar_id, GROUP);

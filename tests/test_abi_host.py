@@ -246,6 +246,10 @@ def test_forward_long_rejects_bad_arguments(wk):
     assert call(*_fwd_long(wk, ws=0x1000 + 0x3000000)) == -1  # workspace overlaps v
     assert call(*_fwd_long(wk, y=0x1000 + 0x9000000)) == -1  # y aliases the workspace
     assert call(*_fwd_long(wk, sT=0x1000 + 0x4000000)) == -1  # sT overlaps a
+    # token rows and (sequence, chunk, head) slots are numbered in 32 bits
+    assert call(*_fwd_long(wk, B=2, T=1 << 30, H=1, wsb=0)) == -2
+    assert call(*_fwd_long(wk, B=1 << 11, T=1 << 20, H=1, wsb=0)) == -2
+    assert call(*_fwd_long(wk, B=1, T=1 << 24, H=1 << 13, wsb=0)) == -2
 
 
 def test_c_program_compiles_and_links(wk, tmp_path):
