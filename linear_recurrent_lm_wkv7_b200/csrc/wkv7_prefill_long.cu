@@ -23,7 +23,9 @@
 // Phase 2 streams the workspace through a ring of bulk copies (4 or 6 stages)
 // issued by a producer warp (full / empty mbarriers, bounded waits), which also
 // prefetches the chunk one ring-depth ahead into L2.  The product is issued as
-// tcgen05 (N = 64, the block's NV columns first in the operand tile, zeros after):
+// tcgen05 (N = 64, the block's NV columns first in the operand tile, zeros after; an
+// N = NV product over a K-major operand, one row per value column, needs NV 2-byte
+// stores per thread and chunk and took 3 % longer per call with NV = 16):
 // a warp-level mma.sync form of it, with the state in accumulator registers, was
 // measured slower on B1 T16384 H40 (268 us with four warps, 329 us with eight,
 // against 176 us: each warp has ~180 dependent instructions per chunk).
@@ -44,14 +46,15 @@ constexpr int NTHR = NCOMP + 32;         // + one producer warp
 constexpr uint64_t WAIT_NS = 1000000000ull;
 constexpr uint32_t ID_KM64 = idesc_f32acc(1, 128, 64, 0, 1);  // bf16, B MN-major, N = 64
 
-// per-block geometry for NV value columns: with 16 columns two blocks share an SM
-// (four chunks in flight each), with 32 or 64 one block holds six or four
+// per-block geometry for NV value columns (16 or 64), four chunks in flight: with 16
+// columns two blocks share an SM
 template <int NV>
 struct ScanGeom {
+    static_assert(NV == 16 || NV == 64, "value columns per block");
     static constexpr uint32_t OUT_PART = NV * 512u;  // this block's columns of OUTpre (NV / 4 quads)
     static constexpr uint32_t BYTES = AS_BYTES + OUT_PART + GAM_BYTES;  // one chunk's bulk copies
     static constexpr uint32_t STAGE = (BYTES + 1023u) / 1024u * 1024u;  // the AS tile is 1024-aligned
-    static constexpr int NST = NV == 32 ? 6 : 4;                         // ring stages
+    static constexpr int NST = 4;                                       // ring stages
     static constexpr uint32_t OFF_ST = NST * STAGE;                     // S0^T, bf16 MN-major (64 x 64)
     static constexpr uint32_t OFF_BAR = OFF_ST + 8192;                  // full[NST], empty[NST], mma, tmem slot
     static constexpr uint32_t SMEM = OFF_BAR + (2 * NST + 2) * 8 + 1024;
@@ -64,7 +67,7 @@ __device__ __forceinline__ void prefetch_l2_bulk(const void* src, uint32_t bytes
     asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
 }
 
-// the first NV fp32 columns of this thread's TMEM lane (NV = 16, 32 or 64)
+// the first NV fp32 columns of this thread's TMEM lane (NV = 16 or 64)
 template <int NV>
 __device__ __forceinline__ void tmem_load_cols(uint32_t taddr, float (&o)[NV]) {
     if constexpr (NV == 16) {
@@ -293,11 +296,12 @@ cudaError_t launch_prefill_long(const PrefillArgs& p, int w_dtype, void* ws, cud
     if (e != cudaSuccess) return e;
     e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     if (e != cudaSuccess) return e;
-    // value columns per block: as few as keep every block of the grid resident at once
-    // (up to two per SM with 16 columns, one with 32)
+    // value columns per block: 16 while the four blocks of every unit stay resident at
+    // once (two per SM), else one block of all 64 columns per unit.  (Two blocks of 32
+    // columns, one per SM, never beat the 16-column split where both fit: 198 against
+    // ~171 us on B1 T16384 H40.)
     const long units = static_cast<long>(p.B) * p.H;
     if (units * 4 <= 2L * sms) return launch_scan<16>(p, q, stream);
-    if (units * 2 <= sms) return launch_scan<32>(p, q, stream);
     return launch_scan<64>(p, q, stream);
 }
 

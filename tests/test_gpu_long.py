@@ -72,8 +72,8 @@ def test_long_dense_lengths(wk, oracle_mod, T, wdt):
 @pytest.mark.parametrize("B,T,H", [(4, 200, 10), (8, 130, 20)])
 def test_long_wider_batches(wk, oracle_mod, B, T, H):
     """40 and 160 (sequence, head) units: the state pass splits each unit over
-    two blocks of 32 value columns, or runs it whole (64), instead of four blocks
-    of 16 for the smaller batches."""
+    four blocks of 16 value columns, or runs it whole (64 columns) when four
+    blocks per unit would not stay resident."""
     check(wk, oracle_mod, W.make_prefill(B, T, H, io="bf16", wdt="f32", s0_std=0.1, seed=820 + B))
 
 
