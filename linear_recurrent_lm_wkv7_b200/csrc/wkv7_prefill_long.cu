@@ -212,16 +212,21 @@ __global__ void __launch_bounds__(NTHR, 1)
             mma_pending = false;
             mma_phase ^= 1u;
             tc_fence_after();
+            // OUTpre and Gamma_L from the stage first (the TMEM read below is fenced against
+            // reordering, so the shared loads are issued ahead of it explicitly)
             const float* pre = reinterpret_cast<const float*>(stage + AS_BYTES) + ts * 4;
+            float4 p4[NV / 4];
+#pragma unroll
+            for (int i = 0; i < NV / 4; ++i) p4[i] = *reinterpret_cast<const float4*>(pre + i * 512);
+            const float GL = ts >= 64 ? reinterpret_cast<const float*>(stage + AS_BYTES + G::OUT_PART)[x] : 1.f;
             float o[NV];
             tmem_load_cols<NV>(tmem + lane_base, o);
 #pragma unroll
             for (int i = 0; i < NV / 4; ++i) {
-                const float4 p4 = *reinterpret_cast<const float4*>(pre + i * 512);
-                o[4 * i] += p4.x;
-                o[4 * i + 1] += p4.y;
-                o[4 * i + 2] += p4.z;
-                o[4 * i + 3] += p4.w;
+                o[4 * i] += p4[i].x;
+                o[4 * i + 1] += p4[i].y;
+                o[4 * i + 2] += p4[i].z;
+                o[4 * i + 3] += p4[i].w;
             }
             if (ts < 64) {
                 if (ts < nv && y != nullptr) {
@@ -233,7 +238,6 @@ __global__ void __launch_bounds__(NTHR, 1)
                                        pack_bf16x2(o[i + 4], o[i + 5]), pack_bf16x2(o[i + 6], o[i + 7]));
                 }
             } else {
-                const float GL = reinterpret_cast<const float*>(stage + AS_BYTES + G::OUT_PART)[x];
                 // 1 / Gamma_t must stay far inside the fp32 / bf16 range (false for NaN too)
                 if (!(GL >= kMinGammaL)) report_status(status, WKV7_ERR_DECAY_RANGE);
 #pragma unroll
