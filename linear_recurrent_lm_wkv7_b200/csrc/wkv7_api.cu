@@ -260,7 +260,7 @@ int wkv7_forward_long(const void* r, const void* w_log, const void* k, const voi
     if (D != wkv7::kHead || io_dtype != WKV7_BF16) return WKV7_ERR_UNSUPPORTED;
     // the first phase numbers token rows and (sequence, chunk, head) slots in 32 bits
     if (static_cast<long long>(B) * T >= (1LL << 31) ||
-        static_cast<long long>(B) * ((T + 63) / 64) * H >= (1LL << 31))
+        static_cast<long long>(B) * ((static_cast<long long>(T) + 63) / 64) * H >= (1LL << 31))
         return WKV7_ERR_UNSUPPORTED;
     if (T > 0 && (!r || !w_log || !k || !v || !a || !b || !y || !workspace)) return WKV7_ERR_INVALID_ARG;
     const void* ptrs[] = {r, w_log, k, v, a, b, s0, y, sT, workspace};

@@ -250,6 +250,8 @@ def test_forward_long_rejects_bad_arguments(wk):
     assert call(*_fwd_long(wk, B=2, T=1 << 30, H=1, wsb=0)) == -2
     assert call(*_fwd_long(wk, B=1 << 11, T=1 << 20, H=1, wsb=0)) == -2
     assert call(*_fwd_long(wk, B=1, T=1 << 24, H=1 << 13, wsb=0)) == -2
+    # T + 63 must not wrap in the slot count: 2^25 chunks x 2^7 heads
+    assert call(*_fwd_long(wk, B=1, T=(1 << 31) - 1, H=1 << 7, wsb=0)) == -2
 
 
 def test_c_program_compiles_and_links(wk, tmp_path):
