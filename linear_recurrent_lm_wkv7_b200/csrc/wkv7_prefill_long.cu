@@ -109,7 +109,7 @@ __global__ void __launch_bounds__(NTHR, 1)
     const int tid = threadIdx.x, warp = tid >> 5;
     const int part = blockIdx.x % NPART, unit = blockIdx.x / NPART, h = unit % H, n = unit / H;
     const int v0 = part * NV;  // this block's value columns v0 .. v0 + NV - 1
-    const int nch = (T + L - 1) / L;
+    const int nch = static_cast<int>((static_cast<long>(T) + L - 1) / L);
     const long cbase = static_cast<long>(n) * nch;  // the sequence's first chunk over the batch
     const long tstride = static_cast<long>(H) * kHead, hoff = static_cast<long>(h) * kHead;
     const long sbase = (static_cast<long>(n) * H + h) * kHead * kHead;
