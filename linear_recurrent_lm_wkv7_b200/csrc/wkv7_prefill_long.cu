@@ -275,7 +275,7 @@ cudaError_t launch_scan(const PrefillArgs& p, const PrefillArgs& q, cudaStream_t
     auto kern = wkv7_long_scan_kernel<NV>;
     const cudaError_t e = configure_smem_once(kern, static_cast<int>(ScanGeom<NV>::SMEM), configured);
     if (e != cudaSuccess) return e;
-    kern<<<static_cast<unsigned>(p.B * p.H * (64 / NV)), NTHR, ScanGeom<NV>::SMEM, stream>>>(
+    kern<<<static_cast<unsigned>(static_cast<long>(p.B) * p.H * (64 / NV)), NTHR, ScanGeom<NV>::SMEM, stream>>>(
         q.ex_as, q.ex_out, q.ex_gam, p.s0, static_cast<__nv_bfloat16*>(p.y), p.sT, p.T, p.H, p.status);
     return cudaGetLastError();
 }
